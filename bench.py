@@ -1,0 +1,592 @@
+#!/usr/bin/env python
+"""Benchmark of the cached GQA attention step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One "step" is one pass of the whole hot path over one batch: for every layer,
+RoPE + cache append (kvattn_rope_append) then attention (kvattn_decode, or
+kvattn_prefill_chunk for the prefill workload), each layer with its own
+cache.  The default workload is batched ragged decode: B=64 sequences, 32
+layers with separate [64, 8192, 8, 128] bf16 caches (64 GiB in HBM, far
+larger than L2, so every step streams its K/V rows from HBM), start positions
+uniform in [512, 8191].
+
+Printed: one JSON line (rank 0) with the KV-cache GB/s of the whole job, the
+decode-kernel roofline, end-to-end GB/s with host buffers, the fp64 oracle's
+throughput on a bounded sample of host cores, and the SM clocks seen during
+the timed region.  With N > 1 (torchrun) every rank runs an independent
+replica on its own GPU; the time is the maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import kvattn_synth as ks  # noqa: E402
+from kvattn_synth.workloads import HEADLINE, WORKLOADS  # noqa: E402
+
+METRIC = "GQA decode: KV-cache HBM GB/s (% of peak) and decode steps/s per layer"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+# ----------------------------------------------------------------- helpers
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    pkg = os.path.join(ROOT, "gqa_decode_attention_kvattn_b200", "csrc")
+    for p in sorted(glob.glob(os.path.join(pkg, "*"))):
+        if p.endswith((".cu", ".cuh", ".h")):
+            with open(p, "rb") as f:
+                h.update(os.path.basename(p).encode())
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel_tag: str, workload: str):
+    """DRAM bytes per launch recorded from an ncu capture, if the kernels have
+    not changed since: profiles/<kernel>__<workload>.md holds
+    `traffic_bytes_per_launch:` and `source_hash:` lines."""
+    path = os.path.join(ROOT, "profiles", f"{kernel_tag}__{workload}.md")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line:
+                k, _, v = line.partition(":")
+                vals[k.strip().strip("-* `")] = v.strip().strip("` ")
+    try:
+        if vals.get("source_hash") != kernel_source_hash():
+            return None
+        return float(vals["traffic_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id: str | None):
+        self.bus_id = bus_id
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+        if self.bus_id:
+            cmd += ["-i", self.bus_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def bus_id_of(dev):
+    import torch
+    try:
+        p = torch.cuda.get_device_properties(dev)
+        return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+    except Exception:
+        return None
+
+
+# ----------------------------------------------------------------- state
+class Layer:
+    pass
+
+
+def build_state(w, seed, device):
+    import torch
+    import gqa_decode_attention_kvattn_b200 as kv
+    sp = w.start_pos(seed)
+    dsp = torch.from_numpy(sp).to(device)
+    rope = kv.LLAMA3_1 if w.scaled_rope else kv.LLAMA3
+    layers = []
+    for l in range(w.layers):
+        L = Layer()
+        L.q = torch.empty((w.B, w.T, w.H, 128), dtype=torch.bfloat16, device=device)
+        L.k = torch.empty((w.B, w.T, w.Hkv, 128), dtype=torch.bfloat16, device=device)
+        L.v = torch.empty_like(L.k)
+        ks.device_normal_bf16(seed, ks.layer_stream(ks.STREAM_Q, l), L.q)
+        ks.device_normal_bf16(seed, ks.layer_stream(ks.STREAM_K_NEW, l), L.k)
+        ks.device_normal_bf16(seed, ks.layer_stream(ks.STREAM_V_NEW, l), L.v)
+        L.ck = torch.empty((w.B, w.S, w.Hkv, 128), dtype=torch.bfloat16, device=device)
+        L.cv = torch.empty_like(L.ck)
+        ks.device_cache_fill(seed, ks.layer_stream(ks.STREAM_CACHE_K, l), L.ck, dsp)
+        ks.device_cache_fill(seed, ks.layer_stream(ks.STREAM_CACHE_V, l), L.cv, dsp)
+        L.q_rot = torch.empty_like(L.q)
+        L.out = torch.empty_like(L.q)
+        layers.append(L)
+    if w.kind == "decode":
+        ws_bytes = kv.kvattn_decode_workspace_bytes(w.B, w.H, w.Hkv, w.S, w.kv_len_hint)
+    else:
+        ws_bytes = kv.kvattn_prefill_workspace_bytes(w.B, w.H, w.Hkv, w.S, w.T, w.kv_len_hint)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    torch.cuda.synchronize(device)
+    return dict(sp=sp, dsp=dsp, rope=rope, layers=layers, ws=ws, ws_bytes=ws_bytes, status=status)
+
+
+def run_step(w, st, events=None):
+    import gqa_decode_attention_kvattn_b200 as kv
+    for i, L in enumerate(st["layers"]):
+        kv.kvattn_rope_append(L.q, L.k, L.v, L.ck, L.cv, st["dsp"], rope=st["rope"], q_rot=L.q_rot,
+                              dev_status=st["status"])
+        if events is not None:
+            events[i][0].record()
+        if w.kind == "decode":
+            kv.kvattn_decode(L.q_rot, L.ck, L.cv, st["dsp"], max_kv_len_hint=w.kv_len_hint, out=L.out,
+                             workspace=st["ws"], dev_status=st["status"])
+        else:
+            kv.kvattn_prefill_chunk(L.q_rot, L.ck, L.cv, st["dsp"], max_kv_len_hint=w.kv_len_hint, out=L.out,
+                                    workspace=st["ws"], dev_status=st["status"])
+        if events is not None:
+            events[i][1].record()
+
+
+def work_units(w, sp):
+    """(algorithmic KV bytes, flops) of the attention of one layer."""
+    import gqa_decode_attention_kvattn_b200 as kv
+    return kv.attention_kv_bytes(sp, w.T, w.Hkv), kv.prefill_flops(sp, w.T, w.H)
+
+
+# ----------------------------------------------------------------- CPU oracle
+def oracle_sample_inputs_from_device(w, st, layer, seqs):
+    """Host copies (exact bf16 bits) of the inputs of some sequences of one
+    layer, taken before the step rewrites nothing they depend on."""
+    import torch
+    L = st["layers"][layer]
+    out = []
+    for b in seqs:
+        spb = int(st["sp"][b])
+        def h(t):
+            return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+        out.append((b, spb, h(L.q[b]), h(L.k[b]), h(L.v[b]), h(L.ck[b, :spb]), h(L.cv[b, :spb])))
+    return out
+
+
+def oracle_sample_inputs_host(w, seed, layer, seqs):
+    """The same bits made by the host generator (no GPU involved)."""
+    sp = w.start_pos(seed)
+    d = 128
+    out = []
+    for b in seqs:
+        spb = int(sp[b])
+        q = ks.normal_bf16(seed, ks.layer_stream(ks.STREAM_Q, layer), b * w.T * w.H * d, w.T * w.H * d)
+        k = ks.normal_bf16(seed, ks.layer_stream(ks.STREAM_K_NEW, layer), b * w.T * w.Hkv * d, w.T * w.Hkv * d)
+        v = ks.normal_bf16(seed, ks.layer_stream(ks.STREAM_V_NEW, layer), b * w.T * w.Hkv * d, w.T * w.Hkv * d)
+        ck = ks.cache_rows(seed, ks.layer_stream(ks.STREAM_CACHE_K, layer), b, w.S, w.Hkv, d, 0, spb, spb)
+        cv = ks.cache_rows(seed, ks.layer_stream(ks.STREAM_CACHE_V, layer), b, w.S, w.Hkv, d, 0, spb, spb)
+        out.append((b, spb, q.reshape(w.T, w.H, d), k.reshape(w.T, w.Hkv, d), v.reshape(w.T, w.Hkv, d), ck, cv))
+    return out
+
+
+def oracle_time(w, samples, rope_scaled):
+    """Run the oracle (rope + append + attention) on each sampled sequence;
+    return (seconds, KV bytes, flops)."""
+    import oracle
+    f = oracle.rope_freqs(128, 500000.0, rope_scaled)
+    secs, nbytes, flops = 0.0, 0, 0
+    for (b, spb, q, k, v, ck_rows, cv_rows) in samples:
+        S = spb + w.T
+        ck = np.zeros((1, S, w.Hkv, 128), np.uint16)
+        cv = np.zeros((1, S, w.Hkv, 128), np.uint16)
+        ck[0, :spb] = ck_rows
+        cv[0, :spb] = cv_rows
+        spa = np.array([spb], np.int32)
+        t0 = time.perf_counter()
+        _, _, rc = oracle.step(q[None].copy(), k[None].copy(), v[None].copy(), ck, cv, spa, f)
+        secs += time.perf_counter() - t0
+        assert rc == 0
+        nbytes += 2 * w.Hkv * 128 * 2 * (spb + w.T) * w.T if w.kind == "prefill" else 2 * w.Hkv * 128 * 2 * (spb + 1)
+        flops += 4 * 128 * w.H * (w.T * (spb + 1) + w.T * (w.T - 1) // 2)
+    return secs, nbytes, flops
+
+
+def cpu_baseline_leg(w, st, seed, target_s=12.0):
+    import oracle
+    cores = oracle.max_threads()
+    seqs = list(range(w.B))
+    total_s = total_b = total_f = 0.0
+    layers_done = 0
+    for layer in range(w.layers):
+        samples = oracle_sample_inputs_from_device(w, st, layer, seqs)
+        s, b, f = oracle_time(w, samples, w.scaled_rope)
+        total_s += s
+        total_b += b
+        total_f += f
+        layers_done += 1
+        if total_s >= target_s or total_s * (layers_done + 1) / layers_done > 30.0:
+            break
+    if w.kind == "decode":
+        value, unit = total_b / total_s / 1e9, "GB/s"
+    else:
+        value, unit = total_f / total_s / 1e12, "TFLOP/s"
+    return {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
+            "sample": f"fp64 C oracle (rope+append+attention) on all {len(seqs)} sequences of "
+                      f"{layers_done} of {w.layers} layer(s) of workload {w.name}, OpenMP over {cores} host threads; "
+                      f"{total_s:.2f} s of oracle time"}
+
+
+# ----------------------------------------------------------------- arms
+def run_ours(args, w, rank, world, device):
+    import torch
+    import torch.distributed as dist
+    import gqa_decode_attention_kvattn_b200 as kv
+
+    st = build_state(w, args.seed, device)
+    nl = len(st["layers"])
+    kv_bytes_layer, flops_layer = work_units(w, st["sp"])
+    merge = 1 if st["ws_bytes"] > 0 else 0
+
+    # warm-up, eager
+    for _ in range(args.warmup):
+        run_step(w, st)
+    torch.cuda.synchronize(device)
+    if int(st["status"].item()) != 0:
+        raise RuntimeError(f"device status {st['status'].item()} after warm-up")
+
+    # capture one step (every layer) with timing events around each attention call
+    events = [(torch.cuda.Event(enable_timing=True, external=True),
+               torch.cuda.Event(enable_timing=True, external=True)) for _ in range(nl)]
+    graph = None
+    if not args.no_graph:
+        stream = torch.cuda.Stream(device)
+        stream.wait_stream(torch.cuda.current_stream(device))
+        with torch.cuda.stream(stream):
+            run_step(w, st)  # one more warm-up on the capture stream
+        torch.cuda.current_stream(device).wait_stream(stream)
+        torch.cuda.synchronize(device)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            run_step(w, st, events)
+        for _ in range(max(1, args.warmup)):
+            graph.replay()
+        torch.cuda.synchronize(device)
+
+    # ---------------- timed region
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    sampler = ClockSampler(bus_id_of(device))
+    sampler.start()
+    time.sleep(0.3)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.steps):
+        if graph is not None:
+            graph.replay()
+        else:
+            run_step(w, st, events)
+    t1.record()
+    torch.cuda.synchronize(device)
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    ms = t0.elapsed_time(t1)
+    attn_ms = [a.elapsed_time(b) for a, b in events]   # the last step's attention calls
+    if world > 1:
+        tt = torch.tensor([ms], dtype=torch.float64, device=device)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    status = int(st["status"].item())
+
+    secs = ms / 1e3
+    ms_per_step = ms / args.steps
+    hbm_peak, tf_peak, peak_src = measured_peaks()
+    attn_avg_ms = float(np.mean(attn_ms))
+    if w.kind == "decode":
+        value = world * args.steps * nl * kv_bytes_layer / secs / 1e9
+        unit = "GB/s"
+        achieved = kv_bytes_layer / (attn_avg_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(achieved / hbm_peak, 4),
+                "traffic": profiled_traffic("decode_splitk", w.name),
+                "kernel": "kvattn_decode (split-K kernel + LSE merge kernel)",
+                "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback 6650 GB/s",
+                "avg_launch_ms": round(attn_avg_ms, 5), "launches_timed": nl,
+                "bytes_per_launch": kv_bytes_layer}
+    else:
+        value = world * args.steps * nl * flops_layer / secs / 1e12
+        unit = "TFLOP/s"
+        achieved = flops_layer / (attn_avg_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": tf_peak, "unit": "TFLOP/s",
+                "frac": round(achieved / tf_peak, 4),
+                "traffic": profiled_traffic("prefill_chunk", w.name),
+                "kernel": "kvattn_prefill_chunk",
+                "peak_source": f"{peak_src} (MEASURED_PEAKS.json bf16_tflops)",
+                "avg_launch_ms": round(attn_avg_ms, 5), "launches_timed": nl,
+                "flops_per_launch": flops_layer}
+
+    # ---------------- end to end with host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, w, st, device, kv_bytes_layer, flops_layer, world)
+
+    line = {
+        "metric": METRIC if w.kind == "decode" else "GQA chunked prefill: attention TFLOP/s (% of bf16 tensor peak)",
+        "value": round(value, 2), "unit": unit, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.B, "new_tokens": w.T, "q_heads": w.H, "kv_heads": w.Hkv,
+                   "head_dim": 128, "cache_rows": w.S, "layers": nl,
+                   "start_pos": f"uniform [{w.sp_lo}, {w.sp_hi}] seed {args.seed}" if w.sp_lo != w.sp_hi else w.sp_lo,
+                   "rope": "llama3.1 scaled, theta 500000" if w.scaled_rope else "theta 500000",
+                   "l2": "inputs larger than L2" if nl * w.B * w.S * w.Hkv * 512 > 256e6 else
+                         "inputs smaller than L2 (latency-bound case)",
+                   "graph": graph is not None,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "pct_of_hbm_peak": round(100 * (value / world) / hbm_peak, 2) if w.kind == "decode" else None,
+        "layer_steps_per_s": round(world * args.steps * nl / secs, 1),
+        "steps_per_s": round(world * args.steps / secs, 2),
+        "roofline": roof,
+        "gpu_launches": args.steps * nl * (2 + merge),
+        "clocks": clocks,
+        "device_status": status,
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_leg(w, st, args.seed)
+    return line
+
+
+def run_e2e(args, w, st, device, kv_bytes_layer, flops_layer, world):
+    """Same step through the C ABI with host buffers: every step copies its
+    inputs (q, k_new, v_new of every layer, start_pos) from pinned host memory
+    and reads every layer's output back."""
+    import torch
+    import torch.distributed as dist
+    layers = st["layers"]
+    h_in = [(L.q.cpu().pin_memory(), L.k.cpu().pin_memory(), L.v.cpu().pin_memory()) for L in layers]
+    h_out = [torch.empty_like(L.out, device="cpu").pin_memory() for L in layers]
+    h_sp = torch.from_numpy(st["sp"]).pin_memory()
+
+    def e2e_step():
+        st["dsp"].copy_(h_sp, non_blocking=True)
+        for (hq, hk, hv), L in zip(h_in, layers):
+            L.q.copy_(hq, non_blocking=True)
+            L.k.copy_(hk, non_blocking=True)
+            L.v.copy_(hv, non_blocking=True)
+        run_step(w, st)
+        for ho, L in zip(h_out, layers):
+            ho.copy_(L.out, non_blocking=True)
+
+    steps = max(3, args.steps // 2)
+    stream = torch.cuda.Stream(device)
+    stream.wait_stream(torch.cuda.current_stream(device))
+    with torch.cuda.stream(stream):
+        e2e_step()
+    torch.cuda.current_stream(device).wait_stream(stream)
+    torch.cuda.synchronize(device)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        e2e_step()
+    graph.replay()
+    torch.cuda.synchronize(device)
+    if world > 1:
+        dist.barrier()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        graph.replay()
+    t1.record()
+    torch.cuda.synchronize(device)
+    ms = t0.elapsed_time(t1)
+    if world > 1:
+        tt = torch.tensor([ms], dtype=torch.float64, device=device)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    secs = ms / 1e3
+    h2d = sum(x.numel() * x.element_size() for trip in h_in for x in trip) + h_sp.numel() * 4
+    d2h = sum(x.numel() * x.element_size() for x in h_out)
+    nl = len(layers)
+    if w.kind == "decode":
+        val, unit = world * steps * nl * kv_bytes_layer / secs / 1e9, "GB/s"
+    else:
+        val, unit = world * steps * nl * flops_layer / secs / 1e12, "TFLOP/s"
+    return {"value": round(val, 2), "unit": unit, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "steps": steps, "ms_per_step": round(ms / steps, 5)}
+
+
+def run_reference(args, w):
+    """The fp64 oracle, as it stands, on the host cores: each step runs it on
+    a bounded sample (the first sequences of layer 0) of the workload."""
+    import oracle
+    cores = oracle.max_threads()
+    nseq = min(w.B, 16 if w.kind == "decode" else 1)
+    seqs = list(range(nseq))
+    try:
+        import torch
+        if torch.cuda.is_available():
+            st = build_state_sample(w, args.seed, seqs)
+            samples = st
+        else:
+            samples = oracle_sample_inputs_host(w, args.seed, 0, seqs)
+    except Exception:
+        samples = oracle_sample_inputs_host(w, args.seed, 0, seqs)
+    for _ in range(args.warmup):
+        oracle_time(w, samples, w.scaled_rope)
+    tot_s = tot_b = tot_f = 0.0
+    for _ in range(args.steps):
+        s, b, f = oracle_time(w, samples, w.scaled_rope)
+        tot_s += s
+        tot_b += b
+        tot_f += f
+    if w.kind == "decode":
+        value, unit = tot_b / tot_s / 1e9, "GB/s"
+    else:
+        value, unit = tot_f / tot_s / 1e12, "TFLOP/s"
+    sample = (f"fp64 C oracle (rope+append+attention) on sequences {seqs[0]}..{seqs[-1]} of layer 0 of "
+              f"workload {w.name} per step, OpenMP over {cores} host threads")
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": unit, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * tot_s / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.B, "new_tokens": w.T, "q_heads": w.H, "kv_heads": w.Hkv,
+                       "head_dim": 128, "cache_rows": w.S, "layers": w.layers},
+            "cpu_baseline": {"value": round(value, 4), "unit": unit, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def build_state_sample(w, seed, seqs):
+    """Inputs of the sampled sequences of layer 0, made by the device
+    generator and copied to the host (exact bits; no product kernel runs)."""
+    import torch
+    dev = torch.device("cuda", 0)
+    sp = w.start_pos(seed)
+    d = 128
+    out = []
+    for b in seqs:
+        spb = int(sp[b])
+        def gen(stream, shape, offset):
+            t = torch.empty(shape, dtype=torch.bfloat16, device=dev)
+            ks.device_normal_bf16(seed, stream, t, offset=offset)
+            return t.view(torch.int16).cpu().numpy().view(np.uint16)
+        q = gen(ks.layer_stream(ks.STREAM_Q, 0), (w.T, w.H, d), b * w.T * w.H * d)
+        k = gen(ks.layer_stream(ks.STREAM_K_NEW, 0), (w.T, w.Hkv, d), b * w.T * w.Hkv * d)
+        v = gen(ks.layer_stream(ks.STREAM_V_NEW, 0), (w.T, w.Hkv, d), b * w.T * w.Hkv * d)
+        row = w.Hkv * d
+        ck = gen(ks.layer_stream(ks.STREAM_CACHE_K, 0), (spb, w.Hkv, d), b * w.S * row) if spb else \
+            np.zeros((0, w.Hkv, d), np.uint16)
+        cv = gen(ks.layer_stream(ks.STREAM_CACHE_V, 0), (spb, w.Hkv, d), b * w.S * row) if spb else \
+            np.zeros((0, w.Hkv, d), np.uint16)
+        out.append((b, spb, q, k, v, ck, cv))
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=HEADLINE)
+    ap.add_argument("--seed", type=int, default=ks.DEFAULT_SEED)
+    ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    w = WORKLOADS[args.workload]
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, w)), flush=True)
+        return 0
+
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    import gqa_decode_attention_kvattn_b200 as kv
+    kv.library()  # fail loudly when the CUDA library is missing
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+    try:
+        line = run_ours(args, w, rank, world, device)
+    finally:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

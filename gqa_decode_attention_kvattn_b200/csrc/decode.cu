@@ -1,0 +1,564 @@
+// K2 + K3: split-K grouped-query attention over the KV cache, on CUDA cores.
+//
+// What it computes ("Llama 3.1 8B KV cache", section "The cache itself is
+// concatenation"; "Llama 3.1 8B · Repeat heads"; the mask comment of model.py
+// 281-302 in "Llama 3 8B · KV cache"): for query token t of sequence b and
+// query head h, with G = H / Hkv and j = floor(h / G),
+//   out[b,t,h,:] = sum_{r < L} softmax_r(scale * q[b,t,h,:] . K[b,r,j,:]) V[b,r,j,:]
+// over the L = start_pos[b] + t + 1 visible cache rows.
+//
+// Work decomposition.  An "item" is (query row set v = (b,t), split s, KV
+// head j): rows [s*C, min((s+1)*C, L)) of KV head j, serving the G query
+// heads of that group from the same tiles (no materialised repeat_kv).  Items
+// are numbered with the KV head fastest, so CTAs that run side by side read
+// the same cache rows of neighbouring heads.  A persistent grid of
+// (SMs x CTAs per SM) walks the items round-robin.
+//
+// Inside a CTA: one producer warp issues TMA tensor loads of 32-row K and V
+// tiles (32 x 256 B each, row stride Hkv*256 B) into a 4-stage shared-memory
+// ring; four consumer warps each take 8 rows of every tile.  Sixteen lanes
+// share one cache row, each holding 8 of its 128 elements, so a half-warp
+// reads a row's 256 bytes from shared memory conflict-free.  Partial dot
+// products of RB rows x G heads are reduce-scattered across the 16 lanes
+// (each lane ends with complete scores), the online softmax runs in log2
+// units (the scale is folded into q), and the probabilities are broadcast
+// through shared memory for the P.V accumulation.  FMAs use the packed
+// fp32x2 form.  At the end of an item the eight half-warp states (max, sum,
+// o) are merged; a single-split row set writes bf16 output directly, others
+// write (o, max, sum) partials that K3 merges by log-sum-exp:
+//   M = max_s m_s,  out = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.
+#include "kvattn_device.cuh"
+#include "kvattn_internal.h"
+
+#include <algorithm>
+
+namespace kvattn {
+namespace {
+
+constexpr int kTileRows = 32;
+constexpr int kStages = 4;
+constexpr int kConsumerWarps = 4;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kHalfWarps = kConsumerWarps * 2;
+constexpr int kMaxRowSets = 4096;  // (b,t) row sets handled with a split table
+constexpr uint32_t kTileBytes = kTileRows * kHeadDim * 2;
+
+constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
+
+template <int G>
+struct Shape {
+  static constexpr int RB = (G >= 8) ? 2 : 4;     // rows per half-warp batch
+  static constexpr int NV = G * RB;                // partial dot products per lane
+  static constexpr int LOG2NV = ilog2(NV);
+  static constexpr int RS = LOG2NV < 4 ? LOG2NV : 4;  // reduce-scatter steps
+  static constexpr int SLOTS = NV >> RS;           // complete scores per lane
+  static constexpr int REP = 1 << (4 - RS);        // lanes holding the same score
+  static constexpr int PASSES = kTileRows / (kHalfWarps * RB);
+  static_assert(kTileRows % (kHalfWarps * RB) == 0, "tile rows");
+  static_assert(NV >= 4 && NV <= 32, "values per lane");
+};
+
+template <int G>
+struct __align__(128) Smem {
+  uint16_t k[kStages][kTileRows][kHeadDim];
+  uint16_t v[kStages][kTileRows][kHeadDim];
+  // per half-warp, double-buffered: probabilities and rescale factors, each
+  // stored twice so that one 8-byte read yields a packed fp32 pair
+  float2 p[2][kHalfWarps][Shape<G>::NV];
+  float2 alpha[2][kHalfWarps][G];
+  float merge_m[kHalfWarps][G];
+  float merge_l[kHalfWarps][G];
+  float merge_o[kConsumerWarps][G][kHeadDim];
+  int row_set_start[kMaxRowSets + 1];
+  int total_items;
+  int abort;  // set when a pipeline wait gave up; later waits return at once
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+};
+
+struct Item {
+  int v, split, kvh, b, t, L, r0, r1, nsplit;
+};
+
+// Number of splits of row set v (0 when the set is invalid).
+__device__ __forceinline__ int splits_of(const DecodeArgs& a, int b, int t, int& L) {
+  const int sp = a.start_pos[b];
+  L = sp + t + 1;
+  if (sp < 0 || (long long)sp + a.Tq > a.S || (long long)sp + a.Tq > a.kv_len_hint) return 0;
+  return (L + a.rows_per_split - 1) / a.rows_per_split;
+}
+
+__device__ __forceinline__ Item decode_item(const DecodeArgs& a, const int* row_set_start, int n_sets,
+                                            int i) {
+  Item it;
+  if (a.max_splits == 1) {
+    it.v = i / a.Hkv;
+    it.split = 0;
+    it.kvh = i - it.v * a.Hkv;
+  } else {
+    int lo = 0, hi = n_sets;  // largest v with row_set_start[v] <= i
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (row_set_start[mid] <= i) lo = mid; else hi = mid;
+    }
+    it.v = lo;
+    const int local = i - row_set_start[lo];
+    it.split = local / a.Hkv;
+    it.kvh = local - it.split * a.Hkv;
+  }
+  it.b = it.v / a.Tq;
+  it.t = it.v - it.b * a.Tq;
+  it.nsplit = splits_of(a, it.b, it.t, it.L);
+  it.r0 = it.split * a.rows_per_split;
+  it.r1 = it.nsplit == 0 ? it.r0 : min(it.r0 + a.rows_per_split, it.L);
+  return it;
+}
+
+template <int G>
+__global__ void __launch_bounds__(kThreads, 2) decode_splitk_kernel(
+    const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+    const DecodeArgs a, const int evict_first) {
+  using Sh = Shape<G>;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  Smem<G>& sm = *reinterpret_cast<Smem<G>*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int n_sets = a.B * a.Tq;
+
+  // ---- item table (only when sequences are split) and barriers
+  if (a.max_splits == 1) {
+    if (tid == 0) sm.total_items = n_sets * a.Hkv;
+    if (blockIdx.x == 0 && tid < 32) {
+      for (int v = lane; v < n_sets; v += 32) {
+        int L;
+        const int b = v / a.Tq;
+        if (splits_of(a, b, v - b * a.Tq, L) == 0) {
+          const int sp = a.start_pos[b];
+          set_status(a.dev_status, (sp < 0 || (long long)sp + a.Tq > a.S) ? KVATTN_DEV_START_POS_RANGE
+                                                                         : KVATTN_DEV_KV_LEN_HINT);
+        }
+      }
+    }
+  } else {
+    // exclusive scan of items per row set over all threads
+    const int per = (n_sets + kThreads - 1) / kThreads;
+    const int beg = min(tid * per, n_sets), end = min(beg + per, n_sets);
+    int local = 0;
+    for (int v = beg; v < end; ++v) {
+      int L;
+      const int b = v / a.Tq;
+      const int ns = splits_of(a, b, v - b * a.Tq, L);
+      if (ns == 0 && blockIdx.x == 0) {
+        const int sp = a.start_pos[b];
+        set_status(a.dev_status, (sp < 0 || (long long)sp + a.Tq > a.S) ? KVATTN_DEV_START_POS_RANGE
+                                                                       : KVATTN_DEV_KV_LEN_HINT);
+      }
+      local += ns * a.Hkv;
+    }
+    // warp-level inclusive scan of the per-thread sums
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    __shared__ int warp_tot[kThreads / 32];
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    int warp_off = 0;
+    for (int w = 0; w < warp; ++w) warp_off += warp_tot[w];
+    int run = warp_off + incl - local;
+    for (int v = beg; v < end; ++v) {
+      int L;
+      const int b = v / a.Tq;
+      sm.row_set_start[v] = run;
+      run += splits_of(a, b, v - b * a.Tq, L) * a.Hkv;
+    }
+    if (tid == kThreads - 1) {
+      int tot = 0;
+      for (int w = 0; w < kThreads / 32; ++w) tot += warp_tot[w];
+      sm.total_items = tot;
+      sm.row_set_start[n_sets] = tot;
+    }
+  }
+  if (tid == 0) {
+    sm.abort = 0;
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], kConsumerWarps);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const int total_items = sm.total_items;
+
+  if (warp == kConsumerWarps) {
+    // ================================================================ producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmap_k);
+      prefetch_tensormap(&tmap_v);
+      uint64_t policy = 0;
+      if (evict_first) policy = l2_policy_evict_first();
+      else asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(policy));
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int i = blockIdx.x; i < total_items && !sm.abort; i += gridDim.x) {
+        const Item it = decode_item(a, sm.row_set_start, n_sets, i);
+        for (int row = it.r0; row < it.r1; row += kTileRows) {
+          if (!mbar_wait(&sm.empty[stage], phase ^ 1, &sm.abort)) {
+            abort_pipeline(&sm.abort, a.dev_status);
+            break;
+          }
+          mbar_arrive_expect_tx(&sm.full[stage], 2 * kTileBytes);
+          tma_load_4d(&sm.k[stage][0][0], &tmap_k, &sm.full[stage], 0, it.kvh, row, it.b, policy);
+          tma_load_4d(&sm.v[stage][0][0], &tmap_v, &sm.full[stage], 0, it.kvh, row, it.b, policy);
+          if (++stage == kStages) { stage = 0; phase ^= 1; }
+        }
+      }
+      // Leave only once every copy into this CTA's shared memory has landed:
+      // wait (bounded) until the consumers have released every stage.
+      for (int s = 0; s < kStages; ++s) {
+        if (!mbar_wait(&sm.empty[stage], phase ^ 1, nullptr)) {
+          abort_pipeline(&sm.abort, a.dev_status);
+          break;
+        }
+        if (++stage == kStages) { stage = 0; phase ^= 1; }
+      }
+    }
+    return;
+  }
+
+  // ================================================================== consumers
+  const int hw = lane >> 4;                 // half-warp within the warp
+  const int l16 = lane & 15;                // 8 elements [8*l16, 8*l16+8) of every row
+  const int hwg = warp * 2 + hw;            // half-warp within the CTA
+
+  // slot bookkeeping: which (head, row) scores this lane ends up holding
+  constexpr int LOGRB = ilog2(Sh::RB);
+  int slot_n0;  // n of slot 0; n = h*RB + j
+  if constexpr (Sh::LOG2NV >= 4) slot_n0 = l16 << (Sh::LOG2NV - 4);
+  else slot_n0 = l16 >> (4 - Sh::LOG2NV);
+  const int my_head = slot_n0 >> LOGRB;     // every slot of a lane has the same head
+  const bool writer = (l16 & (Sh::REP - 1)) == 0;
+  const bool head_writer = writer && ((slot_n0 & (Sh::RB - 1)) == 0);
+
+  int stage = 0;
+  uint32_t phase = 0;
+  int pbuf = 0;
+
+  // Every consumer warp walks the same items and tiles and meets the same
+  // named barriers; after an aborted wait it keeps walking without waiting
+  // (its results are then garbage, flagged in dev_status).
+  for (int i = blockIdx.x; i < total_items; i += gridDim.x) {
+    const Item it = decode_item(a, sm.row_set_start, n_sets, i);
+    if (it.nsplit == 0) continue;
+    // q of the G heads of this group, scaled into log2 units
+    uint64_t q2[G][4];
+    {
+      const uint16_t* qp = a.q_rot + (((size_t)it.b * a.Tq + it.t) * a.H + (size_t)it.kvh * G) * kHeadDim + 8 * l16;
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const uint4 w = *reinterpret_cast<const uint4*>(qp + (size_t)h * kHeadDim);
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          q2[h][k] = f2_pack(bf16lo_to_f32(ws[k]) * a.scale_log2, bf16hi_to_f32(ws[k]) * a.scale_log2);
+      }
+    }
+    uint64_t o2[G][4];
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) o2[h][k] = 0;
+    float m_run = -INFINITY;  // running max of my head (log2 units)
+    float l_run = 0.f;        // running sum of my slots
+
+    for (int row = it.r0; row < it.r1; row += kTileRows) {
+      if (!mbar_wait(&sm.full[stage], phase, &sm.abort)) abort_pipeline(&sm.abort, a.dev_status);
+      const uint16_t* Kt = &sm.k[stage][0][0];
+      const uint16_t* Vt = &sm.v[stage][0][0];
+#pragma unroll
+      for (int pass = 0; pass < Sh::PASSES; ++pass) {
+        const int rbase = pass * kHalfWarps * Sh::RB + hwg * Sh::RB;  // row within the tile
+        // ---- partial scores for RB rows x G heads
+        float part[Sh::NV];
+#pragma unroll
+        for (int j = 0; j < Sh::RB; ++j) {
+          const uint4 kc = lds128(Kt + (rbase + j) * kHeadDim + 8 * l16);
+          const uint64_t k0 = bf16x2_to_f2(kc.x), k1 = bf16x2_to_f2(kc.y);
+          const uint64_t k2 = bf16x2_to_f2(kc.z), k3 = bf16x2_to_f2(kc.w);
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            uint64_t acc = f2_mul(q2[h][0], k0);
+            acc = f2_fma(q2[h][1], k1, acc);
+            acc = f2_fma(q2[h][2], k2, acc);
+            acc = f2_fma(q2[h][3], k3, acc);
+            float x, y;
+            f2_unpack(acc, x, y);
+            part[h * Sh::RB + j] = x + y;
+          }
+        }
+        // ---- reduce-scatter over the 16 lanes of the half-warp
+        int cnt = Sh::NV;
+#pragma unroll
+        for (int st = 0; st < Sh::RS; ++st) {
+          const int m = 8 >> st;
+          const bool upper = (l16 & m) != 0;
+          cnt >>= 1;
+#pragma unroll
+          for (int x = 0; x < Sh::NV / 2; ++x) {
+            if (x < cnt) {
+              const float send = upper ? part[x] : part[x + cnt];
+              const float keep = upper ? part[x + cnt] : part[x];
+              part[x] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+            }
+          }
+        }
+#pragma unroll
+        for (int m = 8 >> Sh::RS; m >= 1; m >>= 1) part[0] += __shfl_xor_sync(0xffffffffu, part[0], m);
+
+        // ---- mask rows beyond this item and take the per-head tile max
+        float s[Sh::SLOTS];
+        float tmax = -INFINITY;
+#pragma unroll
+        for (int x = 0; x < Sh::SLOTS; ++x) {
+          const int j = (slot_n0 + x) & (Sh::RB - 1);
+          s[x] = (row + rbase + j < it.r1) ? part[x] : -INFINITY;
+          tmax = fmaxf(tmax, s[x]);
+        }
+        // lanes holding the other rows of my head differ in the lane bits that
+        // carry n's low LOGRB bits
+#pragma unroll
+        for (int k = 0; k < LOGRB; ++k) {
+          int lane_bit;
+          if constexpr (Sh::LOG2NV >= 4) lane_bit = k - (Sh::LOG2NV - 4);
+          else lane_bit = k + (4 - Sh::LOG2NV);
+          if (lane_bit >= 0) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1 << lane_bit));
+        }
+        const float m_new = fmaxf(m_run, tmax);
+        // m_new is -inf only while every row so far was masked (cannot happen
+        // for the first tile of an item, which always has row r0 < r1)
+        const float alpha = (m_new == -INFINITY) ? 1.f : exp2f(m_run - m_new);
+        m_run = m_new;
+        float psum = 0.f;
+        float2* pb = sm.p[pbuf][hwg];
+#pragma unroll
+        for (int x = 0; x < Sh::SLOTS; ++x) {
+          const float p = (s[x] == -INFINITY) ? 0.f : exp2f(s[x] - m_new);
+          psum += p;
+          if (writer) pb[slot_n0 + x] = make_float2(p, p);
+        }
+        l_run = l_run * alpha + psum;
+        if (head_writer) sm.alpha[pbuf][hwg][my_head] = make_float2(alpha, alpha);
+        const bool any_rescale = __any_sync(0xffffffffu, alpha != 1.f);
+        __syncwarp();
+
+        // ---- rescale o and accumulate P.V
+        if (any_rescale) {
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const uint64_t al = *reinterpret_cast<const uint64_t*>(&sm.alpha[pbuf][hwg][h]);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) o2[h][k] = f2_mul(o2[h][k], al);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < Sh::RB; ++j) {
+          if (row + rbase + j < it.r1) {
+            const uint4 vc = lds128(Vt + (rbase + j) * kHeadDim + 8 * l16);
+            const uint64_t v0 = bf16x2_to_f2(vc.x), v1 = bf16x2_to_f2(vc.y);
+            const uint64_t v2 = bf16x2_to_f2(vc.z), v3 = bf16x2_to_f2(vc.w);
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+              const uint64_t p2 = *reinterpret_cast<const uint64_t*>(&pb[h * Sh::RB + j]);
+              o2[h][0] = f2_fma(p2, v0, o2[h][0]);
+              o2[h][1] = f2_fma(p2, v1, o2[h][1]);
+              o2[h][2] = f2_fma(p2, v2, o2[h][2]);
+              o2[h][3] = f2_fma(p2, v3, o2[h][3]);
+            }
+          }
+        }
+        pbuf ^= 1;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.empty[stage]);
+      if (++stage == kStages) { stage = 0; phase ^= 1; }
+    }
+
+    // ---- merge the eight half-warp states of this item
+    // complete the running sum of my head over the lanes of its rows
+    float l_head = l_run;
+#pragma unroll
+    for (int k = 0; k < LOGRB; ++k) {
+      int lane_bit;
+      if constexpr (Sh::LOG2NV >= 4) lane_bit = k - (Sh::LOG2NV - 4);
+      else lane_bit = k + (4 - Sh::LOG2NV);
+      if (lane_bit >= 0) l_head += __shfl_xor_sync(0xffffffffu, l_head, 1 << lane_bit);
+    }
+    if (head_writer) {
+      sm.merge_m[hwg][my_head] = m_run;
+      sm.merge_l[hwg][my_head] = l_head;
+    }
+    named_bar_sync(1, kConsumerWarps * 32);
+    float Mh[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float mx = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < kHalfWarps; ++k) mx = fmaxf(mx, sm.merge_m[k][h]);
+      Mh[h] = mx;
+      const float mine = sm.merge_m[hwg][h];
+      const float f = (mine == -INFINITY) ? 0.f : exp2f(mine - mx);
+      const uint64_t f2 = f2_pack(f, f);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        o2[h][k] = f2_mul(o2[h][k], f2);
+        float x, y;
+        f2_unpack(o2[h][k], x, y);
+        x += __shfl_xor_sync(0xffffffffu, x, 16);
+        y += __shfl_xor_sync(0xffffffffu, y, 16);
+        o2[h][k] = f2_pack(x, y);
+      }
+    }
+    if (hw == 0) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float4* dst = reinterpret_cast<float4*>(&sm.merge_o[warp][h][8 * l16]);
+        float x0, x1, x2, x3, x4, x5, x6, x7;
+        f2_unpack(o2[h][0], x0, x1);
+        f2_unpack(o2[h][1], x2, x3);
+        f2_unpack(o2[h][2], x4, x5);
+        f2_unpack(o2[h][3], x6, x7);
+        dst[0] = make_float4(x0, x1, x2, x3);
+        dst[1] = make_float4(x4, x5, x6, x7);
+      }
+    }
+    named_bar_sync(1, kConsumerWarps * 32);
+    {
+      const int c = tid;  // 0..127: one output element per head
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float o = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) o += sm.merge_o[w][h][c];
+        float Ls = 0.f;
+#pragma unroll
+        for (int k = 0; k < kHalfWarps; ++k) {
+          const float mk = sm.merge_m[k][h];
+          if (mk != -INFINITY) Ls += sm.merge_l[k][h] * exp2f(mk - Mh[h]);
+        }
+        const int head = it.kvh * G + h;
+        if (it.nsplit == 1) {
+          const float r = o / Ls;
+          const uint32_t bits = f32_to_bf16_bits(r);
+          a.out[(((size_t)it.b * a.Tq + it.t) * a.H + head) * kHeadDim + c] = (uint16_t)bits;
+        } else {
+          const size_t slot = ((size_t)it.v * a.max_splits + it.split) * a.H + head;
+          a.ws_o[slot * kHeadDim + c] = o;
+          if (c == 0) {
+            a.ws_ml[slot * 2 + 0] = Mh[h];
+            a.ws_ml[slot * 2 + 1] = Ls;
+          }
+        }
+      }
+    }
+    named_bar_sync(1, kConsumerWarps * 32);
+  }
+}
+
+// K3: log-sum-exp merge of the split partials.  One CTA per (head, row set),
+// one thread per output element.
+__global__ void __launch_bounds__(kHeadDim) decode_merge_kernel(const DecodeArgs a) {
+  const int head = blockIdx.x;
+  const int v = blockIdx.y;
+  const int b = v / a.Tq, t = v - b * a.Tq;
+  int L;
+  const int ns = splits_of(a, b, t, L);
+  if (ns <= 1) return;
+  const int c = threadIdx.x;
+  const size_t base = (size_t)v * a.max_splits * a.H + head;
+  float M = -INFINITY;
+  for (int s = 0; s < ns; ++s) M = fmaxf(M, a.ws_ml[(base + (size_t)s * a.H) * 2]);
+  float num = 0.f, den = 0.f;
+  for (int s = 0; s < ns; ++s) {
+    const size_t slot = base + (size_t)s * a.H;
+    const float f = exp2f(a.ws_ml[slot * 2] - M);
+    num += f * a.ws_o[slot * kHeadDim + c];
+    den += f * a.ws_ml[slot * 2 + 1];
+  }
+  a.out[(((size_t)b * a.Tq + t) * a.H + head) * kHeadDim + c] = (uint16_t)f32_to_bf16_bits(num / den);
+}
+
+template <int G>
+size_t smem_bytes() {
+  return sizeof(Smem<G>) + 1024;
+}
+
+template <int G>
+cudaError_t launch_g(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st) {
+  const size_t smem = smem_bytes<G>();
+  static bool configured[64] = {false};
+  int dev = 0;
+  cudaError_t e0 = cudaGetDevice(&dev);
+  if (e0 != cudaSuccess) return e0;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(decode_splitk_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  const int evict_first = a.Tq == 1 ? 1 : 0;
+  decode_splitk_kernel<G><<<a.grid, kThreads, smem, st>>>(tk, tv, a, evict_first);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (a.max_splits > 1) {
+    dim3 grid(a.H, a.B * a.Tq);
+    decode_merge_kernel<<<grid, kHeadDim, 0, st>>>(a);
+    e = cudaGetLastError();
+  }
+  return e;
+}
+
+}  // namespace
+
+DecodePlan plan_decode(int B, int Tq, int H, int Hkv, int kv_len_hint, int sm_count) {
+  DecodePlan p;
+  const int G = H / Hkv;
+  const size_t smem = G == 1 ? smem_bytes<1>() : G == 2 ? smem_bytes<2>() : G == 4 ? smem_bytes<4>() : smem_bytes<8>();
+  const int ctas_per_sm = (int)std::max<size_t>(1, std::min<size_t>(4, (227 * 1024) / (smem + 1024)));
+  const int slots = sm_count * ctas_per_sm;
+  const long long row_sets = (long long)B * Tq;
+  // Aim for ~16 items per resident CTA so the round-robin stays balanced when
+  // lengths are ragged; never split below 64 rows, and do not split at all
+  // when the (b, t, head) units alone already give that much parallelism.
+  long long want = (row_sets * Hkv * (long long)kv_len_hint) / (16LL * slots);
+  int C = 64;
+  while (C < 4096 && (long long)C * 2 <= want) C *= 2;
+  if (row_sets > kMaxRowSets || row_sets * Hkv >= 16LL * slots || Tq > 1) C = kv_len_hint;
+  C = ((C + kTileRows - 1) / kTileRows) * kTileRows;
+  if (C >= kv_len_hint) C = ((kv_len_hint + kTileRows - 1) / kTileRows) * kTileRows;
+  p.rows_per_split = std::max(C, kTileRows);
+  p.max_splits = (kv_len_hint + p.rows_per_split - 1) / p.rows_per_split;
+  if (p.max_splits < 1) p.max_splits = 1;
+  const long long items_bound = row_sets * Hkv * p.max_splits;
+  p.grid = (int)std::min<long long>(items_bound, slots);
+  if (p.grid < 1) p.grid = 1;
+  p.ws_bytes = p.max_splits > 1 ? (size_t)row_sets * p.max_splits * H * (kHeadDim + 2) * sizeof(float) : 0;
+  return p;
+}
+
+cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st) {
+  switch (a.H / a.Hkv) {
+    case 1: return launch_g<1>(a, tk, tv, st);
+    case 2: return launch_g<2>(a, tk, tv, st);
+    case 4: return launch_g<4>(a, tk, tv, st);
+    case 8: return launch_g<8>(a, tk, tv, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace kvattn

@@ -1,0 +1,253 @@
+// C-ABI layer of libkvattn.so: host-side validation, the RoPE frequency
+// table, TMA descriptors for the caches, and the launches.  Declared in
+// include/kvattn.h, which states each call's contract.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "kvattn.h"
+#include "kvattn_internal.h"
+
+namespace {
+
+using kvattn::kMaxRopePairs;
+
+constexpr int kHeadDim = 128;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool group_supported(int G) { return G == 1 || G == 2 || G == 4 || G == 8; }
+
+int check_dims(const kvattn_dims* d) {
+  if (!d) return KVATTN_ERR_INVALID_ARG;
+  if (d->batch < 1 || d->n_heads < 1 || d->n_kv_heads < 1 || d->max_seq_len < 1) return KVATTN_ERR_INVALID_ARG;
+  if (d->n_heads % d->n_kv_heads != 0) return KVATTN_ERR_INVALID_ARG;
+  if (d->head_dim != kHeadDim) return KVATTN_ERR_UNSUPPORTED;
+  return KVATTN_OK;
+}
+
+// f_i = theta^(-2i/d), i < d/2, with the optional Llama-3.1 scaling rule
+// (stated in include/kvattn.h beside kvattn_rope_params).
+int make_rope_table(const kvattn_rope_params* r, kvattn::RopeTable* tab) {
+  if (!r || !std::isfinite(r->theta) || !(r->theta > 0.0)) return KVATTN_ERR_INVALID_ARG;
+  if (r->use_scaled) {
+    if (!(r->factor > 0.0) || !(r->low_freq_factor > 0.0) || !(r->high_freq_factor > r->low_freq_factor) ||
+        !(r->original_max_pos > 0.0))
+      return KVATTN_ERR_INVALID_ARG;
+  }
+  const double two_pi = 6.283185307179586476925286766559;
+  for (int i = 0; i < kHeadDim / 2; ++i) {
+    double f = std::pow(r->theta, -(2.0 * i) / kHeadDim);
+    if (r->use_scaled) {
+      const double wavelength = two_pi / f;
+      const double short_wl = r->original_max_pos / r->high_freq_factor;  // kept below this
+      const double long_wl = r->original_max_pos / r->low_freq_factor;    // divided above this
+      if (wavelength > long_wl) {
+        f /= r->factor;
+      } else if (wavelength >= short_wl) {
+        const double s = (r->original_max_pos / wavelength - r->low_freq_factor) /
+                         (r->high_freq_factor - r->low_freq_factor);
+        f = (1.0 - s) * (f / r->factor) + s * f;
+      }
+    }
+    tab->freq[i] = f;
+  }
+  for (int i = kHeadDim / 2; i < kMaxRopePairs; ++i) tab->freq[i] = 0.0;
+  return KVATTN_OK;
+}
+
+// ------------------------------------------------------------ device queries
+int current_sm_count(int* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KVATTN_ERR_CUDA;
+  static std::mutex mu;
+  static int cached[64] = {0};
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev < 0 || dev >= 64) return KVATTN_ERR_CUDA;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      return KVATTN_ERR_CUDA;
+    cached[dev] = n;
+  }
+  *out = cached[dev];
+  return KVATTN_OK;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Cache [B, S, Hkv, 128] bf16 viewed as a 4-D tensor (d, head, row, batch);
+// one box is `rows` consecutive rows of one head of one sequence.
+int encode_cache_map(CUtensorMap* map, const void* base, int B, int S, int Hkv, int rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return KVATTN_ERR_CUDA;
+  const cuuint64_t dims[4] = {(cuuint64_t)kHeadDim, (cuuint64_t)Hkv, (cuuint64_t)S, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)Hkv * kHeadDim * 2,
+                                 (cuuint64_t)S * Hkv * kHeadDim * 2};
+  const cuuint32_t box[4] = {(cuuint32_t)kHeadDim, 1, (cuuint32_t)rows, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? KVATTN_OK : KVATTN_ERR_CUDA;
+}
+
+int hint_or_default(int32_t hint, int S) { return hint <= 0 ? S : hint; }
+
+int run_attention(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, const uint16_t* cache_k,
+                  const uint16_t* cache_v, const int32_t* start_pos, int32_t max_kv_len_hint, float scale,
+                  uint16_t* out, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                  kvattn_stream_t stream) {
+  int rc = check_dims(dims);
+  if (rc != KVATTN_OK) return rc;
+  if (T < 1) return KVATTN_ERR_INVALID_ARG;
+  if (!group_supported(dims->n_heads / dims->n_kv_heads)) return KVATTN_ERR_UNSUPPORTED;
+  if (!q_rot || !cache_k || !cache_v || !start_pos || !out) return KVATTN_ERR_INVALID_ARG;
+  if (!aligned16(q_rot) || !aligned16(cache_k) || !aligned16(cache_v) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(start_pos) & 3u))
+    return KVATTN_ERR_INVALID_ARG;
+  const int hint = hint_or_default(max_kv_len_hint, dims->max_seq_len);
+  if (hint > dims->max_seq_len || hint < T) return KVATTN_ERR_OUT_OF_RANGE;
+  if (!(scale > 0.f)) scale = 1.0f / std::sqrt((float)kHeadDim);
+  if (!std::isfinite(scale)) return KVATTN_ERR_INVALID_ARG;
+  if ((long long)dims->batch * T > (1LL << 24)) return KVATTN_ERR_UNSUPPORTED;
+
+  int sms = 0;
+  rc = current_sm_count(&sms);
+  if (rc != KVATTN_OK) return rc;
+  const kvattn::DecodePlan plan =
+      kvattn::plan_decode(dims->batch, T, dims->n_heads, dims->n_kv_heads, hint, sms);
+  if (plan.ws_bytes > 0) {
+    if (!workspace || workspace_bytes < plan.ws_bytes || !aligned16(workspace)) return KVATTN_ERR_WORKSPACE;
+  }
+
+  CUtensorMap tk, tv;
+  rc = encode_cache_map(&tk, cache_k, dims->batch, dims->max_seq_len, dims->n_kv_heads, 32);
+  if (rc != KVATTN_OK) return rc;
+  rc = encode_cache_map(&tv, cache_v, dims->batch, dims->max_seq_len, dims->n_kv_heads, 32);
+  if (rc != KVATTN_OK) return rc;
+
+  kvattn::DecodeArgs a;
+  a.B = dims->batch;
+  a.Tq = T;
+  a.H = dims->n_heads;
+  a.Hkv = dims->n_kv_heads;
+  a.S = dims->max_seq_len;
+  a.kv_len_hint = hint;
+  a.rows_per_split = plan.rows_per_split;
+  a.max_splits = plan.max_splits;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.q_rot = q_rot;
+  a.out = out;
+  a.start_pos = start_pos;
+  float* ws = static_cast<float*>(workspace);
+  const size_t n_slots = (size_t)dims->batch * T * plan.max_splits * dims->n_heads;
+  a.ws_o = plan.ws_bytes ? ws : nullptr;
+  a.ws_ml = plan.ws_bytes ? ws + n_slots * kHeadDim : nullptr;
+  a.dev_status = dev_status;
+  a.grid = plan.grid;
+  return kvattn::launch_decode(a, tk, tv, (cudaStream_t)stream) == cudaSuccess ? KVATTN_OK : KVATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kvattn_rope_append(const kvattn_dims* dims, const kvattn_rope_params* rope, int32_t T, const uint16_t* q,
+                       uint16_t* q_rot, const uint16_t* k_new, const uint16_t* v_new, uint16_t* cache_k,
+                       uint16_t* cache_v, const int32_t* start_pos, int32_t* dev_status, kvattn_stream_t stream) {
+  int rc = check_dims(dims);
+  if (rc != KVATTN_OK) return rc;
+  if (T < 1) return KVATTN_ERR_INVALID_ARG;
+  if (!q || !q_rot || !k_new || !v_new || !cache_k || !cache_v || !start_pos) return KVATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(q_rot) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(cache_k) ||
+      !aligned16(cache_v) || (reinterpret_cast<uintptr_t>(start_pos) & 3u))
+    return KVATTN_ERR_INVALID_ARG;
+  if (T > dims->max_seq_len) return KVATTN_ERR_OUT_OF_RANGE;
+  kvattn::RopeTable tab;
+  rc = make_rope_table(rope, &tab);
+  if (rc != KVATTN_OK) return rc;
+  kvattn::RopeAppendArgs a;
+  a.B = dims->batch;
+  a.T = T;
+  a.H = dims->n_heads;
+  a.Hkv = dims->n_kv_heads;
+  a.S = dims->max_seq_len;
+  a.q = q;
+  a.q_rot = q_rot;
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.cache_k = cache_k;
+  a.cache_v = cache_v;
+  a.start_pos = start_pos;
+  a.dev_status = dev_status;
+  return kvattn::launch_rope_append(a, tab, (cudaStream_t)stream) == cudaSuccess ? KVATTN_OK : KVATTN_ERR_CUDA;
+}
+
+size_t kvattn_decode_workspace_bytes(const kvattn_dims* dims, int32_t max_kv_len_hint) {
+  if (check_dims(dims) != KVATTN_OK) return 0;
+  const int hint = hint_or_default(max_kv_len_hint, dims->max_seq_len);
+  if (hint > dims->max_seq_len || hint < 1) return 0;
+  int sms = 0;
+  if (current_sm_count(&sms) != KVATTN_OK) return 0;
+  return kvattn::plan_decode(dims->batch, 1, dims->n_heads, dims->n_kv_heads, hint, sms).ws_bytes;
+}
+
+int kvattn_decode(const kvattn_dims* dims, const uint16_t* q_rot, const uint16_t* cache_k, const uint16_t* cache_v,
+                  const int32_t* start_pos, int32_t max_kv_len_hint, float scale, uint16_t* out, void* workspace,
+                  size_t workspace_bytes, int32_t* dev_status, kvattn_stream_t stream) {
+  return run_attention(dims, 1, q_rot, cache_k, cache_v, start_pos, max_kv_len_hint, scale, out, workspace,
+                       workspace_bytes, dev_status, stream);
+}
+
+size_t kvattn_prefill_workspace_bytes(const kvattn_dims* dims, int32_t T, int32_t max_kv_len_hint) {
+  if (check_dims(dims) != KVATTN_OK || T < 1) return 0;
+  const int hint = hint_or_default(max_kv_len_hint, dims->max_seq_len);
+  if (hint > dims->max_seq_len || hint < T) return 0;
+  int sms = 0;
+  if (current_sm_count(&sms) != KVATTN_OK) return 0;
+  return kvattn::plan_decode(dims->batch, T, dims->n_heads, dims->n_kv_heads, hint, sms).ws_bytes;
+}
+
+int kvattn_prefill_chunk(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, const uint16_t* cache_k,
+                         const uint16_t* cache_v, const int32_t* start_pos, int32_t max_kv_len_hint, float scale,
+                         uint16_t* out, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                         kvattn_stream_t stream) {
+  return run_attention(dims, T, q_rot, cache_k, cache_v, start_pos, max_kv_len_hint, scale, out, workspace,
+                       workspace_bytes, dev_status, stream);
+}
+
+const char* kvattn_status_string(int status) {
+  switch (status) {
+    case KVATTN_OK: return "ok";
+    case KVATTN_ERR_INVALID_ARG: return "invalid argument";
+    case KVATTN_ERR_UNSUPPORTED: return "unsupported shape";
+    case KVATTN_ERR_OUT_OF_RANGE: return "length outside the cache";
+    case KVATTN_ERR_WORKSPACE: return "workspace missing or too small";
+    case KVATTN_ERR_CUDA: return "CUDA error";
+    default: return "unknown status";
+  }
+}
+
+int kvattn_version(void) { return 100; }
+
+}  // extern "C"

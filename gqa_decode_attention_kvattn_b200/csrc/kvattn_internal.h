@@ -1,0 +1,63 @@
+// Internal launch interfaces between the C-ABI layer (kvattn_api.cu) and the
+// kernels.  Not part of the public ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace kvattn {
+
+constexpr int kMaxRopePairs = 64;  // d/2 for d = 128
+
+struct RopeTable {
+  double freq[kMaxRopePairs];  // f_i, already scaled when Llama-3.1 scaling is on
+};
+
+struct RopeAppendArgs {
+  int B, T, H, Hkv, S;
+  const uint16_t* q;
+  uint16_t* q_rot;
+  const uint16_t* k_new;
+  const uint16_t* v_new;
+  uint16_t* cache_k;
+  uint16_t* cache_v;
+  const int32_t* start_pos;
+  int32_t* dev_status;
+};
+
+cudaError_t launch_rope_append(const RopeAppendArgs& a, const RopeTable& tab, cudaStream_t stream);
+
+// Split-K attention over the cache for Tq query tokens per sequence.  Each
+// (sequence, token) pair is a "query row set" of G heads per KV head; its
+// visible length is start_pos[b] + t + 1.
+struct DecodeArgs {
+  int B, Tq, H, Hkv, S;
+  int kv_len_hint;     // upper bound on start_pos[b] + Tq
+  int rows_per_split;  // C, a multiple of the tile rows
+  int max_splits;      // ceil(kv_len_hint / C)
+  float scale_log2;    // softmax scale * log2(e)
+  const uint16_t* q_rot;  // [B, Tq, H, d]
+  uint16_t* out;          // [B, Tq, H, d]
+  const int32_t* start_pos;
+  float* ws_o;   // [B*Tq, max_splits, H, d]   unnormalised partial outputs
+  float* ws_ml;  // [B*Tq, max_splits, H, 2]   (running max in log2 units, sum)
+  int32_t* dev_status;
+  int grid;      // persistent CTAs
+};
+
+struct DecodePlan {
+  int rows_per_split;
+  int max_splits;
+  int grid;
+  size_t ws_bytes;
+};
+
+// Split size, persistent grid and workspace for these shapes on this device.
+DecodePlan plan_decode(int B, int Tq, int H, int Hkv, int kv_len_hint, int sm_count);
+
+cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tmap_k, const CUtensorMap& tmap_v,
+                          cudaStream_t stream);
+
+}  // namespace kvattn

@@ -1,0 +1,85 @@
+// K1: RoPE with a position offset, then the KV-cache append.
+//
+// For token t of sequence b the position is p = start_pos[b] + t (the past
+// length is the offset: "Llama 3.1 8B KV cache", section "RoPE has to know
+// where it is").  Each interleaved pair (x_2i, x_2i+1) of every query head and
+// every new key head is rotated by p * f_i; the rotated keys and the values go
+// to cache row p ("Llama 3 8B · KV cache", cache write C_K[p] <- K_r,
+// C_V[p] <- V).  Angles, sin/cos and the rotation run in fp64, which keeps the
+// bf16 result within one rounding of the exact value up to p = 131071 (an fp32
+// angle would already be off by ~1e-2 rad there).
+//
+// One CTA per (b, t); its threads first build the 64 (cos, sin) pairs of that
+// position, then sweep the (H + Hkv) * 64 pairs with coalesced 4-byte
+// accesses, and copy the Hkv value rows with 16-byte accesses.  The kernel
+// moves B*T*(2H + 3Hkv)*256 bytes, a negligible share of a decode step.
+#include "kvattn_device.cuh"
+#include "kvattn_internal.h"
+
+namespace kvattn {
+namespace {
+
+constexpr int kRopeThreads = 256;
+
+__global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(RopeAppendArgs a, RopeTable tab) {
+  const int bt = blockIdx.x;
+  const int b = bt / a.T;
+  const int t = bt - b * a.T;
+  const int sp = a.start_pos[b];
+  if (sp < 0 || (long long)sp + a.T > a.S) {
+    if (t == 0 && threadIdx.x == 0) set_status(a.dev_status, KVATTN_DEV_START_POS_RANGE);
+    return;
+  }
+  const long long pos = (long long)sp + t;
+
+  __shared__ double s_cos[kMaxRopePairs];
+  __shared__ double s_sin[kMaxRopePairs];
+  for (int i = threadIdx.x; i < kHeadDim / 2; i += blockDim.x) {
+    const double ang = (double)pos * tab.freq[i];
+    double s, c;
+    sincos(ang, &s, &c);
+    s_cos[i] = c;
+    s_sin[i] = s;
+  }
+  __syncthreads();
+
+  constexpr int kPairs = kHeadDim / 2;
+  const int q_pairs = a.H * kPairs;
+  const int total = (a.H + a.Hkv) * kPairs;
+  const uint32_t* q_in = reinterpret_cast<const uint32_t*>(a.q) + (size_t)bt * q_pairs;
+  uint32_t* q_out = reinterpret_cast<uint32_t*>(a.q_rot) + (size_t)bt * q_pairs;
+  const uint32_t* k_in = reinterpret_cast<const uint32_t*>(a.k_new) + (size_t)bt * a.Hkv * kPairs;
+  uint32_t* k_out = reinterpret_cast<uint32_t*>(a.cache_k) + ((size_t)b * a.S + pos) * a.Hkv * kPairs;
+
+  for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {
+    const int i = idx & (kPairs - 1);
+    const bool is_q = idx < q_pairs;
+    const uint32_t w = is_q ? q_in[idx] : k_in[idx - q_pairs];
+    const double x0 = (double)bf16lo_to_f32(w);
+    const double x1 = (double)bf16hi_to_f32(w);
+    const double c = s_cos[i], s = s_sin[i];
+    const double y0 = x0 * c - x1 * s;
+    const double y1 = x0 * s + x1 * c;
+    const uint32_t r = f64_to_bf16_bits(y0) | (f64_to_bf16_bits(y1) << 16);
+    if (is_q)
+      q_out[idx] = r;
+    else
+      k_out[idx - q_pairs] = r;
+  }
+
+  // values: bit copy of Hkv rows of 256 bytes
+  const uint4* v_in = reinterpret_cast<const uint4*>(a.v_new) + (size_t)bt * a.Hkv * (kHeadDim / 8);
+  uint4* v_out = reinterpret_cast<uint4*>(a.cache_v) + ((size_t)b * a.S + pos) * a.Hkv * (kHeadDim / 8);
+  for (int idx = threadIdx.x; idx < a.Hkv * (kHeadDim / 8); idx += blockDim.x) v_out[idx] = v_in[idx];
+}
+
+}  // namespace
+
+cudaError_t launch_rope_append(const RopeAppendArgs& a, const RopeTable& tab, cudaStream_t stream) {
+  const long long blocks = (long long)a.B * a.T;
+  if (blocks > 0x7FFFFFFFll) return cudaErrorInvalidValue;
+  rope_append_kernel<<<(unsigned)blocks, kRopeThreads, 0, stream>>>(a, tab);
+  return cudaGetLastError();
+}
+
+}  // namespace kvattn

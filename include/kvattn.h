@@ -1,0 +1,173 @@
+/*
+ * kvattn.h -- C ABI of libkvattn.so: the cached grouped-query-attention step
+ * of a Llama-3.1-style decoder on NVIDIA B200 (sm_100a).
+ *
+ * One call of the step, as "Llama 3 8B · KV cache" (model.py 160-177 and
+ * 281-302 excerpts) and "Llama 3.1 8B KV cache" (sections "RoPE has to know
+ * where it is" and "The cache itself is concatenation") describe it:
+ *   1. rotate the new queries and keys with RoPE at absolute positions
+ *      start_pos .. start_pos+T-1                    -> kvattn_rope_append
+ *   2. write the rotated keys and the values into cache rows
+ *      start_pos .. start_pos+T-1                    -> kvattn_rope_append
+ *   3. attend softmax(q K^T / sqrt(d)) V over rows 0 .. start_pos+t with the
+ *      rectangular causal mask, query head h reading KV head floor(h/G)
+ *      ("Llama 3.1 8B · Repeat heads")               -> kvattn_decode (T = 1)
+ *                                                    -> kvattn_prefill_chunk (T >= 1)
+ *
+ * Conventions shared by every entry point
+ *  - Tensors are caller-owned, contiguous DEVICE memory.  bf16 tensors are
+ *    passed as uint16_t bit patterns.  Every tensor pointer must be 16-byte
+ *    aligned.
+ *  - Layouts follow the code layout of "Llama 3 8B · KV cache" ([B,
+ *    positions, heads, d]):
+ *      q, q_rot, out        [B, T, H,   d]
+ *      k_new, v_new         [B, T, Hkv, d]
+ *      cache_k, cache_v     [B, S, Hkv, d]   (S = max_seq_len rows, allocated up front)
+ *      start_pos            int32 [B] on the device: the past length of each
+ *                           sequence, i.e. the first row this call writes.
+ *  - Calls are asynchronous on `stream` (NULL = legacy default stream); the
+ *    library performs no host synchronisation and allocates no memory.
+ *  - Return value: KVATTN_OK, or a kvattn_status for problems found on the
+ *    host before anything is launched (nothing is launched then).
+ *  - Problems only the device can see (a start_pos outside the cache, a
+ *    sequence longer than max_kv_len_hint, an in-kernel wait that gave up)
+ *    skip the affected sequence's writes and OR a KVATTN_DEV_* bit into
+ *    *dev_status (a device int32 the caller zeroes; may be NULL).
+ */
+#ifndef KVATTN_H
+#define KVATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define KVATTN_API __attribute__((visibility("default")))
+#else
+#define KVATTN_API
+#endif
+
+struct CUstream_st;
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* kvattn_stream_t;
+
+typedef enum kvattn_status {
+  KVATTN_OK = 0,
+  KVATTN_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, H % Hkv != 0 */
+  KVATTN_ERR_UNSUPPORTED = 2, /* head_dim != 128, group size G = H/Hkv not in {1,2,4,8} */
+  KVATTN_ERR_OUT_OF_RANGE = 3, /* a host-visible length outside the cache */
+  KVATTN_ERR_WORKSPACE = 4,    /* workspace missing or smaller than required */
+  KVATTN_ERR_CUDA = 5          /* a CUDA launch or query failed */
+} kvattn_status;
+
+/* Bits OR-ed into *dev_status by the kernels. */
+#define KVATTN_DEV_START_POS_RANGE 0x1 /* start_pos[b] < 0 or start_pos[b]+T > max_seq_len */
+#define KVATTN_DEV_KV_LEN_HINT 0x2     /* start_pos[b]+T > max_kv_len_hint */
+#define KVATTN_DEV_WAIT_TIMEOUT 0x4    /* an in-kernel pipeline wait gave up */
+
+typedef struct kvattn_dims {
+  int32_t batch;       /* B: sequences in this call (rows 0..B-1 of the caches) */
+  int32_t n_heads;     /* H: query heads (32 for Llama 3.1 8B, 64 for 70B) */
+  int32_t n_kv_heads;  /* Hkv: key/value heads (8); G = H / Hkv query heads share one */
+  int32_t head_dim;    /* d: must be 128 */
+  int32_t max_seq_len; /* S: rows the caches were allocated with */
+} kvattn_dims;
+
+/* RoPE parameters: f_i = theta^(-2i/d) ("Llama 3.1 8B KV cache", section
+ * "RoPE has to know where it is"), with optional Llama-3.1 frequency scaling
+ * (use_scaled_rope in "Llama 3.1 8B · Repeat heads", sku_list.py excerpt):
+ * wavelengths 2*pi/f_i shorter than original_max_pos/high_freq_factor are
+ * kept, longer than original_max_pos/low_freq_factor are divided by
+ * `factor`, and in between f becomes (1-s) f/factor + s f with
+ * s = (original_max_pos/wavelength - low_freq_factor) /
+ *     (high_freq_factor - low_freq_factor). */
+typedef struct kvattn_rope_params {
+  double theta;            /* 500000 for Llama 3 / 3.1 */
+  int32_t use_scaled;      /* 0 or 1 */
+  double factor;           /* 8 */
+  double low_freq_factor;  /* 1 */
+  double high_freq_factor; /* 4 */
+  double original_max_pos; /* 8192 */
+} kvattn_rope_params;
+
+/* Steps 1-2 (cache write "C_K[p] <- K_r, C_V[p] <- V" of "Llama 3 8B · KV
+ * cache"; the position offset of "Llama 3.1 8B KV cache", section "RoPE has to
+ * know where it is").
+ * For every b < B and t < T, with p = start_pos[b] + t:
+ *   q_rot[b,t,h,:]   = RoPE_p(q[b,t,h,:])      for h < H
+ *   cache_k[b,p,j,:] = RoPE_p(k_new[b,t,j,:])  for j < Hkv
+ *   cache_v[b,p,j,:] = v_new[b,t,j,:]          (bit copy)
+ * RoPE_p rotates each interleaved pair (x_2i, x_2i+1) counter-clockwise by
+ * p*f_i (the complex product (x_2i + i x_2i+1) e^{i p f_i}).  Angles, cos/sin
+ * and the rotation are computed in fp64 and rounded once to bf16 (nearest,
+ * ties to even).  q_rot may equal q (in place); it must not partially overlap
+ * q.  No other cache row is touched.  A sequence with start_pos[b] < 0 or
+ * start_pos[b] + T > max_seq_len writes nothing and sets
+ * KVATTN_DEV_START_POS_RANGE.
+ * Host errors: INVALID_ARG (null/misaligned pointer, T < 1, B < 1, S < 1,
+ * H % Hkv != 0, non-finite or non-positive theta), UNSUPPORTED (d != 128). */
+KVATTN_API int kvattn_rope_append(const kvattn_dims* dims, const kvattn_rope_params* rope, int32_t T,
+                       const uint16_t* q, uint16_t* q_rot, const uint16_t* k_new,
+                       const uint16_t* v_new, uint16_t* cache_k, uint16_t* cache_v,
+                       const int32_t* start_pos, int32_t* dev_status, kvattn_stream_t stream);
+
+/* Bytes of device workspace kvattn_decode needs for these dims and
+ * max_kv_len_hint on the CURRENT device (the split size depends on its SM
+ * count).  0 on invalid arguments. */
+KVATTN_API size_t kvattn_decode_workspace_bytes(const kvattn_dims* dims, int32_t max_kv_len_hint);
+
+/* Step 3 for one new token per sequence (T = 1; the decode step of "Llama 3 8B
+ * · KV cache" at p = 1000: write row 1000, read rows 0..1000).
+ *   out[b,0,h,:] = sum_{r <= start_pos[b]} softmax_r(scale * q_rot[b,0,h,:] .
+ *                  cache_k[b,r,floor(h/G),:]) * cache_v[b,r,floor(h/G),:]
+ * The cache rows 0..start_pos[b] must already hold the sequence (row
+ * start_pos[b] written by kvattn_rope_append earlier on the same stream).
+ * The rows of each (sequence, KV head) are streamed from HBM once and serve
+ * all G query heads; long rows are split across CTAs and the partial
+ * (o, max, sum) triples are merged by log-sum-exp in a second kernel.
+ * scale <= 0 selects 1/sqrt(d).  max_kv_len_hint (<= 0: max_seq_len) is a
+ * host upper bound on start_pos[b] + 1; it sizes the splits and the
+ * workspace.  A sequence above the hint or outside the cache leaves its
+ * output untouched and sets a KVATTN_DEV_* bit.  out is bf16 [B,1,H,d].
+ * workspace: device memory of kvattn_decode_workspace_bytes() bytes, 16-byte
+ * aligned, owned by the caller, contents need no initialisation; calls that
+ * share a workspace must be ordered on one stream.
+ * Host errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
+KVATTN_API int kvattn_decode(const kvattn_dims* dims, const uint16_t* q_rot, const uint16_t* cache_k,
+                  const uint16_t* cache_v, const int32_t* start_pos, int32_t max_kv_len_hint,
+                  float scale, uint16_t* out, void* workspace, size_t workspace_bytes,
+                  int32_t* dev_status, kvattn_stream_t stream);
+
+/* Bytes of device workspace kvattn_prefill_chunk needs (may be 0). */
+KVATTN_API size_t kvattn_prefill_workspace_bytes(const kvattn_dims* dims, int32_t T, int32_t max_kv_len_hint);
+
+/* Step 3 for a chunk of T new tokens per sequence (chunked prefill into an
+ * existing cache).  Row t of the chunk sits at position start_pos[b]+t and
+ * sees cache rows 0 .. start_pos[b]+t: the rectangular causal mask whose only
+ * masked entries are (t, r) with r > start_pos + t (comment in model.py
+ * 281-302 of "Llama 3 8B · KV cache").
+ *   out[b,t,h,:] = sum_{r <= start_pos[b]+t} softmax_r(scale * q_rot[b,t,h,:] .
+ *                  cache_k[b,r,floor(h/G),:]) * cache_v[b,r,floor(h/G),:]
+ * q_rot and out are bf16 [B,T,H,d]; the chunk's rows must already be in the
+ * cache (kvattn_rope_append with the same T).  max_kv_len_hint bounds
+ * start_pos[b] + T.  Errors and workspace rules as kvattn_decode. */
+KVATTN_API int kvattn_prefill_chunk(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot,
+                         const uint16_t* cache_k, const uint16_t* cache_v,
+                         const int32_t* start_pos, int32_t max_kv_len_hint, float scale,
+                         uint16_t* out, void* workspace, size_t workspace_bytes,
+                         int32_t* dev_status, kvattn_stream_t stream);
+
+/* Human-readable name of a kvattn_status value. */
+KVATTN_API const char* kvattn_status_string(int status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+KVATTN_API int kvattn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVATTN_H */

@@ -1,0 +1,216 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle on the
+same seeded inputs, at small shapes that span several tiles, ragged tails
+and split boundaries, plus indexing, error-flag and schedule checks."""
+import numpy as np
+import pytest
+
+import kvattn_synth as ks
+import oracle
+from tests import kvattn_testutil as U
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+kv = pytest.importorskip("gqa_decode_attention_kvattn_b200")
+
+
+def _dev_step(q, k, v, ck, cv, sp, rope, T, kind, hint=0, in_place=False):
+    """Run rope_append then decode/prefill on the GPU; return host copies."""
+    dq, dk, dv, dck, dcv = (U.to_dev(x) for x in (q, k, v, ck, cv))
+    dsp = torch.from_numpy(np.asarray(sp, np.int32)).cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    q_rot = kv.kvattn_rope_append(dq, dk, dv, dck, dcv, dsp, rope=rope, q_rot=dq if in_place else None,
+                                  dev_status=status)
+    if kind == "decode":
+        out = kv.kvattn_decode(q_rot, dck, dcv, dsp, max_kv_len_hint=hint, dev_status=status)
+    else:
+        out = kv.kvattn_prefill_chunk(q_rot, dck, dcv, dsp, max_kv_len_hint=hint, dev_status=status)
+    torch.cuda.synchronize()
+    return (U.to_host(q_rot), U.to_host(dck), U.to_host(dcv), U.to_host(out), int(status.item()))
+
+
+def _check_step(seed, B, T, H, Hkv, S, sp, rope, kind, hint=0, in_place=False):
+    q, k, v, ck, cv = U.host_inputs(seed, B, T, H, Hkv, S, sp)
+    g_qrot, g_ck, g_cv, g_out, st = _dev_step(q, k, v, ck, cv, sp, rope, T, kind, hint, in_place)
+    assert st == 0
+    # the oracle on the same bits
+    o_ck, o_cv = ck.copy(), cv.copy()
+    q_rot, out, rc = oracle.step(q, k, v, o_ck, o_cv, np.asarray(sp, np.int32), U.oracle_freqs(rope))
+    assert rc == 0
+    assert U.ulp_distance(g_qrot, q_rot).max() <= 1
+    assert U.ulp_distance(g_ck, o_ck).max() <= 1
+    assert np.array_equal(g_cv, o_cv)
+    for b in range(B):  # rows outside the new ones are bit-identical to the input
+        keep = np.ones(S, bool)
+        keep[sp[b]:sp[b] + T] = False
+        assert np.array_equal(g_ck[b, keep], ck[b, keep])
+    return U.assert_attention_close(g_out, out, f"{kind} B={B} T={T} H={H}/{Hkv} sp={list(sp)}")
+
+
+@pytest.mark.parametrize("case", [
+    (3, 32, 8, 64, [0, 17, 63], kv.LLAMA3),
+    (2, 32, 8, 200, [31, 32], kv.LLAMA3),
+    (2, 32, 8, 200, [33, 199], kv.LLAMA3_1),
+    (4, 16, 16, 130, [63, 64, 65, 129], kv.LLAMA3),     # G = 1 (MHA)
+    (3, 16, 8, 300, [0, 95, 257], kv.LLAMA3),           # G = 2
+    (5, 64, 8, 520, [1, 127, 128, 511, 519], kv.LLAMA3),  # G = 8
+])
+def test_decode_step_small(case):
+    B, H, Hkv, S, sp, rope = case
+    _check_step(11, B, 1, H, Hkv, S, sp, rope, "decode")
+
+
+def test_decode_step_in_place_rotation():
+    _check_step(12, 2, 1, 32, 8, 96, [5, 70], kv.LLAMA3, "decode", in_place=True)
+
+
+@pytest.mark.parametrize("hint", [0, 1500, 3000, 4096])
+def test_decode_split_sizes_agree(hint):
+    # different hints give different split sizes; each must match the oracle
+    sp = [1499, 700, 64, 1000]
+    _check_step(13, 4, 1, 32, 8, 4096, sp, kv.LLAMA3, "decode", hint=hint)
+
+
+def test_decode_many_splits_long_rows():
+    _check_step(14, 2, 1, 32, 8, 20000, [19999, 12345], kv.LLAMA3_1, "decode")
+
+
+@pytest.mark.parametrize("case", [
+    (2, 2, 32, 8, 80, [0, 40]),
+    (2, 7, 32, 8, 120, [33, 100]),
+    (1, 128, 32, 8, 400, [200]),
+    (2, 9, 64, 8, 64, [0, 55]),
+    (1, 33, 16, 16, 100, [31]),
+])
+def test_prefill_step_small(case):
+    B, T, H, Hkv, S, sp = case
+    _check_step(21, B, T, H, Hkv, S, sp, kv.LLAMA3, "prefill")
+
+
+def test_rope_append_large_positions_scaled():
+    # positions up to 131071: fp64 angles keep the rotation within one ulp
+    B, T, H, Hkv, S = 2, 1, 32, 8, 131072
+    sp = [131071, 65536]
+    q = ks.tensor_normal(3, ks.STREAM_Q, (B, T, H, 128))
+    k = ks.tensor_normal(3, ks.STREAM_K_NEW, (B, T, Hkv, 128))
+    v = ks.tensor_normal(3, ks.STREAM_V_NEW, (B, T, Hkv, 128))
+    dck = torch.zeros((B, S, Hkv, 128), dtype=torch.bfloat16, device="cuda")
+    dcv = torch.zeros_like(dck)
+    dsp = torch.tensor(sp, dtype=torch.int32, device="cuda")
+    q_rot = kv.kvattn_rope_append(U.to_dev(q), U.to_dev(k), U.to_dev(v), dck, dcv, dsp, rope=kv.LLAMA3_1)
+    torch.cuda.synchronize()
+    g_q = U.to_host(q_rot)
+    f = U.oracle_freqs(kv.LLAMA3_1)
+    for b in range(B):
+        ck = np.zeros((1, sp[b] + T, Hkv, 128), np.uint16)
+        cv = np.zeros_like(ck)
+        qr, rc = oracle.rope_append(q[b:b + 1].copy(), k[b:b + 1].copy(), v[b:b + 1].copy(), ck, cv,
+                                    np.array([sp[b]], np.int32), f)
+        assert rc == 0
+        assert U.ulp_distance(g_q[b], qr[0]).max() <= 1
+        row = U.to_host(dck[b, sp[b]:sp[b] + T])
+        assert U.ulp_distance(row, ck[0, sp[b]:]).max() <= 1
+        assert np.array_equal(U.to_host(dcv[b, sp[b]:sp[b] + T]), cv[0, sp[b]:])
+
+
+@pytest.mark.parametrize("kind,T", [("decode", 1), ("prefill", 4)])
+def test_planted_row_indexing(kind, T):
+    # q aligned with one planted K row gives it all the weight; V rows carry
+    # their index as a code, so the output names the row read, exactly.
+    B, H, Hkv, S = 2, 32, 8, 300
+    sp = np.array([150, 37], np.int32)
+    K = np.full((B, S, Hkv, 128), -1.0 / 128)
+    V = np.zeros((B, S, Hkv, 128))
+    for r in range(S):
+        V[:, r] = float(r % 250 + 1)
+    qv = np.full((B, T, H, 128), 4.0)
+    cases = []
+    for b in range(B):
+        for t in range(T):
+            L = sp[b] + t + 1
+            cases.append((b, t, L - 1, True))
+    for b, t, r_star, vis in cases:
+        K2 = K.copy()
+        K2[b, r_star, :, :] = 1.0
+        dk = U.to_dev(ks.f64_to_bf16_bits(K2))
+        dv = U.to_dev(ks.f64_to_bf16_bits(V))
+        dq = U.to_dev(ks.f64_to_bf16_bits(qv))
+        dsp = torch.from_numpy(sp).cuda()
+        if kind == "decode":
+            out = kv.kvattn_decode(dq, dk, dv, dsp)
+        else:
+            out = kv.kvattn_prefill_chunk(dq, dk, dv, dsp)
+        o = ks.bf16_bits_to_f64(U.to_host(out))
+        assert np.all(o[b, t] == float(r_star % 250 + 1))
+        # the next row (r_star + 1) is invisible to token t: plant there and
+        # the output must stay a mean of visible codes
+        if r_star + 1 < S and t == T - 1:
+            K3 = K.copy()
+            K3[b, r_star + 1, :, :] = 1.0
+            out = (kv.kvattn_decode if kind == "decode" else kv.kvattn_prefill_chunk)(
+                dq, U.to_dev(ks.f64_to_bf16_bits(K3)), dv, dsp)
+            o = ks.bf16_bits_to_f64(U.to_host(out))
+            vis_codes = np.array([float(r % 250 + 1) for r in range(r_star + 1)])
+            assert abs(o[b, t, 0, 0] - vis_codes.mean()) < 0.02 * vis_codes.mean()
+
+
+def test_out_of_range_start_pos_is_flagged_and_skipped():
+    B, H, Hkv, S, T = 3, 32, 8, 64, 2
+    sp = np.array([-1, 10, 63], np.int32)       # 63 + 2 > 64
+    q, k, v, ck, cv = U.host_inputs(5, B, T, H, Hkv, S, [0, 10, 0])
+    dq, dk, dv, dck, dcv = (U.to_dev(x) for x in (q, k, v, ck, cv))
+    dsp = torch.from_numpy(sp).cuda()
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    q_rot = kv.kvattn_rope_append(dq, dk, dv, dck, dcv, dsp, dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() & kv.KVATTN_DEV_START_POS_RANGE
+    g_ck = U.to_host(dck)
+    assert np.array_equal(g_ck[0], ck[0]) and np.array_equal(g_ck[2], ck[2])
+    sentinel = torch.full((B, T, H, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+    st.zero_()
+    out = kv.kvattn_prefill_chunk(q_rot, dck, dcv, dsp, out=sentinel, dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() & kv.KVATTN_DEV_START_POS_RANGE
+    o = U.to_host(out)
+    assert np.all(ks.bf16_bits_to_f64(o[0]) == 7.0) and np.all(ks.bf16_bits_to_f64(o[2]) == 7.0)
+    # the valid sequence is still right
+    qr, kr, ref = U.oracle_sequence(q[1], k[1], v[1], ck[1], cv[1], 10, T, kv.LLAMA3)
+    U.assert_attention_close(o[1], ref, "valid sequence beside bad ones")
+
+
+def test_kv_len_hint_exceeded_is_flagged():
+    B, H, Hkv, S = 2, 32, 8, 256
+    sp = np.array([200, 20], np.int32)
+    q, k, v, ck, cv = U.host_inputs(6, B, 1, H, Hkv, S, sp)
+    dsp = torch.from_numpy(sp).cuda()
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sentinel = torch.full((B, 1, H, 128), 3.0, dtype=torch.bfloat16, device="cuda")
+    out = kv.kvattn_decode(U.to_dev(q), U.to_dev(ck), U.to_dev(cv), dsp, max_kv_len_hint=100,
+                           out=sentinel, dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() & kv.KVATTN_DEV_KV_LEN_HINT
+    o = ks.bf16_bits_to_f64(U.to_host(out))
+    assert np.all(o[0] == 3.0) and not np.all(o[1] == 3.0)
+
+
+def test_prefill_equals_prefill_then_decode_steps():
+    # 12 tokens at once vs 8 then 4 single decode steps (the schedule test of
+    # "Grouped-query attention: a smaller KV cache", 9:42) on the GPU path
+    B, H, Hkv, S, T, T1 = 2, 32, 8, 128, 12, 8
+    sp = np.array([3, 70], np.int32)
+    q, k, v, ck, cv = U.host_inputs(7, B, T, H, Hkv, S, sp)
+    _, ckA, cvA, outA, st = _dev_step(q, k, v, ck, cv, sp, kv.LLAMA3, T, "prefill")
+    assert st == 0
+    _, ckB, cvB, outB1, st = _dev_step(q[:, :T1].copy(), k[:, :T1].copy(), v[:, :T1].copy(), ck, cv, sp,
+                                       kv.LLAMA3, T1, "prefill")
+    outs = [outB1]
+    for t in range(T1, T):
+        _, ckB, cvB, o, st = _dev_step(q[:, t:t + 1].copy(), k[:, t:t + 1].copy(), v[:, t:t + 1].copy(),
+                                       ckB, cvB, sp + t, kv.LLAMA3, 1, "decode")
+        assert st == 0
+        outs.append(o)
+    outB = np.concatenate(outs, axis=1)
+    assert np.array_equal(ckA, ckB) and np.array_equal(cvA, cvB)
+    a = ks.bf16_bits_to_f64(outA)
+    b = ks.bf16_bits_to_f64(outB)
+    assert np.abs(a - b).max() <= 2 * U.MAX_ABS / 4
