@@ -284,3 +284,51 @@ def prefill_flops(start_pos, T: int, n_heads: int, head_dim: int = HEAD_DIM) -> 
 
 def default_scale(head_dim: int = HEAD_DIM) -> float:
     return 1.0 / math.sqrt(head_dim)
+
+
+# ------------------------------------------------- allocation-free decode
+_noalloc = None
+
+
+def _load_noalloc():
+    """ctypes handle of kvattn_decode_noalloc (argument types set once)."""
+    global _noalloc
+    if _noalloc is None:
+        lib = _load()
+        P = ctypes.c_void_p
+        fn = lib.kvattn_decode_noalloc
+        fn.restype = ctypes.c_int
+        fn.argtypes = [ctypes.POINTER(kvattn_dims), P, P, P, P, ctypes.c_int32, ctypes.c_float, P, P, P]
+        lib.kvattn_decode_noalloc_scratch_bytes.restype = ctypes.c_size_t
+        lib.kvattn_decode_noalloc_scratch_bytes.argtypes = []
+        _noalloc = fn
+    return _noalloc
+
+
+def kvattn_decode_noalloc_scratch_bytes() -> int:
+    _load_noalloc()
+    return int(_load().kvattn_decode_noalloc_scratch_bytes())
+
+
+def kvattn_decode_noalloc(q_rot, cache_k, cache_v, start_pos, max_kv_len_hint: int = 0, scale: float = 0.0,
+                          out=None, dev_status=None, stream=None):
+    """kvattn_decode without a workspace: for callers that cannot allocate
+    device memory on the decode path (the library keeps one static 64 MiB
+    array per GPU for the split partials instead).  Calls that overlap on the
+    GPU share that array and race; the first call on a device looks up its
+    address and should come before any stream capture.  Only ``out`` is
+    allocated here, and only when it is not given."""
+    import torch
+    fn = _load_noalloc()
+    _check_bf16("q_rot", q_rot, 4)
+    _check_bf16("cache_k", cache_k, 4)
+    _check_bf16("cache_v", cache_v, 4)
+    if q_rot.shape[1] != 1:
+        raise ValueError("kvattn_decode_noalloc takes one token per sequence (q_rot [B,1,H,d])")
+    dims = _dims_from_cache(q_rot, cache_k)
+    if out is None:
+        out = torch.empty_like(q_rot)
+    rc = fn(ctypes.byref(dims), _ptr(q_rot), _ptr(cache_k), _ptr(cache_v), _ptr(start_pos), int(max_kv_len_hint),
+            float(scale), _ptr(out), _ptr(dev_status), _stream(stream))
+    _check_status(rc, "kvattn_decode_noalloc")
+    return out

@@ -141,6 +141,33 @@ KVATTN_API int kvattn_decode(const kvattn_dims* dims, const uint16_t* q_rot, con
                   float scale, uint16_t* out, void* workspace, size_t workspace_bytes,
                   int32_t* dev_status, kvattn_stream_t stream);
 
+/* Size of the static device array behind kvattn_decode_noalloc: 64 MiB. */
+#define KVATTN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+/* Allocation-free variant of kvattn_decode.  The pages have no counterpart:
+ * this exists for callers that cannot give the library device memory -- a
+ * plugin whose host framework owns every allocation and offers no allocator,
+ * an engine that has reserved nearly all of HBM for its caches and allows no
+ * allocation on the decode path, or a latency-critical loop that cannot pay
+ * for cudaMalloc/cudaFree.  Arguments and results are those of kvattn_decode
+ * without the workspace: the split partials go to a file-scope device array of
+ * KVATTN_NOALLOC_SCRATCH_BYTES that every GPU using this entry point keeps
+ * until the process exits.  The entry point itself allocates nothing.
+ *  - The array's device address is looked up on the first call on each
+ *    device; make that first call before any stream capture.
+ *  - Every call shares the one array: calls whose kernels overlap on the GPU
+ *    (other streams, other host threads) race and must be serialised by the
+ *    caller.  Nothing in the array needs to start at zero.
+ *  - Shapes whose partials need more than the array (see
+ *    kvattn_decode_workspace_bytes) return KVATTN_ERR_WORKSPACE and launch
+ *    nothing. */
+KVATTN_API int kvattn_decode_noalloc(const kvattn_dims* dims, const uint16_t* q_rot, const uint16_t* cache_k,
+                                     const uint16_t* cache_v, const int32_t* start_pos, int32_t max_kv_len_hint,
+                                     float scale, uint16_t* out, int32_t* dev_status, kvattn_stream_t stream);
+
+/* KVATTN_NOALLOC_SCRATCH_BYTES, as built into the library. */
+KVATTN_API size_t kvattn_decode_noalloc_scratch_bytes(void);
+
 /* Bytes of device workspace kvattn_prefill_chunk needs (may be 0). */
 KVATTN_API size_t kvattn_prefill_workspace_bytes(const kvattn_dims* dims, int32_t T, int32_t max_kv_len_hint);
 
