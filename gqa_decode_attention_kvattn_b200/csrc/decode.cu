@@ -31,49 +31,73 @@
 #include "kvattn_internal.h"
 
 #include <algorithm>
+#include <type_traits>
 
 namespace kvattn {
 namespace {
 
+#ifndef KVATTN_DECODE_STAGES
+#define KVATTN_DECODE_STAGES 3
+#endif
+#ifndef KVATTN_DECODE_MIN_BLOCKS
+#define KVATTN_DECODE_MIN_BLOCKS 3
+#endif
+
 constexpr int kTileRows = 32;
-constexpr int kStages = 4;
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kHalfWarps = kConsumerWarps * 2;
-constexpr int kMaxRowSets = 4096;  // (b,t) row sets handled with a split table
+constexpr int kMaxRowSets = 512;  // (b,t) row sets handled with a split table
 constexpr uint32_t kTileBytes = kTileRows * kHeadDim * 2;
 
 constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
+
+// Shared-memory transpose buffer of the score reduction: per half-warp, 16
+// rows (one per lane) of up to 16 partial sums; the 80-byte row pitch keeps
+// the 16-byte stores of 8 lanes on distinct banks, and the 336-float region
+// pitch puts the two half-warps of a warp on opposite bank halves.
+constexpr int kRedPitch = 20;
+constexpr int kRedRegion = 336;
 
 template <int G>
 struct Shape {
   static constexpr int RB = (G >= 8) ? 2 : 4;     // rows per half-warp batch
   static constexpr int NV = G * RB;                // partial dot products per lane
   static constexpr int LOG2NV = ilog2(NV);
-  static constexpr int RS = LOG2NV < 4 ? LOG2NV : 4;  // reduce-scatter steps
-  static constexpr int SLOTS = NV >> RS;           // complete scores per lane
-  static constexpr int REP = 1 << (4 - RS);        // lanes holding the same score
+  static constexpr int REP = NV >= 16 ? 1 : 16 / NV;  // lanes that end up with the same score
   static constexpr int PASSES = kTileRows / (kHalfWarps * RB);
+  // pipeline depth and resident CTAs per SM: G <= 4 fits three CTAs (about
+  // 124 registers a thread); G = 8 holds twice the q/o registers and fits two
+  static constexpr int STAGES = (G <= 4) ? KVATTN_DECODE_STAGES : 4;
+  static constexpr int MIN_BLOCKS = (G <= 4) ? KVATTN_DECODE_MIN_BLOCKS : 2;
   static_assert(kTileRows % (kHalfWarps * RB) == 0, "tile rows");
-  static_assert(NV >= 4 && NV <= 32, "values per lane");
+  static_assert(NV >= 4 && NV <= 16 && NV % 4 == 0, "values per lane");
 };
 
 template <int G>
 struct __align__(128) Smem {
-  uint16_t k[kStages][kTileRows][kHeadDim];
-  uint16_t v[kStages][kTileRows][kHeadDim];
+  uint16_t k[Shape<G>::STAGES][kTileRows][kHeadDim];
+  uint16_t v[Shape<G>::STAGES][kTileRows][kHeadDim];
+  // q of the G heads of an item, delivered with the item's first tile
+  uint16_t q[Shape<G>::STAGES][G][kHeadDim];
+  // the score-reduction buffer is only used inside the tile loop and the
+  // merge buffer only between the named barriers of an item's epilogue
+  union {
+    float red[kHalfWarps * kRedRegion];
+    float merge_o[kConsumerWarps][G][kHeadDim];
+  } u;
   // per half-warp, double-buffered: probabilities and rescale factors, each
   // stored twice so that one 8-byte read yields a packed fp32 pair
   float2 p[2][kHalfWarps][Shape<G>::NV];
   float2 alpha[2][kHalfWarps][G];
   float merge_m[kHalfWarps][G];
   float merge_l[kHalfWarps][G];
-  float merge_o[kConsumerWarps][G][kHeadDim];
   int row_set_start[kMaxRowSets + 1];
+  int row_set_len[kMaxRowSets];  // visible rows of each row set (0: invalid)
   int total_items;
   int abort;  // set when a pipeline wait gave up; later waits return at once
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
+  uint64_t full[Shape<G>::STAGES];
+  uint64_t empty[Shape<G>::STAGES];
 };
 
 struct Item {
@@ -88,8 +112,8 @@ __device__ __forceinline__ int splits_of(const DecodeArgs& a, int b, int t, int&
   return (L + a.rows_per_split - 1) / a.rows_per_split;
 }
 
-__device__ __forceinline__ Item decode_item(const DecodeArgs& a, const int* row_set_start, int n_sets,
-                                            int i) {
+__device__ __forceinline__ Item decode_item(const DecodeArgs& a, const int* row_set_start,
+                                            const int* row_set_len, int n_sets, int i) {
   Item it;
   if (a.max_splits == 1) {
     it.v = i / a.Hkv;
@@ -108,20 +132,29 @@ __device__ __forceinline__ Item decode_item(const DecodeArgs& a, const int* row_
   }
   it.b = it.v / a.Tq;
   it.t = it.v - it.b * a.Tq;
-  it.nsplit = splits_of(a, it.b, it.t, it.L);
+  if (a.max_splits == 1) {
+    it.nsplit = splits_of(a, it.b, it.t, it.L);
+  } else {
+    it.L = row_set_len[it.v];
+    it.nsplit = it.L > 0 ? (it.L + a.rows_per_split - 1) / a.rows_per_split : 0;
+  }
   it.r0 = it.split * a.rows_per_split;
   it.r1 = it.nsplit == 0 ? it.r0 : min(it.r0 + a.rows_per_split, it.L);
   return it;
 }
 
 template <int G>
-__global__ void __launch_bounds__(kThreads, 2) decode_splitk_kernel(
+__global__ void __launch_bounds__(kThreads, Shape<G>::MIN_BLOCKS) decode_splitk_kernel(
     const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
     const DecodeArgs a, const int evict_first) {
   using Sh = Shape<G>;
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
-  Smem<G>& sm = *reinterpret_cast<Smem<G>*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr int kStages = Sh::STAGES;
+  constexpr uint32_t kQBytes = G * kHeadDim * 2;
+  // dynamic shared memory starts 128-byte aligned (the declaration asks for
+  // it); casting the array itself keeps the shared state space visible to
+  // the compiler, so accesses through `sm` become LDS/STS
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  Smem<G>& sm = *reinterpret_cast<Smem<G>*>(smem_raw);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -175,7 +208,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_splitk_kernel(
       int L;
       const int b = v / a.Tq;
       sm.row_set_start[v] = run;
-      run += splits_of(a, b, v - b * a.Tq, L) * a.Hkv;
+      const int ns = splits_of(a, b, v - b * a.Tq, L);
+      sm.row_set_len[v] = ns > 0 ? L : 0;
+      run += ns * a.Hkv;
     }
     if (tid == kThreads - 1) {
       int tot = 0;
@@ -206,13 +241,18 @@ __global__ void __launch_bounds__(kThreads, 2) decode_splitk_kernel(
       int stage = 0;
       uint32_t phase = 0;
       for (int i = blockIdx.x; i < total_items && !sm.abort; i += gridDim.x) {
-        const Item it = decode_item(a, sm.row_set_start, n_sets, i);
+        const Item it = decode_item(a, sm.row_set_start, sm.row_set_len, n_sets, i);
         for (int row = it.r0; row < it.r1; row += kTileRows) {
           if (!mbar_wait(&sm.empty[stage], phase ^ 1, &sm.abort)) {
             abort_pipeline(&sm.abort, a.dev_status);
             break;
           }
-          mbar_arrive_expect_tx(&sm.full[stage], 2 * kTileBytes);
+          const bool first = row == it.r0;
+          mbar_arrive_expect_tx(&sm.full[stage], 2 * kTileBytes + (first ? kQBytes : 0u));
+          if (first) {
+            const uint16_t* qsrc = a.q_rot + (((size_t)it.b * a.Tq + it.t) * a.H + (size_t)it.kvh * G) * kHeadDim;
+            bulk_load(&sm.q[stage][0][0], qsrc, kQBytes, &sm.full[stage]);
+          }
           tma_load_4d(&sm.k[stage][0][0], &tmap_k, &sm.full[stage], 0, it.kvh, row, it.b, policy);
           tma_load_4d(&sm.v[stage][0][0], &tmap_v, &sm.full[stage], 0, it.kvh, row, it.b, policy);
           if (++stage == kStages) { stage = 0; phase ^= 1; }
@@ -236,14 +276,15 @@ __global__ void __launch_bounds__(kThreads, 2) decode_splitk_kernel(
   const int l16 = lane & 15;                // 8 elements [8*l16, 8*l16+8) of every row
   const int hwg = warp * 2 + hw;            // half-warp within the CTA
 
-  // slot bookkeeping: which (head, row) scores this lane ends up holding
+  // score bookkeeping: after the reduction lane l16 holds the complete score
+  // n = h*RB + j (head h, row j of the batch) with n = l16 / REP
   constexpr int LOGRB = ilog2(Sh::RB);
-  int slot_n0;  // n of slot 0; n = h*RB + j
-  if constexpr (Sh::LOG2NV >= 4) slot_n0 = l16 << (Sh::LOG2NV - 4);
-  else slot_n0 = l16 >> (4 - Sh::LOG2NV);
-  const int my_head = slot_n0 >> LOGRB;     // every slot of a lane has the same head
+  constexpr int LOGREP = ilog2(Sh::REP);
+  const int slot_n0 = l16 >> LOGREP;
+  const int my_head = slot_n0 >> LOGRB;
   const bool writer = (l16 & (Sh::REP - 1)) == 0;
   const bool head_writer = writer && ((slot_n0 & (Sh::RB - 1)) == 0);
+  float* const red = sm.u.red + hwg * kRedRegion;
 
   int stage = 0;
   uint32_t phase = 0;
@@ -253,21 +294,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_splitk_kernel(
   // named barriers; after an aborted wait it keeps walking without waiting
   // (its results are then garbage, flagged in dev_status).
   for (int i = blockIdx.x; i < total_items; i += gridDim.x) {
-    const Item it = decode_item(a, sm.row_set_start, n_sets, i);
+    const Item it = decode_item(a, sm.row_set_start, sm.row_set_len, n_sets, i);
     if (it.nsplit == 0) continue;
-    // q of the G heads of this group, scaled into log2 units
-    uint64_t q2[G][4];
-    {
-      const uint16_t* qp = a.q_rot + (((size_t)it.b * a.Tq + it.t) * a.H + (size_t)it.kvh * G) * kHeadDim + 8 * l16;
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const uint4 w = *reinterpret_cast<const uint4*>(qp + (size_t)h * kHeadDim);
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          q2[h][k] = f2_pack(bf16lo_to_f32(ws[k]) * a.scale_log2, bf16hi_to_f32(ws[k]) * a.scale_log2);
-      }
-    }
+    uint64_t q2[G][4];  // q of the G heads, scaled into log2 units (read at the first tile)
     uint64_t o2[G][4];
 #pragma unroll
     for (int h = 0; h < G; ++h)
@@ -278,10 +307,22 @@ __global__ void __launch_bounds__(kThreads, 2) decode_splitk_kernel(
 
     for (int row = it.r0; row < it.r1; row += kTileRows) {
       if (!mbar_wait(&sm.full[stage], phase, &sm.abort)) abort_pipeline(&sm.abort, a.dev_status);
+      if (row == it.r0) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const uint4 w = lds128(&sm.q[stage][h][8 * l16]);
+          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            q2[h][k] = f2_pack(bf16lo_to_f32(ws[k]) * a.scale_log2, bf16hi_to_f32(ws[k]) * a.scale_log2);
+        }
+      }
       const uint16_t* Kt = &sm.k[stage][0][0];
       const uint16_t* Vt = &sm.v[stage][0][0];
-#pragma unroll
-      for (int pass = 0; pass < Sh::PASSES; ++pass) {
+      // One batch: RB rows per half-warp.  MASKED is true only on the last
+      // tile of an item, where some rows may lie past the item's end.
+      auto batch = [&](int pass, auto masked_tag) {
+        constexpr bool MASKED = decltype(masked_tag)::value;
         const int rbase = pass * kHalfWarps * Sh::RB + hwg * Sh::RB;  // row within the tile
         // ---- partial scores for RB rows x G heads
         float part[Sh::NV];
@@ -301,62 +342,47 @@ __global__ void __launch_bounds__(kThreads, 2) decode_splitk_kernel(
             part[h * Sh::RB + j] = x + y;
           }
         }
-        // ---- reduce-scatter over the 16 lanes of the half-warp
-        int cnt = Sh::NV;
+        // ---- reduce over the 16 lanes through shared memory: lane l16
+        // stores its NV partials as row l16, then sums column n = l16/REP
 #pragma unroll
-        for (int st = 0; st < Sh::RS; ++st) {
-          const int m = 8 >> st;
-          const bool upper = (l16 & m) != 0;
-          cnt >>= 1;
+        for (int x = 0; x < Sh::NV; x += 4)
+          *reinterpret_cast<float4*>(red + l16 * kRedPitch + x) =
+              make_float4(part[x], part[x + 1], part[x + 2], part[x + 3]);
+        __syncwarp();
+        float col[16];
 #pragma unroll
-          for (int x = 0; x < Sh::NV / 2; ++x) {
-            if (x < cnt) {
-              const float send = upper ? part[x] : part[x + cnt];
-              const float keep = upper ? part[x + cnt] : part[x];
-              part[x] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-            }
-          }
+        for (int k = 0; k < 16; ++k) col[k] = red[k * kRedPitch + slot_n0];
+#pragma unroll
+        for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+          for (int k = 0; k < w; ++k) col[k] += col[k + w];
+        float sc = col[0];
+        if constexpr (MASKED) {
+          if (row + rbase + (slot_n0 & (Sh::RB - 1)) >= it.r1) sc = -INFINITY;
         }
-#pragma unroll
-        for (int m = 8 >> Sh::RS; m >= 1; m >>= 1) part[0] += __shfl_xor_sync(0xffffffffu, part[0], m);
 
-        // ---- mask rows beyond this item and take the per-head tile max
-        float s[Sh::SLOTS];
-        float tmax = -INFINITY;
+        // ---- online softmax in log2 units with a lazily moved reference:
+        // the reference max m_run only moves when the tile max exceeds it by
+        // more than 8 (so every probability stays <= 2^8); o and l are
+        // rescaled only then, and the final normalisation uses the same
+        // reference, so the result is unchanged.
+        float tmax = sc;
 #pragma unroll
-        for (int x = 0; x < Sh::SLOTS; ++x) {
-          const int j = (slot_n0 + x) & (Sh::RB - 1);
-          s[x] = (row + rbase + j < it.r1) ? part[x] : -INFINITY;
-          tmax = fmaxf(tmax, s[x]);
-        }
-        // lanes holding the other rows of my head differ in the lane bits that
-        // carry n's low LOGRB bits
-#pragma unroll
-        for (int k = 0; k < LOGRB; ++k) {
-          int lane_bit;
-          if constexpr (Sh::LOG2NV >= 4) lane_bit = k - (Sh::LOG2NV - 4);
-          else lane_bit = k + (4 - Sh::LOG2NV);
-          if (lane_bit >= 0) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1 << lane_bit));
-        }
-        const float m_new = fmaxf(m_run, tmax);
-        // m_new is -inf only while every row so far was masked (cannot happen
-        // for the first tile of an item, which always has row r0 < r1)
-        const float alpha = (m_new == -INFINITY) ? 1.f : exp2f(m_run - m_new);
+        for (int k = 0; k < LOGRB; ++k) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1 << (k + LOGREP)));
+        const bool move = tmax > m_run + 8.f;  // also true while m_run is -inf
+        const float m_new = move ? tmax : m_run;
+        const float alpha = move ? fast_exp2(m_run - m_new) : 1.f;  // 2^-inf = 0 on the first move
         m_run = m_new;
-        float psum = 0.f;
         float2* pb = sm.p[pbuf][hwg];
-#pragma unroll
-        for (int x = 0; x < Sh::SLOTS; ++x) {
-          const float p = (s[x] == -INFINITY) ? 0.f : exp2f(s[x] - m_new);
-          psum += p;
-          if (writer) pb[slot_n0 + x] = make_float2(p, p);
-        }
-        l_run = l_run * alpha + psum;
+        // m_new == -inf only while every row so far was masked
+        const float p = (m_new == -INFINITY) ? 0.f : fast_exp2(sc - m_new);
+        if (writer) pb[slot_n0] = make_float2(p, p);
+        l_run = l_run * alpha + p;
         if (head_writer) sm.alpha[pbuf][hwg][my_head] = make_float2(alpha, alpha);
-        const bool any_rescale = __any_sync(0xffffffffu, alpha != 1.f);
+        const bool any_rescale = __any_sync(0xffffffffu, move);
         __syncwarp();
 
-        // ---- rescale o and accumulate P.V
+        // ---- rescale o (rare) and accumulate P.V
         if (any_rescale) {
 #pragma unroll
           for (int h = 0; h < G; ++h) {
@@ -365,23 +391,43 @@ __global__ void __launch_bounds__(kThreads, 2) decode_splitk_kernel(
             for (int k = 0; k < 4; ++k) o2[h][k] = f2_mul(o2[h][k], al);
           }
         }
+        // two rows at a time: one 16-byte read gives both rows' probability
+        // of a head as packed pairs.  On a masked tile, rows past the item
+        // may hold any bits (even NaN), so their V words are replaced by
+        // zeros rather than multiplied by a zero probability.
 #pragma unroll
-        for (int j = 0; j < Sh::RB; ++j) {
-          if (row + rbase + j < it.r1) {
-            const uint4 vc = lds128(Vt + (rbase + j) * kHeadDim + 8 * l16);
-            const uint64_t v0 = bf16x2_to_f2(vc.x), v1 = bf16x2_to_f2(vc.y);
-            const uint64_t v2 = bf16x2_to_f2(vc.z), v3 = bf16x2_to_f2(vc.w);
+        for (int j = 0; j < Sh::RB; j += 2) {
+          uint4 va = lds128(Vt + (rbase + j) * kHeadDim + 8 * l16);
+          uint4 vb = lds128(Vt + (rbase + j + 1) * kHeadDim + 8 * l16);
+          if constexpr (MASKED) {
+            const bool ok0 = row + rbase + j < it.r1;
+            const bool ok1 = row + rbase + j + 1 < it.r1;
+            va.x = ok0 ? va.x : 0u; va.y = ok0 ? va.y : 0u; va.z = ok0 ? va.z : 0u; va.w = ok0 ? va.w : 0u;
+            vb.x = ok1 ? vb.x : 0u; vb.y = ok1 ? vb.y : 0u; vb.z = ok1 ? vb.z : 0u; vb.w = ok1 ? vb.w : 0u;
+          }
+          const uint64_t a0 = bf16x2_to_f2(va.x), a1 = bf16x2_to_f2(va.y);
+          const uint64_t a2 = bf16x2_to_f2(va.z), a3 = bf16x2_to_f2(va.w);
+          const uint64_t b0 = bf16x2_to_f2(vb.x), b1 = bf16x2_to_f2(vb.y);
+          const uint64_t b2 = bf16x2_to_f2(vb.z), b3 = bf16x2_to_f2(vb.w);
 #pragma unroll
-            for (int h = 0; h < G; ++h) {
-              const uint64_t p2 = *reinterpret_cast<const uint64_t*>(&pb[h * Sh::RB + j]);
-              o2[h][0] = f2_fma(p2, v0, o2[h][0]);
-              o2[h][1] = f2_fma(p2, v1, o2[h][1]);
-              o2[h][2] = f2_fma(p2, v2, o2[h][2]);
-              o2[h][3] = f2_fma(p2, v3, o2[h][3]);
-            }
+          for (int h = 0; h < G; ++h) {
+            const uint4 pp = lds128(&pb[h * Sh::RB + j]);
+            const uint64_t pa = ((uint64_t)pp.y << 32) | pp.x;
+            const uint64_t pbb = ((uint64_t)pp.w << 32) | pp.z;
+            o2[h][0] = f2_fma(pbb, b0, f2_fma(pa, a0, o2[h][0]));
+            o2[h][1] = f2_fma(pbb, b1, f2_fma(pa, a1, o2[h][1]));
+            o2[h][2] = f2_fma(pbb, b2, f2_fma(pa, a2, o2[h][2]));
+            o2[h][3] = f2_fma(pbb, b3, f2_fma(pa, a3, o2[h][3]));
           }
         }
         pbuf ^= 1;
+      };
+      if (row + kTileRows <= it.r1) {
+#pragma unroll
+        for (int pass = 0; pass < Sh::PASSES; ++pass) batch(pass, std::false_type{});
+      } else {
+#pragma unroll
+        for (int pass = 0; pass < Sh::PASSES; ++pass) batch(pass, std::true_type{});
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.empty[stage]);
@@ -392,12 +438,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_splitk_kernel(
     // complete the running sum of my head over the lanes of its rows
     float l_head = l_run;
 #pragma unroll
-    for (int k = 0; k < LOGRB; ++k) {
-      int lane_bit;
-      if constexpr (Sh::LOG2NV >= 4) lane_bit = k - (Sh::LOG2NV - 4);
-      else lane_bit = k + (4 - Sh::LOG2NV);
-      if (lane_bit >= 0) l_head += __shfl_xor_sync(0xffffffffu, l_head, 1 << lane_bit);
-    }
+    for (int k = 0; k < LOGRB; ++k) l_head += __shfl_xor_sync(0xffffffffu, l_head, 1 << (k + LOGREP));
     if (head_writer) {
       sm.merge_m[hwg][my_head] = m_run;
       sm.merge_l[hwg][my_head] = l_head;
@@ -411,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_splitk_kernel(
       for (int k = 0; k < kHalfWarps; ++k) mx = fmaxf(mx, sm.merge_m[k][h]);
       Mh[h] = mx;
       const float mine = sm.merge_m[hwg][h];
-      const float f = (mine == -INFINITY) ? 0.f : exp2f(mine - mx);
+      const float f = (mine == -INFINITY) ? 0.f : fast_exp2(mine - mx);
       const uint64_t f2 = f2_pack(f, f);
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
@@ -426,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_splitk_kernel(
     if (hw == 0) {
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        float4* dst = reinterpret_cast<float4*>(&sm.merge_o[warp][h][8 * l16]);
+        float4* dst = reinterpret_cast<float4*>(&sm.u.merge_o[warp][h][8 * l16]);
         float x0, x1, x2, x3, x4, x5, x6, x7;
         f2_unpack(o2[h][0], x0, x1);
         f2_unpack(o2[h][1], x2, x3);
@@ -443,12 +484,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_splitk_kernel(
       for (int h = 0; h < G; ++h) {
         float o = 0.f;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) o += sm.merge_o[w][h][c];
+        for (int w = 0; w < kConsumerWarps; ++w) o += sm.u.merge_o[w][h][c];
         float Ls = 0.f;
 #pragma unroll
         for (int k = 0; k < kHalfWarps; ++k) {
           const float mk = sm.merge_m[k][h];
-          if (mk != -INFINITY) Ls += sm.merge_l[k][h] * exp2f(mk - Mh[h]);
+          if (mk != -INFINITY) Ls += sm.merge_l[k][h] * fast_exp2(mk - Mh[h]);
         }
         const int head = it.kvh * G + h;
         if (it.nsplit == 1) {
@@ -485,7 +526,7 @@ __global__ void __launch_bounds__(kHeadDim) decode_merge_kernel(const DecodeArgs
   float num = 0.f, den = 0.f;
   for (int s = 0; s < ns; ++s) {
     const size_t slot = base + (size_t)s * a.H;
-    const float f = exp2f(a.ws_ml[slot * 2] - M);
+    const float f = fast_exp2(a.ws_ml[slot * 2] - M);
     num += f * a.ws_o[slot * kHeadDim + c];
     den += f * a.ws_ml[slot * 2 + 1];
   }
@@ -494,7 +535,7 @@ __global__ void __launch_bounds__(kHeadDim) decode_merge_kernel(const DecodeArgs
 
 template <int G>
 size_t smem_bytes() {
-  return sizeof(Smem<G>) + 1024;
+  return sizeof(Smem<G>);
 }
 
 template <int G>
@@ -525,11 +566,43 @@ cudaError_t launch_g(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorM
 
 }  // namespace
 
+// Resident CTAs per SM of the decode kernel for group size G (occupancy
+// query: registers and shared memory both count).
+template <int G>
+int resident_ctas() {
+  int n = 0;
+  if (cudaFuncSetAttribute(decode_splitk_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem_bytes<G>()) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_splitk_kernel<G>, kThreads, smem_bytes<G>()) !=
+          cudaSuccess ||
+      n < 1)
+    n = 1;
+  return n;
+}
+
+int resident_ctas_for(int G) {
+  static int cached[64][4] = {};  // [device][log2 G], 0 = not yet queried
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+  const int gi = G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : 3;
+  int n = __atomic_load_n(&cached[dev][gi], __ATOMIC_RELAXED);
+  if (n == 0) {
+    switch (G) {
+      case 1: n = resident_ctas<1>(); break;
+      case 2: n = resident_ctas<2>(); break;
+      case 4: n = resident_ctas<4>(); break;
+      default: n = resident_ctas<8>(); break;
+    }
+    __atomic_store_n(&cached[dev][gi], n, __ATOMIC_RELAXED);
+  }
+  return n;
+}
+
 DecodePlan plan_decode(int B, int Tq, int H, int Hkv, int kv_len_hint, int sm_count) {
   DecodePlan p;
   const int G = H / Hkv;
-  const size_t smem = G == 1 ? smem_bytes<1>() : G == 2 ? smem_bytes<2>() : G == 4 ? smem_bytes<4>() : smem_bytes<8>();
-  const int ctas_per_sm = (int)std::max<size_t>(1, std::min<size_t>(4, (227 * 1024) / (smem + 1024)));
+  const int ctas_per_sm = resident_ctas_for(G);
+  p.ctas_per_sm = ctas_per_sm;
   const int slots = sm_count * ctas_per_sm;
   const long long row_sets = (long long)B * Tq;
   // Aim for ~16 items per resident CTA so the round-robin stays balanced when

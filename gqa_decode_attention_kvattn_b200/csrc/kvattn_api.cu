@@ -236,6 +236,24 @@ int kvattn_prefill_chunk(const kvattn_dims* dims, int32_t T, const uint16_t* q_r
                        workspace_bytes, dev_status, stream);
 }
 
+int kvattn_decode_plan(const kvattn_dims* dims, int32_t max_kv_len_hint, int32_t* rows_per_split,
+                       int32_t* max_splits, int32_t* grid, int32_t* ctas_per_sm) {
+  int rc = check_dims(dims);
+  if (rc != KVATTN_OK) return rc;
+  if (!group_supported(dims->n_heads / dims->n_kv_heads)) return KVATTN_ERR_UNSUPPORTED;
+  const int hint = hint_or_default(max_kv_len_hint, dims->max_seq_len);
+  if (hint > dims->max_seq_len || hint < 1) return KVATTN_ERR_OUT_OF_RANGE;
+  int sms = 0;
+  rc = current_sm_count(&sms);
+  if (rc != KVATTN_OK) return rc;
+  const kvattn::DecodePlan p = kvattn::plan_decode(dims->batch, 1, dims->n_heads, dims->n_kv_heads, hint, sms);
+  if (rows_per_split) *rows_per_split = p.rows_per_split;
+  if (max_splits) *max_splits = p.max_splits;
+  if (grid) *grid = p.grid;
+  if (ctas_per_sm) *ctas_per_sm = p.ctas_per_sm;
+  return KVATTN_OK;
+}
+
 const char* kvattn_status_string(int status) {
   switch (status) {
     case KVATTN_OK: return "ok";

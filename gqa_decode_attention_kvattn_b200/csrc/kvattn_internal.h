@@ -51,6 +51,7 @@ struct DecodePlan {
   int rows_per_split;
   int max_splits;
   int grid;
+  int ctas_per_sm;
   size_t ws_bytes;
 };
 

@@ -141,6 +141,14 @@ KVATTN_API int kvattn_decode(const kvattn_dims* dims, const uint16_t* q_rot, con
                   float scale, uint16_t* out, void* workspace, size_t workspace_bytes,
                   int32_t* dev_status, kvattn_stream_t stream);
 
+/* How kvattn_decode will split the work for these dims and max_kv_len_hint
+ * on the CURRENT device: rows per split (C), the most splits a sequence can
+ * have, the persistent grid (CTAs) and the CTAs resident per SM.  Any output
+ * pointer may be NULL.  Returns a kvattn_status (host-side only, launches
+ * nothing). */
+KVATTN_API int kvattn_decode_plan(const kvattn_dims* dims, int32_t max_kv_len_hint, int32_t* rows_per_split,
+                                  int32_t* max_splits, int32_t* grid, int32_t* ctas_per_sm);
+
 /* Size of the static device array behind kvattn_decode_noalloc: 64 MiB. */
 #define KVATTN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 
