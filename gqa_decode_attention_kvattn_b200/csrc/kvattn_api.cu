@@ -168,6 +168,66 @@ int run_attention(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, con
   return kvattn::launch_decode(a, tk, tv, (cudaStream_t)stream) == cudaSuccess ? KVATTN_OK : KVATTN_ERR_CUDA;
 }
 
+
+// 4-D view (d, head, row, seq) of a [B, R, heads, 128] bf16 tensor with
+// 128-byte swizzled boxes of 64 elements x box_heads x box_rows.
+int encode_sw128_map(CUtensorMap* map, const void* base, int B, int R, int heads, int box_heads, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return KVATTN_ERR_CUDA;
+  const cuuint64_t dims[4] = {(cuuint64_t)kHeadDim, (cuuint64_t)heads, (cuuint64_t)R, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)heads * kHeadDim * 2,
+                                 (cuuint64_t)R * heads * kHeadDim * 2};
+  const cuuint32_t box[4] = {64, (cuuint32_t)box_heads, (cuuint32_t)box_rows, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? KVATTN_OK : KVATTN_ERR_CUDA;
+}
+
+int run_prefill_tc(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, const uint16_t* cache_k,
+                   const uint16_t* cache_v, const int32_t* start_pos, int32_t max_kv_len_hint, float scale,
+                   uint16_t* out, int32_t* dev_status, kvattn_stream_t stream) {
+  int rc = check_dims(dims);
+  if (rc != KVATTN_OK) return rc;
+  if (T < 1) return KVATTN_ERR_INVALID_ARG;
+  const int G = dims->n_heads / dims->n_kv_heads;
+  if (!group_supported(G)) return KVATTN_ERR_UNSUPPORTED;
+  if (!q_rot || !cache_k || !cache_v || !start_pos || !out) return KVATTN_ERR_INVALID_ARG;
+  if (!aligned16(q_rot) || !aligned16(cache_k) || !aligned16(cache_v) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(start_pos) & 3u))
+    return KVATTN_ERR_INVALID_ARG;
+  const int hint = hint_or_default(max_kv_len_hint, dims->max_seq_len);
+  if (hint > dims->max_seq_len || hint < T) return KVATTN_ERR_OUT_OF_RANGE;
+  if (!(scale > 0.f)) scale = 1.0f / std::sqrt((float)kHeadDim);
+  if (!std::isfinite(scale)) return KVATTN_ERR_INVALID_ARG;
+  const int tt = kvattn::prefill_tokens_per_tile(G);
+  const long long n_mtiles = ((long long)T + tt - 1) / tt;
+  if (n_mtiles * dims->n_kv_heads * dims->batch > 0x7FFFFFFFll) return KVATTN_ERR_UNSUPPORTED;
+
+  CUtensorMap tq, tk, tv;
+  rc = encode_sw128_map(&tq, q_rot, dims->batch, T, dims->n_heads, G, tt);
+  if (rc != KVATTN_OK) return rc;
+  rc = encode_sw128_map(&tk, cache_k, dims->batch, dims->max_seq_len, dims->n_kv_heads, 1, 128);
+  if (rc != KVATTN_OK) return rc;
+  rc = encode_sw128_map(&tv, cache_v, dims->batch, dims->max_seq_len, dims->n_kv_heads, 1, 128);
+  if (rc != KVATTN_OK) return rc;
+
+  kvattn::PrefillArgs a;
+  a.B = dims->batch;
+  a.T = T;
+  a.H = dims->n_heads;
+  a.Hkv = dims->n_kv_heads;
+  a.S = dims->max_seq_len;
+  a.kv_len_hint = hint;
+  a.n_mtiles = (int)n_mtiles;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.start_pos = start_pos;
+  a.out = out;
+  a.dev_status = dev_status;
+  return kvattn::launch_prefill(a, tq, tk, tv, (cudaStream_t)stream) == cudaSuccess ? KVATTN_OK : KVATTN_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -220,20 +280,20 @@ int kvattn_decode(const kvattn_dims* dims, const uint16_t* q_rot, const uint16_t
 }
 
 size_t kvattn_prefill_workspace_bytes(const kvattn_dims* dims, int32_t T, int32_t max_kv_len_hint) {
-  if (check_dims(dims) != KVATTN_OK || T < 1) return 0;
-  const int hint = hint_or_default(max_kv_len_hint, dims->max_seq_len);
-  if (hint > dims->max_seq_len || hint < T) return 0;
-  int sms = 0;
-  if (current_sm_count(&sms) != KVATTN_OK) return 0;
-  return kvattn::plan_decode(dims->batch, T, dims->n_heads, dims->n_kv_heads, hint, sms).ws_bytes;
+  (void)dims;
+  (void)T;
+  (void)max_kv_len_hint;
+  return 0;  // the tensor-core prefill keeps its partial state in TMEM
 }
 
 int kvattn_prefill_chunk(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, const uint16_t* cache_k,
                          const uint16_t* cache_v, const int32_t* start_pos, int32_t max_kv_len_hint, float scale,
                          uint16_t* out, void* workspace, size_t workspace_bytes, int32_t* dev_status,
                          kvattn_stream_t stream) {
-  return run_attention(dims, T, q_rot, cache_k, cache_v, start_pos, max_kv_len_hint, scale, out, workspace,
-                       workspace_bytes, dev_status, stream);
+  (void)workspace;
+  (void)workspace_bytes;
+  return run_prefill_tc(dims, T, q_rot, cache_k, cache_v, start_pos, max_kv_len_hint, scale, out, dev_status,
+                        stream);
 }
 
 int kvattn_decode_plan(const kvattn_dims* dims, int32_t max_kv_len_hint, int32_t* rows_per_split,

@@ -61,4 +61,21 @@ DecodePlan plan_decode(int B, int Tq, int H, int Hkv, int kv_len_hint, int sm_co
 cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tmap_k, const CUtensorMap& tmap_v,
                           cudaStream_t stream);
 
+// Chunked prefill on tcgen05: one CTA per (128-row M tile, KV head, sequence).
+struct PrefillArgs {
+  int B, T, H, Hkv, S;
+  int kv_len_hint;  // upper bound on start_pos[b] + T
+  int n_mtiles;     // ceil(T / tokens per tile)
+  float scale_log2; // softmax scale * log2(e)
+  const int32_t* start_pos;
+  uint16_t* out;    // [B, T, H, d]
+  int32_t* dev_status;
+};
+
+// Tokens per 128-row M tile for group size G (128 / G).
+int prefill_tokens_per_tile(int G);
+
+cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& tmap_q, const CUtensorMap& tmap_k,
+                           const CUtensorMap& tmap_v, cudaStream_t stream);
+
 }  // namespace kvattn

@@ -1,0 +1,476 @@
+// K4: chunked-prefill attention on the 5th-generation tensor cores (tcgen05,
+// accumulators in tensor memory).
+//
+// What it computes ("Llama 3 8B · KV cache", model.py 281-302 excerpt: the
+// scores of T new tokens against cache_len + T keys, where entry (i, j) is
+// masked iff j > cache_len + i; softmax(q K^T / sqrt(d)) V of "Llama 3.1 8B KV
+// cache", section "The cache itself is concatenation"; KV head floor(h/G) of
+// "Llama 3.1 8B · Repeat heads"): for token t of sequence b and query head h,
+//   out[b,t,h,:] = sum_{r <= sp+t} softmax_r(scale * q[b,t,h,:] . K[b,r,j,:]) V[b,r,j,:]
+// with sp = start_pos[b] and j = floor(h/G).
+//
+// Tiling.  The G query heads of one KV head and 128/G consecutive tokens form
+// one 128-row M tile (row m = token * G + head), so the grouped heads share
+// every K/V tile without a materialised repeat.  One CTA owns one (M tile, KV
+// head, sequence) and walks the key rows in 128-row tiles up to the last key
+// its last token sees.  Per KV tile j:
+//   S_j = Q K_j^T        tcgen05.mma M=128 N=128 K=16 x8, bf16 -> fp32 in TMEM
+//   P_j = softmax part   4 warps, one query row per thread, read S from TMEM,
+//                        mask, exponentiate (log2 units), write bf16 P into a
+//                        128B-swizzled shared tile
+//   O  += P_j V_j        tcgen05.mma with V as an MN-major operand, fp32 in TMEM
+// S is double buffered in TMEM so that S_{j+1} = Q K_{j+1}^T runs on the
+// tensor cores while the softmax warps work on S_j; O stays in TMEM.  The
+// reference max of a row only moves when a tile's max exceeds it by more than
+// 8 (probabilities stay <= 2^8), so O is rescaled rarely.
+//
+// Warps: 0 = TMA producer, 1 = TMEM owner and MMA issuer (one thread),
+// 2..5 = softmax and epilogue (warp w reads TMEM lanes 32*(w%4)..+31).
+#include "kvattn_device.cuh"
+#include "kvattn_internal.h"
+
+#include <algorithm>
+
+namespace kvattn {
+namespace {
+
+constexpr int kBM = 128;            // query rows per tile
+constexpr int kBN = 128;            // key rows per tile
+constexpr int kHalf = 128 * 64 * 2; // one 128-row x 64-element bf16 half tile (16 KB)
+constexpr int kPrefillThreads = 192;
+constexpr uint32_t kTmemCols = 512; // S0 [0,128), S1 [128,256), O [256,384)
+constexpr uint32_t kColO = 256;
+
+// shared memory layout (offsets from a 1024-byte aligned base)
+constexpr uint32_t kOffQ = 0;                       // 2 halves
+constexpr uint32_t kOffK = kOffQ + 2 * kHalf;       // [stage 2][half 2]
+constexpr uint32_t kOffV = kOffK + 4 * kHalf;       // [stage 2][half 2]
+constexpr uint32_t kOffP = kOffV + 4 * kHalf;       // 2 halves
+constexpr uint32_t kOffBar = kOffP + 2 * kHalf;
+// barrier slots (8 bytes each)
+constexpr uint32_t kBarQFull = 0, kBarKFull = 1, kBarKEmpty = 3, kBarVFull = 5, kBarVEmpty = 7, kBarSFull = 9,
+                   kBarSEmpty = 11, kBarPFull = 13, kBarPVDone = 14, kBarMmaDone = 15, kNumBars = 16;
+constexpr uint32_t kOffTmemSlot = kOffBar + 8 * kNumBars;
+constexpr uint32_t kOffAbort = kOffTmemSlot + 8;
+constexpr uint32_t kPrefillSmemBytes = kOffAbort + 8 + 1024;  // + alignment slack
+
+// ------------------------------------------------------------ raw smem helpers
+__device__ __forceinline__ void bar_init(uint32_t a, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(a), "r"(count) : "memory");
+}
+__device__ __forceinline__ void bar_arrive(uint32_t a) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(a) : "memory");
+}
+__device__ __forceinline__ void bar_expect_tx(uint32_t a, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(a), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool bar_try_wait(uint32_t a, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(a), "r"(parity), "r"(1u << 20)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ int ld_shared_i32(uint32_t a) {
+  int v;
+  asm volatile("ld.volatile.shared.b32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void st_shared_i32(uint32_t a, int v) {
+  asm volatile("st.volatile.shared.b32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
+// Bounded wait (see kWaitLimitNs); gives up at once when the CTA's abort flag
+// is set, and sets it (plus the status bit) when it gives up itself.
+__device__ __forceinline__ bool bar_wait(uint32_t a, uint32_t parity, uint32_t abort_addr, int32_t* dev_status) {
+  if (ld_shared_i32(abort_addr)) return false;
+  if (bar_try_wait(a, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    if (bar_try_wait(a, parity)) return true;
+    if (ld_shared_i32(abort_addr)) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      st_shared_i32(abort_addr, 1);
+      if (dev_status) atomicOr(dev_status, KVATTN_DEV_WAIT_TIMEOUT);
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ void tma_load_4d_raw(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1,
+                                                int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+      "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
+}
+
+// ------------------------------------------------------------ tcgen05 helpers
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor (sm_100 UMMA format): start address,
+// leading / stride byte offsets (all >> 4), version 1, 128-byte swizzle.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFF) << 16) |
+         ((uint64_t)((sbo_bytes >> 4) & 0x3FFF) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor of kind::f16: bf16 A and B, fp32 D, M=128, N=128;
+// b_mn_major selects an N-contiguous B operand.
+__host__ __device__ constexpr uint32_t idesc_bf16_m128_n128(bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((128u >> 3) << 17) |
+         ((128u >> 4) << 24);
+}
+
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+#define KV_R32(r)                                                                                               \
+  "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),    \
+      "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),     \
+      "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),    \
+      "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+#define KV_W32(r)                                                                                                 \
+  "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),   \
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), \
+      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), \
+      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+
+// 32 consecutive 32-bit TMEM columns of this thread's lane (warp-collective).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
+      "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : KV_R32(r)
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,"
+      "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      KV_W32(r)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+template <int G>
+__global__ void __launch_bounds__(kPrefillThreads, 1)
+    prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                      const __grid_constant__ CUtensorMap tmap_v, const PrefillArgs a) {
+  constexpr int TT = kBM / G;  // tokens per M tile
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const uint32_t sQ = base + kOffQ, sK = base + kOffK, sV = base + kOffV, sP = base + kOffP;
+  auto bar = [&](uint32_t slot) { return base + kOffBar + 8u * slot; };
+  const uint32_t abort_addr = base + kOffAbort;
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+
+  // heaviest M tiles (latest tokens, most keys) first
+  const int per_tile = a.Hkv * a.B;
+  const int mtile = a.n_mtiles - 1 - (int)(blockIdx.x / per_tile);
+  const int rem = (int)(blockIdx.x % per_tile);
+  const int kvh = rem % a.Hkv;
+  const int b = rem / a.Hkv;
+  const int sp = a.start_pos[b];
+  if (sp < 0 || (long long)sp + a.T > a.S || (long long)sp + a.T > a.kv_len_hint) {
+    if (mtile == 0 && kvh == 0 && tid == 0)
+      set_status(a.dev_status, (sp < 0 || (long long)sp + a.T > a.S) ? KVATTN_DEV_START_POS_RANGE
+                                                                    : KVATTN_DEV_KV_LEN_HINT);
+    return;
+  }
+  const int t0 = mtile * TT;
+  const int t_last = min(t0 + TT, a.T) - 1;
+  const int Lmax = sp + t_last + 1;          // keys the tile's last token sees
+  const int n_kv = (Lmax + kBN - 1) / kBN;
+
+  if (tid == 0) {
+    bar_init(bar(kBarQFull), 1);
+    for (int s = 0; s < 2; ++s) {
+      bar_init(bar(kBarKFull + s), 1);
+      bar_init(bar(kBarKEmpty + s), 1);
+      bar_init(bar(kBarVFull + s), 1);
+      bar_init(bar(kBarVEmpty + s), 1);
+      bar_init(bar(kBarSFull + s), 1);
+      bar_init(bar(kBarSEmpty + s), 4);
+    }
+    bar_init(bar(kBarPFull), 4);
+    bar_init(bar(kBarPVDone), 1);
+    bar_init(bar(kBarMmaDone), 1);
+    st_shared_i32(abort_addr, 0);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(base + kOffTmemSlot),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = (uint32_t)ld_shared_i32(base + kOffTmemSlot);
+
+  if (warp == 0) {
+    // ================================================================ producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmap_q);
+      prefetch_tensormap(&tmap_k);
+      prefetch_tensormap(&tmap_v);
+      bar_expect_tx(bar(kBarQFull), 2 * kHalf);
+      tma_load_4d_raw(sQ, &tmap_q, bar(kBarQFull), 0, kvh * G, t0, b);
+      tma_load_4d_raw(sQ + kHalf, &tmap_q, bar(kBarQFull), 64, kvh * G, t0, b);
+      for (int j = 0; j < n_kv; ++j) {
+        const int s = j & 1;
+        const uint32_t par = ((j >> 1) & 1) ^ 1;
+        if (!bar_wait(bar(kBarKEmpty + s), par, abort_addr, a.dev_status)) break;
+        bar_expect_tx(bar(kBarKFull + s), 2 * kHalf);
+        tma_load_4d_raw(sK + (2 * s) * kHalf, &tmap_k, bar(kBarKFull + s), 0, kvh, j * kBN, b);
+        tma_load_4d_raw(sK + (2 * s + 1) * kHalf, &tmap_k, bar(kBarKFull + s), 64, kvh, j * kBN, b);
+        if (!bar_wait(bar(kBarVEmpty + s), par, abort_addr, a.dev_status)) break;
+        bar_expect_tx(bar(kBarVFull + s), 2 * kHalf);
+        tma_load_4d_raw(sV + (2 * s) * kHalf, &tmap_v, bar(kBarVFull + s), 0, kvh, j * kBN, b);
+        tma_load_4d_raw(sV + (2 * s + 1) * kHalf, &tmap_v, bar(kBarVFull + s), 64, kvh, j * kBN, b);
+      }
+    }
+  } else if (warp == 1) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_m128_n128(false);
+      constexpr uint32_t idesc_pv = idesc_bf16_m128_n128(true);
+      bool ok = bar_wait(bar(kBarQFull), 0, abort_addr, a.dev_status);
+      tc_fence_after();
+      auto issue_qk = [&](int j) {
+        const int s = j & 1;
+        if (!bar_wait(bar(kBarKFull + s), (j >> 1) & 1, abort_addr, a.dev_status)) return false;
+        if (!bar_wait(bar(kBarSEmpty + s), ((j >> 1) & 1) ^ 1, abort_addr, a.dev_status)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t da = sw128_desc(sQ + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024);
+          const uint64_t db = sw128_desc(sK + (2 * s + (kk >> 2)) * kHalf + (kk & 3) * 32, 16, 1024);
+          tc_mma(tmem + (uint32_t)s * 128u, da, db, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(bar(kBarSFull + s));
+        tc_commit(bar(kBarKEmpty + s));
+        return true;
+      };
+      if (ok) ok = issue_qk(0);
+      for (int j = 0; j < n_kv && ok; ++j) {
+        if (j + 1 < n_kv && !issue_qk(j + 1)) break;
+        const int s = j & 1;
+        if (!bar_wait(bar(kBarPFull), j & 1, abort_addr, a.dev_status)) break;
+        if (!bar_wait(bar(kBarVFull + s), (j >> 1) & 1, abort_addr, a.dev_status)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t da = sw128_desc(sP + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024);
+          // V tile as B = [keys x dims], dims contiguous: 64-dim atoms one half
+          // apart (LBO), 8-key groups 1 KB apart (SBO); 16 keys per step
+          const uint64_t db = sw128_desc(sV + (2 * s) * kHalf + kk * 2048, kHalf, 1024);
+          tc_mma(tmem + kColO, da, db, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(bar(kBarVEmpty + s));
+        tc_commit(bar(kBarPVDone));
+      }
+      tc_commit(bar(kBarMmaDone));
+      // every MMA issued above has finished once this completes
+      bar_wait(bar(kBarMmaDone), 0, abort_addr, nullptr);
+    }
+  } else {
+    // ================================================================ softmax / epilogue
+    const int quarter = warp & 3;         // TMEM lanes 32*quarter .. +31
+    const int m = 32 * quarter + lane;    // query row of this thread
+    const int tok = t0 + m / G;
+    const int head = kvh * G + (m % G);
+    const int lim = sp + min(tok, a.T - 1);  // last visible key (rows past T borrow the last token's)
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * quarter) << 16);
+    const int st = tid - 64;              // 0..127 among the softmax threads
+    float m_ref = -INFINITY;
+    float l = 0.f;
+
+    for (int j = 0; j < n_kv; ++j) {
+      const int s = j & 1;
+      bar_wait(bar(kBarSFull + s), (j >> 1) & 1, abort_addr, a.dev_status);
+      tc_fence_after();
+      float sv[128];
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+        uint32_t r[32];
+        tmem_ld32(lane_addr + (uint32_t)s * 128u + 32u * c4, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 32; ++c) sv[32 * c4 + c] = __uint_as_float(r[c]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) bar_arrive(bar(kBarSEmpty + s));
+
+      const int kbase = j * kBN;
+      float mx = -INFINITY;
+      if (kbase + kBN - 1 > lim) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const float x = (kbase + c <= lim) ? sv[c] * a.scale_log2 : -INFINITY;
+          sv[c] = x;
+          mx = fmaxf(mx, x);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const float x = sv[c] * a.scale_log2;
+          sv[c] = x;
+          mx = fmaxf(mx, x);
+        }
+      }
+      const bool move = mx > m_ref + 8.f;
+      const float m_new = move ? mx : m_ref;
+      const float alpha = move ? fast_exp2(m_ref - m_new) : 1.f;
+      m_ref = m_new;
+      uint32_t pk[64];
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 128; c += 2) {
+        const float p0 = (m_new == -INFINITY) ? 0.f : fast_exp2(sv[c] - m_new);
+        const float p1 = (m_new == -INFINITY) ? 0.f : fast_exp2(sv[c + 1] - m_new);
+        sum += p0 + p1;
+        pk[c >> 1] = pack_bf16x2_rn(p0, p1);
+      }
+      l = l * alpha + sum;
+
+      if (j > 0) {
+        // PV_{j-1} done: the P buffer is free and O is stable
+        bar_wait(bar(kBarPVDone), (j - 1) & 1, abort_addr, a.dev_status);
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, move)) {
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            uint32_t r[32];
+            tmem_ld32(lane_addr + kColO + 32u * c4, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
+            tmem_st32(lane_addr + kColO + 32u * c4, r);
+          }
+          tmem_wait_st();
+        }
+      }
+      if (j == n_kv - 1 && Lmax < kbase + kBN) {
+        // rows of the last V tile past the last visible key may hold any bits;
+        // zero them so that 0 * (garbage) cannot reach O
+        bar_wait(bar(kBarVFull + s), (j >> 1) & 1, abort_addr, a.dev_status);
+        const int first_bad = Lmax - kbase;
+        const int nchunks = (kBN - first_bad) * 16;  // 16-byte chunks over both halves
+        for (int c = st; c < nchunks; c += 128) {
+          const int r = first_bad + (c >> 4);
+          const int half = (c >> 3) & 1;
+          const int cc = c & 7;
+          st_shared_v4(sV + (2 * s + half) * kHalf + r * 128 + cc * 16, 0u, 0u, 0u, 0u);
+        }
+      }
+      // P row m into the 128B-swizzled K-major tile: chunk cc of half h of row m
+      // lives at h*16KB + m*128 + ((cc ^ (m & 7)) * 16)
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const int half = c >> 3, cc = c & 7;
+        st_shared_v4(sP + half * kHalf + m * 128 + ((cc ^ (m & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
+                     pk[4 * c + 3]);
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) bar_arrive(bar(kBarPFull));
+    }
+
+    // ---- epilogue: O / l -> bf16 rows
+    bar_wait(bar(kBarPVDone), (n_kv - 1) & 1, abort_addr, a.dev_status);
+    tc_fence_after();
+    const float inv_l = 1.f / l;
+    const bool store = tok < a.T;
+    uint16_t* dst = a.out + (((size_t)b * a.T + (store ? tok : 0)) * a.H + head) * kHeadDim;
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4) {
+      uint32_t r[32];
+      tmem_ld32(lane_addr + kColO + 32u * c4, r);
+      tmem_wait_ld();
+      if (store) {
+#pragma unroll
+        for (int c = 0; c < 32; c += 8) {
+          uint4 w;
+          w.x = pack_bf16x2_rn(__uint_as_float(r[c]) * inv_l, __uint_as_float(r[c + 1]) * inv_l);
+          w.y = pack_bf16x2_rn(__uint_as_float(r[c + 2]) * inv_l, __uint_as_float(r[c + 3]) * inv_l);
+          w.z = pack_bf16x2_rn(__uint_as_float(r[c + 4]) * inv_l, __uint_as_float(r[c + 5]) * inv_l);
+          w.w = pack_bf16x2_rn(__uint_as_float(r[c + 6]) * inv_l, __uint_as_float(r[c + 7]) * inv_l);
+          *reinterpret_cast<uint4*>(dst + 32 * c4 + c) = w;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+  }
+}
+
+template <int G>
+cudaError_t launch_prefill_g(const PrefillArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
+                             const CUtensorMap& tv, cudaStream_t st) {
+  static bool configured[64] = {false};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!configured[dev]) {
+    e = cudaFuncSetAttribute(prefill_tc_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kPrefillSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  const long long grid = (long long)a.n_mtiles * a.Hkv * a.B;
+  if (grid <= 0 || grid > 0x7FFFFFFFll) return cudaErrorInvalidValue;
+  prefill_tc_kernel<G><<<(unsigned)grid, kPrefillThreads, kPrefillSmemBytes, st>>>(tq, tk, tv, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int prefill_tokens_per_tile(int G) { return kBM / G; }
+
+cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           cudaStream_t st) {
+  switch (a.H / a.Hkv) {
+    case 1: return launch_prefill_g<1>(a, tq, tk, tv, st);
+    case 2: return launch_prefill_g<2>(a, tq, tk, tv, st);
+    case 4: return launch_prefill_g<4>(a, tq, tk, tv, st);
+    case 8: return launch_prefill_g<8>(a, tq, tk, tv, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace kvattn

@@ -214,3 +214,33 @@ def test_prefill_equals_prefill_then_decode_steps():
     a = ks.bf16_bits_to_f64(outA)
     b = ks.bf16_bits_to_f64(outB)
     assert np.abs(a - b).max() <= 2 * U.MAX_ABS / 4
+
+
+@pytest.mark.parametrize("case", [
+    (2, 77, 32, 8, 400, [0, 250]),      # G=4: 3 M tiles (32 tokens each), ragged tail
+    (1, 300, 16, 8, 700, [123]),        # G=2: 64-token tiles, several key tiles
+    (2, 20, 64, 8, 300, [0, 129]),      # G=8: 16-token tiles
+    (1, 130, 8, 8, 260, [127]),         # G=1 (MHA): 128-token tiles
+    (3, 1, 32, 8, 300, [0, 127, 128]),  # one token per sequence through the prefill path
+])
+def test_prefill_tiles_and_groups(case):
+    B, T, H, Hkv, S, sp = case
+    _check_step(23, B, T, H, Hkv, S, sp, kv.LLAMA3, "prefill")
+
+
+@pytest.mark.parametrize("kind,T", [("decode", 1), ("prefill", 40)])
+def test_rows_past_the_sequence_may_hold_nan(kind, T):
+    # cache rows at and beyond start_pos+T are outside every mask; filling them
+    # with NaN must not change any output (no 0 * NaN may reach the result)
+    B, H, Hkv, S = 2, 32, 8, 512
+    sp = np.array([100, 300], np.int32)
+    q, k, v, ck, cv = U.host_inputs(24, B, T, H, Hkv, S, sp)
+    for b in range(B):
+        ck[b, sp[b]:] = 0x7FC0
+        cv[b, sp[b]:] = 0x7FC0
+    _, g_ck, g_cv, g_out, st = _dev_step(q, k, v, ck, cv, sp, kv.LLAMA3, T, kind)
+    assert st == 0
+    o_ck, o_cv = ck.copy(), cv.copy()
+    _, out, rc = oracle.step(q, k, v, o_ck, o_cv, sp, U.oracle_freqs(kv.LLAMA3))
+    assert rc == 0
+    U.assert_attention_close(g_out, out, f"{kind} with NaN past the sequence")
