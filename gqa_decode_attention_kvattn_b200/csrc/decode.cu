@@ -47,7 +47,8 @@ constexpr int kTileRows = 32;
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kHalfWarps = kConsumerWarps * 2;
-constexpr int kMaxRowSets = 512;  // (b,t) row sets handled with a split table
+constexpr int kMaxRowSets = 512;
+constexpr int kMaxBuckets = 129;  // last-split sizes in tiles: 1 .. 4096/32  // (b,t) row sets handled with a split table
 constexpr uint32_t kTileBytes = kTileRows * kHeadDim * 2;
 
 constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
@@ -92,55 +93,142 @@ struct __align__(128) Smem {
   float2 alpha[2][kHalfWarps][G];
   float merge_m[kHalfWarps][G];
   float merge_l[kHalfWarps][G];
-  int row_set_start[kMaxRowSets + 1];
-  int row_set_len[kMaxRowSets];  // visible rows of each row set (0: invalid)
-  int total_items;
+  // work table (split path): visible rows per row set, first full-split item
+  // of each row set, and the valid row sets ordered by the size of their
+  // last (partial) split, largest first
+  int set_len[kMaxRowSets];
+  int full_start[kMaxRowSets + 1];
+  int sorted_set[kMaxRowSets];
+  int bucket[kMaxBuckets + 1];
+  int n_full, total_items;
+  int stage_item[Shape<G>::STAGES];  // item whose tile fills the stage; -1: no more work
   int abort;  // set when a pipeline wait gave up; later waits return at once
   uint64_t full[Shape<G>::STAGES];
   uint64_t empty[Shape<G>::STAGES];
+  uint64_t cons;  // the four consumer warps' epilogue barrier
 };
 
 struct Item {
   int v, split, kvh, b, t, L, r0, r1, nsplit;
 };
 
-// Number of splits of row set v (0 when the set is invalid).
-__device__ __forceinline__ int splits_of(const DecodeArgs& a, int b, int t, int& L) {
+// Visible rows of row set v = (b, t), or 0 when its start position is out of
+// range; the number of splits of C rows it needs.
+__device__ __forceinline__ int set_length(const DecodeArgs& a, int v) {
+  const int b = v / a.Tq;
   const int sp = a.start_pos[b];
-  L = sp + t + 1;
   if (sp < 0 || (long long)sp + a.Tq > a.S || (long long)sp + a.Tq > a.kv_len_hint) return 0;
-  return (L + a.rows_per_split - 1) / a.rows_per_split;
+  return sp + (v - b * a.Tq) + 1;
 }
 
-__device__ __forceinline__ Item decode_item(const DecodeArgs& a, const int* row_set_start,
-                                            const int* row_set_len, int n_sets, int i) {
+// Item numbering.  Without splits (max_splits == 1): item i is row set
+// i / Hkv, KV head i % Hkv.  With splits: first every full split of every row
+// set (row-set major, KV head fastest), then the last split of each valid row
+// set in the order of sorted_set (largest first), so that work handed out
+// from a counter ends with the smallest pieces.
+template <class SM>
+__device__ __forceinline__ Item decode_item(const DecodeArgs& a, const SM& sm, int n_sets, int i) {
   Item it;
+  const int C = a.rows_per_split;
   if (a.max_splits == 1) {
     it.v = i / a.Hkv;
-    it.split = 0;
     it.kvh = i - it.v * a.Hkv;
-  } else {
-    int lo = 0, hi = n_sets;  // largest v with row_set_start[v] <= i
+    it.split = 0;
+    it.L = set_length(a, it.v);
+    it.nsplit = it.L > 0 ? 1 : 0;
+  } else if (i < sm.n_full) {
+    int lo = 0, hi = n_sets;  // largest v with full_start[v] <= i
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
-      if (row_set_start[mid] <= i) lo = mid; else hi = mid;
+      if (sm.full_start[mid] <= i) lo = mid; else hi = mid;
     }
     it.v = lo;
-    const int local = i - row_set_start[lo];
+    const int local = i - sm.full_start[lo];
     it.split = local / a.Hkv;
     it.kvh = local - it.split * a.Hkv;
+    it.L = sm.set_len[lo];
+    it.nsplit = (it.L + C - 1) / C;
+  } else {
+    const int r = (i - sm.n_full) / a.Hkv;
+    it.kvh = (i - sm.n_full) - r * a.Hkv;
+    it.v = sm.sorted_set[r];
+    it.L = sm.set_len[it.v];
+    it.nsplit = (it.L + C - 1) / C;
+    it.split = it.nsplit - 1;
   }
   it.b = it.v / a.Tq;
   it.t = it.v - it.b * a.Tq;
-  if (a.max_splits == 1) {
-    it.nsplit = splits_of(a, it.b, it.t, it.L);
-  } else {
-    it.L = row_set_len[it.v];
-    it.nsplit = it.L > 0 ? (it.L + a.rows_per_split - 1) / a.rows_per_split : 0;
-  }
-  it.r0 = it.split * a.rows_per_split;
-  it.r1 = it.nsplit == 0 ? it.r0 : min(it.r0 + a.rows_per_split, it.L);
+  it.r0 = it.split * C;
+  it.r1 = it.nsplit == 0 ? it.r0 : min(it.r0 + C, it.L);
   return it;
+}
+
+// Warp 0 builds the work table of the split path (deterministically, so that
+// every CTA derives the same numbering).
+template <class SM>
+__device__ void build_work_table(const DecodeArgs& a, SM& sm, int n_sets, int lane) {
+  const int C = a.rows_per_split;
+  const int nb = C / kTileRows + 1;  // bucket k holds last splits of C/32 - k + ... tiles
+  for (int k = lane; k <= nb; k += 32) sm.bucket[k] = 0;
+  __syncwarp();
+  // lengths, full-split prefix (warp scan over chunks of 32) and bucket counts
+  int run = 0;
+  for (int base = 0; base < n_sets; base += 32) {
+    const int v = base + lane;
+    int L = 0, full = 0;
+    if (v < n_sets) {
+      L = set_length(a, v);
+      sm.set_len[v] = L;
+      if (L > 0) {
+        const int ns = (L + C - 1) / C;
+        full = (ns - 1) * a.Hkv;
+        const int last_tiles = (L - (ns - 1) * C + kTileRows - 1) / kTileRows;
+        atomicAdd(&sm.bucket[C / kTileRows - last_tiles], 1);  // larger pieces, smaller key
+      }
+    }
+    int incl = full;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (v < n_sets) sm.full_start[v] = run + incl - full;
+    run += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (lane == 0) {
+    sm.full_start[n_sets] = run;
+    sm.n_full = run;
+  }
+  __syncwarp();
+  // exclusive prefix of the bucket counts (lane 0; at most 129 entries)
+  if (lane == 0) {
+    int acc = 0;
+    for (int k = 0; k < nb; ++k) {
+      const int c = sm.bucket[k];
+      sm.bucket[k] = acc;
+      acc += c;
+    }
+    sm.bucket[nb] = acc;  // valid row sets
+    sm.total_items = run + acc * a.Hkv;
+  }
+  __syncwarp();
+  // stable placement in row-set order: equal keys keep increasing v
+  for (int base = 0; base < n_sets; base += 32) {
+    const int v = base + lane;
+    const int L = v < n_sets ? sm.set_len[v] : 0;
+    int key = -1;
+    if (L > 0) {
+      const int ns = (L + C - 1) / C;
+      key = C / kTileRows - (L - (ns - 1) * C + kTileRows - 1) / kTileRows;
+    }
+    const unsigned same = __match_any_sync(0xffffffffu, key);
+    const int before = __popc(same & ((1u << lane) - 1u));
+    if (key >= 0) sm.sorted_set[sm.bucket[key] + before] = v;
+    __syncwarp();
+    const int last = 31 - __clz(same);  // highest lane holding this key
+    if (key >= 0 && lane == last) sm.bucket[key] += before + 1;
+    __syncwarp();
+  }
 }
 
 template <int G>
@@ -161,70 +249,30 @@ __global__ void __launch_bounds__(kThreads, Shape<G>::MIN_BLOCKS) decode_splitk_
   const int lane = tid & 31;
   const int n_sets = a.B * a.Tq;
 
-  // ---- item table (only when sequences are split) and barriers
-  if (a.max_splits == 1) {
-    if (tid == 0) sm.total_items = n_sets * a.Hkv;
-    if (blockIdx.x == 0 && tid < 32) {
+  // ---- work table and barriers
+  if (warp == 0) {
+    if (a.max_splits == 1) {
+      if (lane == 0) sm.total_items = n_sets * a.Hkv;
+    } else {
+      build_work_table(a, sm, n_sets, lane);
+    }
+    if (blockIdx.x == 0) {
       for (int v = lane; v < n_sets; v += 32) {
-        int L;
-        const int b = v / a.Tq;
-        if (splits_of(a, b, v - b * a.Tq, L) == 0) {
-          const int sp = a.start_pos[b];
+        if (set_length(a, v) == 0) {
+          const int sp = a.start_pos[v / a.Tq];
           set_status(a.dev_status, (sp < 0 || (long long)sp + a.Tq > a.S) ? KVATTN_DEV_START_POS_RANGE
                                                                          : KVATTN_DEV_KV_LEN_HINT);
         }
       }
     }
-  } else {
-    // exclusive scan of items per row set over all threads
-    const int per = (n_sets + kThreads - 1) / kThreads;
-    const int beg = min(tid * per, n_sets), end = min(beg + per, n_sets);
-    int local = 0;
-    for (int v = beg; v < end; ++v) {
-      int L;
-      const int b = v / a.Tq;
-      const int ns = splits_of(a, b, v - b * a.Tq, L);
-      if (ns == 0 && blockIdx.x == 0) {
-        const int sp = a.start_pos[b];
-        set_status(a.dev_status, (sp < 0 || (long long)sp + a.Tq > a.S) ? KVATTN_DEV_START_POS_RANGE
-                                                                       : KVATTN_DEV_KV_LEN_HINT);
-      }
-      local += ns * a.Hkv;
-    }
-    // warp-level inclusive scan of the per-thread sums
-    int incl = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    __shared__ int warp_tot[kThreads / 32];
-    if (lane == 31) warp_tot[warp] = incl;
-    __syncthreads();
-    int warp_off = 0;
-    for (int w = 0; w < warp; ++w) warp_off += warp_tot[w];
-    int run = warp_off + incl - local;
-    for (int v = beg; v < end; ++v) {
-      int L;
-      const int b = v / a.Tq;
-      sm.row_set_start[v] = run;
-      const int ns = splits_of(a, b, v - b * a.Tq, L);
-      sm.row_set_len[v] = ns > 0 ? L : 0;
-      run += ns * a.Hkv;
-    }
-    if (tid == kThreads - 1) {
-      int tot = 0;
-      for (int w = 0; w < kThreads / 32; ++w) tot += warp_tot[w];
-      sm.total_items = tot;
-      sm.row_set_start[n_sets] = tot;
-    }
   }
-  if (tid == 0) {
+  if (tid == 32) {
     sm.abort = 0;
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], kConsumerWarps);
     }
+    mbar_init(&sm.cons, kConsumerWarps);
     fence_barrier_init();
   }
   __syncthreads();
@@ -240,14 +288,37 @@ __global__ void __launch_bounds__(kThreads, Shape<G>::MIN_BLOCKS) decode_splitk_
       else asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(policy));
       int stage = 0;
       uint32_t phase = 0;
-      for (int i = blockIdx.x; i < total_items && !sm.abort; i += gridDim.x) {
-        const Item it = decode_item(a, sm.row_set_start, sm.row_set_len, n_sets, i);
+      // Items come from the per-call counter when there is one (dynamic
+      // balance), else round-robin over the grid.
+      int next_static = blockIdx.x;
+      for (;;) {
+        int i;
+        if (a.counter) i = atomicAdd(a.counter, 1);
+        else { i = next_static; next_static += gridDim.x; }
+        const bool done = i >= total_items || sm.abort;
+        Item it;
+        if (!done) {
+          it = decode_item(a, sm, n_sets, i);
+          if (it.nsplit == 0) continue;  // invalid row set: nothing to stream
+        }
+        if (done) {
+          // hand the consumers the end marker through the next stage
+          if (mbar_wait(&sm.empty[stage], phase ^ 1, &sm.abort)) {
+            sm.stage_item[stage] = -1;
+            mbar_arrive(&sm.full[stage]);
+          } else {
+            abort_pipeline(&sm.abort, a.dev_status);
+          }
+          if (++stage == kStages) { stage = 0; phase ^= 1; }
+          break;
+        }
         for (int row = it.r0; row < it.r1; row += kTileRows) {
           if (!mbar_wait(&sm.empty[stage], phase ^ 1, &sm.abort)) {
             abort_pipeline(&sm.abort, a.dev_status);
             break;
           }
           const bool first = row == it.r0;
+          sm.stage_item[stage] = i;
           mbar_arrive_expect_tx(&sm.full[stage], 2 * kTileBytes + (first ? kQBytes : 0u));
           if (first) {
             const uint16_t* qsrc = a.q_rot + (((size_t)it.b * a.Tq + it.t) * a.H + (size_t)it.kvh * G) * kHeadDim;
@@ -290,12 +361,27 @@ __global__ void __launch_bounds__(kThreads, Shape<G>::MIN_BLOCKS) decode_splitk_
   uint32_t phase = 0;
   int pbuf = 0;
 
-  // Every consumer warp walks the same items and tiles and meets the same
-  // named barriers; after an aborted wait it keeps walking without waiting
-  // (its results are then garbage, flagged in dev_status).
-  for (int i = blockIdx.x; i < total_items; i += gridDim.x) {
-    const Item it = decode_item(a, sm.row_set_start, sm.row_set_len, n_sets, i);
-    if (it.nsplit == 0) continue;
+  uint32_t cons_phase = 0;
+  // the four consumer warps meet here in an item's epilogue (bounded wait)
+  auto cons_sync = [&]() {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.cons);
+    mbar_wait(&sm.cons, cons_phase, &sm.abort);
+    cons_phase ^= 1;
+    __syncwarp();
+  };
+
+  // Every consumer warp reads the same item sequence from the stages the
+  // producer fills.  After an aborted wait the warps stop at their next item.
+  for (;;) {
+    if (!mbar_wait(&sm.full[stage], phase, &sm.abort)) abort_pipeline(&sm.abort, a.dev_status);
+    const int i = sm.stage_item[stage];
+    if (i < 0 || sm.abort) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.empty[stage]);
+      break;
+    }
+    const Item it = decode_item(a, sm, n_sets, i);
     uint64_t q2[G][4];  // q of the G heads, scaled into log2 units (read at the first tile)
     uint64_t o2[G][4];
 #pragma unroll
@@ -306,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, Shape<G>::MIN_BLOCKS) decode_splitk_
     float l_run = 0.f;        // running sum of my slots
 
     for (int row = it.r0; row < it.r1; row += kTileRows) {
-      if (!mbar_wait(&sm.full[stage], phase, &sm.abort)) abort_pipeline(&sm.abort, a.dev_status);
+      if (row != it.r0 && !mbar_wait(&sm.full[stage], phase, &sm.abort)) abort_pipeline(&sm.abort, a.dev_status);
       if (row == it.r0) {
 #pragma unroll
         for (int h = 0; h < G; ++h) {
@@ -443,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, Shape<G>::MIN_BLOCKS) decode_splitk_
       sm.merge_m[hwg][my_head] = m_run;
       sm.merge_l[hwg][my_head] = l_head;
     }
-    named_bar_sync(1, kConsumerWarps * 32);
+    cons_sync();
     float Mh[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
@@ -477,7 +563,7 @@ __global__ void __launch_bounds__(kThreads, Shape<G>::MIN_BLOCKS) decode_splitk_
         dst[1] = make_float4(x4, x5, x6, x7);
       }
     }
-    named_bar_sync(1, kConsumerWarps * 32);
+    cons_sync();
     {
       const int c = tid;  // 0..127: one output element per head
 #pragma unroll
@@ -506,29 +592,32 @@ __global__ void __launch_bounds__(kThreads, Shape<G>::MIN_BLOCKS) decode_splitk_
         }
       }
     }
-    named_bar_sync(1, kConsumerWarps * 32);
+    cons_sync();
   }
 }
 
 // K3: log-sum-exp merge of the split partials.  One CTA per (head, row set),
-// one thread per output element.
+// one thread per output element; one pass with a running maximum.
 __global__ void __launch_bounds__(kHeadDim) decode_merge_kernel(const DecodeArgs a) {
   const int head = blockIdx.x;
   const int v = blockIdx.y;
+  const int L = set_length(a, v);
+  const int ns = (L + a.rows_per_split - 1) / a.rows_per_split;
+  if (L == 0 || ns <= 1) return;  // invalid, or written directly by K2
   const int b = v / a.Tq, t = v - b * a.Tq;
-  int L;
-  const int ns = splits_of(a, b, t, L);
-  if (ns <= 1) return;
   const int c = threadIdx.x;
   const size_t base = (size_t)v * a.max_splits * a.H + head;
-  float M = -INFINITY;
-  for (int s = 0; s < ns; ++s) M = fmaxf(M, a.ws_ml[(base + (size_t)s * a.H) * 2]);
-  float num = 0.f, den = 0.f;
+  float M = -INFINITY, num = 0.f, den = 0.f;
   for (int s = 0; s < ns; ++s) {
     const size_t slot = base + (size_t)s * a.H;
-    const float f = fast_exp2(a.ws_ml[slot * 2] - M);
-    num += f * a.ws_o[slot * kHeadDim + c];
-    den += f * a.ws_ml[slot * 2 + 1];
+    const float2 ml = *reinterpret_cast<const float2*>(a.ws_ml + slot * 2);
+    const float o = a.ws_o[slot * kHeadDim + c];
+    const float Mn = fmaxf(M, ml.x);
+    const float f_old = (M == -INFINITY) ? 0.f : fast_exp2(M - Mn);
+    const float f_new = fast_exp2(ml.x - Mn);
+    num = num * f_old + o * f_new;
+    den = den * f_old + ml.y * f_new;
+    M = Mn;
   }
   a.out[(((size_t)b * a.Tq + t) * a.H + head) * kHeadDim + c] = (uint16_t)f32_to_bf16_bits(num / den);
 }
@@ -553,6 +642,10 @@ cudaError_t launch_g(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorM
     configured[dev] = true;
   }
   const int evict_first = a.Tq == 1 ? 1 : 0;
+  if (a.counter) {
+    cudaError_t e1 = cudaMemsetAsync(a.counter, 0, sizeof(int), st);
+    if (e1 != cudaSuccess) return e1;
+  }
   decode_splitk_kernel<G><<<a.grid, kThreads, smem, st>>>(tk, tv, a, evict_first);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -620,8 +713,24 @@ DecodePlan plan_decode(int B, int Tq, int H, int Hkv, int kv_len_hint, int sm_co
   const long long items_bound = row_sets * Hkv * p.max_splits;
   p.grid = (int)std::min<long long>(items_bound, slots);
   if (p.grid < 1) p.grid = 1;
-  p.ws_bytes = p.max_splits > 1 ? (size_t)row_sets * p.max_splits * H * (kHeadDim + 2) * sizeof(float) : 0;
+  // partial (o, max, sum) per (row set, split, head), then the work counter
+  p.ws_bytes =
+      p.max_splits > 1 ? (size_t)row_sets * p.max_splits * H * (kHeadDim + 2) * sizeof(float) + 16 : 0;
   return p;
+}
+
+void bind_decode_workspace(DecodeArgs& a, const DecodePlan& plan, void* workspace) {
+  if (plan.ws_bytes == 0 || !workspace) {
+    a.ws_o = nullptr;
+    a.ws_ml = nullptr;
+    a.counter = nullptr;
+    return;
+  }
+  const size_t n_slots = (size_t)a.B * a.Tq * plan.max_splits * a.H;
+  float* ws = static_cast<float*>(workspace);
+  a.ws_o = ws;
+  a.ws_ml = ws + n_slots * kHeadDim;
+  a.counter = reinterpret_cast<int*>(ws + n_slots * (kHeadDim + 2));
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st) {

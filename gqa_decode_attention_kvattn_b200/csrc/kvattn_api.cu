@@ -159,10 +159,7 @@ int run_attention(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, con
   a.q_rot = q_rot;
   a.out = out;
   a.start_pos = start_pos;
-  float* ws = static_cast<float*>(workspace);
-  const size_t n_slots = (size_t)dims->batch * T * plan.max_splits * dims->n_heads;
-  a.ws_o = plan.ws_bytes ? ws : nullptr;
-  a.ws_ml = plan.ws_bytes ? ws + n_slots * kHeadDim : nullptr;
+  kvattn::bind_decode_workspace(a, plan, workspace);
   a.dev_status = dev_status;
   a.grid = plan.grid;
   return kvattn::launch_decode(a, tk, tv, (cudaStream_t)stream) == cudaSuccess ? KVATTN_OK : KVATTN_ERR_CUDA;

@@ -43,6 +43,7 @@ struct DecodeArgs {
   const int32_t* start_pos;
   float* ws_o;   // [B*Tq, max_splits, H, d]   unnormalised partial outputs
   float* ws_ml;  // [B*Tq, max_splits, H, 2]   (running max in log2 units, sum)
+  int* counter;  // work counter (split path), reset by the launch; null: round-robin
   int32_t* dev_status;
   int grid;      // persistent CTAs
 };
@@ -57,6 +58,9 @@ struct DecodePlan {
 
 // Split size, persistent grid and workspace for these shapes on this device.
 DecodePlan plan_decode(int B, int Tq, int H, int Hkv, int kv_len_hint, int sm_count);
+
+// Points ws_o / ws_ml / counter of `a` into a workspace of plan.ws_bytes.
+void bind_decode_workspace(DecodeArgs& a, const DecodePlan& plan, void* workspace);
 
 cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tmap_k, const CUtensorMap& tmap_v,
                           cudaStream_t stream);
