@@ -15,17 +15,22 @@
 // head, sequence) and walks the key rows in 128-row tiles up to the last key
 // its last token sees.  Per KV tile j:
 //   S_j = Q K_j^T        tcgen05.mma M=128 N=128 K=16 x8, bf16 -> fp32 in TMEM
-//   P_j = softmax part   4 warps, one query row per thread, read S from TMEM,
-//                        mask, exponentiate (log2 units), write bf16 P into a
-//                        128B-swizzled shared tile
-//   O  += P_j V_j        tcgen05.mma with V as an MN-major operand, fp32 in TMEM
-// S is double buffered in TMEM so that S_{j+1} = Q K_{j+1}^T runs on the
-// tensor cores while the softmax warps work on S_j; O stays in TMEM.  The
+//   P_j = softmax part   8 warps, each row split over two threads, read S
+//                        from TMEM, mask, exponentiate (log2 units), write
+//                        bf16 P back into TMEM
+//   O  += P_j V_j        tcgen05.mma with P read from TMEM and V from shared
+//                        memory as an MN-major operand, fp32 in TMEM
+// S and P are double buffered in TMEM so that S_{j+1} = Q K_{j+1}^T runs on
+// the tensor cores while the softmax warps work on S_j; O stays in TMEM.  P
+// never touches shared memory, which leaves shared-memory bandwidth to the
+// TMA writes and the Q, K, V operand reads.  The
 // reference max of a row only moves when a tile's max exceeds it by more than
 // 8 (probabilities stay <= 2^8), so O is rescaled rarely.
 //
 // Warps: 0 = TMA producer, 1 = TMEM owner and MMA issuer (one thread),
-// 2..5 = softmax and epilogue (warp w reads TMEM lanes 32*(w%4)..+31).
+// 2..9 = softmax and epilogue: warp w reads TMEM lanes 32*(w%4)..+31 and
+// takes column half (w-2)/4 of every S and O row; the two warps that share
+// rows exchange their partial row maxima through shared memory.
 #include "kvattn_device.cuh"
 #include "kvattn_internal.h"
 
@@ -37,22 +42,25 @@ namespace {
 constexpr int kBM = 128;            // query rows per tile
 constexpr int kBN = 128;            // key rows per tile
 constexpr int kHalf = 128 * 64 * 2; // one 128-row x 64-element bf16 half tile (16 KB)
-constexpr int kPrefillThreads = 192;
-constexpr uint32_t kTmemCols = 512; // S0 [0,128), S1 [128,256), O [256,384)
+constexpr int kPrefillThreads = 320;  // 10 warps
+constexpr int kSoftmaxWarps = 8;
+constexpr uint32_t kTmemCols = 512; // S0 [0,128), S1 [128,256), O [256,384), P0 [384,448), P1 [448,512)
 constexpr uint32_t kColO = 256;
+constexpr uint32_t kColP = 384;     // bf16 P, two per 32-bit column: 64 columns per buffer
 
 // shared memory layout (offsets from a 1024-byte aligned base)
 constexpr uint32_t kOffQ = 0;                       // 2 halves
 constexpr uint32_t kOffK = kOffQ + 2 * kHalf;       // [stage 2][half 2]
 constexpr uint32_t kOffV = kOffK + 4 * kHalf;       // [stage 2][half 2]
-constexpr uint32_t kOffP = kOffV + 4 * kHalf;       // 2 halves
-constexpr uint32_t kOffBar = kOffP + 2 * kHalf;
+constexpr uint32_t kOffBar = kOffV + 4 * kHalf;
 // barrier slots (8 bytes each)
 constexpr uint32_t kBarQFull = 0, kBarKFull = 1, kBarKEmpty = 3, kBarVFull = 5, kBarVEmpty = 7, kBarSFull = 9,
                    kBarSEmpty = 11, kBarPFull = 13, kBarPVDone = 14, kBarMmaDone = 15, kNumBars = 16;
 constexpr uint32_t kOffTmemSlot = kOffBar + 8 * kNumBars;
 constexpr uint32_t kOffAbort = kOffTmemSlot + 8;
-constexpr uint32_t kPrefillSmemBytes = kOffAbort + 8 + 1024;  // + alignment slack
+constexpr uint32_t kOffXmax = kOffAbort + 8;        // [2 column halves][128 rows] fp32
+constexpr uint32_t kOffXsum = kOffXmax + 2 * 128 * 4;
+constexpr uint32_t kPrefillSmemBytes = kOffXsum + 2 * 128 * 4 + 1024;  // + alignment slack
 
 // ------------------------------------------------------------ raw smem helpers
 __device__ __forceinline__ void bar_init(uint32_t a, uint32_t count) {
@@ -135,6 +143,15 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// A operand from tensor memory (rows in lanes, two bf16 per column).
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
@@ -181,7 +198,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   constexpr int TT = kBM / G;  // tokens per M tile
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
-  const uint32_t sQ = base + kOffQ, sK = base + kOffK, sV = base + kOffV, sP = base + kOffP;
+  const uint32_t sQ = base + kOffQ, sK = base + kOffK, sV = base + kOffV;
   auto bar = [&](uint32_t slot) { return base + kOffBar + 8u * slot; };
   const uint32_t abort_addr = base + kOffAbort;
 
@@ -215,9 +232,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       bar_init(bar(kBarVFull + s), 1);
       bar_init(bar(kBarVEmpty + s), 1);
       bar_init(bar(kBarSFull + s), 1);
-      bar_init(bar(kBarSEmpty + s), 4);
+      bar_init(bar(kBarSEmpty + s), kSoftmaxWarps);
     }
-    bar_init(bar(kBarPFull), 4);
+    bar_init(bar(kBarPFull), kSoftmaxWarps);
     bar_init(bar(kBarPVDone), 1);
     bar_init(bar(kBarMmaDone), 1);
     st_shared_i32(abort_addr, 0);
@@ -287,11 +304,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t da = sw128_desc(sP + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024);
+          // P_j from TMEM: keys 16kk..16kk+15 are columns 8kk..8kk+7 of its buffer
+          const uint32_t pa = tmem + kColP + 64u * (uint32_t)s + 8u * kk;
           // V tile as B = [keys x dims], dims contiguous: 64-dim atoms one half
           // apart (LBO), 8-key groups 1 KB apart (SBO); 16 keys per step
           const uint64_t db = sw128_desc(sV + (2 * s) * kHalf + kk * 2048, kHalf, 1024);
-          tc_mma(tmem + kColO, da, db, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_ts(tmem + kColO, pa, db, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
         tc_commit(bar(kBarVEmpty + s));
         tc_commit(bar(kBarPVDone));
@@ -303,62 +321,75 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   } else {
     // ================================================================ softmax / epilogue
     const int quarter = warp & 3;         // TMEM lanes 32*quarter .. +31
+    const int ch = (warp - 2) >> 2;       // column half: S/O columns 64*ch .. +63
     const int m = 32 * quarter + lane;    // query row of this thread
     const int tok = t0 + m / G;
     const int head = kvh * G + (m % G);
     const int lim = sp + min(tok, a.T - 1);  // last visible key (rows past T borrow the last token's)
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * quarter) << 16);
-    const int st = tid - 64;              // 0..127 among the softmax threads
+    const int st = tid - 64;              // 0..255 among the softmax threads
+    const uint32_t xmax_mine = base + kOffXmax + (uint32_t)(ch * 128 + m) * 4;
+    const uint32_t xmax_other = base + kOffXmax + (uint32_t)((1 - ch) * 128 + m) * 4;
+    const int pair_bar = 1 + quarter;     // named barrier of the two warps sharing these rows
     float m_ref = -INFINITY;
-    float l = 0.f;
+    float l = 0.f;                        // sum over this thread's column half
 
     for (int j = 0; j < n_kv; ++j) {
       const int s = j & 1;
       bar_wait(bar(kBarSFull + s), (j >> 1) & 1, abort_addr, a.dev_status);
       tc_fence_after();
-      float sv[128];
+      // this thread's 64 columns of the S row: two 32-column loads, one wait
+      uint32_t sr[2][32];
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        uint32_t r[32];
-        tmem_ld32(lane_addr + (uint32_t)s * 128u + 32u * c4, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 32; ++c) sv[32 * c4 + c] = __uint_as_float(r[c]);
-      }
+      for (int c2 = 0; c2 < 2; ++c2) tmem_ld32(lane_addr + (uint32_t)s * 128u + 64u * ch + 32u * c2, sr[c2]);
+      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) bar_arrive(bar(kBarSEmpty + s));
 
-      const int kbase = j * kBN;
-      float mx = -INFINITY;
-      if (kbase + kBN - 1 > lim) {
+      // mask (raw scores; the scale is folded into the exponent below) and
+      // partial row max over eight independent accumulators
+      const int kbase = j * kBN + 64 * ch;
+      if (kbase + 63 > lim) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const float x = (kbase + c <= lim) ? sv[c] * a.scale_log2 : -INFINITY;
-          sv[c] = x;
-          mx = fmaxf(mx, x);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const float x = sv[c] * a.scale_log2;
-          sv[c] = x;
-          mx = fmaxf(mx, x);
-        }
+        for (int c = 0; c < 64; ++c)
+          if (kbase + c > lim) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
       }
+      float mx8[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mx8[k] = __uint_as_float(sr[0][k]);
+#pragma unroll
+      for (int c = 8; c < 64; c += 8)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], __uint_as_float(sr[c >> 5][(c & 31) + k]));
+      const float mx_half = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                  fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      // combine with the other column half: both threads of a row take the
+      // same decisions from the same numbers
+      asm volatile("st.shared.f32 [%0], %1;" ::"r"(xmax_mine), "f"(mx_half) : "memory");
+      named_bar_sync(pair_bar, 64);
+      float mx_other;
+      asm volatile("ld.shared.f32 %0, [%1];" : "=f"(mx_other) : "r"(xmax_other) : "memory");
+      named_bar_sync(pair_bar, 64);  // both read before either writes the next tile's value
+      const float mx = fmaxf(mx_half, mx_other) * a.scale_log2;
       const bool move = mx > m_ref + 8.f;
       const float m_new = move ? mx : m_ref;
       const float alpha = move ? fast_exp2(m_ref - m_new) : 1.f;
       m_ref = m_new;
-      uint32_t pk[64];
-      float sum = 0.f;
+      // p = 2^(s * scale_log2 - m): one FFMA and one ex2 per score
+      const float neg_m = (m_new == -INFINITY) ? 0.f : -m_new;
+      uint32_t pk[32];
+      float sum8[8];
 #pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        const float p0 = (m_new == -INFINITY) ? 0.f : fast_exp2(sv[c] - m_new);
-        const float p1 = (m_new == -INFINITY) ? 0.f : fast_exp2(sv[c + 1] - m_new);
-        sum += p0 + p1;
+      for (int k = 0; k < 8; ++k) sum8[k] = 0.f;
+#pragma unroll
+      for (int c = 0; c < 64; c += 2) {
+        const float p0 = fast_exp2(fmaf(__uint_as_float(sr[c >> 5][c & 31]), a.scale_log2, neg_m));
+        const float p1 = fast_exp2(fmaf(__uint_as_float(sr[(c + 1) >> 5][(c + 1) & 31]), a.scale_log2, neg_m));
+        sum8[(c >> 1) & 7] += p0 + p1;
         pk[c >> 1] = pack_bf16x2_rn(p0, p1);
       }
+      const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
       l = l * alpha + sum;
 
       if (j > 0) {
@@ -367,54 +398,55 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         tc_fence_after();
         if (__any_sync(0xffffffffu, move)) {
 #pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {
+          for (int c2 = 0; c2 < 2; ++c2) {
             uint32_t r[32];
-            tmem_ld32(lane_addr + kColO + 32u * c4, r);
+            tmem_ld32(lane_addr + kColO + 64u * ch + 32u * c2, r);
             tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
-            tmem_st32(lane_addr + kColO + 32u * c4, r);
+            tmem_st32(lane_addr + kColO + 64u * ch + 32u * c2, r);
           }
           tmem_wait_st();
         }
       }
-      if (j == n_kv - 1 && Lmax < kbase + kBN) {
+      if (j == n_kv - 1 && Lmax < j * kBN + kBN) {
         // rows of the last V tile past the last visible key may hold any bits;
         // zero them so that 0 * (garbage) cannot reach O
         bar_wait(bar(kBarVFull + s), (j >> 1) & 1, abort_addr, a.dev_status);
-        const int first_bad = Lmax - kbase;
+        const int first_bad = Lmax - j * kBN;
         const int nchunks = (kBN - first_bad) * 16;  // 16-byte chunks over both halves
-        for (int c = st; c < nchunks; c += 128) {
+        for (int c = st; c < nchunks; c += kSoftmaxWarps * 32) {
           const int r = first_bad + (c >> 4);
           const int half = (c >> 3) & 1;
           const int cc = c & 7;
           st_shared_v4(sV + (2 * s + half) * kHalf + r * 128 + cc * 16, 0u, 0u, 0u, 0u);
         }
       }
-      // P row m into the 128B-swizzled K-major tile: chunk cc of half h of row m
-      // lives at h*16KB + m*128 + ((cc ^ (m & 7)) * 16)
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const int half = c >> 3, cc = c & 7;
-        st_shared_v4(sP + half * kHalf + m * 128 + ((cc ^ (m & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
-                     pk[4 * c + 3]);
-      }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      // P row m, keys 64*ch .. +63: columns 32*ch .. +31 of P buffer j%2
+      tmem_st32(lane_addr + kColP + 64u * (uint32_t)s + 32u * ch, pk);
+      tmem_wait_st();
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the zeroed V rows, if any
       tc_fence_before();
       __syncwarp();
       if (lane == 0) bar_arrive(bar(kBarPFull));
     }
 
-    // ---- epilogue: O / l -> bf16 rows
+    // ---- epilogue: O / l -> bf16 rows (this thread's 64 columns)
+    const uint32_t xsum_mine = base + kOffXsum + (uint32_t)(ch * 128 + m) * 4;
+    const uint32_t xsum_other = base + kOffXsum + (uint32_t)((1 - ch) * 128 + m) * 4;
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(xsum_mine), "f"(l) : "memory");
+    named_bar_sync(pair_bar, 64);
+    float l_other;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(l_other) : "r"(xsum_other) : "memory");
     bar_wait(bar(kBarPVDone), (n_kv - 1) & 1, abort_addr, a.dev_status);
     tc_fence_after();
-    const float inv_l = 1.f / l;
+    const float inv_l = 1.f / (l + l_other);
     const bool store = tok < a.T;
-    uint16_t* dst = a.out + (((size_t)b * a.T + (store ? tok : 0)) * a.H + head) * kHeadDim;
+    uint16_t* dst = a.out + (((size_t)b * a.T + (store ? tok : 0)) * a.H + head) * kHeadDim + 64 * ch;
 #pragma unroll
-    for (int c4 = 0; c4 < 4; ++c4) {
+    for (int c2 = 0; c2 < 2; ++c2) {
       uint32_t r[32];
-      tmem_ld32(lane_addr + kColO + 32u * c4, r);
+      tmem_ld32(lane_addr + kColO + 64u * ch + 32u * c2, r);
       tmem_wait_ld();
       if (store) {
 #pragma unroll
@@ -424,7 +456,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           w.y = pack_bf16x2_rn(__uint_as_float(r[c + 2]) * inv_l, __uint_as_float(r[c + 3]) * inv_l);
           w.z = pack_bf16x2_rn(__uint_as_float(r[c + 4]) * inv_l, __uint_as_float(r[c + 5]) * inv_l);
           w.w = pack_bf16x2_rn(__uint_as_float(r[c + 6]) * inv_l, __uint_as_float(r[c + 7]) * inv_l);
-          *reinterpret_cast<uint4*>(dst + 32 * c4 + c) = w;
+          *reinterpret_cast<uint4*>(dst + 32 * c2 + c) = w;
         }
       }
     }
