@@ -54,14 +54,21 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
-def kernel_source_hash():
+KERNEL_SOURCES = {
+    "decode_splitk": ("decode.cu", "kvattn_device.cuh"),
+    "prefill_chunk": ("prefill.cu", "kvattn_device.cuh"),
+}
+
+
+def kernel_source_hash(kernel_tag: str):
+    """Hash of the source files a kernel is built from (its .cu and the
+    shared device header), to tell whether a recorded profile still applies."""
     h = hashlib.sha256()
     pkg = os.path.join(ROOT, "gqa_decode_attention_kvattn_b200", "csrc")
-    for p in sorted(glob.glob(os.path.join(pkg, "*"))):
-        if p.endswith((".cu", ".cuh", ".h")):
-            with open(p, "rb") as f:
-                h.update(os.path.basename(p).encode())
-                h.update(f.read())
+    for name in KERNEL_SOURCES[kernel_tag]:
+        with open(os.path.join(pkg, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
@@ -79,7 +86,7 @@ def profiled_traffic(kernel_tag: str, workload: str):
                 k, _, v = line.partition(":")
                 vals[k.strip().strip("-* `")] = v.strip().strip("` ")
     try:
-        if vals.get("source_hash") != kernel_source_hash():
+        if vals.get("source_hash") != kernel_source_hash(kernel_tag):
             return None
         return float(vals["traffic_bytes_per_launch"])
     except Exception:
