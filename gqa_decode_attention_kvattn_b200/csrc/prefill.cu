@@ -54,8 +54,10 @@ constexpr uint32_t kOffK = kOffQ + 2 * kHalf;       // [stage 2][half 2]
 constexpr uint32_t kOffV = kOffK + 4 * kHalf;       // [stage 2][half 2]
 constexpr uint32_t kOffBar = kOffV + 4 * kHalf;
 // barrier slots (8 bytes each)
+// (every pipeline barrier exists once per buffer, so a waiter is never more
+// than one phase behind the barrier it waits on)
 constexpr uint32_t kBarQFull = 0, kBarKFull = 1, kBarKEmpty = 3, kBarVFull = 5, kBarVEmpty = 7, kBarSFull = 9,
-                   kBarSEmpty = 11, kBarPFull = 13, kBarPVDone = 14, kBarMmaDone = 15, kNumBars = 16;
+                   kBarSEmpty = 11, kBarPFull = 13, kBarPVDone = 15, kBarMmaDone = 17, kNumBars = 18;
 constexpr uint32_t kOffTmemSlot = kOffBar + 8 * kNumBars;
 constexpr uint32_t kOffAbort = kOffTmemSlot + 8;
 constexpr uint32_t kOffXmax = kOffAbort + 8;        // [2 column halves][128 rows] fp32
@@ -72,13 +74,30 @@ __device__ __forceinline__ void bar_arrive(uint32_t a) {
 __device__ __forceinline__ void bar_expect_tx(uint32_t a, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(a), "r"(bytes) : "memory");
 }
-__device__ __forceinline__ bool bar_try_wait(uint32_t a, uint32_t parity) {
+#ifndef KVATTN_PREFILL_SPIN_MMA
+#define KVATTN_PREFILL_SPIN_MMA 0
+#endif
+#ifndef KVATTN_PREFILL_SPIN_ALL
+#define KVATTN_PREFILL_SPIN_ALL 1
+#endif
+// One try of a phase wait.  With `suspend` the thread sleeps in hardware
+// until the phase completes (or ~1 ms passes); without it the call returns at
+// once and the caller spins, which wakes sooner but costs issue slots.
+__device__ __forceinline__ bool bar_try_wait(uint32_t a, uint32_t parity, bool suspend) {
   uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(a), "r"(parity), "r"(1u << 20)
-      : "memory");
+  if (suspend) {
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(a), "r"(parity), "r"(1u << 20)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(a), "r"(parity)
+        : "memory");
+  }
   return ok != 0;
 }
 __device__ __forceinline__ int ld_shared_i32(uint32_t a) {
@@ -91,12 +110,13 @@ __device__ __forceinline__ void st_shared_i32(uint32_t a, int v) {
 }
 // Bounded wait (see kWaitLimitNs); gives up at once when the CTA's abort flag
 // is set, and sets it (plus the status bit) when it gives up itself.
-__device__ __forceinline__ bool bar_wait(uint32_t a, uint32_t parity, uint32_t abort_addr, int32_t* dev_status) {
+__device__ __forceinline__ bool bar_wait(uint32_t a, uint32_t parity, uint32_t abort_addr, int32_t* dev_status,
+                                         bool suspend = !KVATTN_PREFILL_SPIN_ALL) {
   if (ld_shared_i32(abort_addr)) return false;
-  if (bar_try_wait(a, parity)) return true;
+  if (bar_try_wait(a, parity, suspend)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (;;) {
-    if (bar_try_wait(a, parity)) return true;
+    if (bar_try_wait(a, parity, suspend)) return true;
     if (ld_shared_i32(abort_addr)) return false;
     if (globaltimer_ns() - t0 > kWaitLimitNs) {
       st_shared_i32(abort_addr, 1);
@@ -233,9 +253,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       bar_init(bar(kBarVEmpty + s), 1);
       bar_init(bar(kBarSFull + s), 1);
       bar_init(bar(kBarSEmpty + s), kSoftmaxWarps);
+      bar_init(bar(kBarPFull + s), kSoftmaxWarps);
+      bar_init(bar(kBarPVDone + s), 1);
     }
-    bar_init(bar(kBarPFull), kSoftmaxWarps);
-    bar_init(bar(kBarPVDone), 1);
     bar_init(bar(kBarMmaDone), 1);
     st_shared_i32(abort_addr, 0);
     fence_barrier_init();
@@ -278,12 +298,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_m128_n128(false);
       constexpr uint32_t idesc_pv = idesc_bf16_m128_n128(true);
+      constexpr bool kMmaSuspend = !(KVATTN_PREFILL_SPIN_MMA || KVATTN_PREFILL_SPIN_ALL);
       bool ok = bar_wait(bar(kBarQFull), 0, abort_addr, a.dev_status);
       tc_fence_after();
       auto issue_qk = [&](int j) {
         const int s = j & 1;
-        if (!bar_wait(bar(kBarKFull + s), (j >> 1) & 1, abort_addr, a.dev_status)) return false;
-        if (!bar_wait(bar(kBarSEmpty + s), ((j >> 1) & 1) ^ 1, abort_addr, a.dev_status)) return false;
+        if (!bar_wait(bar(kBarKFull + s), (j >> 1) & 1, abort_addr, a.dev_status, kMmaSuspend)) return false;
+        if (!bar_wait(bar(kBarSEmpty + s), ((j >> 1) & 1) ^ 1, abort_addr, a.dev_status, kMmaSuspend)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -299,8 +320,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       for (int j = 0; j < n_kv && ok; ++j) {
         if (j + 1 < n_kv && !issue_qk(j + 1)) break;
         const int s = j & 1;
-        if (!bar_wait(bar(kBarPFull), j & 1, abort_addr, a.dev_status)) break;
-        if (!bar_wait(bar(kBarVFull + s), (j >> 1) & 1, abort_addr, a.dev_status)) break;
+        if (!bar_wait(bar(kBarPFull + s), (j >> 1) & 1, abort_addr, a.dev_status, kMmaSuspend)) break;
+        if (!bar_wait(bar(kBarVFull + s), (j >> 1) & 1, abort_addr, a.dev_status, kMmaSuspend)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -312,7 +333,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           tc_mma_ts(tmem + kColO, pa, db, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
         tc_commit(bar(kBarVEmpty + s));
-        tc_commit(bar(kBarPVDone));
+        tc_commit(bar(kBarPVDone + s));
       }
       tc_commit(bar(kBarMmaDone));
       // every MMA issued above has finished once this completes
@@ -376,27 +397,33 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       const float m_new = move ? mx : m_ref;
       const float alpha = move ? fast_exp2(m_ref - m_new) : 1.f;
       m_ref = m_new;
-      // p = 2^(s * scale_log2 - m): one FFMA and one ex2 per score
+      // p = 2^(s * scale_log2 - m): packed FMA for two scores, one ex2 each,
+      // packed sums in four accumulators
       const float neg_m = (m_new == -INFINITY) ? 0.f : -m_new;
+      const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2);
+      const uint64_t nm2 = f2_pack(neg_m, neg_m);
       uint32_t pk[32];
-      float sum8[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) sum8[k] = 0.f;
+      uint64_t sum2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
       for (int c = 0; c < 64; c += 2) {
-        const float p0 = fast_exp2(fmaf(__uint_as_float(sr[c >> 5][c & 31]), a.scale_log2, neg_m));
-        const float p1 = fast_exp2(fmaf(__uint_as_float(sr[(c + 1) >> 5][(c + 1) & 31]), a.scale_log2, neg_m));
-        sum8[(c >> 1) & 7] += p0 + p1;
+        const uint64_t sv = ((uint64_t)sr[c >> 5][(c & 31) + 1] << 32) | sr[c >> 5][c & 31];
+        float x0, x1;
+        f2_unpack(f2_fma(sv, sc2, nm2), x0, x1);
+        const float p0 = fast_exp2(x0);
+        const float p1 = fast_exp2(x1);
+        sum2[(c >> 1) & 3] = f2_add(sum2[(c >> 1) & 3], f2_pack(p0, p1));
         pk[c >> 1] = pack_bf16x2_rn(p0, p1);
       }
-      const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+      float sa, sb;
+      f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), sa, sb);
+      const float sum = sa + sb;
       l = l * alpha + sum;
 
-      if (j > 0) {
-        // PV_{j-1} done: the P buffer is free and O is stable
-        bar_wait(bar(kBarPVDone), (j - 1) & 1, abort_addr, a.dev_status);
+      if (j > 0 && __any_sync(0xffffffffu, move)) {
+        // a row's reference moved: rescale its O once PV_{j-1} has finished
+        bar_wait(bar(kBarPVDone + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort_addr, a.dev_status);
         tc_fence_after();
-        if (__any_sync(0xffffffffu, move)) {
+        {
 #pragma unroll
           for (int c2 = 0; c2 < 2; ++c2) {
             uint32_t r[32];
@@ -408,6 +435,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           }
           tmem_wait_st();
         }
+      }
+      if (j >= 2) {
+        // P buffer j%2 is free once PV_{j-2} has read it
+        bar_wait(bar(kBarPVDone + s), ((j >> 1) - 1) & 1, abort_addr, a.dev_status);
+        tc_fence_after();
       }
       if (j == n_kv - 1 && Lmax < j * kBN + kBN) {
         // rows of the last V tile past the last visible key may hold any bits;
@@ -428,7 +460,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the zeroed V rows, if any
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) bar_arrive(bar(kBarPFull));
+      if (lane == 0) bar_arrive(bar(kBarPFull + s));
     }
 
     // ---- epilogue: O / l -> bf16 rows (this thread's 64 columns)
@@ -438,7 +470,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     named_bar_sync(pair_bar, 64);
     float l_other;
     asm volatile("ld.shared.f32 %0, [%1];" : "=f"(l_other) : "r"(xsum_other) : "memory");
-    bar_wait(bar(kBarPVDone), (n_kv - 1) & 1, abort_addr, a.dev_status);
+    bar_wait(bar(kBarPVDone + ((n_kv - 1) & 1)), ((n_kv - 1) >> 1) & 1, abort_addr, a.dev_status);
     tc_fence_after();
     const float inv_l = 1.f / (l + l_other);
     const bool store = tok < a.T;
