@@ -27,6 +27,7 @@ KVATTN_ERR_CUDA = 5
 KVATTN_DEV_START_POS_RANGE = 0x1
 KVATTN_DEV_KV_LEN_HINT = 0x2
 KVATTN_DEV_WAIT_TIMEOUT = 0x4
+KVATTN_DEV_INTERNAL = 0x8
 
 HEAD_DIM = 128
 

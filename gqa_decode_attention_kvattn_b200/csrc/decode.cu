@@ -62,7 +62,7 @@ constexpr int kRedRegion = 336;
 
 template <int G>
 struct Shape {
-  static constexpr int RB = (G >= 8) ? 2 : 4;     // rows per half-warp batch
+  static constexpr int RB = (G >= 16) ? 1 : (G >= 8) ? 2 : 4;  // rows per half-warp batch
   static constexpr int NV = G * RB;                // partial dot products per lane
   static constexpr int LOG2NV = ilog2(NV);
   static constexpr int REP = NV >= 16 ? 1 : 16 / NV;  // lanes that end up with the same score
@@ -622,6 +622,381 @@ __global__ void __launch_bounds__(kHeadDim) decode_merge_kernel(const DecodeArgs
   a.out[(((size_t)b * a.Tq + t) * a.H + head) * kHeadDim + c] = (uint16_t)f32_to_bf16_bits(num / den);
 }
 
+// ======================================================================
+// Tensor-core decode for G >= 8 (legacy warp-level mma.sync, m16n8k16).
+//
+// At G = 8 the decode does 16 flop per cache byte, above what the fp32 FMA
+// units can sustain at HBM speed (about 74 TFLOP/s / 6.5 TB/s = 11 flop/B),
+// so the contraction goes to the tensor cores: the G query heads are the M
+// dimension (padded to 16), 16 cache rows per warp are K (for P.V) or N (for
+// q.K^T).  Per warp and 16 rows: S = q K^T as 2 n-tiles x 8 k-steps, then
+// O += P V as 16 n-tiles of 8 dims, P taken straight from the S accumulator
+// registers (their layout is the A-fragment layout).  Each lane's S values and
+// O values belong to the same head (lane/4, and lane/4+8 when G = 16), so the
+// online softmax rescales O without any exchange between lanes.  K and V
+// arrive by TMA as 128B-swizzled 64-element halves, read with ldmatrix.
+constexpr int kMmaTileRows = 64;
+constexpr int kMmaStages = 2;
+constexpr uint32_t kMmaHalfBytes = kMmaTileRows * 64 * 2;  // 8 KB
+
+template <int G>
+struct __align__(1024) SmemMma {
+  uint16_t k[kMmaStages][2][kMmaTileRows * 64];  // [stage][d half][row*64 + swizzled elem]
+  uint16_t v[kMmaStages][2][kMmaTileRows * 64];
+  uint16_t q[kMmaStages][G][kHeadDim];
+  float merge_o[kConsumerWarps][G][kHeadDim];
+  float merge_m[kConsumerWarps][G];
+  float merge_l[kConsumerWarps][G];
+  int set_len[kMaxRowSets];
+  int full_start[kMaxRowSets + 1];
+  int sorted_set[kMaxRowSets];
+  int bucket[kMaxBuckets + 1];
+  int n_full, total_items;
+  int stage_item[kMmaStages];
+  int abort;
+  uint64_t full[kMmaStages];
+  uint64_t empty[kMmaStages];
+  uint64_t cons;
+};
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+// byte offset of the 16-byte chunk holding elements 8*chunk.. of `row` in a
+// 128B-swizzled [rows][64] half tile
+__device__ __forceinline__ uint32_t sw128_off(int row, int chunk) {
+  return (uint32_t)(row * 128 + (((chunk ^ row) & 7) << 4));
+}
+
+template <int G>
+__global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(
+    const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+    const DecodeArgs a, const int evict_first) {
+  static_assert(G == 8 || G == 16, "tensor-core decode handles G = 8 or 16");
+  constexpr uint32_t kQBytes = G * kHeadDim * 2;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  SmemMma<G>& sm = *reinterpret_cast<SmemMma<G>*>(smem_raw);
+  // the 128B-swizzled tiles need a 1024-byte aligned base; refuse otherwise
+  if ((smem_u32(smem_raw) & 1023u) != 0) {
+    if (threadIdx.x == 0) set_status(a.dev_status, KVATTN_DEV_INTERNAL);
+    return;
+  }
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int n_sets = a.B * a.Tq;
+
+  if (warp == 0) {
+    if (a.max_splits == 1) {
+      if (lane == 0) sm.total_items = n_sets * a.Hkv;
+    } else {
+      build_work_table(a, sm, n_sets, lane);
+    }
+    if (blockIdx.x == 0) {
+      for (int v = lane; v < n_sets; v += 32) {
+        if (set_length(a, v) == 0) {
+          const int sp = a.start_pos[v / a.Tq];
+          set_status(a.dev_status, (sp < 0 || (long long)sp + a.Tq > a.S) ? KVATTN_DEV_START_POS_RANGE
+                                                                         : KVATTN_DEV_KV_LEN_HINT);
+        }
+      }
+    }
+  }
+  if (tid == 32) {
+    sm.abort = 0;
+    for (int s = 0; s < kMmaStages; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], kConsumerWarps);
+    }
+    mbar_init(&sm.cons, kConsumerWarps);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const int total_items = sm.total_items;
+
+  if (warp == kConsumerWarps) {
+    // ================================================================ producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmap_k);
+      prefetch_tensormap(&tmap_v);
+      uint64_t policy = 0;
+      if (evict_first) policy = l2_policy_evict_first();
+      else asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(policy));
+      int stage = 0;
+      uint32_t phase = 0;
+      int next_static = blockIdx.x;
+      for (;;) {
+        int i;
+        if (a.counter) i = atomicAdd(a.counter, 1);
+        else { i = next_static; next_static += gridDim.x; }
+        const bool done = i >= total_items || sm.abort;
+        Item it;
+        if (!done) {
+          it = decode_item(a, sm, n_sets, i);
+          if (it.nsplit == 0) continue;
+        }
+        if (done) {
+          if (mbar_wait(&sm.empty[stage], phase ^ 1, &sm.abort)) {
+            sm.stage_item[stage] = -1;
+            mbar_arrive(&sm.full[stage]);
+          } else {
+            abort_pipeline(&sm.abort, a.dev_status);
+          }
+          if (++stage == kMmaStages) { stage = 0; phase ^= 1; }
+          break;
+        }
+        for (int row = it.r0; row < it.r1; row += kMmaTileRows) {
+          if (!mbar_wait(&sm.empty[stage], phase ^ 1, &sm.abort)) {
+            abort_pipeline(&sm.abort, a.dev_status);
+            break;
+          }
+          const bool first = row == it.r0;
+          sm.stage_item[stage] = i;
+          mbar_arrive_expect_tx(&sm.full[stage], 4 * kMmaHalfBytes + (first ? kQBytes : 0u));
+          if (first) {
+            const uint16_t* qsrc = a.q_rot + (((size_t)it.b * a.Tq + it.t) * a.H + (size_t)it.kvh * G) * kHeadDim;
+            bulk_load(&sm.q[stage][0][0], qsrc, kQBytes, &sm.full[stage]);
+          }
+          tma_load_4d(&sm.k[stage][0][0], &tmap_k, &sm.full[stage], 0, it.kvh, row, it.b, policy);
+          tma_load_4d(&sm.k[stage][1][0], &tmap_k, &sm.full[stage], 64, it.kvh, row, it.b, policy);
+          tma_load_4d(&sm.v[stage][0][0], &tmap_v, &sm.full[stage], 0, it.kvh, row, it.b, policy);
+          tma_load_4d(&sm.v[stage][1][0], &tmap_v, &sm.full[stage], 64, it.kvh, row, it.b, policy);
+          if (++stage == kMmaStages) { stage = 0; phase ^= 1; }
+        }
+      }
+      for (int s = 0; s < kMmaStages; ++s) {
+        if (!mbar_wait(&sm.empty[stage], phase ^ 1, nullptr)) {
+          abort_pipeline(&sm.abort, a.dev_status);
+          break;
+        }
+        if (++stage == kMmaStages) { stage = 0; phase ^= 1; }
+      }
+    }
+    return;
+  }
+
+  // ================================================================== consumers
+  const int g = lane >> 2;   // head of this lane's accumulator rows (and g + 8)
+  const int c4 = lane & 3;   // column pair within an 8-wide fragment
+  const int wrow = 16 * warp;  // this warp's 16 rows of each 64-row tile
+  int stage = 0;
+  uint32_t phase = 0;
+  uint32_t cons_phase = 0;
+  auto cons_sync = [&]() {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.cons);
+    mbar_wait(&sm.cons, cons_phase, &sm.abort);
+    cons_phase ^= 1;
+    __syncwarp();
+  };
+
+  for (;;) {
+    if (!mbar_wait(&sm.full[stage], phase, &sm.abort)) abort_pipeline(&sm.abort, a.dev_status);
+    const int i = sm.stage_item[stage];
+    if (i < 0 || sm.abort) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.empty[stage]);
+      break;
+    }
+    const Item it = decode_item(a, sm, n_sets, i);
+
+    // q as A fragments (rows = heads g and g+8, columns = head dims)
+    uint32_t qa[8][4];
+    float o[16][4];
+#pragma unroll
+    for (int dt = 0; dt < 16; ++dt)
+#pragma unroll
+      for (int x = 0; x < 4; ++x) o[dt][x] = 0.f;
+    float m_run[2] = {-INFINITY, -INFINITY};  // heads g, g+8 (log2 units)
+    float l_run[2] = {0.f, 0.f};
+
+    for (int row = it.r0; row < it.r1; row += kMmaTileRows) {
+      if (row != it.r0 && !mbar_wait(&sm.full[stage], phase, &sm.abort)) abort_pipeline(&sm.abort, a.dev_status);
+      if (row == it.r0) {
+        const uint32_t* qw = reinterpret_cast<const uint32_t*>(&sm.q[stage][0][0]);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const int col = 8 * kk + c4;  // word index of dims 16kk + 2*c4
+          qa[kk][0] = qw[g * 64 + col];
+          qa[kk][2] = qw[g * 64 + col + 4];
+          if constexpr (G == 16) {
+            qa[kk][1] = qw[(g + 8) * 64 + col];
+            qa[kk][3] = qw[(g + 8) * 64 + col + 4];
+          } else {
+            qa[kk][1] = 0u;
+            qa[kk][3] = 0u;
+          }
+        }
+      }
+      const uint32_t kbase = smem_u32(&sm.k[stage][0][0]);
+      const uint32_t vbase = smem_u32(&sm.v[stage][0][0]);
+      const bool masked = row + kMmaTileRows > it.r1;
+      if (masked) {
+        // rows of this warp past the item may hold any bits; zero their V so
+        // that no 0 * NaN reaches O (the warp reads only its own 16 rows)
+        for (int x = lane; x < 16 * 16; x += 32) {
+          const int r = wrow + (x >> 4);
+          if (row + r >= it.r1) {
+            const int half = (x >> 3) & 1, ch = x & 7;
+            *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(&sm.v[stage][half][0]) + r * 128 + ch * 16) =
+                make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+        __syncwarp();
+      }
+
+      // ---- S = q K^T for the warp's 16 rows: n-tile nt covers rows wrow+8nt..+7
+      float sacc[2][4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+        for (int x = 0; x < 4; ++x) sacc[nt][x] = 0.f;
+        const int r = wrow + 8 * nt + (lane & 7);
+#pragma unroll
+        for (int kp = 0; kp < 4; ++kp) {
+          // matrices: dims chunks 4kp + (lane>>3): k-steps 2kp (chunks 4kp, 4kp+1) and 2kp+1
+          const int chunk = 4 * kp + (lane >> 3);
+          const uint32_t addr = kbase + (uint32_t)(chunk >> 3) * kMmaHalfBytes + sw128_off(r, chunk & 7);
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(addr, b0, b1, b2, b3);
+          mma_bf16_16816(sacc[nt], qa[2 * kp][0], qa[2 * kp][1], qa[2 * kp][2], qa[2 * kp][3], b0, b1);
+          mma_bf16_16816(sacc[nt], qa[2 * kp + 1][0], qa[2 * kp + 1][1], qa[2 * kp + 1][2], qa[2 * kp + 1][3], b2,
+                         b3);
+        }
+      }
+      // ---- online softmax per head (lanes with the same g share a head)
+      // sacc[nt][0..1]: head g, rows wrow+8nt+2c4+{0,1}; [2..3]: head g+8
+      float pv[2][4];
+#pragma unroll
+      for (int hh = 0; hh < (G == 16 ? 2 : 1); ++hh) {
+        float sv[4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int rr = row + wrow + 8 * nt + 2 * c4 + e;
+            const float x = sacc[nt][2 * hh + e] * a.scale_log2;
+            sv[2 * nt + e] = (masked && rr >= it.r1) ? -INFINITY : x;
+          }
+        float tmax = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
+        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
+        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
+        const bool move = tmax > m_run[hh] + 8.f;
+        const float m_new = move ? tmax : m_run[hh];
+        const float alpha = move ? fast_exp2(m_run[hh] - m_new) : 1.f;
+        m_run[hh] = m_new;
+        float ps = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float p = (m_new == -INFINITY) ? 0.f : fast_exp2(sv[e] - m_new);
+          pv[hh][e] = p;
+          ps += p;
+        }
+        l_run[hh] = l_run[hh] * alpha + ps;
+        if (alpha != 1.f) {
+#pragma unroll
+          for (int dt = 0; dt < 16; ++dt) {
+            o[dt][2 * hh] *= alpha;
+            o[dt][2 * hh + 1] *= alpha;
+          }
+        }
+      }
+      // P as the A fragment: a0 = head g rows 2c4..+1, a2 = rows 8+2c4..+1,
+      // a1/a3 the same for head g+8 (zero when G = 8)
+      uint32_t pa0 = pack_bf16x2(pv[0][0], pv[0][1]);
+      uint32_t pa2 = pack_bf16x2(pv[0][2], pv[0][3]);
+      uint32_t pa1 = 0u, pa3 = 0u;
+      if constexpr (G == 16) {
+        pa1 = pack_bf16x2(pv[1][0], pv[1][1]);
+        pa3 = pack_bf16x2(pv[1][2], pv[1][3]);
+      }
+      // ---- O += P V: n-tile dt covers dims 8dt..8dt+7
+#pragma unroll
+      for (int dp = 0; dp < 8; ++dp) {
+        // matrices (rows wrow..+7 | wrow+8..+15) x (dims chunk 2dp | 2dp+1)
+        const int mi = lane >> 3;
+        const int r = wrow + 8 * (mi & 1) + (lane & 7);
+        const int chunk = 2 * dp + (mi >> 1);
+        const uint32_t addr = vbase + (uint32_t)(chunk >> 3) * kMmaHalfBytes + sw128_off(r, chunk & 7);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(addr, b0, b1, b2, b3);
+        mma_bf16_16816(o[2 * dp], pa0, pa1, pa2, pa3, b0, b1);
+        mma_bf16_16816(o[2 * dp + 1], pa0, pa1, pa2, pa3, b2, b3);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.empty[stage]);
+      if (++stage == kMmaStages) { stage = 0; phase ^= 1; }
+    }
+
+    // ---- merge the four warps' states of this item
+#pragma unroll
+    for (int hh = 0; hh < (G == 16 ? 2 : 1); ++hh) {
+      float lsum = l_run[hh];
+      lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
+      lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
+      if (c4 == 0) {
+        sm.merge_m[warp][g + 8 * hh] = m_run[hh];
+        sm.merge_l[warp][g + 8 * hh] = lsum;
+      }
+#pragma unroll
+      for (int dt = 0; dt < 16; ++dt)
+        *reinterpret_cast<float2*>(&sm.merge_o[warp][g + 8 * hh][8 * dt + 2 * c4]) =
+            make_float2(o[dt][2 * hh], o[dt][2 * hh + 1]);
+    }
+    cons_sync();
+    {
+      const int c = tid;  // 0..127: one output element per head
+#pragma unroll 1
+      for (int h = 0; h < G; ++h) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm.merge_m[w][h]);
+        float o_sum = 0.f, Ls = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          const float mw = sm.merge_m[w][h];
+          const float f = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
+          o_sum += f * sm.merge_o[w][h][c];
+          Ls += f * sm.merge_l[w][h];
+        }
+        const int head = it.kvh * G + h;
+        if (it.nsplit == 1) {
+          a.out[(((size_t)it.b * a.Tq + it.t) * a.H + head) * kHeadDim + c] = (uint16_t)f32_to_bf16_bits(o_sum / Ls);
+        } else {
+          const size_t slot = ((size_t)it.v * a.max_splits + it.split) * a.H + head;
+          a.ws_o[slot * kHeadDim + c] = o_sum;
+          if (c == 0) {
+            a.ws_ml[slot * 2 + 0] = M;
+            a.ws_ml[slot * 2 + 1] = Ls;
+          }
+        }
+      }
+    }
+    cons_sync();
+  }
+}
+
+template <int G>
+size_t smem_bytes_mma() {
+  return sizeof(SmemMma<G>);
+}
+
 template <int G>
 size_t smem_bytes() {
   return sizeof(Smem<G>);
@@ -629,15 +1004,19 @@ size_t smem_bytes() {
 
 template <int G>
 cudaError_t launch_g(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st) {
-  const size_t smem = smem_bytes<G>();
+  constexpr bool kMma = G >= 8;
+  auto kernel = [] {
+    if constexpr (kMma) return decode_mma_kernel<G>;
+    else return decode_splitk_kernel<G>;
+  }();
+  const size_t smem = kMma ? smem_bytes_mma<G>() : smem_bytes<G>();
   static bool configured[64] = {false};
   int dev = 0;
   cudaError_t e0 = cudaGetDevice(&dev);
   if (e0 != cudaSuccess) return e0;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(decode_splitk_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
@@ -646,7 +1025,7 @@ cudaError_t launch_g(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorM
     cudaError_t e1 = cudaMemsetAsync(a.counter, 0, sizeof(int), st);
     if (e1 != cudaSuccess) return e1;
   }
-  decode_splitk_kernel<G><<<a.grid, kThreads, smem, st>>>(tk, tv, a, evict_first);
+  kernel<<<a.grid, kThreads, smem, st>>>(tk, tv, a, evict_first);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (a.max_splits > 1) {
@@ -663,28 +1042,32 @@ cudaError_t launch_g(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorM
 // query: registers and shared memory both count).
 template <int G>
 int resident_ctas() {
+  constexpr bool kMma = G >= 8;
+  auto kernel = [] {
+    if constexpr (kMma) return decode_mma_kernel<G>;
+    else return decode_splitk_kernel<G>;
+  }();
+  const size_t smem = kMma ? smem_bytes_mma<G>() : smem_bytes<G>();
   int n = 0;
-  if (cudaFuncSetAttribute(decode_splitk_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem_bytes<G>()) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_splitk_kernel<G>, kThreads, smem_bytes<G>()) !=
-          cudaSuccess ||
-      n < 1)
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kThreads, smem) != cudaSuccess || n < 1)
     n = 1;
   return n;
 }
 
 int resident_ctas_for(int G) {
-  static int cached[64][4] = {};  // [device][log2 G], 0 = not yet queried
+  static int cached[64][5] = {};  // [device][log2 G], 0 = not yet queried
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
-  const int gi = G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : 3;
+  const int gi = G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : G == 8 ? 3 : 4;
   int n = __atomic_load_n(&cached[dev][gi], __ATOMIC_RELAXED);
   if (n == 0) {
     switch (G) {
       case 1: n = resident_ctas<1>(); break;
       case 2: n = resident_ctas<2>(); break;
       case 4: n = resident_ctas<4>(); break;
-      default: n = resident_ctas<8>(); break;
+      case 8: n = resident_ctas<8>(); break;
+      default: n = resident_ctas<16>(); break;
     }
     __atomic_store_n(&cached[dev][gi], n, __ATOMIC_RELAXED);
   }
@@ -739,8 +1122,11 @@ cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tk, const CUte
     case 2: return launch_g<2>(a, tk, tv, st);
     case 4: return launch_g<4>(a, tk, tv, st);
     case 8: return launch_g<8>(a, tk, tv, st);
+    case 16: return launch_g<16>(a, tk, tv, st);
     default: return cudaErrorInvalidValue;
   }
 }
+
+bool decode_uses_tensor_cores(int G) { return G >= 8; }
 
 }  // namespace kvattn

@@ -67,8 +67,9 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 // Same cache view as kvattn_decode uses: (d, head, row, batch), boxes of 32
-// rows of one head of one sequence.
-int cache_map(CUtensorMap* map, const void* base, int B, int S, int Hkv) {
+// rows x 128 elements of one head, or 128B-swizzled boxes of 64 rows x 64
+// elements for the tensor-core decode (G >= 8).
+int cache_map(CUtensorMap* map, const void* base, int B, int S, int Hkv, bool swizzled) {
   static EncodeTiledFn fn = nullptr;
   static std::once_flag once;
   std::call_once(once, [] {
@@ -82,11 +83,11 @@ int cache_map(CUtensorMap* map, const void* base, int B, int S, int Hkv) {
   const cuuint64_t dims[4] = {(cuuint64_t)kHeadDim, (cuuint64_t)Hkv, (cuuint64_t)S, (cuuint64_t)B};
   const cuuint64_t strides[3] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)Hkv * kHeadDim * 2,
                                  (cuuint64_t)S * Hkv * kHeadDim * 2};
-  const cuuint32_t box[4] = {(cuuint32_t)kHeadDim, 1, 32, 1};
+  const cuuint32_t box[4] = {swizzled ? 64u : (cuuint32_t)kHeadDim, 1, swizzled ? 64u : 32u, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzled ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS
              ? KVATTN_OK
              : KVATTN_ERR_CUDA;
 }
@@ -107,7 +108,7 @@ extern "C" KVATTN_API int kvattn_decode_noalloc(const kvattn_dims* dims, const u
     return KVATTN_ERR_INVALID_ARG;
   if (dims->head_dim != kHeadDim) return KVATTN_ERR_UNSUPPORTED;
   const int G = dims->n_heads / dims->n_kv_heads;
-  if (G != 1 && G != 2 && G != 4 && G != 8) return KVATTN_ERR_UNSUPPORTED;
+  if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return KVATTN_ERR_UNSUPPORTED;
   if (!q_rot || !cache_k || !cache_v || !start_pos || !out) return KVATTN_ERR_INVALID_ARG;
   if (!aligned16(q_rot) || !aligned16(cache_k) || !aligned16(cache_v) || !aligned16(out) ||
       (reinterpret_cast<uintptr_t>(start_pos) & 3u))
@@ -129,9 +130,10 @@ extern "C" KVATTN_API int kvattn_decode_noalloc(const kvattn_dims* dims, const u
     if (rc != KVATTN_OK) return rc;
   }
   CUtensorMap tk, tv;
-  rc = cache_map(&tk, cache_k, dims->batch, dims->max_seq_len, dims->n_kv_heads);
+  const bool swizzled = kvattn::decode_uses_tensor_cores(G);
+  rc = cache_map(&tk, cache_k, dims->batch, dims->max_seq_len, dims->n_kv_heads, swizzled);
   if (rc != KVATTN_OK) return rc;
-  rc = cache_map(&tv, cache_v, dims->batch, dims->max_seq_len, dims->n_kv_heads);
+  rc = cache_map(&tv, cache_v, dims->batch, dims->max_seq_len, dims->n_kv_heads, swizzled);
   if (rc != KVATTN_OK) return rc;
 
   kvattn::DecodeArgs a;

@@ -20,7 +20,7 @@ constexpr int kHeadDim = 128;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-bool group_supported(int G) { return G == 1 || G == 2 || G == 4 || G == 8; }
+bool group_supported(int G) { return G == 1 || G == 2 || G == 4 || G == 8 || G == 16; }
 
 int check_dims(const kvattn_dims* d) {
   if (!d) return KVATTN_ERR_INVALID_ARG;
@@ -113,6 +113,23 @@ int encode_cache_map(CUtensorMap* map, const void* base, int B, int S, int Hkv, 
 
 int hint_or_default(int32_t hint, int S) { return hint <= 0 ? S : hint; }
 
+// 4-D view (d, head, row, seq) of a [B, R, heads, 128] bf16 tensor with
+// 128-byte swizzled boxes of 64 elements x box_heads x box_rows.
+int encode_sw128_map(CUtensorMap* map, const void* base, int B, int R, int heads, int box_heads, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return KVATTN_ERR_CUDA;
+  const cuuint64_t dims[4] = {(cuuint64_t)kHeadDim, (cuuint64_t)heads, (cuuint64_t)R, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)heads * kHeadDim * 2,
+                                 (cuuint64_t)R * heads * kHeadDim * 2};
+  const cuuint32_t box[4] = {64, (cuuint32_t)box_heads, (cuuint32_t)box_rows, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? KVATTN_OK : KVATTN_ERR_CUDA;
+}
+
+
 int run_attention(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, const uint16_t* cache_k,
                   const uint16_t* cache_v, const int32_t* start_pos, int32_t max_kv_len_hint, float scale,
                   uint16_t* out, void* workspace, size_t workspace_bytes, int32_t* dev_status,
@@ -141,9 +158,15 @@ int run_attention(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, con
   }
 
   CUtensorMap tk, tv;
-  rc = encode_cache_map(&tk, cache_k, dims->batch, dims->max_seq_len, dims->n_kv_heads, 32);
-  if (rc != KVATTN_OK) return rc;
-  rc = encode_cache_map(&tv, cache_v, dims->batch, dims->max_seq_len, dims->n_kv_heads, 32);
+  if (kvattn::decode_uses_tensor_cores(dims->n_heads / dims->n_kv_heads)) {
+    rc = encode_sw128_map(&tk, cache_k, dims->batch, dims->max_seq_len, dims->n_kv_heads, 1, 64);
+    if (rc != KVATTN_OK) return rc;
+    rc = encode_sw128_map(&tv, cache_v, dims->batch, dims->max_seq_len, dims->n_kv_heads, 1, 64);
+  } else {
+    rc = encode_cache_map(&tk, cache_k, dims->batch, dims->max_seq_len, dims->n_kv_heads, 32);
+    if (rc != KVATTN_OK) return rc;
+    rc = encode_cache_map(&tv, cache_v, dims->batch, dims->max_seq_len, dims->n_kv_heads, 32);
+  }
   if (rc != KVATTN_OK) return rc;
 
   kvattn::DecodeArgs a;
@@ -165,22 +188,6 @@ int run_attention(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, con
   return kvattn::launch_decode(a, tk, tv, (cudaStream_t)stream) == cudaSuccess ? KVATTN_OK : KVATTN_ERR_CUDA;
 }
 
-
-// 4-D view (d, head, row, seq) of a [B, R, heads, 128] bf16 tensor with
-// 128-byte swizzled boxes of 64 elements x box_heads x box_rows.
-int encode_sw128_map(CUtensorMap* map, const void* base, int B, int R, int heads, int box_heads, int box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return KVATTN_ERR_CUDA;
-  const cuuint64_t dims[4] = {(cuuint64_t)kHeadDim, (cuuint64_t)heads, (cuuint64_t)R, (cuuint64_t)B};
-  const cuuint64_t strides[3] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)heads * kHeadDim * 2,
-                                 (cuuint64_t)R * heads * kHeadDim * 2};
-  const cuuint32_t box[4] = {64, (cuuint32_t)box_heads, (cuuint32_t)box_rows, 1};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? KVATTN_OK : KVATTN_ERR_CUDA;
-}
 
 int run_prefill_tc(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, const uint16_t* cache_k,
                    const uint16_t* cache_v, const int32_t* start_pos, int32_t max_kv_len_hint, float scale,

@@ -59,6 +59,10 @@ struct DecodePlan {
 // Split size, persistent grid and workspace for these shapes on this device.
 DecodePlan plan_decode(int B, int Tq, int H, int Hkv, int kv_len_hint, int sm_count);
 
+// G >= 8 runs the tensor-core decode, whose cache view is 128B-swizzled
+// boxes of 64 elements x 64 rows (else plain boxes of 128 elements x 32 rows).
+bool decode_uses_tensor_cores(int G);
+
 // Points ws_o / ws_ml / counter of `a` into a workspace of plan.ws_bytes.
 void bind_decode_workspace(DecodeArgs& a, const DecodePlan& plan, void* workspace);
 

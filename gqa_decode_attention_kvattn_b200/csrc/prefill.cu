@@ -533,6 +533,7 @@ cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& tq, const CU
     case 2: return launch_prefill_g<2>(a, tq, tk, tv, st);
     case 4: return launch_prefill_g<4>(a, tq, tk, tv, st);
     case 8: return launch_prefill_g<8>(a, tq, tk, tv, st);
+    case 16: return launch_prefill_g<16>(a, tq, tk, tv, st);
     default: return cudaErrorInvalidValue;
   }
 }

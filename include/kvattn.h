@@ -57,7 +57,7 @@ typedef struct CUstream_st* kvattn_stream_t;
 typedef enum kvattn_status {
   KVATTN_OK = 0,
   KVATTN_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, H % Hkv != 0 */
-  KVATTN_ERR_UNSUPPORTED = 2, /* head_dim != 128, group size G = H/Hkv not in {1,2,4,8} */
+  KVATTN_ERR_UNSUPPORTED = 2, /* head_dim != 128, group size G = H/Hkv not in {1,2,4,8,16} */
   KVATTN_ERR_OUT_OF_RANGE = 3, /* a host-visible length outside the cache */
   KVATTN_ERR_WORKSPACE = 4,    /* workspace missing or smaller than required */
   KVATTN_ERR_CUDA = 5          /* a CUDA launch or query failed */
@@ -67,6 +67,7 @@ typedef enum kvattn_status {
 #define KVATTN_DEV_START_POS_RANGE 0x1 /* start_pos[b] < 0 or start_pos[b]+T > max_seq_len */
 #define KVATTN_DEV_KV_LEN_HINT 0x2     /* start_pos[b]+T > max_kv_len_hint */
 #define KVATTN_DEV_WAIT_TIMEOUT 0x4    /* an in-kernel pipeline wait gave up */
+#define KVATTN_DEV_INTERNAL 0x8        /* an internal invariant failed (the launch did nothing) */
 
 typedef struct kvattn_dims {
   int32_t batch;       /* B: sequences in this call (rows 0..B-1 of the caches) */

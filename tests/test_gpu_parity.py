@@ -53,7 +53,9 @@ def _check_step(seed, B, T, H, Hkv, S, sp, rope, kind, hint=0, in_place=False):
     (2, 32, 8, 200, [33, 199], kv.LLAMA3_1),
     (4, 16, 16, 130, [63, 64, 65, 129], kv.LLAMA3),     # G = 1 (MHA)
     (3, 16, 8, 300, [0, 95, 257], kv.LLAMA3),           # G = 2
-    (5, 64, 8, 520, [1, 127, 128, 511, 519], kv.LLAMA3),  # G = 8
+    (5, 64, 8, 520, [1, 127, 128, 511, 519], kv.LLAMA3),  # G = 8 (tensor cores)
+    (3, 32, 2, 700, [0, 63, 64, 699][:3], kv.LLAMA3),     # G = 16 (tensor cores)
+    (4, 64, 8, 3000, [2999, 64, 65, 1000], kv.LLAMA3_1),  # G = 8, several splits
 ])
 def test_decode_step_small(case):
     B, H, Hkv, S, sp, rope = case
@@ -221,6 +223,7 @@ def test_prefill_equals_prefill_then_decode_steps():
     (1, 300, 16, 8, 700, [123]),        # G=2: 64-token tiles, several key tiles
     (2, 20, 64, 8, 300, [0, 129]),      # G=8: 16-token tiles
     (1, 130, 8, 8, 260, [127]),         # G=1 (MHA): 128-token tiles
+    (2, 11, 32, 2, 150, [0, 120]),      # G=16: 8-token tiles
     (3, 1, 32, 8, 300, [0, 127, 128]),  # one token per sequence through the prefill path
 ])
 def test_prefill_tiles_and_groups(case):

@@ -107,9 +107,9 @@ def test_rope_append_rejects_bad_pointers_and_params(lib):
 def test_attention_entry_points_reject_bad_args(lib):
     d = _dims()
     P = [FAKE] * 4
-    # group size 32/2 = 16 is not built
-    d16 = _dims(n_kv_heads=2)
-    assert lib.kvattn_decode(ctypes.byref(d16), *P, 0, 0.0, FAKE, None, 0, None, None) == 2
+    # group size 32/1 = 32 is not built
+    d32 = _dims(n_kv_heads=1)
+    assert lib.kvattn_decode(ctypes.byref(d32), *P, 0, 0.0, FAKE, None, 0, None, None) == 2
     # null output
     assert lib.kvattn_decode(ctypes.byref(d), *P, 0, 0.0, None, None, 0, None, None) == 1
     # hint beyond the cache
