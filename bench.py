@@ -161,6 +161,32 @@ def bus_id_of(dev):
         return None
 
 
+# ----------------------------------------------------------------- ranks
+def max_over_ranks(ms: float, world: int, device=None) -> float:
+    """The slowest rank's time: every rank contributes its own device-timed
+    milliseconds and all of them get the maximum (replicas are timed as one
+    job).  A no-op for a single process."""
+    if world <= 1:
+        return float(ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank_step: float, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job rate: the units every rank processed over the slowest rank's
+    time (weak scaling: each replica does the same work)."""
+    return world * steps * units_per_rank_step / (max_ms / 1e3)
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
 # ----------------------------------------------------------------- state
 class Layer:
     pass
@@ -336,8 +362,7 @@ def run_ours(args, w, rank, world, device):
         torch.cuda.synchronize(device)
 
     # ---------------- timed region
-    if world > 1:
-        dist.barrier()
+    barrier(world)
     torch.cuda.synchronize(device)
     sampler = ClockSampler(bus_id_of(device))
     sampler.start()
@@ -353,14 +378,10 @@ def run_ours(args, w, rank, world, device):
     t1.record()
     torch.cuda.synchronize(device)
     clocks = sampler.stop()
-    if world > 1:
-        dist.barrier()
+    barrier(world)
     ms = t0.elapsed_time(t1)
     attn_ms = [a.elapsed_time(b) for a, b in events]   # the last step's attention calls
-    if world > 1:
-        tt = torch.tensor([ms], dtype=torch.float64, device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(ms, world, device)
     status = int(st["status"].item())
 
     secs = ms / 1e3
@@ -368,7 +389,7 @@ def run_ours(args, w, rank, world, device):
     hbm_peak, tf_peak, peak_src = measured_peaks()
     attn_avg_ms = float(np.mean(attn_ms))
     if w.kind == "decode":
-        value = world * args.steps * nl * kv_bytes_layer / secs / 1e9
+        value = job_throughput(nl * kv_bytes_layer, args.steps, world, ms) / 1e9
         unit = "GB/s"
         achieved = kv_bytes_layer / (attn_avg_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
@@ -379,7 +400,7 @@ def run_ours(args, w, rank, world, device):
                 "avg_launch_ms": round(attn_avg_ms, 5), "launches_timed": nl,
                 "bytes_per_launch": kv_bytes_layer}
     else:
-        value = world * args.steps * nl * flops_layer / secs / 1e12
+        value = job_throughput(nl * flops_layer, args.steps, world, ms) / 1e12
         unit = "TFLOP/s"
         achieved = flops_layer / (attn_avg_ms / 1e3) / 1e12
         roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": tf_peak, "unit": "TFLOP/s",
@@ -456,8 +477,7 @@ def run_e2e(args, w, st, device, kv_bytes_layer, flops_layer, world):
         e2e_step()
     graph.replay()
     torch.cuda.synchronize(device)
-    if world > 1:
-        dist.barrier()
+    barrier(world)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record()
@@ -466,10 +486,7 @@ def run_e2e(args, w, st, device, kv_bytes_layer, flops_layer, world):
     t1.record()
     torch.cuda.synchronize(device)
     ms = t0.elapsed_time(t1)
-    if world > 1:
-        tt = torch.tensor([ms], dtype=torch.float64, device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(ms, world, device)
     secs = ms / 1e3
     h2d = sum(x.numel() * x.element_size() for trip in h_in for x in trip) + h_sp.numel() * 4
     d2h = sum(x.numel() * x.element_size() for x in h_out)
