@@ -48,11 +48,12 @@ def _load():
                                           ctypes.c_double, _f64p]
         lib.oracle_rope_rotate_f64.restype = ctypes.c_int
         lib.oracle_rope_rotate_f64.argtypes = [ctypes.c_int, ctypes.c_int, _f64p, ctypes.c_long,
-                                               _f64p, _f64p]
+                                               _f64p, _f64p, ctypes.c_int, ctypes.c_int]
         lib.oracle_rope_append.restype = ctypes.c_int
         lib.oracle_rope_append.argtypes = [ctypes.c_int] * 6 + [_f64p, _i32p, _u16p, _u16p, _u16p,
                                                                 _u16p, _u16p, _u16p,
-                                                                ctypes.c_void_p, ctypes.c_void_p]
+                                                                ctypes.c_void_p, ctypes.c_void_p,
+                                                                ctypes.c_int, ctypes.c_int]
         lib.oracle_attention.restype = ctypes.c_int
         lib.oracle_attention.argtypes = [ctypes.c_int] * 6 + [_i32p, ctypes.c_double, _u16p, _u16p,
                                                               _u16p, _f64p, ctypes.c_int]
@@ -88,18 +89,20 @@ def rope_freqs(head_dim: int = 128, theta: float = 500000.0, use_scaled: bool = 
     return out
 
 
-def rope_rotate_f64(x: np.ndarray, freqs: np.ndarray, pos: int) -> np.ndarray:
+def rope_rotate_f64(x: np.ndarray, freqs: np.ndarray, pos: int, layout: int = 0, rotary_dim: int = 0) -> np.ndarray:
+    """layout 0: interleaved pairs (2i, 2i+1); 1: half-split pairs (i, i+r/2);
+    the first rotary_dim elements (0: all d) rotate, the rest pass through."""
     x = np.ascontiguousarray(x, dtype=np.float64)
     d = x.shape[-1]
     y = np.empty_like(x)
     rc = _load().oracle_rope_rotate_f64(x.size // d, d, np.ascontiguousarray(freqs), int(pos),
-                                        x.reshape(-1), y.reshape(-1))
+                                        x.reshape(-1), y.reshape(-1), int(layout), int(rotary_dim))
     if rc != OK:
         raise ValueError(f"oracle_rope_rotate_f64 rc={rc}")
     return y
 
 
-def rope_append(q, k_new, v_new, cache_k, cache_v, start_pos, freqs, want_exact=False):
+def rope_append(q, k_new, v_new, cache_k, cache_v, start_pos, freqs, want_exact=False, layout=0, rotary_dim=0):
     """Rotate q and k_new, append k_rot / v_new into the caches IN PLACE.
 
     q [B,T,H,d], k_new/v_new [B,T,Hkv,d], caches [B,S,Hkv,d]: uint16 bf16 bits.
@@ -115,7 +118,8 @@ def rope_append(q, k_new, v_new, cache_k, cache_v, start_pos, freqs, want_exact=
         B, T, H, Hkv, d, S, np.ascontiguousarray(freqs, np.float64),
         np.ascontiguousarray(start_pos, np.int32), np.ascontiguousarray(q),
         np.ascontiguousarray(k_new), np.ascontiguousarray(v_new), q_rot, cache_k, cache_v,
-        qe.ctypes.data if want_exact else None, ke.ctypes.data if want_exact else None)
+        qe.ctypes.data if want_exact else None, ke.ctypes.data if want_exact else None, int(layout),
+        int(rotary_dim))
     if want_exact:
         return q_rot, qe, ke, rc
     return q_rot, rc
@@ -135,9 +139,10 @@ def attention(q_rot, cache_k, cache_v, start_pos, scale=None, n_threads=0):
     return out, rc
 
 
-def step(q, k_new, v_new, cache_k, cache_v, start_pos, freqs, scale=None, n_threads=0):
+def step(q, k_new, v_new, cache_k, cache_v, start_pos, freqs, scale=None, n_threads=0, layout=0, rotary_dim=0):
     """One whole cached-attention call: rope + append (caches updated in
     place), then attention over rows 0..start_pos+t.  Returns (q_rot, out)."""
-    q_rot, rc = rope_append(q, k_new, v_new, cache_k, cache_v, start_pos, freqs)
+    q_rot, rc = rope_append(q, k_new, v_new, cache_k, cache_v, start_pos, freqs, layout=layout,
+                            rotary_dim=rotary_dim)
     out, rc2 = attention(q_rot, cache_k, cache_v, start_pos, scale, n_threads)
     return q_rot, out, max(rc, rc2)

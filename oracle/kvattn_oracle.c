@@ -21,11 +21,15 @@
  *     token after 4096 cached ones is rotated at angle 4097*f_i (same section
  *     of "Llama 3.1 8B KV cache"; freqs_cis[start_pos:start_pos+seqlen] in the
  *     model.py 281-302 excerpt of "Llama 3 8B · KV cache").
- *  3. Rotation of each interleaved pair (2i, 2i+1) of q and k by angle p*f_i,
- *     as the complex product (x_2i + i x_2i+1) e^{i p f_i}: Meta's
- *     apply_rotary_emb (model.py 160-177 excerpt of "Llama 3 8B · KV cache";
- *     its body is not printed; interleaved pairs and the counter-clockwise
- *     sense are the reading taken).  Angle, cos/sin and rotation in fp64.
+ *  3. Rotation of each pair of q and k by angle p*f_i, as the complex product
+ *     (x_a + i x_b) e^{i p f_i}: Meta's apply_rotary_emb (model.py 160-177
+ *     excerpt of "Llama 3 8B · KV cache"; its body is not printed;
+ *     interleaved pairs (a, b) = (2i, 2i+1) and the counter-clockwise sense
+ *     are the reading taken).  "The Modern Decoder Block" (module L7.3) also
+ *     names the half-split layout, pairs (i, i + r/2), and partial rotary,
+ *     where only the first r elements rotate (frequencies theta^(-2i/r)) and
+ *     the rest pass through; both are offered.  Angle, cos/sin and rotation
+ *     in fp64.
  *  4. Storage: q_rot and k_rot rounded to bf16 (round to nearest even), the
  *     cache dtype following the activations (cache.to(xq), bf16 default
  *     tensor type: "Llama 3 8B · KV cache", model.py 160-177 and
@@ -47,7 +51,9 @@
  * caches [B,S,Hkv,d].  bf16 tensors are passed as their uint16 bit patterns.
  *
  * Pins (tests/test_oracle_pins.py, tests/test_oracle_bruteforce.py): RoPE is
- * the identity at p = 0, preserves pair norms, gives dot products that depend
+ * the identity at p = 0, preserves pair norms, the half-split layout is the
+ * interleaved one conjugated by the pair permutation, partial rotary passes
+ * the tail through and rotates the head like a full RoPE of that width, gives dot products that depend
  * only on the relative offset, rotates (1,0) by 90 degrees to (0,1) at angle
  * pi/2, composes additively; the unscaled frequency table has f_0 = 1,
  * f_{d/4} = 1/sqrt(theta) and a constant ratio; the scaled table keeps the
@@ -134,22 +140,31 @@ int oracle_rope_freqs(int head_dim, double theta, int use_scaled, double factor,
   return ORACLE_OK;
 }
 
-/* Step 3 on one vector of d elements at position p (fp64 in, fp64 out). */
-static void rotate_f64(const double* x, double* y, int d, const double* freqs, long p) {
-  for (int i = 0; i < d / 2; ++i) {
+/* Step 3 on one vector of d elements at position p (fp64 in, fp64 out).
+ * layout 0: pairs (2i, 2i+1); layout 1: pairs (i, i + r/2); the first
+ * r = rotary_dim elements rotate, elements r..d-1 are copied. */
+static void rotate_f64(const double* x, double* y, int d, const double* freqs, long p, int layout, int r) {
+  for (int c = r; c < d; ++c) y[c] = x[c];
+  for (int i = 0; i < r / 2; ++i) {
+    const int ia = layout ? i : 2 * i;
+    const int ib = layout ? i + r / 2 : 2 * i + 1;
     double a = (double)p * freqs[i];
     double c = cos(a), s = sin(a);
-    double x0 = x[2 * i], x1 = x[2 * i + 1];
-    y[2 * i] = x0 * c - x1 * s;
-    y[2 * i + 1] = x0 * s + x1 * c;
+    double x0 = x[ia], x1 = x[ib];
+    y[ia] = x0 * c - x1 * s;
+    y[ib] = x0 * s + x1 * c;
   }
 }
 
-/* Exposed for the RoPE pins: rotate n_vec vectors of d doubles at position p. */
-int oracle_rope_rotate_f64(int n_vec, int d, const double* freqs, long p, const double* x,
-                           double* y) {
+/* Exposed for the RoPE pins: rotate n_vec vectors of d doubles at position p
+ * (rotary_dim 0 means d). */
+int oracle_rope_rotate_f64(int n_vec, int d, const double* freqs, long p, const double* x, double* y, int layout,
+                           int rotary_dim) {
   if (n_vec < 0 || d <= 0 || (d & 1) || !freqs || !x || !y) return ORACLE_ERR_ARG;
-  for (int v = 0; v < n_vec; ++v) rotate_f64(x + (size_t)v * d, y + (size_t)v * d, d, freqs, p);
+  if (rotary_dim == 0) rotary_dim = d;
+  if (rotary_dim < 2 || rotary_dim > d || (rotary_dim & 1) || (layout != 0 && layout != 1)) return ORACLE_ERR_ARG;
+  for (int v = 0; v < n_vec; ++v)
+    rotate_f64(x + (size_t)v * d, y + (size_t)v * d, d, freqs, p, layout, rotary_dim);
   return ORACLE_OK;
 }
 
@@ -161,8 +176,11 @@ int oracle_rope_rotate_f64(int n_vec, int d, const double* freqs, long p, const 
 int oracle_rope_append(int B, int T, int H, int Hkv, int d, int S, const double* freqs,
                        const int32_t* start_pos, const uint16_t* q, const uint16_t* k_new,
                        const uint16_t* v_new, uint16_t* q_rot, uint16_t* cache_k,
-                       uint16_t* cache_v, double* q_rot_exact, double* k_rot_exact) {
+                       uint16_t* cache_v, double* q_rot_exact, double* k_rot_exact, int layout,
+                       int rotary_dim) {
   if (B < 0 || T < 0 || H <= 0 || Hkv <= 0 || d <= 0 || (d & 1) || S < 0) return ORACLE_ERR_ARG;
+  if (rotary_dim == 0) rotary_dim = d;
+  if (rotary_dim < 2 || rotary_dim > d || (rotary_dim & 1) || (layout != 0 && layout != 1)) return ORACLE_ERR_ARG;
   if (!freqs || !start_pos || !q || !k_new || !v_new || !q_rot || !cache_k || !cache_v)
     return ORACLE_ERR_ARG;
   int rc = ORACLE_OK;
@@ -179,7 +197,7 @@ int oracle_rope_append(int B, int T, int H, int Hkv, int d, int S, const double*
       for (int h = 0; h < H; ++h) {
         size_t off = (((size_t)b * T + t) * H + h) * d;
         for (int c = 0; c < d; ++c) x[c] = bf16_to_f64(q[off + c]);
-        rotate_f64(x, y, d, freqs, p);
+        rotate_f64(x, y, d, freqs, p, layout, rotary_dim);
         for (int c = 0; c < d; ++c) {
           q_rot[off + c] = f64_to_bf16(y[c]);
           if (q_rot_exact) q_rot_exact[off + c] = y[c];
@@ -189,7 +207,7 @@ int oracle_rope_append(int B, int T, int H, int Hkv, int d, int S, const double*
         size_t in = (((size_t)b * T + t) * Hkv + j) * d;
         size_t row = (((size_t)b * S + p) * Hkv + j) * d;
         for (int c = 0; c < d; ++c) x[c] = bf16_to_f64(k_new[in + c]);
-        rotate_f64(x, y, d, freqs, p);
+        rotate_f64(x, y, d, freqs, p, layout, rotary_dim);
         for (int c = 0; c < d; ++c) {
           cache_k[row + c] = f64_to_bf16(y[c]);
           if (k_rot_exact) k_rot_exact[in + c] = y[c];

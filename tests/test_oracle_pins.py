@@ -327,3 +327,43 @@ def test_attention_rejects_out_of_range_start_pos():
     out, rc = oracle.attention(q, ck, cv, np.array([9, 1], np.int32))
     assert rc == oracle.ERR_RANGE
     assert np.all(out[0] == 0) and np.any(out[1] != 0)
+
+
+# ------------------------------------------- half-split layout, partial rotary
+def test_half_split_is_interleaved_under_the_pair_permutation():
+    # pairs (i, i + d/2) instead of (2i, 2i+1): moving element i to 2i and
+    # element i + d/2 to 2i + 1 must turn one layout into the other exactly
+    d = 16
+    f = oracle.rope_freqs(d, 10000.0)
+    x = RNG.standard_normal((3, d))
+    perm = np.empty(d, int)
+    perm[0::2] = np.arange(d // 2)
+    perm[1::2] = np.arange(d // 2) + d // 2
+    for p in (0, 7, 1234):
+        half = oracle.rope_rotate_f64(x, f, p, layout=1)
+        inter = oracle.rope_rotate_f64(x[:, perm], f, p, layout=0)
+        assert np.array_equal(half[:, perm], inter)
+        if p:
+            assert not np.allclose(half, oracle.rope_rotate_f64(x, f, p, layout=0))
+
+
+def test_partial_rotary_passes_the_tail_and_rotates_the_head():
+    d, r = 16, 6
+    f = oracle.rope_freqs(r, 10000.0)              # frequencies over the rotated width
+    x = RNG.standard_normal((4, d))
+    for layout in (0, 1):
+        y = oracle.rope_rotate_f64(x, f, 321, layout=layout, rotary_dim=r)
+        assert np.array_equal(y[:, r:], x[:, r:])
+        assert np.array_equal(y[:, :r], oracle.rope_rotate_f64(x[:, :r].copy(), f, 321, layout=layout))
+        # still a rotation: norms of the rotated part are kept
+        assert np.allclose(np.linalg.norm(y[:, :r], axis=1), np.linalg.norm(x[:, :r], axis=1), rtol=1e-13)
+
+
+def test_half_split_relative_offset():
+    d = 32
+    f = oracle.rope_freqs(d, 500000.0)
+    q = RNG.standard_normal(d)
+    k = RNG.standard_normal(d)
+    a = oracle.rope_rotate_f64(q, f, 40, layout=1) @ oracle.rope_rotate_f64(k, f, 10, layout=1)
+    b = oracle.rope_rotate_f64(q, f, 1030, layout=1) @ oracle.rope_rotate_f64(k, f, 1000, layout=1)
+    assert abs(a - b) <= 1e-10 * (1 + abs(a))
