@@ -50,7 +50,11 @@ class kvattn_dims(ctypes.Structure):
 class kvattn_rope_params(ctypes.Structure):
     _fields_ = [("theta", ctypes.c_double), ("use_scaled", ctypes.c_int32), ("factor", ctypes.c_double),
                 ("low_freq_factor", ctypes.c_double), ("high_freq_factor", ctypes.c_double),
-                ("original_max_pos", ctypes.c_double)]
+                ("original_max_pos", ctypes.c_double), ("layout", ctypes.c_int32), ("rotary_dim", ctypes.c_int32)]
+
+
+KVATTN_ROPE_INTERLEAVED = 0
+KVATTN_ROPE_HALF_SPLIT = 1
 
 
 @dataclass(frozen=True)
@@ -62,10 +66,13 @@ class RopeParams:
     low_freq_factor: float = 1.0
     high_freq_factor: float = 4.0
     original_max_pos: float = 8192.0
+    layout: int = KVATTN_ROPE_INTERLEAVED   # or KVATTN_ROPE_HALF_SPLIT
+    rotary_dim: int = 0                     # 0: the whole head
 
     def as_c(self) -> kvattn_rope_params:
         return kvattn_rope_params(self.theta, int(self.use_scaled), self.factor, self.low_freq_factor,
-                                  self.high_freq_factor, self.original_max_pos)
+                                  self.high_freq_factor, self.original_max_pos, int(self.layout),
+                                  int(self.rotary_dim))
 
 
 LLAMA3 = RopeParams()                     # rope_theta 500000, use_scaled_rope False

@@ -30,8 +30,8 @@ int check_dims(const kvattn_dims* d) {
   return KVATTN_OK;
 }
 
-// f_i = theta^(-2i/d), i < d/2, with the optional Llama-3.1 scaling rule
-// (stated in include/kvattn.h beside kvattn_rope_params).
+// f_i = theta^(-2i/r), i < r/2 (r = rotary_dim), with the optional Llama-3.1
+// scaling rule (stated in include/kvattn.h beside kvattn_rope_params).
 int make_rope_table(const kvattn_rope_params* r, kvattn::RopeTable* tab) {
   if (!r || !std::isfinite(r->theta) || !(r->theta > 0.0)) return KVATTN_ERR_INVALID_ARG;
   if (r->use_scaled) {
@@ -39,9 +39,12 @@ int make_rope_table(const kvattn_rope_params* r, kvattn::RopeTable* tab) {
         !(r->original_max_pos > 0.0))
       return KVATTN_ERR_INVALID_ARG;
   }
+  if (r->layout != KVATTN_ROPE_INTERLEAVED && r->layout != KVATTN_ROPE_HALF_SPLIT) return KVATTN_ERR_INVALID_ARG;
+  const int rd = r->rotary_dim == 0 ? kHeadDim : r->rotary_dim;
+  if (rd < 2 || rd > kHeadDim || (rd & 1)) return KVATTN_ERR_INVALID_ARG;
   const double two_pi = 6.283185307179586476925286766559;
-  for (int i = 0; i < kHeadDim / 2; ++i) {
-    double f = std::pow(r->theta, -(2.0 * i) / kHeadDim);
+  for (int i = 0; i < rd / 2; ++i) {
+    double f = std::pow(r->theta, -(2.0 * i) / rd);
     if (r->use_scaled) {
       const double wavelength = two_pi / f;
       const double short_wl = r->original_max_pos / r->high_freq_factor;  // kept below this
@@ -56,7 +59,9 @@ int make_rope_table(const kvattn_rope_params* r, kvattn::RopeTable* tab) {
     }
     tab->freq[i] = f;
   }
-  for (int i = kHeadDim / 2; i < kMaxRopePairs; ++i) tab->freq[i] = 0.0;
+  for (int i = rd / 2; i < kMaxRopePairs; ++i) tab->freq[i] = 0.0;
+  tab->layout = r->layout;
+  tab->rotary_dim = rd;
   return KVATTN_OK;
 }
 

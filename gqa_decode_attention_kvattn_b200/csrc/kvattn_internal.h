@@ -13,6 +13,8 @@ constexpr int kMaxRopePairs = 64;  // d/2 for d = 128
 
 struct RopeTable {
   double freq[kMaxRopePairs];  // f_i, already scaled when Llama-3.1 scaling is on
+  int layout;                  // 0: pairs (2i, 2i+1); 1: pairs (i, i + r/2)
+  int rotary_dim;              // r: elements 0..r-1 rotate, the rest are copied
 };
 
 struct RopeAppendArgs {

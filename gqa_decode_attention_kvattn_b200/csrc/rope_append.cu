@@ -34,7 +34,8 @@ __global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(RopeAppendArg
 
   __shared__ double s_cos[kMaxRopePairs];
   __shared__ double s_sin[kMaxRopePairs];
-  for (int i = threadIdx.x; i < kHeadDim / 2; i += blockDim.x) {
+  const int rp = tab.rotary_dim / 2;  // rotated pairs
+  for (int i = threadIdx.x; i < rp; i += blockDim.x) {
     const double ang = (double)pos * tab.freq[i];
     double s, c;
     sincos(ang, &s, &c);
@@ -51,20 +52,55 @@ __global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(RopeAppendArg
   const uint32_t* k_in = reinterpret_cast<const uint32_t*>(a.k_new) + (size_t)bt * a.Hkv * kPairs;
   uint32_t* k_out = reinterpret_cast<uint32_t*>(a.cache_k) + ((size_t)b * a.S + pos) * a.Hkv * kPairs;
 
-  for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {
-    const int i = idx & (kPairs - 1);
-    const bool is_q = idx < q_pairs;
-    const uint32_t w = is_q ? q_in[idx] : k_in[idx - q_pairs];
-    const double x0 = (double)bf16lo_to_f32(w);
-    const double x1 = (double)bf16hi_to_f32(w);
-    const double c = s_cos[i], s = s_sin[i];
-    const double y0 = x0 * c - x1 * s;
-    const double y1 = x0 * s + x1 * c;
-    const uint32_t r = f64_to_bf16_bits(y0) | (f64_to_bf16_bits(y1) << 16);
-    if (is_q)
-      q_out[idx] = r;
-    else
-      k_out[idx - q_pairs] = r;
+  if (tab.layout == 0 && rp == kPairs) {
+    // Meta layout over the whole head: each pair is one 32-bit word
+    for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {
+      const int i = idx & (kPairs - 1);
+      const bool is_q = idx < q_pairs;
+      const uint32_t w = is_q ? q_in[idx] : k_in[idx - q_pairs];
+      const double x0 = (double)bf16lo_to_f32(w);
+      const double x1 = (double)bf16hi_to_f32(w);
+      const double c = s_cos[i], s = s_sin[i];
+      const double y0 = x0 * c - x1 * s;
+      const double y1 = x0 * s + x1 * c;
+      const uint32_t r = f64_to_bf16_bits(y0) | (f64_to_bf16_bits(y1) << 16);
+      if (is_q)
+        q_out[idx] = r;
+      else
+        k_out[idx - q_pairs] = r;
+    }
+  } else {
+    // any layout / rotary width: slot j < rp rotates pair (a, b); slots
+    // j >= rp copy elements rd + 2(j - rp) and the next one unchanged
+    const int rd = 2 * rp;
+    for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {
+      const int vec = idx >> 6;
+      const int j = idx & (kPairs - 1);
+      const bool is_q = vec < a.H;
+      const uint16_t* in = is_q ? reinterpret_cast<const uint16_t*>(q_in) + (size_t)vec * kHeadDim
+                                : reinterpret_cast<const uint16_t*>(k_in) + (size_t)(vec - a.H) * kHeadDim;
+      uint16_t* outp = is_q ? reinterpret_cast<uint16_t*>(q_out) + (size_t)vec * kHeadDim
+                            : reinterpret_cast<uint16_t*>(k_out) + (size_t)(vec - a.H) * kHeadDim;
+      int ea, eb;
+      if (j < rp) {
+        ea = tab.layout ? j : 2 * j;
+        eb = tab.layout ? j + rp : 2 * j + 1;
+      } else {
+        ea = rd + 2 * (j - rp);
+        eb = ea + 1;
+      }
+      const uint16_t xa = in[ea], xb = in[eb];
+      if (j < rp) {
+        const double x0 = (double)__uint_as_float((uint32_t)xa << 16);
+        const double x1 = (double)__uint_as_float((uint32_t)xb << 16);
+        const double c = s_cos[j], s = s_sin[j];
+        outp[ea] = (uint16_t)f64_to_bf16_bits(x0 * c - x1 * s);
+        outp[eb] = (uint16_t)f64_to_bf16_bits(x0 * s + x1 * c);
+      } else {
+        outp[ea] = xa;
+        outp[eb] = xb;
+      }
+    }
   }
 
   // values: bit copy of Hkv rows of 256 bytes

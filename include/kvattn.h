@@ -77,14 +77,21 @@ typedef struct kvattn_dims {
   int32_t max_seq_len; /* S: rows the caches were allocated with */
 } kvattn_dims;
 
-/* RoPE parameters: f_i = theta^(-2i/d) ("Llama 3.1 8B KV cache", section
- * "RoPE has to know where it is"), with optional Llama-3.1 frequency scaling
- * (use_scaled_rope in "Llama 3.1 8B · Repeat heads", sku_list.py excerpt):
- * wavelengths 2*pi/f_i shorter than original_max_pos/high_freq_factor are
- * kept, longer than original_max_pos/low_freq_factor are divided by
- * `factor`, and in between f becomes (1-s) f/factor + s f with
+/* RoPE parameters: f_i = theta^(-2i/r), i < r/2, r = rotary_dim ("Llama 3.1
+ * 8B KV cache", section "RoPE has to know where it is", with r = d), with
+ * optional Llama-3.1 frequency scaling (use_scaled_rope in "Llama 3.1 8B ·
+ * Repeat heads", sku_list.py excerpt): wavelengths 2*pi/f_i shorter than
+ * original_max_pos/high_freq_factor are kept, longer than
+ * original_max_pos/low_freq_factor are divided by `factor`, and in between f
+ * becomes (1-s) f/factor + s f with
  * s = (original_max_pos/wavelength - low_freq_factor) /
- *     (high_freq_factor - low_freq_factor). */
+ *     (high_freq_factor - low_freq_factor).
+ * layout selects the rotated pairs: KVATTN_ROPE_INTERLEAVED (2i, 2i+1), the
+ * Meta layout, or KVATTN_ROPE_HALF_SPLIT (i, i + r/2) (both listed with
+ * partial rotary for the modern decoder block, "The Modern Decoder Block",
+ * module L7.3).  Elements r..d-1 pass through unchanged. */
+#define KVATTN_ROPE_INTERLEAVED 0
+#define KVATTN_ROPE_HALF_SPLIT 1
 typedef struct kvattn_rope_params {
   double theta;            /* 500000 for Llama 3 / 3.1 */
   int32_t use_scaled;      /* 0 or 1 */
@@ -92,6 +99,8 @@ typedef struct kvattn_rope_params {
   double low_freq_factor;  /* 1 */
   double high_freq_factor; /* 4 */
   double original_max_pos; /* 8192 */
+  int32_t layout;          /* KVATTN_ROPE_INTERLEAVED (0) or KVATTN_ROPE_HALF_SPLIT (1) */
+  int32_t rotary_dim;      /* even, 2..head_dim; 0 means head_dim */
 } kvattn_rope_params;
 
 /* Steps 1-2 (cache write "C_K[p] <- K_r, C_V[p] <- V" of "Llama 3 8B · KV
@@ -101,15 +110,17 @@ typedef struct kvattn_rope_params {
  *   q_rot[b,t,h,:]   = RoPE_p(q[b,t,h,:])      for h < H
  *   cache_k[b,p,j,:] = RoPE_p(k_new[b,t,j,:])  for j < Hkv
  *   cache_v[b,p,j,:] = v_new[b,t,j,:]          (bit copy)
- * RoPE_p rotates each interleaved pair (x_2i, x_2i+1) counter-clockwise by
- * p*f_i (the complex product (x_2i + i x_2i+1) e^{i p f_i}).  Angles, cos/sin
+ * RoPE_p rotates each pair (a, b) of the chosen layout counter-clockwise by
+ * p*f_i (the complex product (x_a + i x_b) e^{i p f_i}); elements at or past
+ * rotary_dim are copied.  Angles, cos/sin
  * and the rotation are computed in fp64 and rounded once to bf16 (nearest,
  * ties to even).  q_rot may equal q (in place); it must not partially overlap
  * q.  No other cache row is touched.  A sequence with start_pos[b] < 0 or
  * start_pos[b] + T > max_seq_len writes nothing and sets
  * KVATTN_DEV_START_POS_RANGE.
  * Host errors: INVALID_ARG (null/misaligned pointer, T < 1, B < 1, S < 1,
- * H % Hkv != 0, non-finite or non-positive theta), UNSUPPORTED (d != 128). */
+ * H % Hkv != 0, non-finite or non-positive theta, bad layout or
+ * rotary_dim), UNSUPPORTED (d != 128). */
 KVATTN_API int kvattn_rope_append(const kvattn_dims* dims, const kvattn_rope_params* rope, int32_t T,
                        const uint16_t* q, uint16_t* q_rot, const uint16_t* k_new,
                        const uint16_t* v_new, uint16_t* cache_k, uint16_t* cache_v,

@@ -65,7 +65,8 @@ def host_inputs(seed, B, T, H, Hkv, S, sp, d=128):
 
 
 def oracle_freqs(rope):
-    return oracle.rope_freqs(128, rope.theta, rope.use_scaled, rope.factor, rope.low_freq_factor,
+    """f_i over the rotated width: rotary_dim (0 means the whole head)."""
+    return oracle.rope_freqs(rope.rotary_dim or 128, rope.theta, rope.use_scaled, rope.factor, rope.low_freq_factor,
                              rope.high_freq_factor, rope.original_max_pos)
 
 
@@ -81,7 +82,8 @@ def oracle_sequence(q_b, k_b, v_b, ck_rows, cv_rows, sp_b, T, rope, scale=None):
     cv[0, :sp_b] = cv_rows[:sp_b]
     spa = np.array([sp_b], np.int32)
     q_rot, out, rc = oracle.step(q_b[None].copy(), k_b[None].copy(), v_b[None].copy(), ck, cv, spa,
-                                 oracle_freqs(rope), scale=scale)
+                                 oracle_freqs(rope), scale=scale, layout=rope.layout,
+                                 rotary_dim=rope.rotary_dim)
     assert rc == 0
     return q_rot[0], ck[0, sp_b:sp_b + T], out[0]
 

@@ -35,7 +35,8 @@ def _check_step(seed, B, T, H, Hkv, S, sp, rope, kind, hint=0, in_place=False):
     assert st == 0
     # the oracle on the same bits
     o_ck, o_cv = ck.copy(), cv.copy()
-    q_rot, out, rc = oracle.step(q, k, v, o_ck, o_cv, np.asarray(sp, np.int32), U.oracle_freqs(rope))
+    q_rot, out, rc = oracle.step(q, k, v, o_ck, o_cv, np.asarray(sp, np.int32), U.oracle_freqs(rope),
+                                 layout=rope.layout, rotary_dim=rope.rotary_dim)
     assert rc == 0
     assert U.ulp_distance(g_qrot, q_rot).max() <= 1
     assert U.ulp_distance(g_ck, o_ck).max() <= 1
@@ -247,3 +248,20 @@ def test_rows_past_the_sequence_may_hold_nan(kind, T):
     _, out, rc = oracle.step(q, k, v, o_ck, o_cv, sp, U.oracle_freqs(kv.LLAMA3))
     assert rc == 0
     U.assert_attention_close(g_out, out, f"{kind} with NaN past the sequence")
+
+
+@pytest.mark.parametrize("layout,rotary_dim,scaled,kind,T", [
+    (1, 0, False, "prefill", 3), (0, 64, False, "prefill", 3), (1, 96, True, "prefill", 3),
+    (0, 2, False, "decode", 1), (1, 64, False, "decode", 1)])
+def test_rope_layouts_and_partial_rotary(layout, rotary_dim, scaled, kind, T):
+    """Half-split pairs (i, i + r/2) and a rotary width r < d, against the
+    oracle: cache and q_rot within one ulp, the unrotated tail bit-copied."""
+    B, H, Hkv, S = 2, 32, 8, 200
+    sp = np.array([0, 150], np.int32)
+    rope = kv.RopeParams(use_scaled=scaled, layout=layout, rotary_dim=rotary_dim)
+    _check_step(37 + layout, B, T, H, Hkv, S, sp, rope, kind)
+    q, k, v, ck, cv = U.host_inputs(31, B, T, H, Hkv, S, sp)
+    g_qrot, _, _, _, st = _dev_step(q, k, v, ck, cv, sp, rope, T, kind)
+    assert st == 0
+    r = rotary_dim or 128
+    assert np.array_equal(g_qrot[..., r:], q[..., r:])

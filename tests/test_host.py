@@ -117,3 +117,12 @@ def test_attention_entry_points_reject_bad_args(lib):
     # prefill: T < 1, and a hint shorter than the chunk
     assert lib.kvattn_prefill_chunk(ctypes.byref(d), 0, *P, 0, 0.0, FAKE, None, 0, None, None) == 1
     assert lib.kvattn_prefill_chunk(ctypes.byref(d), 8, *P, 4, 0.0, FAKE, None, 0, None, None) == 3
+
+
+def test_rope_layout_and_rotary_dim_validation(lib):
+    d = _dims()
+    args = [FAKE] * 7
+    for bad in (kv.RopeParams(layout=2), kv.RopeParams(rotary_dim=3), kv.RopeParams(rotary_dim=130),
+                kv.RopeParams(rotary_dim=-2)):
+        rope = bad.as_c()
+        assert lib.kvattn_rope_append(ctypes.byref(d), ctypes.byref(rope), 1, *args, None, None) == 1
