@@ -103,6 +103,11 @@ def _load():
     lib.kvattn_decode_workspace_bytes.argtypes = [dims_p, ctypes.c_int32]
     lib.kvattn_decode.restype = ctypes.c_int
     lib.kvattn_decode.argtypes = [dims_p, P, P, P, P, ctypes.c_int32, ctypes.c_float, P, P, ctypes.c_size_t, P, P]
+    lib.kvattn_decode_fused_workspace_bytes.restype = ctypes.c_size_t
+    lib.kvattn_decode_fused_workspace_bytes.argtypes = [dims_p, ctypes.c_int32]
+    lib.kvattn_decode_fused.restype = ctypes.c_int
+    lib.kvattn_decode_fused.argtypes = [dims_p, rope_p, P, P, P, P, P, P, P, ctypes.c_int32, ctypes.c_float, P, P,
+                                        ctypes.c_size_t, P, P]
     lib.kvattn_prefill_workspace_bytes.restype = ctypes.c_size_t
     lib.kvattn_prefill_workspace_bytes.argtypes = [dims_p, ctypes.c_int32, ctypes.c_int32]
     lib.kvattn_prefill_chunk.restype = ctypes.c_int
@@ -110,6 +115,10 @@ def _load():
                                          ctypes.c_size_t, P, P]
     lib.kvattn_status_string.restype = ctypes.c_char_p
     lib.kvattn_status_string.argtypes = [ctypes.c_int]
+    lib.kvattn_last_cuda_error.restype = ctypes.c_int
+    lib.kvattn_last_cuda_error.argtypes = []
+    lib.kvattn_last_cuda_error_string.restype = ctypes.c_char_p
+    lib.kvattn_last_cuda_error_string.argtypes = []
     lib.kvattn_version.restype = ctypes.c_int
     lib.kvattn_version.argtypes = []
     _lib = lib
@@ -161,6 +170,9 @@ def _check_bf16(name, t, ndim):
 
 def _check_status(rc: int, where: str):
     if rc != KVATTN_OK:
+        if rc == KVATTN_ERR_CUDA:
+            lib = _load()
+            where = f"{where} [cuda error {lib.kvattn_last_cuda_error()}: {lib.kvattn_last_cuda_error_string().decode()}]"
         raise KvattnError(rc, where)
 
 
@@ -256,6 +268,51 @@ def kvattn_decode(q_rot, cache_k, cache_v, start_pos, max_kv_len_hint: int = 0, 
                            int(max_kv_len_hint), float(scale), _ptr(out), _ptr(workspace), ws_size,
                            _ptr(dev_status), _stream(stream))
     _check_status(rc, "kvattn_decode")
+    return out
+
+
+def kvattn_decode_fused_workspace_bytes(batch, n_heads, n_kv_heads, max_seq_len, max_kv_len_hint=0,
+                                        head_dim=HEAD_DIM) -> int:
+    dims = kvattn_dims(batch, n_heads, n_kv_heads, head_dim, max_seq_len)
+    return int(_load().kvattn_decode_fused_workspace_bytes(ctypes.byref(dims), int(max_kv_len_hint)))
+
+
+def alloc_fused_workspace(nbytes: int, device=None):
+    """A zeroed workspace for kvattn_decode_fused (its counters start at 0
+    and every completed call leaves them at 0)."""
+    import torch
+    return torch.zeros(max(nbytes, 16), dtype=torch.uint8, device=device or "cuda")
+
+
+def kvattn_decode_fused(q, k_new, v_new, cache_k, cache_v, start_pos, rope: RopeParams = LLAMA3,
+                        max_kv_len_hint: int = 0, scale: float = 0.0, out=None, q_rot=None, workspace=None,
+                        dev_status=None, stream=None):
+    """RoPE + cache append + split-K decode + merge in one launch (see
+    include/kvattn.h).  q [B,1,H,d], k_new/v_new [B,1,Hkv,d]; the caches are
+    updated in place; returns out [B,1,H,d].  q_rot (optional, not q)
+    receives the rotated q.  A zeroed workspace is allocated when none is
+    given; a caller-owned one must be zeroed once before its first use."""
+    import torch
+    lib = _load()
+    for name, t in (("q", q), ("k_new", k_new), ("v_new", v_new), ("cache_k", cache_k), ("cache_v", cache_v)):
+        _check_bf16(name, t, 4)
+    if q.shape[1] != 1:
+        raise ValueError("kvattn_decode_fused takes one token per sequence (q [B,1,H,d])")
+    if start_pos.dtype != torch.int32 or not start_pos.is_cuda:
+        raise ValueError("start_pos must be an int32 CUDA tensor")
+    dims = _dims_from_cache(q, cache_k)
+    if out is None:
+        out = torch.empty_like(q)
+    ws_bytes = int(lib.kvattn_decode_fused_workspace_bytes(ctypes.byref(dims), int(max_kv_len_hint)))
+    if workspace is None and ws_bytes > 0:
+        workspace = alloc_fused_workspace(ws_bytes, q.device)
+    ws_size = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    rope_c = rope.as_c()
+    rc = lib.kvattn_decode_fused(ctypes.byref(dims), ctypes.byref(rope_c), _ptr(q), _ptr(q_rot), _ptr(k_new),
+                                 _ptr(v_new), _ptr(cache_k), _ptr(cache_v), _ptr(start_pos), int(max_kv_len_hint),
+                                 float(scale), _ptr(out), _ptr(workspace), ws_size, _ptr(dev_status),
+                                 _stream(stream))
+    _check_status(rc, "kvattn_decode_fused")
     return out
 
 

@@ -29,6 +29,7 @@
 //   M = max_s m_s,  out = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.
 #include "kvattn_device.cuh"
 #include "kvattn_internal.h"
+#include "rope_device.cuh"
 
 #include <algorithm>
 #include <type_traits>
@@ -103,6 +104,7 @@ struct __align__(128) Smem {
   int n_full, total_items;
   int stage_item[Shape<G>::STAGES];  // item whose tile fills the stage; -1: no more work
   int abort;  // set when a pipeline wait gave up; later waits return at once
+  int merge_last;  // fused decode: this CTA stored the last split of the item
   uint64_t full[Shape<G>::STAGES];
   uint64_t empty[Shape<G>::STAGES];
   uint64_t cons;  // the four consumer warps' epilogue barrier
@@ -231,13 +233,202 @@ __device__ void build_work_table(const DecodeArgs& a, SM& sm, int n_sets, int la
   }
 }
 
-template <int G>
+// Log-sum-exp merge of the ns split partials of (row set v, head) for output
+// element c, in split order with a running maximum:
+//   M = max_s m_s,  out = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.
+// The partials may come from other CTAs, so they are read from L2.
+__device__ __forceinline__ float lse_merge_element(const DecodeArgs& a, int v, int head, int ns, int c) {
+  const size_t base = (size_t)v * a.max_splits * a.H + head;
+  float M = -INFINITY, num = 0.f, den = 0.f;
+  for (int s = 0; s < ns; ++s) {
+    const size_t slot = base + (size_t)s * a.H;
+    const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.ws_ml + slot * 2));
+    const float o = __ldcg(a.ws_o + slot * kHeadDim + c);
+    const float Mn = fmaxf(M, ml.x);
+    const float f_old = (M == -INFINITY) ? 0.f : fast_exp2(M - Mn);
+    const float f_new = fast_exp2(ml.x - Mn);
+    num = num * f_old + o * f_new;
+    den = den * f_old + ml.y * f_new;
+    M = Mn;
+  }
+  return num / den;
+}
+
+// Fused decode, after the four consumer warps stored an item's partials: the
+// CTA whose item is the last of its (row set, KV head) to finish merges all
+// its splits into the bf16 output and clears the counter for the next call.
+// Stores, a device-scope fence, then the counter increment on one side; the
+// increment that completes the count, a fence, then the loads on the other.
+template <int G, class Sync>
+__device__ __forceinline__ void merge_if_last(const DecodeArgs& a, const Item& it, int tid, volatile int* flag,
+                                              Sync&& sync) {
+  __threadfence();
+  sync();
+  int* cnt = a.merge_counter + (size_t)it.v * a.Hkv + it.kvh;
+  if (tid == 0) {
+    *flag = atomicAdd(cnt, 1) == it.nsplit - 1;
+    __threadfence();
+  }
+  sync();
+  if (*flag) {
+    __threadfence();
+    for (int h = 0; h < G; ++h) {
+      const int head = it.kvh * G + h;
+      const float r = lse_merge_element(a, it.v, head, it.nsplit, tid);
+      a.out[(((size_t)it.b * a.Tq + it.t) * a.H + head) * kHeadDim + tid] = (uint16_t)f32_to_bf16_bits(r);
+    }
+    if (tid == 0) atomicExch(cnt, 0);
+  }
+}
+
+// The producer warp of both decode kernels.  Lane 0 claims items (from the
+// per-call counter when there is one, else round-robin over the grid), waits
+// for free stages and issues the tile copies (`load` issues one tile's).
+//
+// Unfused, only lane 0 runs this and the item's (already rotated) q arrives
+// by a bulk copy with its first tile.  Fused (one new token per sequence),
+// the whole warp runs it: at an item's first tile each lane takes slots lane
+// and lane + 32 of every head vector, computes their (cos, sin) at the new
+// token's position p = L - 1, and rotates the item's G query heads into the
+// stage's q slot.  The item whose rows end at p (the last split) first
+// rotates the new K row and writes it, and the new V row, to cache row p,
+// then fences the generic-proxy stores against the tensor copies that read
+// that row back.  Only that item reads row p, so no other CTA waits on it.
+template <bool FUSED, int G, int STAGES, int TILE_ROWS, class SM, class Load>
+__device__ __forceinline__ void produce(const DecodeArgs& a, const RopeTable& tab, SM& sm, int n_sets,
+                                        int total_items, uint32_t tile_bytes, int lane, Load&& load) {
+  constexpr uint32_t kQBytes = G * kHeadDim * 2;
+  const bool leader = lane == 0;
+  auto bcast = [&](int x) {
+    if constexpr (FUSED) return __shfl_sync(0xffffffffu, x, 0);
+    else return x;
+  };
+  int stage = 0;
+  uint32_t phase = 0;
+  int next_static = blockIdx.x;
+  for (;;) {
+    int i = 0, stop = 0;
+    if (leader) {
+      i = a.counter ? atomicAdd(a.counter, 1) : next_static;
+      stop = (i >= total_items || sm.abort) ? 1 : 0;
+    }
+    next_static += gridDim.x;
+    i = bcast(i);
+    stop = bcast(stop);
+    if (stop) {
+      // hand the consumers the end marker through the next stage
+      if (leader) {
+        if (mbar_wait(&sm.empty[stage], phase ^ 1, &sm.abort)) {
+          sm.stage_item[stage] = -1;
+          mbar_arrive(&sm.full[stage]);
+        } else {
+          abort_pipeline(&sm.abort, a.dev_status);
+        }
+      }
+      if (++stage == STAGES) { stage = 0; phase ^= 1; }
+      break;
+    }
+    const Item it = decode_item(a, sm, n_sets, i);
+    if (it.nsplit == 0) continue;  // invalid row set: nothing to stream
+    for (int row = it.r0; row < it.r1; row += TILE_ROWS) {
+      int ok = 1;
+      if (leader) ok = mbar_wait(&sm.empty[stage], phase ^ 1, &sm.abort) ? 1 : 0;
+      ok = bcast(ok);
+      if (!ok) {
+        if (leader) abort_pipeline(&sm.abort, a.dev_status);
+        break;
+      }
+      const bool first = row == it.r0;
+      if (!FUSED || !first) {
+        if (leader) {
+          sm.stage_item[stage] = i;
+          mbar_arrive_expect_tx(&sm.full[stage], tile_bytes + (first ? kQBytes : 0u));
+          if (first) {
+            const uint16_t* qsrc = a.q + (((size_t)it.b * a.Tq + it.t) * a.H + (size_t)it.kvh * G) * kHeadDim;
+            bulk_load(&sm.q[stage][0][0], qsrc, kQBytes, &sm.full[stage]);
+          }
+          load(stage, it, row);
+        }
+      } else {
+        const long long pos = it.L - 1;
+        RopeSlot sl[2];
+        double cs[2], sn[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          sl[u] = rope_slot(tab, lane + 32 * u);
+          rope_cos_sin(tab, lane + 32 * u, pos, cs[u], sn[u]);
+        }
+        if (it.r1 == it.L) {
+          const size_t src = ((size_t)it.b * a.Hkv + it.kvh) * kHeadDim;
+          const size_t dst = (((size_t)it.b * a.S + pos) * a.Hkv + it.kvh) * kHeadDim;
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            uint16_t ya, yb;
+            rope_rotate_bits(sl[u].rotate, cs[u], sn[u], a.k_new[src + sl[u].ea], a.k_new[src + sl[u].eb], ya, yb);
+            a.cache_k[dst + sl[u].ea] = ya;
+            a.cache_k[dst + sl[u].eb] = yb;
+          }
+          if (lane < kHeadDim / 8)
+            reinterpret_cast<uint4*>(a.cache_v + dst)[lane] = reinterpret_cast<const uint4*>(a.v_new + src)[lane];
+          asm volatile("fence.proxy.async.global;" ::: "memory");
+          __syncwarp();
+        }
+        if (leader) {
+          sm.stage_item[stage] = i;
+          mbar_expect_tx(&sm.full[stage], tile_bytes);
+          load(stage, it, row);
+        }
+        const size_t qoff = ((size_t)it.b * a.H + (size_t)it.kvh * G) * kHeadDim;
+        uint16_t* qout = (a.q_rot_out && it.split == 0) ? a.q_rot_out + qoff : nullptr;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const uint16_t* qin = a.q + qoff + (size_t)h * kHeadDim;
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            uint16_t ya, yb;
+            rope_rotate_bits(sl[u].rotate, cs[u], sn[u], qin[sl[u].ea], qin[sl[u].eb], ya, yb);
+            sm.q[stage][h][sl[u].ea] = ya;
+            sm.q[stage][h][sl[u].eb] = yb;
+            if (qout) {
+              qout[h * kHeadDim + sl[u].ea] = ya;
+              qout[h * kHeadDim + sl[u].eb] = yb;
+            }
+          }
+        }
+        __syncwarp();
+        if (leader) mbar_arrive(&sm.full[stage]);  // the stage's one arrival: q is in place
+      }
+      if (++stage == STAGES) { stage = 0; phase ^= 1; }
+    }
+  }
+  if (!leader) return;
+  // Leave only once every copy into this CTA's shared memory has landed:
+  // wait (bounded) until the consumers have released every stage.
+  for (int s = 0; s < STAGES; ++s) {
+    if (!mbar_wait(&sm.empty[stage], phase ^ 1, nullptr)) {
+      abort_pipeline(&sm.abort, a.dev_status);
+      break;
+    }
+    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+  }
+  if constexpr (FUSED) {
+    // the last CTA to finish leaves the work counter at zero for the next call
+    if (a.counter) {
+      __threadfence();
+      if (atomicAdd(a.exit_counter, 1) == (int)gridDim.x - 1) {
+        atomicExch(a.counter, 0);
+        atomicExch(a.exit_counter, 0);
+      }
+    }
+  }
+}
+
+template <int G, bool FUSED>
 __global__ void __launch_bounds__(kThreads, Shape<G>::MIN_BLOCKS) decode_splitk_kernel(
     const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
-    const DecodeArgs a, const int evict_first) {
+    const DecodeArgs a, const int evict_first, const __grid_constant__ RopeTable tab) {
   using Sh = Shape<G>;
   constexpr int kStages = Sh::STAGES;
-  constexpr uint32_t kQBytes = G * kHeadDim * 2;
   // dynamic shared memory starts 128-byte aligned (the declaration asks for
   // it); casting the array itself keeps the shared state space visible to
   // the compiler, so accesses through `sm` become LDS/STS
@@ -280,64 +471,19 @@ __global__ void __launch_bounds__(kThreads, Shape<G>::MIN_BLOCKS) decode_splitk_
 
   if (warp == kConsumerWarps) {
     // ================================================================ producer
-    if (lane == 0) {
-      prefetch_tensormap(&tmap_k);
-      prefetch_tensormap(&tmap_v);
+    if (FUSED || lane == 0) {
       uint64_t policy = 0;
-      if (evict_first) policy = l2_policy_evict_first();
-      else asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(policy));
-      int stage = 0;
-      uint32_t phase = 0;
-      // Items come from the per-call counter when there is one (dynamic
-      // balance), else round-robin over the grid.
-      int next_static = blockIdx.x;
-      for (;;) {
-        int i;
-        if (a.counter) i = atomicAdd(a.counter, 1);
-        else { i = next_static; next_static += gridDim.x; }
-        const bool done = i >= total_items || sm.abort;
-        Item it;
-        if (!done) {
-          it = decode_item(a, sm, n_sets, i);
-          if (it.nsplit == 0) continue;  // invalid row set: nothing to stream
-        }
-        if (done) {
-          // hand the consumers the end marker through the next stage
-          if (mbar_wait(&sm.empty[stage], phase ^ 1, &sm.abort)) {
-            sm.stage_item[stage] = -1;
-            mbar_arrive(&sm.full[stage]);
-          } else {
-            abort_pipeline(&sm.abort, a.dev_status);
-          }
-          if (++stage == kStages) { stage = 0; phase ^= 1; }
-          break;
-        }
-        for (int row = it.r0; row < it.r1; row += kTileRows) {
-          if (!mbar_wait(&sm.empty[stage], phase ^ 1, &sm.abort)) {
-            abort_pipeline(&sm.abort, a.dev_status);
-            break;
-          }
-          const bool first = row == it.r0;
-          sm.stage_item[stage] = i;
-          mbar_arrive_expect_tx(&sm.full[stage], 2 * kTileBytes + (first ? kQBytes : 0u));
-          if (first) {
-            const uint16_t* qsrc = a.q_rot + (((size_t)it.b * a.Tq + it.t) * a.H + (size_t)it.kvh * G) * kHeadDim;
-            bulk_load(&sm.q[stage][0][0], qsrc, kQBytes, &sm.full[stage]);
-          }
-          tma_load_4d(&sm.k[stage][0][0], &tmap_k, &sm.full[stage], 0, it.kvh, row, it.b, policy);
-          tma_load_4d(&sm.v[stage][0][0], &tmap_v, &sm.full[stage], 0, it.kvh, row, it.b, policy);
-          if (++stage == kStages) { stage = 0; phase ^= 1; }
-        }
+      if (lane == 0) {
+        prefetch_tensormap(&tmap_k);
+        prefetch_tensormap(&tmap_v);
+        if (evict_first) policy = l2_policy_evict_first();
+        else asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(policy));
       }
-      // Leave only once every copy into this CTA's shared memory has landed:
-      // wait (bounded) until the consumers have released every stage.
-      for (int s = 0; s < kStages; ++s) {
-        if (!mbar_wait(&sm.empty[stage], phase ^ 1, nullptr)) {
-          abort_pipeline(&sm.abort, a.dev_status);
-          break;
-        }
-        if (++stage == kStages) { stage = 0; phase ^= 1; }
-      }
+      produce<FUSED, G, kStages, kTileRows>(a, tab, sm, n_sets, total_items, 2 * kTileBytes, lane,
+                                            [&](int st, const Item& it, int row) {
+        tma_load_4d(&sm.k[st][0][0], &tmap_k, &sm.full[st], 0, it.kvh, row, it.b, policy);
+        tma_load_4d(&sm.v[st][0][0], &tmap_v, &sm.full[st], 0, it.kvh, row, it.b, policy);
+      });
     }
     return;
   }
@@ -592,6 +738,9 @@ __global__ void __launch_bounds__(kThreads, Shape<G>::MIN_BLOCKS) decode_splitk_
         }
       }
     }
+    if constexpr (FUSED) {
+      if (it.nsplit > 1) merge_if_last<G>(a, it, tid, &sm.merge_last, cons_sync);
+    }
     cons_sync();
   }
 }
@@ -606,20 +755,8 @@ __global__ void __launch_bounds__(kHeadDim) decode_merge_kernel(const DecodeArgs
   if (L == 0 || ns <= 1) return;  // invalid, or written directly by K2
   const int b = v / a.Tq, t = v - b * a.Tq;
   const int c = threadIdx.x;
-  const size_t base = (size_t)v * a.max_splits * a.H + head;
-  float M = -INFINITY, num = 0.f, den = 0.f;
-  for (int s = 0; s < ns; ++s) {
-    const size_t slot = base + (size_t)s * a.H;
-    const float2 ml = *reinterpret_cast<const float2*>(a.ws_ml + slot * 2);
-    const float o = a.ws_o[slot * kHeadDim + c];
-    const float Mn = fmaxf(M, ml.x);
-    const float f_old = (M == -INFINITY) ? 0.f : fast_exp2(M - Mn);
-    const float f_new = fast_exp2(ml.x - Mn);
-    num = num * f_old + o * f_new;
-    den = den * f_old + ml.y * f_new;
-    M = Mn;
-  }
-  a.out[(((size_t)b * a.Tq + t) * a.H + head) * kHeadDim + c] = (uint16_t)f32_to_bf16_bits(num / den);
+  const float r = lse_merge_element(a, v, head, ns, c);
+  a.out[(((size_t)b * a.Tq + t) * a.H + head) * kHeadDim + c] = (uint16_t)f32_to_bf16_bits(r);
 }
 
 // ======================================================================
@@ -654,6 +791,7 @@ struct __align__(1024) SmemMma {
   int n_full, total_items;
   int stage_item[kMmaStages];
   int abort;
+  int merge_last;
   uint64_t full[kMmaStages];
   uint64_t empty[kMmaStages];
   uint64_t cons;
@@ -683,12 +821,11 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int chunk) {
   return (uint32_t)(row * 128 + (((chunk ^ row) & 7) << 4));
 }
 
-template <int G>
+template <int G, bool FUSED>
 __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(
     const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
-    const DecodeArgs a, const int evict_first) {
+    const DecodeArgs a, const int evict_first, const __grid_constant__ RopeTable tab) {
   static_assert(G == 8 || G == 16, "tensor-core decode handles G = 8 or 16");
-  constexpr uint32_t kQBytes = G * kHeadDim * 2;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   SmemMma<G>& sm = *reinterpret_cast<SmemMma<G>*>(smem_raw);
   // the 128B-swizzled tiles need a 1024-byte aligned base; refuse otherwise
@@ -732,61 +869,21 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(
 
   if (warp == kConsumerWarps) {
     // ================================================================ producer
-    if (lane == 0) {
-      prefetch_tensormap(&tmap_k);
-      prefetch_tensormap(&tmap_v);
+    if (FUSED || lane == 0) {
       uint64_t policy = 0;
-      if (evict_first) policy = l2_policy_evict_first();
-      else asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(policy));
-      int stage = 0;
-      uint32_t phase = 0;
-      int next_static = blockIdx.x;
-      for (;;) {
-        int i;
-        if (a.counter) i = atomicAdd(a.counter, 1);
-        else { i = next_static; next_static += gridDim.x; }
-        const bool done = i >= total_items || sm.abort;
-        Item it;
-        if (!done) {
-          it = decode_item(a, sm, n_sets, i);
-          if (it.nsplit == 0) continue;
-        }
-        if (done) {
-          if (mbar_wait(&sm.empty[stage], phase ^ 1, &sm.abort)) {
-            sm.stage_item[stage] = -1;
-            mbar_arrive(&sm.full[stage]);
-          } else {
-            abort_pipeline(&sm.abort, a.dev_status);
-          }
-          if (++stage == kMmaStages) { stage = 0; phase ^= 1; }
-          break;
-        }
-        for (int row = it.r0; row < it.r1; row += kMmaTileRows) {
-          if (!mbar_wait(&sm.empty[stage], phase ^ 1, &sm.abort)) {
-            abort_pipeline(&sm.abort, a.dev_status);
-            break;
-          }
-          const bool first = row == it.r0;
-          sm.stage_item[stage] = i;
-          mbar_arrive_expect_tx(&sm.full[stage], 4 * kMmaHalfBytes + (first ? kQBytes : 0u));
-          if (first) {
-            const uint16_t* qsrc = a.q_rot + (((size_t)it.b * a.Tq + it.t) * a.H + (size_t)it.kvh * G) * kHeadDim;
-            bulk_load(&sm.q[stage][0][0], qsrc, kQBytes, &sm.full[stage]);
-          }
-          tma_load_4d(&sm.k[stage][0][0], &tmap_k, &sm.full[stage], 0, it.kvh, row, it.b, policy);
-          tma_load_4d(&sm.k[stage][1][0], &tmap_k, &sm.full[stage], 64, it.kvh, row, it.b, policy);
-          tma_load_4d(&sm.v[stage][0][0], &tmap_v, &sm.full[stage], 0, it.kvh, row, it.b, policy);
-          tma_load_4d(&sm.v[stage][1][0], &tmap_v, &sm.full[stage], 64, it.kvh, row, it.b, policy);
-          if (++stage == kMmaStages) { stage = 0; phase ^= 1; }
-        }
+      if (lane == 0) {
+        prefetch_tensormap(&tmap_k);
+        prefetch_tensormap(&tmap_v);
+        if (evict_first) policy = l2_policy_evict_first();
+        else asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(policy));
       }
-      for (int s = 0; s < kMmaStages; ++s) {
-        if (!mbar_wait(&sm.empty[stage], phase ^ 1, nullptr)) {
-          abort_pipeline(&sm.abort, a.dev_status);
-          break;
-        }
-        if (++stage == kMmaStages) { stage = 0; phase ^= 1; }
-      }
+      produce<FUSED, G, kMmaStages, kMmaTileRows>(a, tab, sm, n_sets, total_items, 4 * kMmaHalfBytes, lane,
+                                                  [&](int st, const Item& it, int row) {
+        tma_load_4d(&sm.k[st][0][0], &tmap_k, &sm.full[st], 0, it.kvh, row, it.b, policy);
+        tma_load_4d(&sm.k[st][1][0], &tmap_k, &sm.full[st], 64, it.kvh, row, it.b, policy);
+        tma_load_4d(&sm.v[st][0][0], &tmap_v, &sm.full[st], 0, it.kvh, row, it.b, policy);
+        tma_load_4d(&sm.v[st][1][0], &tmap_v, &sm.full[st], 64, it.kvh, row, it.b, policy);
+      });
     }
     return;
   }
@@ -988,6 +1085,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(
         }
       }
     }
+    if constexpr (FUSED) {
+      if (it.nsplit > 1) merge_if_last<G>(a, it, tid, &sm.merge_last, cons_sync);
+    }
     cons_sync();
   }
 }
@@ -1002,14 +1102,23 @@ size_t smem_bytes() {
   return sizeof(Smem<G>);
 }
 
+template <int G, bool FUSED>
+auto decode_kernel() {
+  if constexpr (G >= 8) return decode_mma_kernel<G, FUSED>;
+  else return decode_splitk_kernel<G, FUSED>;
+}
+
 template <int G>
-cudaError_t launch_g(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st) {
-  constexpr bool kMma = G >= 8;
-  auto kernel = [] {
-    if constexpr (kMma) return decode_mma_kernel<G>;
-    else return decode_splitk_kernel<G>;
-  }();
-  const size_t smem = kMma ? smem_bytes_mma<G>() : smem_bytes<G>();
+size_t decode_smem_bytes() {
+  if constexpr (G >= 8) return smem_bytes_mma<G>();
+  else return smem_bytes<G>();
+}
+
+template <int G, bool FUSED>
+cudaError_t launch_g(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, const RopeTable& tab,
+                     cudaStream_t st) {
+  auto kernel = decode_kernel<G, FUSED>();
+  const size_t smem = decode_smem_bytes<G>();
   static bool configured[64] = {false};
   int dev = 0;
   cudaError_t e0 = cudaGetDevice(&dev);
@@ -1021,14 +1130,15 @@ cudaError_t launch_g(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorM
     configured[dev] = true;
   }
   const int evict_first = a.Tq == 1 ? 1 : 0;
-  if (a.counter) {
+  if (!FUSED && a.counter) {
+    // the fused kernel leaves its counters at zero itself
     cudaError_t e1 = cudaMemsetAsync(a.counter, 0, sizeof(int), st);
     if (e1 != cudaSuccess) return e1;
   }
-  kernel<<<a.grid, kThreads, smem, st>>>(tk, tv, a, evict_first);
+  kernel<<<a.grid, kThreads, smem, st>>>(tk, tv, a, evict_first, tab);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (a.max_splits > 1) {
+  if (!FUSED && a.max_splits > 1) {
     dim3 grid(a.H, a.B * a.Tq);
     decode_merge_kernel<<<grid, kHeadDim, 0, st>>>(a);
     e = cudaGetLastError();
@@ -1036,23 +1146,33 @@ cudaError_t launch_g(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorM
   return e;
 }
 
+template <int G>
+cudaError_t launch_g(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st,
+                     const RopeTable* fused) {
+  if (fused) return launch_g<G, true>(a, tk, tv, *fused, st);
+  RopeTable unused{};
+  return launch_g<G, false>(a, tk, tv, unused, st);
+}
+
 }  // namespace
 
 // Resident CTAs per SM of the decode kernel for group size G (occupancy
 // query: registers and shared memory both count).
-template <int G>
-int resident_ctas() {
-  constexpr bool kMma = G >= 8;
-  auto kernel = [] {
-    if constexpr (kMma) return decode_mma_kernel<G>;
-    else return decode_splitk_kernel<G>;
-  }();
-  const size_t smem = kMma ? smem_bytes_mma<G>() : smem_bytes<G>();
+template <int G, bool FUSED>
+int resident_ctas_of() {
+  auto kernel = decode_kernel<G, FUSED>();
+  const size_t smem = decode_smem_bytes<G>();
   int n = 0;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess ||
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kThreads, smem) != cudaSuccess || n < 1)
     n = 1;
   return n;
+}
+
+// the persistent grid serves both the unfused and the fused kernel
+template <int G>
+int resident_ctas() {
+  return std::min(resident_ctas_of<G, false>(), resident_ctas_of<G, true>());
 }
 
 int resident_ctas_for(int G) {
@@ -1099,11 +1219,16 @@ DecodePlan plan_decode(int B, int Tq, int H, int Hkv, int kv_len_hint, int sm_co
   // partial (o, max, sum) per (row set, split, head), then the work counter
   p.ws_bytes =
       p.max_splits > 1 ? (size_t)row_sets * p.max_splits * H * (kHeadDim + 2) * sizeof(float) + 16 : 0;
+  // fused: the same, then (work, exit) counters and one merge counter per
+  // (row set, KV head), padded to 16 bytes
+  p.fused_ws_bytes = p.max_splits > 1 ? p.ws_bytes + (((size_t)row_sets * Hkv * sizeof(int) + 15) & ~(size_t)15) : 0;
   return p;
 }
 
-void bind_decode_workspace(DecodeArgs& a, const DecodePlan& plan, void* workspace) {
-  if (plan.ws_bytes == 0 || !workspace) {
+void bind_decode_workspace(DecodeArgs& a, const DecodePlan& plan, void* workspace, bool fused) {
+  a.exit_counter = nullptr;
+  a.merge_counter = nullptr;
+  if ((fused ? plan.fused_ws_bytes : plan.ws_bytes) == 0 || !workspace) {
     a.ws_o = nullptr;
     a.ws_ml = nullptr;
     a.counter = nullptr;
@@ -1114,15 +1239,26 @@ void bind_decode_workspace(DecodeArgs& a, const DecodePlan& plan, void* workspac
   a.ws_o = ws;
   a.ws_ml = ws + n_slots * kHeadDim;
   a.counter = reinterpret_cast<int*>(ws + n_slots * (kHeadDim + 2));
+  if (fused) {
+    a.exit_counter = a.counter + 1;
+    a.merge_counter = a.counter + 4;
+  }
 }
 
-cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st) {
+cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st,
+                          const RopeTable* fused) {
+  // every tensor argument the chosen kernel dereferences must have been set
+  if (!a.q || !a.out || !a.start_pos) return cudaErrorInvalidValue;
+  if (a.max_splits > 1 && (!a.ws_o || !a.ws_ml)) return cudaErrorInvalidValue;
+  if (fused && (a.Tq != 1 || !a.k_new || !a.v_new || !a.cache_k || !a.cache_v ||
+                (a.counter && (!a.exit_counter || !a.merge_counter))))
+    return cudaErrorInvalidValue;
   switch (a.H / a.Hkv) {
-    case 1: return launch_g<1>(a, tk, tv, st);
-    case 2: return launch_g<2>(a, tk, tv, st);
-    case 4: return launch_g<4>(a, tk, tv, st);
-    case 8: return launch_g<8>(a, tk, tv, st);
-    case 16: return launch_g<16>(a, tk, tv, st);
+    case 1: return launch_g<1>(a, tk, tv, st, fused);
+    case 2: return launch_g<2>(a, tk, tv, st, fused);
+    case 4: return launch_g<4>(a, tk, tv, st, fused);
+    case 8: return launch_g<8>(a, tk, tv, st, fused);
+    case 16: return launch_g<16>(a, tk, tv, st, fused);
     default: return cudaErrorInvalidValue;
   }
 }

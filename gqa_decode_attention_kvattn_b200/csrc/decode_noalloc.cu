@@ -136,7 +136,7 @@ extern "C" KVATTN_API int kvattn_decode_noalloc(const kvattn_dims* dims, const u
   rc = cache_map(&tv, cache_v, dims->batch, dims->max_seq_len, dims->n_kv_heads, swizzled);
   if (rc != KVATTN_OK) return rc;
 
-  kvattn::DecodeArgs a;
+  kvattn::DecodeArgs a{};
   a.B = dims->batch;
   a.Tq = 1;
   a.H = dims->n_heads;
@@ -146,11 +146,11 @@ extern "C" KVATTN_API int kvattn_decode_noalloc(const kvattn_dims* dims, const u
   a.rows_per_split = plan.rows_per_split;
   a.max_splits = plan.max_splits;
   a.scale_log2 = scale * 1.4426950408889634f;
-  a.q_rot = q_rot;
+  a.q = q_rot;
   a.out = out;
   a.start_pos = start_pos;
   kvattn::bind_decode_workspace(a, plan, scratch);
   a.dev_status = dev_status;
   a.grid = plan.grid;
-  return kvattn::launch_decode(a, tk, tv, (cudaStream_t)stream) == cudaSuccess ? KVATTN_OK : KVATTN_ERR_CUDA;
+  return kvattn::launch_status(kvattn::launch_decode(a, tk, tv, (cudaStream_t)stream));
 }

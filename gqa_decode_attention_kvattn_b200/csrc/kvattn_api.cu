@@ -12,6 +12,20 @@
 #include "kvattn.h"
 #include "kvattn_internal.h"
 
+namespace kvattn {
+
+namespace {
+thread_local int t_last_cuda_error = 0;
+}
+
+int launch_status(cudaError_t e) {
+  if (e == cudaSuccess) return KVATTN_OK;
+  t_last_cuda_error = (int)e;
+  return KVATTN_ERR_CUDA;
+}
+
+}  // namespace kvattn
+
 namespace {
 
 using kvattn::kMaxRopePairs;
@@ -174,7 +188,7 @@ int run_attention(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, con
   }
   if (rc != KVATTN_OK) return rc;
 
-  kvattn::DecodeArgs a;
+  kvattn::DecodeArgs a{};
   a.B = dims->batch;
   a.Tq = T;
   a.H = dims->n_heads;
@@ -184,13 +198,13 @@ int run_attention(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, con
   a.rows_per_split = plan.rows_per_split;
   a.max_splits = plan.max_splits;
   a.scale_log2 = scale * 1.4426950408889634f;
-  a.q_rot = q_rot;
+  a.q = q_rot;
   a.out = out;
   a.start_pos = start_pos;
   kvattn::bind_decode_workspace(a, plan, workspace);
   a.dev_status = dev_status;
   a.grid = plan.grid;
-  return kvattn::launch_decode(a, tk, tv, (cudaStream_t)stream) == cudaSuccess ? KVATTN_OK : KVATTN_ERR_CUDA;
+  return kvattn::launch_status(kvattn::launch_decode(a, tk, tv, (cudaStream_t)stream));
 }
 
 
@@ -234,7 +248,7 @@ int run_prefill_tc(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, co
   a.start_pos = start_pos;
   a.out = out;
   a.dev_status = dev_status;
-  return kvattn::launch_prefill(a, tq, tk, tv, (cudaStream_t)stream) == cudaSuccess ? KVATTN_OK : KVATTN_ERR_CUDA;
+  return kvattn::launch_status(kvattn::launch_prefill(a, tq, tk, tv, (cudaStream_t)stream));
 }
 
 }  // namespace
@@ -255,7 +269,7 @@ int kvattn_rope_append(const kvattn_dims* dims, const kvattn_rope_params* rope, 
   kvattn::RopeTable tab;
   rc = make_rope_table(rope, &tab);
   if (rc != KVATTN_OK) return rc;
-  kvattn::RopeAppendArgs a;
+  kvattn::RopeAppendArgs a{};
   a.B = dims->batch;
   a.T = T;
   a.H = dims->n_heads;
@@ -269,7 +283,7 @@ int kvattn_rope_append(const kvattn_dims* dims, const kvattn_rope_params* rope, 
   a.cache_v = cache_v;
   a.start_pos = start_pos;
   a.dev_status = dev_status;
-  return kvattn::launch_rope_append(a, tab, (cudaStream_t)stream) == cudaSuccess ? KVATTN_OK : KVATTN_ERR_CUDA;
+  return kvattn::launch_status(kvattn::launch_rope_append(a, tab, (cudaStream_t)stream));
 }
 
 size_t kvattn_decode_workspace_bytes(const kvattn_dims* dims, int32_t max_kv_len_hint) {
@@ -286,6 +300,80 @@ int kvattn_decode(const kvattn_dims* dims, const uint16_t* q_rot, const uint16_t
                   size_t workspace_bytes, int32_t* dev_status, kvattn_stream_t stream) {
   return run_attention(dims, 1, q_rot, cache_k, cache_v, start_pos, max_kv_len_hint, scale, out, workspace,
                        workspace_bytes, dev_status, stream);
+}
+
+size_t kvattn_decode_fused_workspace_bytes(const kvattn_dims* dims, int32_t max_kv_len_hint) {
+  if (check_dims(dims) != KVATTN_OK) return 0;
+  const int hint = hint_or_default(max_kv_len_hint, dims->max_seq_len);
+  if (hint > dims->max_seq_len || hint < 1) return 0;
+  int sms = 0;
+  if (current_sm_count(&sms) != KVATTN_OK) return 0;
+  return kvattn::plan_decode(dims->batch, 1, dims->n_heads, dims->n_kv_heads, hint, sms).fused_ws_bytes;
+}
+
+int kvattn_decode_fused(const kvattn_dims* dims, const kvattn_rope_params* rope, const uint16_t* q,
+                        uint16_t* q_rot, const uint16_t* k_new, const uint16_t* v_new, uint16_t* cache_k,
+                        uint16_t* cache_v, const int32_t* start_pos, int32_t max_kv_len_hint, float scale,
+                        uint16_t* out, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                        kvattn_stream_t stream) {
+  int rc = check_dims(dims);
+  if (rc != KVATTN_OK) return rc;
+  if (!group_supported(dims->n_heads / dims->n_kv_heads)) return KVATTN_ERR_UNSUPPORTED;
+  if (!q || !k_new || !v_new || !cache_k || !cache_v || !start_pos || !out) return KVATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(cache_k) || !aligned16(cache_v) ||
+      !aligned16(out) || (q_rot && !aligned16(q_rot)) || (reinterpret_cast<uintptr_t>(start_pos) & 3u))
+    return KVATTN_ERR_INVALID_ARG;
+  if (q_rot == q) return KVATTN_ERR_INVALID_ARG;  // other items of a sequence still read q
+  kvattn::RopeTable tab;
+  rc = make_rope_table(rope, &tab);
+  if (rc != KVATTN_OK) return rc;
+  const int hint = hint_or_default(max_kv_len_hint, dims->max_seq_len);
+  if (hint > dims->max_seq_len || hint < 1) return KVATTN_ERR_OUT_OF_RANGE;
+  if (!(scale > 0.f)) scale = 1.0f / std::sqrt((float)kHeadDim);
+  if (!std::isfinite(scale)) return KVATTN_ERR_INVALID_ARG;
+  if ((long long)dims->batch > (1LL << 24)) return KVATTN_ERR_UNSUPPORTED;
+
+  int sms = 0;
+  rc = current_sm_count(&sms);
+  if (rc != KVATTN_OK) return rc;
+  const kvattn::DecodePlan plan = kvattn::plan_decode(dims->batch, 1, dims->n_heads, dims->n_kv_heads, hint, sms);
+  if (plan.fused_ws_bytes > 0) {
+    if (!workspace || workspace_bytes < plan.fused_ws_bytes || !aligned16(workspace)) return KVATTN_ERR_WORKSPACE;
+  }
+  CUtensorMap tk, tv;
+  if (kvattn::decode_uses_tensor_cores(dims->n_heads / dims->n_kv_heads)) {
+    rc = encode_sw128_map(&tk, cache_k, dims->batch, dims->max_seq_len, dims->n_kv_heads, 1, 64);
+    if (rc != KVATTN_OK) return rc;
+    rc = encode_sw128_map(&tv, cache_v, dims->batch, dims->max_seq_len, dims->n_kv_heads, 1, 64);
+  } else {
+    rc = encode_cache_map(&tk, cache_k, dims->batch, dims->max_seq_len, dims->n_kv_heads, 32);
+    if (rc != KVATTN_OK) return rc;
+    rc = encode_cache_map(&tv, cache_v, dims->batch, dims->max_seq_len, dims->n_kv_heads, 32);
+  }
+  if (rc != KVATTN_OK) return rc;
+
+  kvattn::DecodeArgs a{};
+  a.B = dims->batch;
+  a.Tq = 1;
+  a.H = dims->n_heads;
+  a.Hkv = dims->n_kv_heads;
+  a.S = dims->max_seq_len;
+  a.kv_len_hint = hint;
+  a.rows_per_split = plan.rows_per_split;
+  a.max_splits = plan.max_splits;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.q = q;
+  a.out = out;
+  a.start_pos = start_pos;
+  kvattn::bind_decode_workspace(a, plan, workspace, true);
+  a.dev_status = dev_status;
+  a.grid = plan.grid;
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.cache_k = cache_k;
+  a.cache_v = cache_v;
+  a.q_rot_out = q_rot;
+  return kvattn::launch_status(kvattn::launch_decode(a, tk, tv, (cudaStream_t)stream, &tab));
 }
 
 size_t kvattn_prefill_workspace_bytes(const kvattn_dims* dims, int32_t T, int32_t max_kv_len_hint) {
@@ -333,6 +421,12 @@ const char* kvattn_status_string(int status) {
     case KVATTN_ERR_CUDA: return "CUDA error";
     default: return "unknown status";
   }
+}
+
+int kvattn_last_cuda_error(void) { return kvattn::t_last_cuda_error; }
+
+const char* kvattn_last_cuda_error_string(void) {
+  return kvattn::t_last_cuda_error ? cudaGetErrorString((cudaError_t)kvattn::t_last_cuda_error) : "no error";
 }
 
 int kvattn_version(void) { return 100; }

@@ -128,6 +128,12 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
 }
+// Raise the phase's expected transaction bytes without arriving; the phase
+// then completes once those bytes have landed and the arrivals are in.
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
 // One bounded wait on the phase with the given parity: the thread is
 // suspended (not spinning) until the phase completes or about `hint_ns`
 // passes.  True when the phase completed.

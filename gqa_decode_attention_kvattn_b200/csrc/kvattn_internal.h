@@ -9,6 +9,10 @@
 
 namespace kvattn {
 
+// Maps a launch result to a kvattn_status (KVATTN_OK or KVATTN_ERR_CUDA) and
+// remembers a failure for kvattn_last_cuda_error() on this host thread.
+int launch_status(cudaError_t e);
+
 constexpr int kMaxRopePairs = 64;  // d/2 for d = 128
 
 struct RopeTable {
@@ -40,14 +44,23 @@ struct DecodeArgs {
   int rows_per_split;  // C, a multiple of the tile rows
   int max_splits;      // ceil(kv_len_hint / C)
   float scale_log2;    // softmax scale * log2(e)
-  const uint16_t* q_rot;  // [B, Tq, H, d]
-  uint16_t* out;          // [B, Tq, H, d]
+  const uint16_t* q;   // [B, Tq, H, d]: rotated, or (fused decode) as projected
+  uint16_t* out;       // [B, Tq, H, d]
   const int32_t* start_pos;
   float* ws_o;   // [B*Tq, max_splits, H, d]   unnormalised partial outputs
   float* ws_ml;  // [B*Tq, max_splits, H, 2]   (running max in log2 units, sum)
-  int* counter;  // work counter (split path), reset by the launch; null: round-robin
+  int* counter;  // work counter (split path); null: round-robin
   int32_t* dev_status;
   int grid;      // persistent CTAs
+  // fused decode only (Tq = 1): the new token's K/V rows to rotate and append,
+  // the optional rotated-q output, and the self-resetting counters
+  const uint16_t* k_new;  // [B, 1, Hkv, d]
+  const uint16_t* v_new;  // [B, 1, Hkv, d]
+  uint16_t* cache_k;      // the same caches the tensor maps view
+  uint16_t* cache_v;
+  uint16_t* q_rot_out;    // [B, 1, H, d] or null
+  int* exit_counter;      // CTAs that finished (counter reset by the last)
+  int* merge_counter;     // [B, Hkv] splits finished per row set and KV head
 };
 
 struct DecodePlan {
@@ -55,7 +68,8 @@ struct DecodePlan {
   int max_splits;
   int grid;
   int ctas_per_sm;
-  size_t ws_bytes;
+  size_t ws_bytes;        // partials + work counter (unfused decode)
+  size_t fused_ws_bytes;  // partials + the counters of the fused decode
 };
 
 // Split size, persistent grid and workspace for these shapes on this device.
@@ -65,11 +79,15 @@ DecodePlan plan_decode(int B, int Tq, int H, int Hkv, int kv_len_hint, int sm_co
 // boxes of 64 elements x 64 rows (else plain boxes of 128 elements x 32 rows).
 bool decode_uses_tensor_cores(int G);
 
-// Points ws_o / ws_ml / counter of `a` into a workspace of plan.ws_bytes.
-void bind_decode_workspace(DecodeArgs& a, const DecodePlan& plan, void* workspace);
+// Points ws_o / ws_ml / counter (and, when `fused`, the fused decode's
+// counters) of `a` into a workspace of plan.ws_bytes (plan.fused_ws_bytes).
+void bind_decode_workspace(DecodeArgs& a, const DecodePlan& plan, void* workspace, bool fused = false);
 
+// Unfused attention (fused == null: q already rotated, cache rows already
+// appended) or the fused decode step (rope + append + attention + merge in
+// one launch, Tq = 1) with the frequency table `fused`.
 cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tmap_k, const CUtensorMap& tmap_v,
-                          cudaStream_t stream);
+                          cudaStream_t stream, const RopeTable* fused = nullptr);
 
 // Chunked prefill on tcgen05: one CTA per (128-row M tile, KV head, sequence).
 struct PrefillArgs {

@@ -15,6 +15,7 @@
 // moves B*T*(2H + 3Hkv)*256 bytes, a negligible share of a decode step.
 #include "kvattn_device.cuh"
 #include "kvattn_internal.h"
+#include "rope_device.cuh"
 
 namespace kvattn {
 namespace {
@@ -36,9 +37,8 @@ __global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(RopeAppendArg
   __shared__ double s_sin[kMaxRopePairs];
   const int rp = tab.rotary_dim / 2;  // rotated pairs
   for (int i = threadIdx.x; i < rp; i += blockDim.x) {
-    const double ang = (double)pos * tab.freq[i];
     double s, c;
-    sincos(ang, &s, &c);
+    rope_cos_sin(tab, i, pos, c, s);
     s_cos[i] = c;
     s_sin[i] = s;
   }
@@ -58,21 +58,16 @@ __global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(RopeAppendArg
       const int i = idx & (kPairs - 1);
       const bool is_q = idx < q_pairs;
       const uint32_t w = is_q ? q_in[idx] : k_in[idx - q_pairs];
-      const double x0 = (double)bf16lo_to_f32(w);
-      const double x1 = (double)bf16hi_to_f32(w);
-      const double c = s_cos[i], s = s_sin[i];
-      const double y0 = x0 * c - x1 * s;
-      const double y1 = x0 * s + x1 * c;
-      const uint32_t r = f64_to_bf16_bits(y0) | (f64_to_bf16_bits(y1) << 16);
+      uint16_t y0, y1;
+      rope_rotate_bits(true, s_cos[i], s_sin[i], (uint16_t)(w & 0xFFFFu), (uint16_t)(w >> 16), y0, y1);
+      const uint32_t r = (uint32_t)y0 | ((uint32_t)y1 << 16);
       if (is_q)
         q_out[idx] = r;
       else
         k_out[idx - q_pairs] = r;
     }
   } else {
-    // any layout / rotary width: slot j < rp rotates pair (a, b); slots
-    // j >= rp copy elements rd + 2(j - rp) and the next one unchanged
-    const int rd = 2 * rp;
+    // any layout / rotary width, one slot (pair or pass-through pair) at a time
     for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {
       const int vec = idx >> 6;
       const int j = idx & (kPairs - 1);
@@ -81,25 +76,12 @@ __global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(RopeAppendArg
                                 : reinterpret_cast<const uint16_t*>(k_in) + (size_t)(vec - a.H) * kHeadDim;
       uint16_t* outp = is_q ? reinterpret_cast<uint16_t*>(q_out) + (size_t)vec * kHeadDim
                             : reinterpret_cast<uint16_t*>(k_out) + (size_t)(vec - a.H) * kHeadDim;
-      int ea, eb;
-      if (j < rp) {
-        ea = tab.layout ? j : 2 * j;
-        eb = tab.layout ? j + rp : 2 * j + 1;
-      } else {
-        ea = rd + 2 * (j - rp);
-        eb = ea + 1;
-      }
-      const uint16_t xa = in[ea], xb = in[eb];
-      if (j < rp) {
-        const double x0 = (double)__uint_as_float((uint32_t)xa << 16);
-        const double x1 = (double)__uint_as_float((uint32_t)xb << 16);
-        const double c = s_cos[j], s = s_sin[j];
-        outp[ea] = (uint16_t)f64_to_bf16_bits(x0 * c - x1 * s);
-        outp[eb] = (uint16_t)f64_to_bf16_bits(x0 * s + x1 * c);
-      } else {
-        outp[ea] = xa;
-        outp[eb] = xb;
-      }
+      const RopeSlot sl = rope_slot(tab, j);
+      uint16_t ya, yb;
+      rope_rotate_bits(sl.rotate, sl.rotate ? s_cos[j] : 1.0, sl.rotate ? s_sin[j] : 0.0, in[sl.ea], in[sl.eb], ya,
+                       yb);
+      outp[sl.ea] = ya;
+      outp[sl.eb] = yb;
     }
   }
 
@@ -112,6 +94,9 @@ __global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(RopeAppendArg
 }  // namespace
 
 cudaError_t launch_rope_append(const RopeAppendArgs& a, const RopeTable& tab, cudaStream_t stream) {
+  // every tensor argument must have been set (callers value-initialise the args)
+  if (!a.q || !a.q_rot || !a.k_new || !a.v_new || !a.cache_k || !a.cache_v || !a.start_pos)
+    return cudaErrorInvalidValue;
   const long long blocks = (long long)a.B * a.T;
   if (blocks > 0x7FFFFFFFll) return cudaErrorInvalidValue;
   rope_append_kernel<<<(unsigned)blocks, kRopeThreads, 0, stream>>>(a, tab);

@@ -161,6 +161,39 @@ KVATTN_API int kvattn_decode(const kvattn_dims* dims, const uint16_t* q_rot, con
 KVATTN_API int kvattn_decode_plan(const kvattn_dims* dims, int32_t max_kv_len_hint, int32_t* rows_per_split,
                                   int32_t* max_splits, int32_t* grid, int32_t* ctas_per_sm);
 
+/* Bytes of device workspace kvattn_decode_fused needs for these dims and
+ * max_kv_len_hint on the CURRENT device (0: none needed, or invalid
+ * arguments). */
+KVATTN_API size_t kvattn_decode_fused_workspace_bytes(const kvattn_dims* dims, int32_t max_kv_len_hint);
+
+/* Steps 1-3 of one decode step in a single kernel launch (T = 1): the
+ * per-token work of "Llama 3 8B · KV cache" (rotate the new q and k at
+ * p = start_pos[b], write cache row p, attend rows 0..p) and the log-sum-exp
+ * merge of the split partials, with the results of kvattn_rope_append
+ * followed by kvattn_decode:
+ *   q_rot[b,0,h,:]   = RoPE_p(q[b,0,h,:])          (only if q_rot != NULL)
+ *   cache_k[b,p,j,:] = RoPE_p(k_new[b,0,j,:]),  cache_v[b,p,j,:] = v_new[b,0,j,:]
+ *   out[b,0,h,:]     = attention of RoPE_p(q[b,0,h,:]) over rows 0..p
+ * q, k_new, v_new are bf16 [B,1,H,d] / [B,1,Hkv,d]; q_rot may be NULL and
+ * must not be q (the kernel reads q until it ends).  Rows other than p are
+ * not written.  A sequence with start_pos[b] outside the cache or above the
+ * hint writes nothing (no cache row, no output) and sets its KVATTN_DEV_*
+ * bit.  rope, scale and max_kv_len_hint are as in kvattn_rope_append and
+ * kvattn_decode.
+ * workspace: kvattn_decode_fused_workspace_bytes() bytes, 16-byte aligned,
+ * owned by the caller (NULL allowed when that size is 0).  Unlike
+ * kvattn_decode's, it holds counters that must be ZERO before the first call
+ * (e.g. cudaMemset once after allocation); every call leaves them zero again
+ * when it completes, so no memset is needed between calls.  After a call
+ * that set KVATTN_DEV_WAIT_TIMEOUT, zero the workspace again.  Calls sharing
+ * a workspace must be ordered on one stream.
+ * Host errors: INVALID_ARG, UNSUPPORTED, OUT_OF_RANGE, WORKSPACE, CUDA. */
+KVATTN_API int kvattn_decode_fused(const kvattn_dims* dims, const kvattn_rope_params* rope, const uint16_t* q,
+                                   uint16_t* q_rot, const uint16_t* k_new, const uint16_t* v_new, uint16_t* cache_k,
+                                   uint16_t* cache_v, const int32_t* start_pos, int32_t max_kv_len_hint, float scale,
+                                   uint16_t* out, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                                   kvattn_stream_t stream);
+
 /* Size of the static device array behind kvattn_decode_noalloc: 64 MiB. */
 #define KVATTN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 
@@ -209,6 +242,11 @@ KVATTN_API int kvattn_prefill_chunk(const kvattn_dims* dims, int32_t T, const ui
 
 /* Human-readable name of a kvattn_status value. */
 KVATTN_API const char* kvattn_status_string(int status);
+
+/* The cudaError_t value behind the most recent KVATTN_ERR_CUDA returned on
+ * this host thread (0 if none yet), and its text. */
+KVATTN_API int kvattn_last_cuda_error(void);
+KVATTN_API const char* kvattn_last_cuda_error_string(void);
 
 /* Library version, major*10000 + minor*100 + patch. */
 KVATTN_API int kvattn_version(void);

@@ -126,3 +126,27 @@ def test_rope_layout_and_rotary_dim_validation(lib):
                 kv.RopeParams(rotary_dim=-2)):
         rope = bad.as_c()
         assert lib.kvattn_rope_append(ctypes.byref(d), ctypes.byref(rope), 1, *args, None, None) == 1
+
+
+def test_fused_decode_rejects_bad_args(lib):
+    d = _dims()
+    rope = kv.LLAMA3.as_c()
+    P7 = [FAKE] * 6  # k_new, v_new, cache_k, cache_v, start_pos
+    # q_rot aliasing q is refused (other items still read q)
+    assert lib.kvattn_decode_fused(ctypes.byref(d), ctypes.byref(rope), FAKE, FAKE, *P7[:5], 0, 0.0, FAKE, None, 0,
+                                   None, None) == 1
+    # a null q / out
+    assert lib.kvattn_decode_fused(ctypes.byref(d), ctypes.byref(rope), None, None, *P7[:5], 0, 0.0, FAKE, None, 0,
+                                   None, None) == 1
+    assert lib.kvattn_decode_fused(ctypes.byref(d), ctypes.byref(rope), FAKE, None, *P7[:5], 0, 0.0, None, None, 0,
+                                   None, None) == 1
+    # group size 32 is not built; a bad rope layout
+    d32 = _dims(n_kv_heads=1)
+    assert lib.kvattn_decode_fused(ctypes.byref(d32), ctypes.byref(rope), FAKE, None, *P7[:5], 0, 0.0, FAKE, None,
+                                   0, None, None) == 2
+    bad = kv.RopeParams(layout=5).as_c()
+    assert lib.kvattn_decode_fused(ctypes.byref(d), ctypes.byref(bad), FAKE, None, *P7[:5], 0, 0.0, FAKE, None, 0,
+                                   None, None) == 1
+    # hint beyond the cache
+    assert lib.kvattn_decode_fused(ctypes.byref(d), ctypes.byref(rope), FAKE, None, *P7[:5], 65, 0.0, FAKE, None, 0,
+                                   None, None) == 3
