@@ -4,9 +4,10 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
 One "step" is one pass of the whole hot path over one batch: for every layer,
-RoPE + cache append (kvattn_rope_append) then attention (kvattn_decode, or
-kvattn_prefill_chunk for the prefill workload), each layer with its own
-cache.  The default workload is batched ragged decode: B=64 sequences, 32
+RoPE + cache append (kvattn_rope_append) then attention (kvattn_decode: the
+split-K kernel and its LSE merge kernel, or kvattn_prefill_chunk for the
+prefill workload), each layer with its own cache.  --path fused times the
+single-launch kvattn_decode_fused instead.  The default workload is batched ragged decode: B=64 sequences, 32
 layers with separate [64, 8192, 8, 128] bf16 caches (64 GiB in HBM, far
 larger than L2, so every step streams its K/V rows from HBM), start positions
 uniform in [512, 8191].
@@ -56,6 +57,7 @@ def measured_peaks():
 
 KERNEL_SOURCES = {
     "decode_splitk": ("decode.cu", "kvattn_device.cuh"),
+    "decode_fused": ("decode.cu", "kvattn_device.cuh", "rope_device.cuh"),
     "prefill_chunk": ("prefill.cu", "kvattn_device.cuh"),
 }
 
@@ -192,7 +194,7 @@ class Layer:
     pass
 
 
-def build_state(w, seed, device):
+def build_state(w, seed, device, path="split"):
     import torch
     import gqa_decode_attention_kvattn_b200 as kv
     sp = w.start_pos(seed)
@@ -214,18 +216,34 @@ def build_state(w, seed, device):
         L.q_rot = torch.empty_like(L.q)
         L.out = torch.empty_like(L.q)
         layers.append(L)
-    if w.kind == "decode":
-        ws_bytes = kv.kvattn_decode_workspace_bytes(w.B, w.H, w.Hkv, w.S, w.kv_len_hint)
+    fused = w.kind == "decode" and path == "fused"
+    if fused:
+        ws_bytes = kv.kvattn_decode_fused_workspace_bytes(w.B, w.H, w.Hkv, w.S, w.kv_len_hint)
+        ws = kv.alloc_fused_workspace(ws_bytes, device)   # zeroed once; every call leaves it zeroed
     else:
-        ws_bytes = kv.kvattn_prefill_workspace_bytes(w.B, w.H, w.Hkv, w.S, w.T, w.kv_len_hint)
-    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=device)
+        if w.kind == "decode":
+            ws_bytes = kv.kvattn_decode_workspace_bytes(w.B, w.H, w.Hkv, w.S, w.kv_len_hint)
+        else:
+            ws_bytes = kv.kvattn_prefill_workspace_bytes(w.B, w.H, w.Hkv, w.S, w.T, w.kv_len_hint)
+        ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=device)
     status = torch.zeros(1, dtype=torch.int32, device=device)
     torch.cuda.synchronize(device)
-    return dict(sp=sp, dsp=dsp, rope=rope, layers=layers, ws=ws, ws_bytes=ws_bytes, status=status)
+    return dict(sp=sp, dsp=dsp, rope=rope, layers=layers, ws=ws, ws_bytes=ws_bytes, status=status, fused=fused)
 
 
 def run_step(w, st, events=None):
     import gqa_decode_attention_kvattn_b200 as kv
+    if st["fused"]:
+        # one launch per layer: rope + append + split-K attention + merge
+        for i, L in enumerate(st["layers"]):
+            if events is not None:
+                events[i][0].record()
+            kv.kvattn_decode_fused(L.q, L.k, L.v, L.ck, L.cv, st["dsp"], rope=st["rope"],
+                                   max_kv_len_hint=w.kv_len_hint, out=L.out, workspace=st["ws"],
+                                   dev_status=st["status"])
+            if events is not None:
+                events[i][1].record()
+        return
     for i, L in enumerate(st["layers"]):
         kv.kvattn_rope_append(L.q, L.k, L.v, L.ck, L.cv, st["dsp"], rope=st["rope"], q_rot=L.q_rot,
                               dev_status=st["status"])
@@ -331,10 +349,11 @@ def run_ours(args, w, rank, world, device):
     import torch.distributed as dist
     import gqa_decode_attention_kvattn_b200 as kv
 
-    st = build_state(w, args.seed, device)
+    st = build_state(w, args.seed, device, args.path)
     nl = len(st["layers"])
     kv_bytes_layer, flops_layer = work_units(w, st["sp"])
     merge = 1 if st["ws_bytes"] > 0 else 0
+    launches_per_layer = 1 if st["fused"] else 2 + merge
 
     # warm-up, eager
     for _ in range(args.warmup):
@@ -394,8 +413,9 @@ def run_ours(args, w, rank, world, device):
         achieved = kv_bytes_layer / (attn_avg_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                 "frac": round(achieved / hbm_peak, 4),
-                "traffic": profiled_traffic("decode_splitk", w.name),
-                "kernel": "kvattn_decode (split-K kernel + LSE merge kernel)",
+                "traffic": profiled_traffic("decode_fused" if st["fused"] else "decode_splitk", w.name),
+                "kernel": ("kvattn_decode_fused (rope + append + split-K attention + LSE merge, one kernel)"
+                           if st["fused"] else "kvattn_decode (split-K kernel + LSE merge kernel)"),
                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback 6650 GB/s",
                 "avg_launch_ms": round(attn_avg_ms, 5), "launches_timed": nl,
                 "bytes_per_launch": kv_bytes_layer}
@@ -428,12 +448,13 @@ def run_ours(args, w, rank, world, device):
                    "l2": "inputs larger than L2" if nl * w.B * w.S * w.Hkv * 512 > 256e6 else
                          "inputs smaller than L2 (latency-bound case)",
                    "graph": graph is not None,
+                   "path": "fused" if st["fused"] else "rope_append + " + ("decode" if w.kind == "decode" else "prefill"),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "pct_of_hbm_peak": round(100 * (value / world) / hbm_peak, 2) if w.kind == "decode" else None,
         "layer_steps_per_s": round(world * args.steps * nl / secs, 1),
         "steps_per_s": round(world * args.steps / secs, 2),
         "roofline": roof,
-        "gpu_launches": args.steps * nl * (2 + merge),
+        "gpu_launches": args.steps * nl * launches_per_layer,
         "clocks": clocks,
         "device_status": status,
     }
@@ -574,6 +595,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=HEADLINE)
     ap.add_argument("--seed", type=int, default=ks.DEFAULT_SEED)
+    ap.add_argument("--path", choices=["fused", "split"], default="split",
+                    help="decode entry points: rope_append + decode (+ merge kernel), the faster on B200 today, "
+                         "or one kvattn_decode_fused launch per layer")
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
