@@ -359,8 +359,10 @@ __device__ __forceinline__ void produce(const DecodeArgs& a, const RopeTable& ta
           rope_cos_sin(tab, lane + 32 * u, pos, cs[u], sn[u]);
         }
         if (it.r1 == it.L) {
-          const size_t src = ((size_t)it.b * a.Hkv + it.kvh) * kHeadDim;
-          const size_t dst = (((size_t)it.b * a.S + pos) * a.Hkv + it.kvh) * kHeadDim;
+          // (with G > 16 every group of the KV head writes the same bits)
+          const int kvp = it.kvh / a.kv_div;
+          const size_t src = ((size_t)it.b * a.Hkv_phys + kvp) * kHeadDim;
+          const size_t dst = (((size_t)it.b * a.S + pos) * a.Hkv_phys + kvp) * kHeadDim;
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             uint16_t ya, yb;
@@ -481,8 +483,9 @@ __global__ void __launch_bounds__(kThreads, Shape<G>::MIN_BLOCKS) decode_splitk_
       }
       produce<FUSED, G, kStages, kTileRows>(a, tab, sm, n_sets, total_items, 2 * kTileBytes, lane,
                                             [&](int st, const Item& it, int row) {
-        tma_load_4d(&sm.k[st][0][0], &tmap_k, &sm.full[st], 0, it.kvh, row, it.b, policy);
-        tma_load_4d(&sm.v[st][0][0], &tmap_v, &sm.full[st], 0, it.kvh, row, it.b, policy);
+        const int kvp = it.kvh / a.kv_div;  // the KV head in the cache
+        tma_load_4d(&sm.k[st][0][0], &tmap_k, &sm.full[st], 0, kvp, row, it.b, policy);
+        tma_load_4d(&sm.v[st][0][0], &tmap_v, &sm.full[st], 0, kvp, row, it.b, policy);
       });
     }
     return;
@@ -879,10 +882,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(
       }
       produce<FUSED, G, kMmaStages, kMmaTileRows>(a, tab, sm, n_sets, total_items, 4 * kMmaHalfBytes, lane,
                                                   [&](int st, const Item& it, int row) {
-        tma_load_4d(&sm.k[st][0][0], &tmap_k, &sm.full[st], 0, it.kvh, row, it.b, policy);
-        tma_load_4d(&sm.k[st][1][0], &tmap_k, &sm.full[st], 64, it.kvh, row, it.b, policy);
-        tma_load_4d(&sm.v[st][0][0], &tmap_v, &sm.full[st], 0, it.kvh, row, it.b, policy);
-        tma_load_4d(&sm.v[st][1][0], &tmap_v, &sm.full[st], 64, it.kvh, row, it.b, policy);
+        const int kvp = it.kvh / a.kv_div;  // the KV head in the cache
+        tma_load_4d(&sm.k[st][0][0], &tmap_k, &sm.full[st], 0, kvp, row, it.b, policy);
+        tma_load_4d(&sm.k[st][1][0], &tmap_k, &sm.full[st], 64, kvp, row, it.b, policy);
+        tma_load_4d(&sm.v[st][0][0], &tmap_v, &sm.full[st], 0, kvp, row, it.b, policy);
+        tma_load_4d(&sm.v[st][1][0], &tmap_v, &sm.full[st], 64, kvp, row, it.b, policy);
       });
     }
     return;

@@ -108,7 +108,8 @@ extern "C" KVATTN_API int kvattn_decode_noalloc(const kvattn_dims* dims, const u
     return KVATTN_ERR_INVALID_ARG;
   if (dims->head_dim != kHeadDim) return KVATTN_ERR_UNSUPPORTED;
   const int G = dims->n_heads / dims->n_kv_heads;
-  if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return KVATTN_ERR_UNSUPPORTED;
+  if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16 && G != 32 && G != 64 && G != 128)
+    return KVATTN_ERR_UNSUPPORTED;
   if (!q_rot || !cache_k || !cache_v || !start_pos || !out) return KVATTN_ERR_INVALID_ARG;
   if (!aligned16(q_rot) || !aligned16(cache_k) || !aligned16(cache_v) || !aligned16(out) ||
       (reinterpret_cast<uintptr_t>(start_pos) & 3u))
@@ -121,7 +122,9 @@ extern "C" KVATTN_API int kvattn_decode_noalloc(const kvattn_dims* dims, const u
   int sms = 0;
   int rc = sm_count(&sms);
   if (rc != KVATTN_OK) return rc;
-  const kvattn::DecodePlan plan = kvattn::plan_decode(dims->batch, 1, dims->n_heads, dims->n_kv_heads, hint, sms);
+  int groups = 0, kv_div = 1;
+  kvattn::decode_group_view(dims->n_heads, dims->n_kv_heads, &groups, &kv_div);
+  const kvattn::DecodePlan plan = kvattn::plan_decode(dims->batch, 1, dims->n_heads, groups, hint, sms);
   if (plan.ws_bytes > kScratchBytes) return KVATTN_ERR_WORKSPACE;  // needs more than the static array
 
   void* scratch = nullptr;
@@ -140,7 +143,9 @@ extern "C" KVATTN_API int kvattn_decode_noalloc(const kvattn_dims* dims, const u
   a.B = dims->batch;
   a.Tq = 1;
   a.H = dims->n_heads;
-  a.Hkv = dims->n_kv_heads;
+  a.Hkv = groups;
+  a.kv_div = kv_div;
+  a.Hkv_phys = dims->n_kv_heads;
   a.S = dims->max_seq_len;
   a.kv_len_hint = hint;
   a.rows_per_split = plan.rows_per_split;

@@ -34,7 +34,16 @@ constexpr int kHeadDim = 128;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-bool group_supported(int G) { return G == 1 || G == 2 || G == 4 || G == 8 || G == 16; }
+bool group_supported(int G) {
+  return G == 1 || G == 2 || G == 4 || G == 8 || G == 16 || G == 32 || G == 64 || G == 128;
+}
+
+// KV-head groups the decode kernels walk for these dims (see decode_group_view).
+int decode_groups(const kvattn_dims* d, int* kv_div) {
+  int groups = 0;
+  kvattn::decode_group_view(d->n_heads, d->n_kv_heads, &groups, kv_div);
+  return groups;
+}
 
 int check_dims(const kvattn_dims* d) {
   if (!d) return KVATTN_ERR_INVALID_ARG;
@@ -170,8 +179,9 @@ int run_attention(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, con
   int sms = 0;
   rc = current_sm_count(&sms);
   if (rc != KVATTN_OK) return rc;
-  const kvattn::DecodePlan plan =
-      kvattn::plan_decode(dims->batch, T, dims->n_heads, dims->n_kv_heads, hint, sms);
+  int kv_div = 1;
+  const int groups = decode_groups(dims, &kv_div);
+  const kvattn::DecodePlan plan = kvattn::plan_decode(dims->batch, T, dims->n_heads, groups, hint, sms);
   if (plan.ws_bytes > 0) {
     if (!workspace || workspace_bytes < plan.ws_bytes || !aligned16(workspace)) return KVATTN_ERR_WORKSPACE;
   }
@@ -192,7 +202,9 @@ int run_attention(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, con
   a.B = dims->batch;
   a.Tq = T;
   a.H = dims->n_heads;
-  a.Hkv = dims->n_kv_heads;
+  a.Hkv = groups;
+  a.kv_div = kv_div;
+  a.Hkv_phys = dims->n_kv_heads;
   a.S = dims->max_seq_len;
   a.kv_len_hint = hint;
   a.rows_per_split = plan.rows_per_split;
@@ -292,7 +304,8 @@ size_t kvattn_decode_workspace_bytes(const kvattn_dims* dims, int32_t max_kv_len
   if (hint > dims->max_seq_len || hint < 1) return 0;
   int sms = 0;
   if (current_sm_count(&sms) != KVATTN_OK) return 0;
-  return kvattn::plan_decode(dims->batch, 1, dims->n_heads, dims->n_kv_heads, hint, sms).ws_bytes;
+  int kv_div = 1;
+  return kvattn::plan_decode(dims->batch, 1, dims->n_heads, decode_groups(dims, &kv_div), hint, sms).ws_bytes;
 }
 
 int kvattn_decode(const kvattn_dims* dims, const uint16_t* q_rot, const uint16_t* cache_k, const uint16_t* cache_v,
@@ -308,7 +321,9 @@ size_t kvattn_decode_fused_workspace_bytes(const kvattn_dims* dims, int32_t max_
   if (hint > dims->max_seq_len || hint < 1) return 0;
   int sms = 0;
   if (current_sm_count(&sms) != KVATTN_OK) return 0;
-  return kvattn::plan_decode(dims->batch, 1, dims->n_heads, dims->n_kv_heads, hint, sms).fused_ws_bytes;
+  int kv_div = 1;
+  return kvattn::plan_decode(dims->batch, 1, dims->n_heads, decode_groups(dims, &kv_div), hint, sms)
+      .fused_ws_bytes;
 }
 
 int kvattn_decode_fused(const kvattn_dims* dims, const kvattn_rope_params* rope, const uint16_t* q,
@@ -336,7 +351,9 @@ int kvattn_decode_fused(const kvattn_dims* dims, const kvattn_rope_params* rope,
   int sms = 0;
   rc = current_sm_count(&sms);
   if (rc != KVATTN_OK) return rc;
-  const kvattn::DecodePlan plan = kvattn::plan_decode(dims->batch, 1, dims->n_heads, dims->n_kv_heads, hint, sms);
+  int kv_div = 1;
+  const int groups = decode_groups(dims, &kv_div);
+  const kvattn::DecodePlan plan = kvattn::plan_decode(dims->batch, 1, dims->n_heads, groups, hint, sms);
   if (plan.fused_ws_bytes > 0) {
     if (!workspace || workspace_bytes < plan.fused_ws_bytes || !aligned16(workspace)) return KVATTN_ERR_WORKSPACE;
   }
@@ -356,7 +373,9 @@ int kvattn_decode_fused(const kvattn_dims* dims, const kvattn_rope_params* rope,
   a.B = dims->batch;
   a.Tq = 1;
   a.H = dims->n_heads;
-  a.Hkv = dims->n_kv_heads;
+  a.Hkv = groups;
+  a.kv_div = kv_div;
+  a.Hkv_phys = dims->n_kv_heads;
   a.S = dims->max_seq_len;
   a.kv_len_hint = hint;
   a.rows_per_split = plan.rows_per_split;
@@ -403,7 +422,8 @@ int kvattn_decode_plan(const kvattn_dims* dims, int32_t max_kv_len_hint, int32_t
   int sms = 0;
   rc = current_sm_count(&sms);
   if (rc != KVATTN_OK) return rc;
-  const kvattn::DecodePlan p = kvattn::plan_decode(dims->batch, 1, dims->n_heads, dims->n_kv_heads, hint, sms);
+  int kv_div = 1;
+  const kvattn::DecodePlan p = kvattn::plan_decode(dims->batch, 1, dims->n_heads, decode_groups(dims, &kv_div), hint, sms);
   if (rows_per_split) *rows_per_split = p.rows_per_split;
   if (max_splits) *max_splits = p.max_splits;
   if (grid) *grid = p.grid;

@@ -39,7 +39,12 @@ cudaError_t launch_rope_append(const RopeAppendArgs& a, const RopeTable& tab, cu
 // (sequence, token) pair is a "query row set" of G heads per KV head; its
 // visible length is start_pos[b] + t + 1.
 struct DecodeArgs {
-  int B, Tq, H, Hkv, S;
+  int B, Tq, H;
+  int Hkv;       // KV-head groups the kernel walks: the KV heads, or for G > 16
+                 // kv_div groups of 16 query heads per KV head
+  int S;
+  int kv_div;    // groups per KV head (1 unless G > 16)
+  int Hkv_phys;  // KV heads in the caches and in k_new / v_new
   int kv_len_hint;     // upper bound on start_pos[b] + Tq
   int rows_per_split;  // C, a multiple of the tile rows
   int max_splits;      // ceil(kv_len_hint / C)
@@ -62,6 +67,16 @@ struct DecodeArgs {
   int* exit_counter;      // CTAs that finished (counter reset by the last)
   int* merge_counter;     // [B, Hkv] splits finished per row set and KV head
 };
+
+// Group view of the decode kernels: G <= 16 query heads per KV head run as
+// one group; G = 32, 64, 128 run as G/16 groups of 16 heads that read the
+// same KV head (neighbouring work items, so the second read of a row is
+// normally served by L2).
+inline void decode_group_view(int H, int Hkv, int* groups, int* kv_div) {
+  const int G = H / Hkv;
+  *kv_div = G > 16 ? G / 16 : 1;
+  *groups = Hkv * *kv_div;
+}
 
 struct DecodePlan {
   int rows_per_split;

@@ -534,6 +534,9 @@ cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& tq, const CU
     case 4: return launch_prefill_g<4>(a, tq, tk, tv, st);
     case 8: return launch_prefill_g<8>(a, tq, tk, tv, st);
     case 16: return launch_prefill_g<16>(a, tq, tk, tv, st);
+    case 32: return launch_prefill_g<32>(a, tq, tk, tv, st);
+    case 64: return launch_prefill_g<64>(a, tq, tk, tv, st);
+    case 128: return launch_prefill_g<128>(a, tq, tk, tv, st);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -57,7 +57,7 @@ typedef struct CUstream_st* kvattn_stream_t;
 typedef enum kvattn_status {
   KVATTN_OK = 0,
   KVATTN_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, H % Hkv != 0 */
-  KVATTN_ERR_UNSUPPORTED = 2, /* head_dim != 128, group size G = H/Hkv not in {1,2,4,8,16} */
+  KVATTN_ERR_UNSUPPORTED = 2, /* head_dim != 128, group size G = H/Hkv not in {1,2,4,...,128} */
   KVATTN_ERR_OUT_OF_RANGE = 3, /* a host-visible length outside the cache */
   KVATTN_ERR_WORKSPACE = 4,    /* workspace missing or smaller than required */
   KVATTN_ERR_CUDA = 5          /* a CUDA launch or query failed */
@@ -138,7 +138,9 @@ KVATTN_API size_t kvattn_decode_workspace_bytes(const kvattn_dims* dims, int32_t
  * The cache rows 0..start_pos[b] must already hold the sequence (row
  * start_pos[b] written by kvattn_rope_append earlier on the same stream).
  * The rows of each (sequence, KV head) are streamed from HBM once and serve
- * all G query heads; long rows are split across CTAs and the partial
+ * all G query heads (G = 32, 64, 128, e.g. multi-query attention, run as
+ * G/16 groups of 16 heads over the same rows, scheduled side by side so the
+ * repeat reads are served by L2); long rows are split across CTAs and the partial
  * (o, max, sum) triples are merged by log-sum-exp in a second kernel.
  * scale <= 0 selects 1/sqrt(d).  max_kv_len_hint (<= 0: max_seq_len) is a
  * host upper bound on start_pos[b] + 1; it sizes the splits and the

@@ -55,6 +55,9 @@ WORKLOADS = {
     "decode_wide_g8_b128": Workload(
         "decode_wide_g8_b128", B=128, T=1, H=64, Hkv=8, S=4096, sp_lo=1, sp_hi=4095,
         note="70B-style 64/8 heads (groups of 8)"),
+    "decode_mqa_g32_b64": Workload(
+        "decode_mqa_g32_b64", B=64, T=1, H=32, Hkv=1, S=32768, sp_lo=4096, sp_hi=32767,
+        note="multi-query attention: all 32 query heads share one KV head"),
 }
 
 # the workload the headline metric is quoted on

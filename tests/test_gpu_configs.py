@@ -48,6 +48,7 @@ def _sample(w, sp):
     ("prefill_b4_t512_sp3584", 0),
     ("decode_long_scaled_b8", 0),
     ("decode_wide_g8_b128", 0),
+    ("decode_mqa_g32_b64", 0),
 ])
 def test_workload_full_size(name, layer):
     w = WORKLOADS[name]

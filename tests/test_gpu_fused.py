@@ -45,6 +45,7 @@ CASES = [
     (3, 16, 8, 900, [0, 95, 857], kv.LLAMA3, 0),                    # G = 2
     (5, 64, 8, 2100, [1, 127, 128, 2047, 2099], kv.LLAMA3, 0),      # G = 8 (tensor cores)
     (3, 32, 2, 3000, [0, 63, 2999], kv.LLAMA3, 0),                  # G = 16 (tensor cores)
+    (3, 32, 1, 2500, [0, 1000, 2499], kv.LLAMA3, 0),                # G = 32 (MQA): two groups per KV head
     (2, 32, 8, 3000, [2999, 600], kv.RopeParams(layout=1), 0),      # half-split pairs
     (2, 32, 8, 3000, [2999, 600], kv.RopeParams(rotary_dim=64, use_scaled=True), 0),  # partial rotary
 ]
@@ -71,7 +72,7 @@ def test_fused_matches_oracle(case):
     U.assert_attention_close(g_out, out, f"fused B={B} H={H}/{Hkv} sp={sp}")
 
 
-@pytest.mark.parametrize("case", [CASES[1], CASES[3], CASES[6], CASES[7], CASES[8]])
+@pytest.mark.parametrize("case", [CASES[1], CASES[3], CASES[6], CASES[7], CASES[8], CASES[9]])
 def test_fused_equals_unfused_bitwise(case):
     """Same rotation, same tiles, same merge order: identical bits."""
     B, H, Hkv, S, sp, rope, hint = case

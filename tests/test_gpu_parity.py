@@ -57,6 +57,9 @@ def _check_step(seed, B, T, H, Hkv, S, sp, rope, kind, hint=0, in_place=False):
     (5, 64, 8, 520, [1, 127, 128, 511, 519], kv.LLAMA3),  # G = 8 (tensor cores)
     (3, 32, 2, 700, [0, 63, 64, 699][:3], kv.LLAMA3),     # G = 16 (tensor cores)
     (4, 64, 8, 3000, [2999, 64, 65, 1000], kv.LLAMA3_1),  # G = 8, several splits
+    (3, 32, 1, 2500, [0, 1000, 2499], kv.LLAMA3),       # G = 32 (MQA): two 16-head groups per KV head
+    (2, 64, 2, 1500, [1499, 700], kv.LLAMA3),           # G = 32 with two KV heads
+    (2, 64, 1, 900, [899, 33], kv.LLAMA3_1),            # G = 64 (MQA, 64 heads)
 ])
 def test_decode_step_small(case):
     B, H, Hkv, S, sp, rope = case
@@ -225,6 +228,9 @@ def test_prefill_equals_prefill_then_decode_steps():
     (2, 20, 64, 8, 300, [0, 129]),      # G=8: 16-token tiles
     (1, 130, 8, 8, 260, [127]),         # G=1 (MHA): 128-token tiles
     (2, 11, 32, 2, 150, [0, 120]),      # G=16: 8-token tiles
+    (2, 9, 32, 1, 300, [0, 200]),       # G=32 (MQA, 32 heads): 4-token tiles
+    (1, 5, 64, 1, 200, [150]),          # G=64 (MQA, 64 heads): 2-token tiles
+    (2, 3, 128, 1, 140, [7, 130]),      # G=128: one token per tile
     (3, 1, 32, 8, 300, [0, 127, 128]),  # one token per sequence through the prefill path
 ])
 def test_prefill_tiles_and_groups(case):

@@ -107,9 +107,10 @@ def test_rope_append_rejects_bad_pointers_and_params(lib):
 def test_attention_entry_points_reject_bad_args(lib):
     d = _dims()
     P = [FAKE] * 4
-    # group size 32/1 = 32 is not built
-    d32 = _dims(n_kv_heads=1)
-    assert lib.kvattn_decode(ctypes.byref(d32), *P, 0, 0.0, FAKE, None, 0, None, None) == 2
+    # group sizes that are not powers of two up to 128 are not built (48, 256)
+    for bad_g in (_dims(n_heads=48, n_kv_heads=1), _dims(n_heads=256, n_kv_heads=1)):
+        assert lib.kvattn_decode(ctypes.byref(bad_g), *P, 0, 0.0, FAKE, None, 0, None, None) == 2
+        assert lib.kvattn_prefill_chunk(ctypes.byref(bad_g), 1, *P, 0, 0.0, FAKE, None, 0, None, None) == 2
     # null output
     assert lib.kvattn_decode(ctypes.byref(d), *P, 0, 0.0, None, None, 0, None, None) == 1
     # hint beyond the cache
@@ -141,7 +142,7 @@ def test_fused_decode_rejects_bad_args(lib):
     assert lib.kvattn_decode_fused(ctypes.byref(d), ctypes.byref(rope), FAKE, None, *P7[:5], 0, 0.0, None, None, 0,
                                    None, None) == 1
     # group size 32 is not built; a bad rope layout
-    d32 = _dims(n_kv_heads=1)
+    d32 = _dims(n_heads=48, n_kv_heads=1)
     assert lib.kvattn_decode_fused(ctypes.byref(d32), ctypes.byref(rope), FAKE, None, *P7[:5], 0, 0.0, FAKE, None,
                                    0, None, None) == 2
     bad = kv.RopeParams(layout=5).as_c()
