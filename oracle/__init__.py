@@ -57,6 +57,10 @@ def _load():
         lib.oracle_attention.restype = ctypes.c_int
         lib.oracle_attention.argtypes = [ctypes.c_int] * 6 + [_i32p, ctypes.c_double, _u16p, _u16p,
                                                               _u16p, _f64p, ctypes.c_int]
+        lib.oracle_attention_masked.restype = ctypes.c_int
+        lib.oracle_attention_masked.argtypes = [ctypes.c_int] * 6 + [_i32p, ctypes.c_double, ctypes.c_int,
+                                                                     ctypes.c_int, ctypes.c_void_p, _u16p,
+                                                                     _u16p, _u16p, _f64p, ctypes.c_int]
         lib.oracle_f64_to_bf16.restype = ctypes.c_uint16
         lib.oracle_f64_to_bf16.argtypes = [ctypes.c_double]
         lib.oracle_bf16_to_f64.restype = ctypes.c_double
@@ -125,24 +129,39 @@ def rope_append(q, k_new, v_new, cache_k, cache_v, start_pos, freqs, want_exact=
     return q_rot, rc
 
 
-def attention(q_rot, cache_k, cache_v, start_pos, scale=None, n_threads=0):
-    """fp64 masked GQA softmax attention: returns (out [B,T,H,d] f64, rc)."""
+def attention(q_rot, cache_k, cache_v, start_pos, scale=None, n_threads=0, window=0, n_sink=0,
+              sink_logits=None):
+    """fp64 masked GQA softmax attention: returns (out [B,T,H,d] f64, rc).
+
+    window > 0: token at position p sees rows p-window < r <= p, plus the
+    first n_sink rows; sink_logits [H] (f64, or None): learned sink logits in
+    the units of the scaled scores, added to each head's softmax denominator."""
     B, T, H, d = q_rot.shape
     S, Hkv = cache_k.shape[1], cache_k.shape[2]
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     out = np.zeros((B, T, H, d), np.float64)
-    rc = _load().oracle_attention(B, T, H, Hkv, d, S, np.ascontiguousarray(start_pos, np.int32),
-                                  float(scale), np.ascontiguousarray(q_rot),
-                                  np.ascontiguousarray(cache_k), np.ascontiguousarray(cache_v),
-                                  out, int(n_threads))
+    args = (B, T, H, Hkv, d, S, np.ascontiguousarray(start_pos, np.int32), float(scale))
+    tail = (np.ascontiguousarray(q_rot), np.ascontiguousarray(cache_k), np.ascontiguousarray(cache_v), out,
+            int(n_threads))
+    if window <= 0 and sink_logits is None:
+        rc = _load().oracle_attention(*args, *tail)
+    else:
+        sl = None if sink_logits is None else np.ascontiguousarray(sink_logits, np.float64)
+        if sl is not None and sl.shape != (H,):
+            raise ValueError("sink_logits must have one entry per query head")
+        rc = _load().oracle_attention_masked(*args, int(window), int(n_sink),
+                                             None if sl is None else sl.ctypes.data, *tail)
     return out, rc
 
 
-def step(q, k_new, v_new, cache_k, cache_v, start_pos, freqs, scale=None, n_threads=0, layout=0, rotary_dim=0):
+def step(q, k_new, v_new, cache_k, cache_v, start_pos, freqs, scale=None, n_threads=0, layout=0, rotary_dim=0,
+         window=0, n_sink=0, sink_logits=None):
     """One whole cached-attention call: rope + append (caches updated in
-    place), then attention over rows 0..start_pos+t.  Returns (q_rot, out)."""
+    place), then attention over rows 0..start_pos+t (or the window and
+    sinks).  Returns (q_rot, out, rc)."""
     q_rot, rc = rope_append(q, k_new, v_new, cache_k, cache_v, start_pos, freqs, layout=layout,
                             rotary_dim=rotary_dim)
-    out, rc2 = attention(q_rot, cache_k, cache_v, start_pos, scale, n_threads)
+    out, rc2 = attention(q_rot, cache_k, cache_v, start_pos, scale, n_threads, window=window, n_sink=n_sink,
+                         sink_logits=sink_logits)
     return q_rot, out, max(rc, rc2)

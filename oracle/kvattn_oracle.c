@@ -45,6 +45,15 @@
  *     scale = 1/sqrt(d); w = softmax(s) with the maximum subtracted;
  *     out = sum_r w_r V_r -- all in fp64 ("Llama 3.1 8B KV cache", section
  *     "The cache itself is concatenation").  The output is fp64, unrounded.
+ *  6. Optional masks of "The Modern Decoder Block" (modules L7.5 and L7.7:
+ *     sliding window, StreamingLLM sinks, learned sinks).  The page names
+ *     them without defining them; the readings taken are the plain ones of
+ *     the cited works: with a window W > 0 the query at position p sees rows
+ *     p - W < r <= p; the first n_sink rows (attention sinks) stay visible as
+ *     well; positions stay absolute (rows are positions in this cache).  A
+ *     learned sink is one logit sigma_h per query head, in the units of the
+ *     scaled scores, that joins the softmax denominator and carries no value:
+ *     out = sum_r e^{s_r} V_r / (e^{sigma_h} + sum_r e^{s_r}).
  *
  * Layouts (the code layout of "Llama 3 8B · KV cache": [B, positions,
  * heads, d]): q, q_rot, out [B,T,H,d]; k_new, v_new [B,T,Hkv,d];
@@ -225,11 +234,15 @@ int oracle_rope_append(int B, int T, int H, int Hkv, int d, int S, const double*
  * as they stand (the caller has already appended the new rows).  Sequences
  * with start_pos < 0 or start_pos + T > S are skipped (out untouched) and the
  * call returns ORACLE_ERR_RANGE.  n_threads <= 0 uses every core. */
-int oracle_attention(int B, int T, int H, int Hkv, int d, int S, const int32_t* start_pos,
-                     double scale, const uint16_t* q_rot, const uint16_t* cache_k,
-                     const uint16_t* cache_v, double* out, int n_threads) {
+/* Attention with the optional masks of step 6: window <= 0 means no window,
+ * n_sink rows always visible when a window is set, sink_logits (length H,
+ * may be NULL) the learned sink logits. */
+int oracle_attention_masked(int B, int T, int H, int Hkv, int d, int S, const int32_t* start_pos,
+                            double scale, int window, int n_sink, const double* sink_logits,
+                            const uint16_t* q_rot, const uint16_t* cache_k, const uint16_t* cache_v,
+                            double* out, int n_threads) {
   if (B < 0 || T < 0 || H <= 0 || Hkv <= 0 || d <= 0 || S < 0) return ORACLE_ERR_ARG;
-  if (H % Hkv != 0) return ORACLE_ERR_ARG;
+  if (H % Hkv != 0 || n_sink < 0) return ORACLE_ERR_ARG;
   if (!start_pos || !q_rot || !cache_k || !cache_v || !out) return ORACLE_ERR_ARG;
   const int G = H / Hkv;
   int rc = ORACLE_OK;
@@ -247,7 +260,8 @@ int oracle_attention(int B, int T, int H, int Hkv, int d, int S, const int32_t* 
     const long sp = start_pos[b];
     if (sp < 0 || sp + T > S) continue;
     const int j = h / G;
-    const long L = sp + t + 1;
+    const long p = sp + t;          /* this token's position */
+    const long L = p + 1;           /* rows 0..p */
     const size_t qoff = (((size_t)b * T + t) * H + h) * d;
     double* qv = (double*)malloc(sizeof(double) * d);
     double* s = (double*)malloc(sizeof(double) * L);
@@ -255,14 +269,21 @@ int oracle_attention(int B, int T, int H, int Hkv, int d, int S, const int32_t* 
     for (int c = 0; c < d; ++c) qv[c] = bf16_to_f64(q_rot[qoff + c]);
     double m = -INFINITY;
     for (long r = 0; r < L; ++r) {
+      const int visible = window <= 0 || r > p - window || r < n_sink;
+      if (!visible) {
+        s[r] = -INFINITY;
+        continue;
+      }
       const uint16_t* kr = cache_k + (((size_t)b * S + r) * Hkv + j) * d;
       double dot = 0.0;
       for (int c = 0; c < d; ++c) dot += qv[c] * bf16_to_f64(kr[c]);
       s[r] = dot * scale;
       if (s[r] > m) m = s[r];
     }
-    double z = 0.0;
+    if (sink_logits && sink_logits[h] > m) m = sink_logits[h];
+    double z = sink_logits ? exp(sink_logits[h] - m) : 0.0;
     for (long r = 0; r < L; ++r) {
+      if (s[r] == -INFINITY) continue;
       const double w = exp(s[r] - m);
       z += w;
       const uint16_t* vr = cache_v + (((size_t)b * S + r) * Hkv + j) * d;
@@ -274,6 +295,14 @@ int oracle_attention(int B, int T, int H, int Hkv, int d, int S, const int32_t* 
     free(acc);
   }
   return rc;
+}
+
+/* Step 5: every row 0..start_pos[b]+t visible, no sink. */
+int oracle_attention(int B, int T, int H, int Hkv, int d, int S, const int32_t* start_pos,
+                     double scale, const uint16_t* q_rot, const uint16_t* cache_k,
+                     const uint16_t* cache_v, double* out, int n_threads) {
+  return oracle_attention_masked(B, T, H, Hkv, d, S, start_pos, scale, 0, 0, NULL, q_rot, cache_k, cache_v,
+                                 out, n_threads);
 }
 
 int oracle_max_threads(void) {

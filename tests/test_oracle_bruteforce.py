@@ -101,3 +101,36 @@ def test_bruteforce_tiny(seed):
                 z = sum(w)
                 o = [sum(w[r] * rows_v[r][c] for r in range(L)) / z for c in range(d)]
                 assert np.allclose(out[b, t, h], o, atol=1e-13)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_bruteforce_window_sinks(seed):
+    """Direct-softmax formula over an explicitly listed row set, with a learned
+    sink term in the denominator, against the oracle's masked attention."""
+    rnd = random.Random(100 + seed)
+    Hkv, G = rnd.choice([1, 2]), rnd.choice([1, 2, 4])
+    H, d, B, T, S = Hkv * G, rnd.choice([4, 8]), 2, rnd.choice([1, 3]), 16
+    sp = [rnd.randint(3, S - T) for _ in range(B)]
+    W, n_sink = rnd.randint(1, 6), rnd.randint(0, 3)
+    sig = [rnd.uniform(-2, 2) for _ in range(H)] if seed % 2 else None
+    q = ks.tensor_normal(seed, 11, (B, T, H, d))
+    ck = ks.cache_fill(seed, 14, B, S, Hkv, d, [s + T for s in sp])
+    cv = ks.cache_fill(seed, 15, B, S, Hkv, d, [s + T for s in sp])
+    scale = 1.0 / math.sqrt(d)
+    out, rc = oracle.attention(q, ck, cv, np.array(sp, np.int32), scale, window=W, n_sink=n_sink,
+                               sink_logits=None if sig is None else np.array(sig))
+    assert rc == 0
+    for b in range(B):
+        for t in range(T):
+            p = sp[b] + t
+            rows = [r for r in range(0, p + 1) if (p - r) < W or r < n_sink]
+            for h in range(H):
+                j = h // G
+                qv = [_bits_to_float(x) for x in q[b, t, h]]
+                s = [sum(a * _bits_to_float(c) for a, c in zip(qv, ck[b, r, j])) * scale for r in rows]
+                terms = s + ([sig[h]] if sig else [])
+                mx = max(terms)
+                w = [math.exp(x - mx) for x in s]
+                z = sum(w) + (math.exp(sig[h] - mx) if sig else 0.0)
+                o = [sum(w[i] * _bits_to_float(cv[b, r, j, c]) for i, r in enumerate(rows)) / z for c in range(d)]
+                assert np.allclose(out[b, t, h], o, atol=1e-13)

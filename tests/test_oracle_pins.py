@@ -367,3 +367,84 @@ def test_half_split_relative_offset():
     a = oracle.rope_rotate_f64(q, f, 40, layout=1) @ oracle.rope_rotate_f64(k, f, 10, layout=1)
     b = oracle.rope_rotate_f64(q, f, 1030, layout=1) @ oracle.rope_rotate_f64(k, f, 1000, layout=1)
     assert abs(a - b) <= 1e-10 * (1 + abs(a))
+
+
+# ---- sliding window, StreamingLLM sinks, learned sinks ("The Modern Decoder Block", L7.5 / L7.7)
+
+def _cache_inputs(seed=7, B=2, T=3, H=4, Hkv=2, d=8, S=40, sp=(20, 33)):
+    sp = np.array(sp, np.int32)
+    q, k, v, ck, cv = _inputs(B, T, H, Hkv, d, S, sp, seed=seed)
+    f = oracle.rope_freqs(d)
+    q_rot, rc = oracle.rope_append(q, k, v, ck, cv, sp, f)
+    assert rc == 0
+    return q_rot, ck, cv, sp
+
+
+def test_window_covering_everything_changes_nothing():
+    q_rot, ck, cv, sp = _cache_inputs()
+    ref, _ = oracle.attention(q_rot, ck, cv, sp)
+    for W, n in ((10**6, 0), (ck.shape[1], 3), (40, 40)):
+        out, rc = oracle.attention(q_rot, ck, cv, sp, window=W, n_sink=n)
+        assert rc == 0 and np.array_equal(out, ref)
+
+
+def test_window_one_returns_the_token_s_own_value():
+    q_rot, ck, cv, sp = _cache_inputs()
+    out, rc = oracle.attention(q_rot, ck, cv, sp, window=1)
+    assert rc == 0
+    V = ks.bf16_bits_to_f64(cv)
+    for b in range(2):
+        for t in range(3):
+            for h in range(4):
+                assert np.array_equal(out[b, t, h], V[b, sp[b] + t, h // 2])
+
+
+@pytest.mark.parametrize("W,n", [(5, 0), (5, 2), (1, 3), (17, 4), (8, 30)])
+def test_window_and_sinks_equal_plain_attention_over_the_gathered_rows(W, n):
+    """The visible rows of token t at position p are p-W < r <= p and r < n;
+    plain attention over a cache holding exactly those rows gives the same
+    output (an off-by-one in either bound changes the set)."""
+    q_rot, ck, cv, sp = _cache_inputs()
+    out, rc = oracle.attention(q_rot, ck, cv, sp, window=W, n_sink=n)
+    assert rc == 0
+    B, T, H, d = q_rot.shape
+    for b in range(B):
+        for t in range(T):
+            p = int(sp[b]) + t
+            rows = [r for r in range(p + 1) if r > p - W or r < n]
+            gk = ck[b:b + 1, rows]
+            gv = cv[b:b + 1, rows]
+            ref, rc2 = oracle.attention(q_rot[b:b + 1, t:t + 1], gk, gv, np.array([len(rows) - 1], np.int32))
+            assert rc2 == 0
+            assert np.allclose(out[b, t], ref[0, 0], atol=1e-15, rtol=0)
+
+
+def test_learned_sink_limits_and_closed_forms():
+    q_rot, ck, cv, sp = _cache_inputs()
+    H = q_rot.shape[2]
+    ref, _ = oracle.attention(q_rot, ck, cv, sp)
+    # a sink at -infinity takes no mass
+    out, rc = oracle.attention(q_rot, ck, cv, sp, sink_logits=np.full(H, -1e300))
+    assert rc == 0 and np.array_equal(out, ref)
+    # zero query: all scores 0, so out = mean(V) * L / (L + e^sigma)
+    qz = np.zeros_like(q_rot)
+    sig = np.array([-1.0, 0.0, 0.5, 2.0])
+    out, rc = oracle.attention(qz, ck, cv, sp, sink_logits=sig)
+    V = ks.bf16_bits_to_f64(cv)
+    for b in range(2):
+        for t in range(3):
+            L = int(sp[b]) + t + 1
+            for h in range(H):
+                expect = V[b, :L, h // 2].mean(axis=0) * L / (L + math.exp(sig[h]))
+                assert np.allclose(out[b, t, h], expect, atol=1e-14, rtol=1e-13)
+    # one visible row (window 1): out = V_p * e^s / (e^s + e^sigma)
+    out, rc = oracle.attention(q_rot, ck, cv, sp, window=1, sink_logits=sig)
+    Q = ks.bf16_bits_to_f64(q_rot)
+    K = ks.bf16_bits_to_f64(ck)
+    for b in range(2):
+        for t in range(3):
+            p = int(sp[b]) + t
+            for h in range(H):
+                s = float(Q[b, t, h] @ K[b, p, h // 2]) / math.sqrt(8)
+                wt = 1.0 / (1.0 + math.exp(sig[h] - s))
+                assert np.allclose(out[b, t, h], V[b, p, h // 2] * wt, atol=1e-14, rtol=1e-12)
