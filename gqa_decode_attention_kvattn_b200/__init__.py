@@ -47,6 +47,10 @@ class kvattn_dims(ctypes.Structure):
                 ("head_dim", ctypes.c_int32), ("max_seq_len", ctypes.c_int32)]
 
 
+class kvattn_attn_mask(ctypes.Structure):
+    _fields_ = [("window", ctypes.c_int32), ("n_sink", ctypes.c_int32), ("sink_logits", ctypes.c_void_p)]
+
+
 class kvattn_rope_params(ctypes.Structure):
     _fields_ = [("theta", ctypes.c_double), ("use_scaled", ctypes.c_int32), ("factor", ctypes.c_double),
                 ("low_freq_factor", ctypes.c_double), ("high_freq_factor", ctypes.c_double),
@@ -108,6 +112,15 @@ def _load():
     lib.kvattn_decode_fused.restype = ctypes.c_int
     lib.kvattn_decode_fused.argtypes = [dims_p, rope_p, P, P, P, P, P, P, P, ctypes.c_int32, ctypes.c_float, P, P,
                                         ctypes.c_size_t, P, P]
+    mask_p = ctypes.POINTER(kvattn_attn_mask)
+    lib.kvattn_decode_masked_workspace_bytes.restype = ctypes.c_size_t
+    lib.kvattn_decode_masked_workspace_bytes.argtypes = [dims_p, ctypes.c_int32, mask_p]
+    lib.kvattn_decode_masked.restype = ctypes.c_int
+    lib.kvattn_decode_masked.argtypes = [dims_p, P, P, P, P, ctypes.c_int32, ctypes.c_float, mask_p, P, P,
+                                         ctypes.c_size_t, P, P]
+    lib.kvattn_prefill_chunk_masked.restype = ctypes.c_int
+    lib.kvattn_prefill_chunk_masked.argtypes = [dims_p, ctypes.c_int32, P, P, P, P, ctypes.c_int32, ctypes.c_float,
+                                                mask_p, P, P, ctypes.c_size_t, P, P]
     lib.kvattn_prefill_workspace_bytes.restype = ctypes.c_size_t
     lib.kvattn_prefill_workspace_bytes.argtypes = [dims_p, ctypes.c_int32, ctypes.c_int32]
     lib.kvattn_prefill_chunk.restype = ctypes.c_int
@@ -244,12 +257,30 @@ def alloc_workspace(nbytes: int, device=None):
     return torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device or "cuda")
 
 
+def _mask(window, n_sink, sink_logits):
+    """kvattn_attn_mask for the optional masks, or None when none is set.
+    sink_logits: a float32 CUDA tensor [H] (learned sink logits)."""
+    if window <= 0 and sink_logits is None:
+        return None
+    if sink_logits is not None:
+        import torch
+        if sink_logits.dtype != torch.float32 or not sink_logits.is_cuda or not sink_logits.is_contiguous():
+            raise ValueError("sink_logits must be a contiguous float32 CUDA tensor [H]")
+    return kvattn_attn_mask(int(max(window, 0)), int(n_sink), None if sink_logits is None else sink_logits.data_ptr())
+
+
 def kvattn_decode(q_rot, cache_k, cache_v, start_pos, max_kv_len_hint: int = 0, scale: float = 0.0,
-                  out=None, workspace=None, dev_status=None, stream=None):
+                  out=None, workspace=None, dev_status=None, stream=None, window: int = 0, n_sink: int = 0,
+                  sink_logits=None):
     """Split-K GQA decode for one new token per sequence (see include/kvattn.h).
 
     q_rot [B,1,H,d]; returns out [B,1,H,d] bf16.  A workspace is allocated
-    with torch when none is given."""
+    with torch when none is given.  window / n_sink / sink_logits select the
+    masked entry point (sliding window, attention sinks, learned sinks)."""
+    mask = _mask(window, n_sink, sink_logits)
+    if mask is not None:
+        return _decode_masked(q_rot, cache_k, cache_v, start_pos, max_kv_len_hint, scale, mask, out, workspace,
+                              dev_status, stream)
     import torch
     lib = _load()
     _check_bf16("q_rot", q_rot, 4)
@@ -316,12 +347,47 @@ def kvattn_decode_fused(q, k_new, v_new, cache_k, cache_v, start_pos, rope: Rope
     return out
 
 
-def kvattn_prefill_chunk(q_rot, cache_k, cache_v, start_pos, max_kv_len_hint: int = 0, scale: float = 0.0,
-                         out=None, workspace=None, dev_status=None, stream=None):
-    """Chunked-prefill attention with the rectangular causal mask (see
-    include/kvattn.h).  q_rot [B,T,H,d]; returns out [B,T,H,d] bf16."""
+def _decode_masked(q_rot, cache_k, cache_v, start_pos, max_kv_len_hint, scale, mask, out, workspace, dev_status,
+                   stream):
     import torch
     lib = _load()
+    _check_bf16("q_rot", q_rot, 4)
+    _check_bf16("cache_k", cache_k, 4)
+    _check_bf16("cache_v", cache_v, 4)
+    if q_rot.shape[1] != 1:
+        raise ValueError("kvattn_decode takes one token per sequence (q_rot [B,1,H,d])")
+    dims = _dims_from_cache(q_rot, cache_k)
+    if out is None:
+        out = torch.empty_like(q_rot)
+    ws_bytes = int(lib.kvattn_decode_masked_workspace_bytes(ctypes.byref(dims), int(max_kv_len_hint),
+                                                            ctypes.byref(mask)))
+    if workspace is None and ws_bytes > 0:
+        workspace = alloc_workspace(ws_bytes, q_rot.device)
+    ws_size = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    rc = lib.kvattn_decode_masked(ctypes.byref(dims), _ptr(q_rot), _ptr(cache_k), _ptr(cache_v), _ptr(start_pos),
+                                  int(max_kv_len_hint), float(scale), ctypes.byref(mask), _ptr(out),
+                                  _ptr(workspace), ws_size, _ptr(dev_status), _stream(stream))
+    _check_status(rc, "kvattn_decode_masked")
+    return out
+
+
+def kvattn_decode_masked_workspace_bytes(batch, n_heads, n_kv_heads, max_seq_len, max_kv_len_hint=0, window=0,
+                                         n_sink=0, head_dim=HEAD_DIM) -> int:
+    dims = kvattn_dims(batch, n_heads, n_kv_heads, head_dim, max_seq_len)
+    mask = kvattn_attn_mask(int(window), int(n_sink), None)
+    return int(_load().kvattn_decode_masked_workspace_bytes(ctypes.byref(dims), int(max_kv_len_hint),
+                                                            ctypes.byref(mask)))
+
+
+def kvattn_prefill_chunk(q_rot, cache_k, cache_v, start_pos, max_kv_len_hint: int = 0, scale: float = 0.0,
+                         out=None, workspace=None, dev_status=None, stream=None, window: int = 0, n_sink: int = 0,
+                         sink_logits=None):
+    """Chunked-prefill attention with the rectangular causal mask (see
+    include/kvattn.h).  q_rot [B,T,H,d]; returns out [B,T,H,d] bf16.
+    window / n_sink / sink_logits select the masked entry point."""
+    import torch
+    lib = _load()
+    mask = _mask(window, n_sink, sink_logits)
     _check_bf16("q_rot", q_rot, 4)
     _check_bf16("cache_k", cache_k, 4)
     _check_bf16("cache_v", cache_v, 4)
@@ -333,9 +399,14 @@ def kvattn_prefill_chunk(q_rot, cache_k, cache_v, start_pos, max_kv_len_hint: in
     if workspace is None and ws_bytes > 0:
         workspace = alloc_workspace(ws_bytes, q_rot.device)
     ws_size = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    rc = lib.kvattn_prefill_chunk(ctypes.byref(dims), T, _ptr(q_rot), _ptr(cache_k), _ptr(cache_v),
-                                  _ptr(start_pos), int(max_kv_len_hint), float(scale), _ptr(out), _ptr(workspace),
-                                  ws_size, _ptr(dev_status), _stream(stream))
+    if mask is not None:
+        rc = lib.kvattn_prefill_chunk_masked(ctypes.byref(dims), T, _ptr(q_rot), _ptr(cache_k), _ptr(cache_v),
+                                             _ptr(start_pos), int(max_kv_len_hint), float(scale), ctypes.byref(mask),
+                                             _ptr(out), _ptr(workspace), ws_size, _ptr(dev_status), _stream(stream))
+    else:
+        rc = lib.kvattn_prefill_chunk(ctypes.byref(dims), T, _ptr(q_rot), _ptr(cache_k), _ptr(cache_v),
+                                      _ptr(start_pos), int(max_kv_len_hint), float(scale), _ptr(out),
+                                      _ptr(workspace), ws_size, _ptr(dev_status), _stream(stream))
     _check_status(rc, "kvattn_prefill_chunk")
     return out
 

@@ -110,17 +110,69 @@ struct __align__(128) Smem {
   uint64_t cons;  // the four consumer warps' epilogue barrier
 };
 
+// One work item: row set v = (b, t), split `split` of nsplit, KV-head group
+// kvh.  Rows are counted in a compacted (virtual) index u in [0, Lv): the
+// visible rows of the row set form at most two segments that start on
+// 64-row boundaries, u < a_len maps to row u (attention sinks) and u >= a_len
+// to row b0 + (u - a_len) (the window, ending at row L - 1).  Rows g0 <= r <
+// g1 inside those segments are not visible.  Without a window: a_len = b0 =
+// 0, Lv = L and no gap.
 struct Item {
-  int v, split, kvh, b, t, L, r0, r1, nsplit;
+  int v, split, kvh, b, t, L, Lv, a_len, b0, g0, g1, r0, r1, nsplit;
 };
 
-// Visible rows of row set v = (b, t), or 0 when its start position is out of
-// range; the number of splits of C rows it needs.
-__device__ __forceinline__ int set_length(const DecodeArgs& a, int v) {
+struct RowView {
+  int L, Lv, a_len, b0, g0, g1;
+};
+
+// Visible rows of row set v = (b, t) (Lv = 0 when its start position is out of
+// range or above the hint).
+template <bool WINDOW>
+__device__ __forceinline__ RowView row_view(const DecodeArgs& a, int v) {
+  RowView r{0, 0, 0, 0, 0, 0};
   const int b = v / a.Tq;
   const int sp = a.start_pos[b];
-  if (sp < 0 || (long long)sp + a.Tq > a.S || (long long)sp + a.Tq > a.kv_len_hint) return 0;
-  return sp + (v - b * a.Tq) + 1;
+  if (sp < 0 || (long long)sp + a.Tq > a.S || (long long)sp + a.Tq > a.kv_len_hint) return r;
+  r.L = sp + (v - b * a.Tq) + 1;
+  r.Lv = r.L;
+  if (!WINDOW || a.window <= 0 || r.L <= a.window) return r;
+  const int lo = r.L - a.window;        // first row of the window
+  const int ns = min(a.n_sink, lo);     // sink rows below it
+  const int lo_al = lo & ~63;
+  const int ns_al = (ns + 63) & ~63;
+  r.g0 = ns;
+  r.g1 = lo;
+  if (ns == 0) {
+    r.b0 = lo_al;                       // the window alone
+  } else if (ns_al < lo_al) {
+    r.a_len = ns_al;                    // sinks, then the window
+    r.b0 = lo_al;
+  }                                     // else one segment from row 0 with a short gap
+  r.Lv = r.a_len + (r.L - r.b0);
+  return r;
+}
+
+template <bool WINDOW>
+__device__ __forceinline__ int set_length(const DecodeArgs& a, int v) { return row_view<WINDOW>(a, v).Lv; }
+
+// the cache row of compacted index u
+__device__ __forceinline__ int item_row(const Item& it, int u) { return u < it.a_len ? u : it.b0 + (u - it.a_len); }
+
+// out = num / den, with a learned sink s2 (log2 units, -inf: none) added to
+// the denominator; num and den are relative to the reference max m.
+__device__ __forceinline__ float normalise_with_sink(float num, float den, float m, float s2) {
+  if (s2 != -INFINITY) {
+    const float mn = fmaxf(m, s2);
+    const float f = (m == -INFINITY) ? 0.f : fast_exp2(m - mn);
+    num *= f;
+    den = den * f + fast_exp2(s2 - mn);
+  }
+  return num / den;
+}
+
+// Learned sink of `head` in log2 units, or -inf.
+__device__ __forceinline__ float sink_log2(const DecodeArgs& a, int head) {
+  return a.sink_logits ? __ldg(a.sink_logits + head) * 1.4426950408889634f : -INFINITY;
 }
 
 // Item numbering.  Without splits (max_splits == 1): item i is row set
@@ -128,7 +180,7 @@ __device__ __forceinline__ int set_length(const DecodeArgs& a, int v) {
 // set (row-set major, KV head fastest), then the last split of each valid row
 // set in the order of sorted_set (largest first), so that work handed out
 // from a counter ends with the smallest pieces.
-template <class SM>
+template <bool WINDOW, class SM>
 __device__ __forceinline__ Item decode_item(const DecodeArgs& a, const SM& sm, int n_sets, int i) {
   Item it;
   const int C = a.rows_per_split;
@@ -136,8 +188,6 @@ __device__ __forceinline__ Item decode_item(const DecodeArgs& a, const SM& sm, i
     it.v = i / a.Hkv;
     it.kvh = i - it.v * a.Hkv;
     it.split = 0;
-    it.L = set_length(a, it.v);
-    it.nsplit = it.L > 0 ? 1 : 0;
   } else if (i < sm.n_full) {
     int lo = 0, hi = n_sets;  // largest v with full_start[v] <= i
     while (hi - lo > 1) {
@@ -148,26 +198,37 @@ __device__ __forceinline__ Item decode_item(const DecodeArgs& a, const SM& sm, i
     const int local = i - sm.full_start[lo];
     it.split = local / a.Hkv;
     it.kvh = local - it.split * a.Hkv;
-    it.L = sm.set_len[lo];
-    it.nsplit = (it.L + C - 1) / C;
   } else {
     const int r = (i - sm.n_full) / a.Hkv;
     it.kvh = (i - sm.n_full) - r * a.Hkv;
     it.v = sm.sorted_set[r];
-    it.L = sm.set_len[it.v];
-    it.nsplit = (it.L + C - 1) / C;
-    it.split = it.nsplit - 1;
+    it.split = -1;  // the last split, set below
   }
+  if constexpr (WINDOW) {
+    const RowView rv = row_view<true>(a, it.v);
+    it.L = rv.L;
+    it.Lv = rv.Lv;
+    it.a_len = rv.a_len;
+    it.b0 = rv.b0;
+    it.g0 = rv.g0;
+    it.g1 = rv.g1;
+  } else {
+    it.L = a.max_splits == 1 ? set_length<false>(a, it.v) : sm.set_len[it.v];
+    it.Lv = it.L;
+    it.a_len = it.b0 = it.g0 = it.g1 = 0;
+  }
+  it.nsplit = (it.Lv + C - 1) / C;
+  if (it.split < 0) it.split = it.nsplit - 1;
   it.b = it.v / a.Tq;
   it.t = it.v - it.b * a.Tq;
   it.r0 = it.split * C;
-  it.r1 = it.nsplit == 0 ? it.r0 : min(it.r0 + C, it.L);
+  it.r1 = it.nsplit == 0 ? it.r0 : min(it.r0 + C, it.Lv);
   return it;
 }
 
 // Warp 0 builds the work table of the split path (deterministically, so that
 // every CTA derives the same numbering).
-template <class SM>
+template <bool WINDOW, class SM>
 __device__ void build_work_table(const DecodeArgs& a, SM& sm, int n_sets, int lane) {
   const int C = a.rows_per_split;
   const int nb = C / kTileRows + 1;  // bucket k holds last splits of C/32 - k + ... tiles
@@ -179,7 +240,7 @@ __device__ void build_work_table(const DecodeArgs& a, SM& sm, int n_sets, int la
     const int v = base + lane;
     int L = 0, full = 0;
     if (v < n_sets) {
-      L = set_length(a, v);
+      L = set_length<WINDOW>(a, v);
       sm.set_len[v] = L;
       if (L > 0) {
         const int ns = (L + C - 1) / C;
@@ -251,7 +312,7 @@ __device__ __forceinline__ float lse_merge_element(const DecodeArgs& a, int v, i
     den = den * f_old + ml.y * f_new;
     M = Mn;
   }
-  return num / den;
+  return normalise_with_sink(num, den, M, sink_log2(a, head));
 }
 
 // Fused decode, after the four consumer warps stored an item's partials: the
@@ -294,7 +355,7 @@ __device__ __forceinline__ void merge_if_last(const DecodeArgs& a, const Item& i
 // rotates the new K row and writes it, and the new V row, to cache row p,
 // then fences the generic-proxy stores against the tensor copies that read
 // that row back.  Only that item reads row p, so no other CTA waits on it.
-template <bool FUSED, int G, int STAGES, int TILE_ROWS, class SM, class Load>
+template <bool FUSED, bool WINDOW, int G, int STAGES, int TILE_ROWS, class SM, class Load>
 __device__ __forceinline__ void produce(const DecodeArgs& a, const RopeTable& tab, SM& sm, int n_sets,
                                         int total_items, uint32_t tile_bytes, int lane, Load&& load) {
   constexpr uint32_t kQBytes = G * kHeadDim * 2;
@@ -328,7 +389,7 @@ __device__ __forceinline__ void produce(const DecodeArgs& a, const RopeTable& ta
       if (++stage == STAGES) { stage = 0; phase ^= 1; }
       break;
     }
-    const Item it = decode_item(a, sm, n_sets, i);
+    const Item it = decode_item<WINDOW>(a, sm, n_sets, i);
     if (it.nsplit == 0) continue;  // invalid row set: nothing to stream
     for (int row = it.r0; row < it.r1; row += TILE_ROWS) {
       int ok = 1;
@@ -347,7 +408,7 @@ __device__ __forceinline__ void produce(const DecodeArgs& a, const RopeTable& ta
             const uint16_t* qsrc = a.q + (((size_t)it.b * a.Tq + it.t) * a.H + (size_t)it.kvh * G) * kHeadDim;
             bulk_load(&sm.q[stage][0][0], qsrc, kQBytes, &sm.full[stage]);
           }
-          load(stage, it, row);
+          load(stage, it, item_row(it, row));
         }
       } else {
         const long long pos = it.L - 1;
@@ -358,7 +419,7 @@ __device__ __forceinline__ void produce(const DecodeArgs& a, const RopeTable& ta
           sl[u] = rope_slot(tab, lane + 32 * u);
           rope_cos_sin(tab, lane + 32 * u, pos, cs[u], sn[u]);
         }
-        if (it.r1 == it.L) {
+        if (it.r1 == it.Lv) {  // the last split: its last row is the new one
           // (with G > 16 every group of the KV head writes the same bits)
           const int kvp = it.kvh / a.kv_div;
           const size_t src = ((size_t)it.b * a.Hkv_phys + kvp) * kHeadDim;
@@ -378,7 +439,7 @@ __device__ __forceinline__ void produce(const DecodeArgs& a, const RopeTable& ta
         if (leader) {
           sm.stage_item[stage] = i;
           mbar_expect_tx(&sm.full[stage], tile_bytes);
-          load(stage, it, row);
+          load(stage, it, item_row(it, row));
         }
         const size_t qoff = ((size_t)it.b * a.H + (size_t)it.kvh * G) * kHeadDim;
         uint16_t* qout = (a.q_rot_out && it.split == 0) ? a.q_rot_out + qoff : nullptr;
@@ -425,7 +486,7 @@ __device__ __forceinline__ void produce(const DecodeArgs& a, const RopeTable& ta
   }
 }
 
-template <int G, bool FUSED>
+template <int G, bool FUSED, bool WINDOW>
 __global__ void __launch_bounds__(kThreads, Shape<G>::MIN_BLOCKS) decode_splitk_kernel(
     const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
     const DecodeArgs a, const int evict_first, const __grid_constant__ RopeTable tab) {
@@ -447,11 +508,11 @@ __global__ void __launch_bounds__(kThreads, Shape<G>::MIN_BLOCKS) decode_splitk_
     if (a.max_splits == 1) {
       if (lane == 0) sm.total_items = n_sets * a.Hkv;
     } else {
-      build_work_table(a, sm, n_sets, lane);
+      build_work_table<WINDOW>(a, sm, n_sets, lane);
     }
     if (blockIdx.x == 0) {
       for (int v = lane; v < n_sets; v += 32) {
-        if (set_length(a, v) == 0) {
+        if (set_length<WINDOW>(a, v) == 0) {
           const int sp = a.start_pos[v / a.Tq];
           set_status(a.dev_status, (sp < 0 || (long long)sp + a.Tq > a.S) ? KVATTN_DEV_START_POS_RANGE
                                                                          : KVATTN_DEV_KV_LEN_HINT);
@@ -481,7 +542,7 @@ __global__ void __launch_bounds__(kThreads, Shape<G>::MIN_BLOCKS) decode_splitk_
         if (evict_first) policy = l2_policy_evict_first();
         else asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(policy));
       }
-      produce<FUSED, G, kStages, kTileRows>(a, tab, sm, n_sets, total_items, 2 * kTileBytes, lane,
+      produce<FUSED, WINDOW, G, kStages, kTileRows>(a, tab, sm, n_sets, total_items, 2 * kTileBytes, lane,
                                             [&](int st, const Item& it, int row) {
         const int kvp = it.kvh / a.kv_div;  // the KV head in the cache
         tma_load_4d(&sm.k[st][0][0], &tmap_k, &sm.full[st], 0, kvp, row, it.b, policy);
@@ -530,7 +591,7 @@ __global__ void __launch_bounds__(kThreads, Shape<G>::MIN_BLOCKS) decode_splitk_
       if (lane == 0) mbar_arrive(&sm.empty[stage]);
       break;
     }
-    const Item it = decode_item(a, sm, n_sets, i);
+    const Item it = decode_item<WINDOW>(a, sm, n_sets, i);
     uint64_t q2[G][4];  // q of the G heads, scaled into log2 units (read at the first tile)
     uint64_t o2[G][4];
 #pragma unroll
@@ -554,6 +615,14 @@ __global__ void __launch_bounds__(kThreads, Shape<G>::MIN_BLOCKS) decode_splitk_
       }
       const uint16_t* Kt = &sm.k[stage][0][0];
       const uint16_t* Vt = &sm.v[stage][0][0];
+      // rows of this tile that are not visible: past the item, or in the gap
+      // between the attention sinks and the window
+      // (the window kernels also hide the rows between the sinks and the window)
+      const int act = WINDOW ? item_row(it, row) : row;
+      auto hidden = [&](int k) {
+        if constexpr (WINDOW) return row + k >= it.r1 || (act + k >= it.g0 && act + k < it.g1);
+        else return row + k >= it.r1;
+      };
       // One batch: RB rows per half-warp.  MASKED is true only on the last
       // tile of an item, where some rows may lie past the item's end.
       auto batch = [&](int pass, auto masked_tag) {
@@ -593,7 +662,7 @@ __global__ void __launch_bounds__(kThreads, Shape<G>::MIN_BLOCKS) decode_splitk_
           for (int k = 0; k < w; ++k) col[k] += col[k + w];
         float sc = col[0];
         if constexpr (MASKED) {
-          if (row + rbase + (slot_n0 & (Sh::RB - 1)) >= it.r1) sc = -INFINITY;
+          if (hidden(rbase + (slot_n0 & (Sh::RB - 1)))) sc = -INFINITY;
         }
 
         // ---- online softmax in log2 units with a lazily moved reference:
@@ -635,8 +704,8 @@ __global__ void __launch_bounds__(kThreads, Shape<G>::MIN_BLOCKS) decode_splitk_
           uint4 va = lds128(Vt + (rbase + j) * kHeadDim + 8 * l16);
           uint4 vb = lds128(Vt + (rbase + j + 1) * kHeadDim + 8 * l16);
           if constexpr (MASKED) {
-            const bool ok0 = row + rbase + j < it.r1;
-            const bool ok1 = row + rbase + j + 1 < it.r1;
+            const bool ok0 = !hidden(rbase + j);
+            const bool ok1 = !hidden(rbase + j + 1);
             va.x = ok0 ? va.x : 0u; va.y = ok0 ? va.y : 0u; va.z = ok0 ? va.z : 0u; va.w = ok0 ? va.w : 0u;
             vb.x = ok1 ? vb.x : 0u; vb.y = ok1 ? vb.y : 0u; vb.z = ok1 ? vb.z : 0u; vb.w = ok1 ? vb.w : 0u;
           }
@@ -657,7 +726,7 @@ __global__ void __launch_bounds__(kThreads, Shape<G>::MIN_BLOCKS) decode_splitk_
         }
         pbuf ^= 1;
       };
-      if (row + kTileRows <= it.r1) {
+      if (row + kTileRows <= it.r1 && !(WINDOW && act < it.g1 && act + kTileRows > it.g0)) {
 #pragma unroll
         for (int pass = 0; pass < Sh::PASSES; ++pass) batch(pass, std::false_type{});
       } else {
@@ -727,7 +796,7 @@ __global__ void __launch_bounds__(kThreads, Shape<G>::MIN_BLOCKS) decode_splitk_
           if (mk != -INFINITY) Ls += sm.merge_l[k][h] * fast_exp2(mk - Mh[h]);
         }
         const int head = it.kvh * G + h;
-        if (it.nsplit == 1) {
+        if (it.nsplit == 1 && !a.sink_logits) {
           const float r = o / Ls;
           const uint32_t bits = f32_to_bf16_bits(r);
           a.out[(((size_t)it.b * a.Tq + it.t) * a.H + head) * kHeadDim + c] = (uint16_t)bits;
@@ -753,9 +822,9 @@ __global__ void __launch_bounds__(kThreads, Shape<G>::MIN_BLOCKS) decode_splitk_
 __global__ void __launch_bounds__(kHeadDim) decode_merge_kernel(const DecodeArgs a) {
   const int head = blockIdx.x;
   const int v = blockIdx.y;
-  const int L = set_length(a, v);
+  const int L = set_length<true>(a, v);
   const int ns = (L + a.rows_per_split - 1) / a.rows_per_split;
-  if (L == 0 || ns <= 1) return;  // invalid, or written directly by K2
+  if (L == 0 || (ns <= 1 && !a.sink_logits)) return;  // invalid, or written directly by K2
   const int b = v / a.Tq, t = v - b * a.Tq;
   const int c = threadIdx.x;
   const float r = lse_merge_element(a, v, head, ns, c);
@@ -824,7 +893,7 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int chunk) {
   return (uint32_t)(row * 128 + (((chunk ^ row) & 7) << 4));
 }
 
-template <int G, bool FUSED>
+template <int G, bool FUSED, bool WINDOW>
 __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(
     const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
     const DecodeArgs a, const int evict_first, const __grid_constant__ RopeTable tab) {
@@ -846,11 +915,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(
     if (a.max_splits == 1) {
       if (lane == 0) sm.total_items = n_sets * a.Hkv;
     } else {
-      build_work_table(a, sm, n_sets, lane);
+      build_work_table<WINDOW>(a, sm, n_sets, lane);
     }
     if (blockIdx.x == 0) {
       for (int v = lane; v < n_sets; v += 32) {
-        if (set_length(a, v) == 0) {
+        if (set_length<WINDOW>(a, v) == 0) {
           const int sp = a.start_pos[v / a.Tq];
           set_status(a.dev_status, (sp < 0 || (long long)sp + a.Tq > a.S) ? KVATTN_DEV_START_POS_RANGE
                                                                          : KVATTN_DEV_KV_LEN_HINT);
@@ -880,7 +949,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(
         if (evict_first) policy = l2_policy_evict_first();
         else asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(policy));
       }
-      produce<FUSED, G, kMmaStages, kMmaTileRows>(a, tab, sm, n_sets, total_items, 4 * kMmaHalfBytes, lane,
+      produce<FUSED, WINDOW, G, kMmaStages, kMmaTileRows>(a, tab, sm, n_sets, total_items, 4 * kMmaHalfBytes, lane,
                                                   [&](int st, const Item& it, int row) {
         const int kvp = it.kvh / a.kv_div;  // the KV head in the cache
         tma_load_4d(&sm.k[st][0][0], &tmap_k, &sm.full[st], 0, kvp, row, it.b, policy);
@@ -915,7 +984,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(
       if (lane == 0) mbar_arrive(&sm.empty[stage]);
       break;
     }
-    const Item it = decode_item(a, sm, n_sets, i);
+    const Item it = decode_item<WINDOW>(a, sm, n_sets, i);
 
     // q as A fragments (rows = heads g and g+8, columns = head dims)
     uint32_t qa[8][4];
@@ -947,13 +1016,19 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(
       }
       const uint32_t kbase = smem_u32(&sm.k[stage][0][0]);
       const uint32_t vbase = smem_u32(&sm.v[stage][0][0]);
-      const bool masked = row + kMmaTileRows > it.r1;
+      // (the window kernels also hide the rows between the sinks and the window)
+      const int act = WINDOW ? item_row(it, row) : row;
+      auto hidden = [&](int k) {
+        if constexpr (WINDOW) return row + k >= it.r1 || (act + k >= it.g0 && act + k < it.g1);
+        else return row + k >= it.r1;
+      };
+      const bool masked = row + kMmaTileRows > it.r1 || (WINDOW && act < it.g1 && act + kMmaTileRows > it.g0);
       if (masked) {
         // rows of this warp past the item may hold any bits; zero their V so
         // that no 0 * NaN reaches O (the warp reads only its own 16 rows)
         for (int x = lane; x < 16 * 16; x += 32) {
           const int r = wrow + (x >> 4);
-          if (row + r >= it.r1) {
+          if (hidden(r)) {
             const int half = (x >> 3) & 1, ch = x & 7;
             *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(&sm.v[stage][half][0]) + r * 128 + ch * 16) =
                 make_uint4(0u, 0u, 0u, 0u);
@@ -993,7 +1068,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(
           for (int e = 0; e < 2; ++e) {
             const int rr = row + wrow + 8 * nt + 2 * c4 + e;
             const float x = sacc[nt][2 * hh + e] * a.scale_log2;
-            sv[2 * nt + e] = (masked && rr >= it.r1) ? -INFINITY : x;
+            sv[2 * nt + e] = (masked && hidden(rr - row)) ? -INFINITY : x;
           }
         float tmax = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
         tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
@@ -1077,7 +1152,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(
           Ls += f * sm.merge_l[w][h];
         }
         const int head = it.kvh * G + h;
-        if (it.nsplit == 1) {
+        if (it.nsplit == 1 && !a.sink_logits) {
           a.out[(((size_t)it.b * a.Tq + it.t) * a.H + head) * kHeadDim + c] = (uint16_t)f32_to_bf16_bits(o_sum / Ls);
         } else {
           const size_t slot = ((size_t)it.v * a.max_splits + it.split) * a.H + head;
@@ -1106,10 +1181,10 @@ size_t smem_bytes() {
   return sizeof(Smem<G>);
 }
 
-template <int G, bool FUSED>
+template <int G, bool FUSED, bool WINDOW>
 auto decode_kernel() {
-  if constexpr (G >= 8) return decode_mma_kernel<G, FUSED>;
-  else return decode_splitk_kernel<G, FUSED>;
+  if constexpr (G >= 8) return decode_mma_kernel<G, FUSED, WINDOW>;
+  else return decode_splitk_kernel<G, FUSED, WINDOW>;
 }
 
 template <int G>
@@ -1118,10 +1193,10 @@ size_t decode_smem_bytes() {
   else return smem_bytes<G>();
 }
 
-template <int G, bool FUSED>
+template <int G, bool FUSED, bool WINDOW>
 cudaError_t launch_g(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, const RopeTable& tab,
                      cudaStream_t st) {
-  auto kernel = decode_kernel<G, FUSED>();
+  auto kernel = decode_kernel<G, FUSED, WINDOW>();
   const size_t smem = decode_smem_bytes<G>();
   static bool configured[64] = {false};
   int dev = 0;
@@ -1142,7 +1217,7 @@ cudaError_t launch_g(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorM
   kernel<<<a.grid, kThreads, smem, st>>>(tk, tv, a, evict_first, tab);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (!FUSED && a.max_splits > 1) {
+  if (!FUSED && (a.max_splits > 1 || a.sink_logits)) {
     dim3 grid(a.H, a.B * a.Tq);
     decode_merge_kernel<<<grid, kHeadDim, 0, st>>>(a);
     e = cudaGetLastError();
@@ -1153,18 +1228,19 @@ cudaError_t launch_g(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorM
 template <int G>
 cudaError_t launch_g(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st,
                      const RopeTable* fused) {
-  if (fused) return launch_g<G, true>(a, tk, tv, *fused, st);
+  if (fused) return launch_g<G, true, false>(a, tk, tv, *fused, st);
   RopeTable unused{};
-  return launch_g<G, false>(a, tk, tv, unused, st);
+  if (a.window > 0) return launch_g<G, false, true>(a, tk, tv, unused, st);
+  return launch_g<G, false, false>(a, tk, tv, unused, st);
 }
 
 }  // namespace
 
 // Resident CTAs per SM of the decode kernel for group size G (occupancy
 // query: registers and shared memory both count).
-template <int G, bool FUSED>
+template <int G, bool FUSED, bool WINDOW>
 int resident_ctas_of() {
-  auto kernel = decode_kernel<G, FUSED>();
+  auto kernel = decode_kernel<G, FUSED, WINDOW>();
   const size_t smem = decode_smem_bytes<G>();
   int n = 0;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess ||
@@ -1173,10 +1249,11 @@ int resident_ctas_of() {
   return n;
 }
 
-// the persistent grid serves both the unfused and the fused kernel
+// the persistent grid serves the unfused, the fused and the window kernels
 template <int G>
 int resident_ctas() {
-  return std::min(resident_ctas_of<G, false>(), resident_ctas_of<G, true>());
+  return std::min(std::min(resident_ctas_of<G, false, false>(), resident_ctas_of<G, true, false>()),
+                  resident_ctas_of<G, false, true>());
 }
 
 int resident_ctas_for(int G) {
@@ -1198,7 +1275,7 @@ int resident_ctas_for(int G) {
   return n;
 }
 
-DecodePlan plan_decode(int B, int Tq, int H, int Hkv, int kv_len_hint, int sm_count) {
+DecodePlan plan_decode(int B, int Tq, int H, int Hkv, int kv_len_hint, int sm_count, bool always_partials) {
   DecodePlan p;
   const int G = H / Hkv;
   const int ctas_per_sm = resident_ctas_for(G);
@@ -1221,8 +1298,9 @@ DecodePlan plan_decode(int B, int Tq, int H, int Hkv, int kv_len_hint, int sm_co
   p.grid = (int)std::min<long long>(items_bound, slots);
   if (p.grid < 1) p.grid = 1;
   // partial (o, max, sum) per (row set, split, head), then the work counter
-  p.ws_bytes =
-      p.max_splits > 1 ? (size_t)row_sets * p.max_splits * H * (kHeadDim + 2) * sizeof(float) + 16 : 0;
+  p.ws_bytes = (p.max_splits > 1 || always_partials)
+                   ? (size_t)row_sets * p.max_splits * H * (kHeadDim + 2) * sizeof(float) + 16
+                   : 0;
   // fused: the same, then (work, exit) counters and one merge counter per
   // (row set, KV head), padded to 16 bytes
   p.fused_ws_bytes = p.max_splits > 1 ? p.ws_bytes + (((size_t)row_sets * Hkv * sizeof(int) + 15) & ~(size_t)15) : 0;
@@ -1253,7 +1331,9 @@ cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tk, const CUte
                           const RopeTable* fused) {
   // every tensor argument the chosen kernel dereferences must have been set
   if (!a.q || !a.out || !a.start_pos) return cudaErrorInvalidValue;
-  if (a.max_splits > 1 && (!a.ws_o || !a.ws_ml)) return cudaErrorInvalidValue;
+  if ((a.max_splits > 1 || a.sink_logits) && (!a.ws_o || !a.ws_ml)) return cudaErrorInvalidValue;
+  if (fused && a.sink_logits) return cudaErrorInvalidValue;  // the fused decode has no learned sinks
+  if (fused && a.window > 0) return cudaErrorInvalidValue;  // the fused decode has no window
   if (fused && (a.Tq != 1 || !a.k_new || !a.v_new || !a.cache_k || !a.cache_v ||
                 (a.counter && (!a.exit_counter || !a.merge_counter))))
     return cudaErrorInvalidValue;

@@ -141,6 +141,27 @@ int encode_cache_map(CUtensorMap* map, const void* base, int B, int S, int Hkv, 
 
 int hint_or_default(int32_t hint, int S) { return hint <= 0 ? S : hint; }
 
+int check_mask(const kvattn_attn_mask* m) {
+  if (!m) return KVATTN_OK;
+  if (m->window < 0 || m->n_sink < 0) return KVATTN_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(m->sink_logits) & 3u) return KVATTN_ERR_INVALID_ARG;
+  return KVATTN_OK;
+}
+
+// Rows a sequence can have visible: the hint, or with a window at most the
+// window plus the 64-row-aligned sink segment and one tile of alignment.
+int visible_len_bound(int hint, const kvattn_attn_mask* m) {
+  if (!m || m->window <= 0) return hint;
+  const long long bound = (long long)m->window + (((long long)m->n_sink + 63) & ~63ll) + 64;
+  return bound < hint ? (int)bound : hint;
+}
+
+void apply_mask(kvattn::DecodeArgs& a, const kvattn_attn_mask* m) {
+  a.window = m ? m->window : 0;
+  a.n_sink = (m && m->window > 0) ? m->n_sink : 0;
+  a.sink_logits = m ? m->sink_logits : nullptr;
+}
+
 // 4-D view (d, head, row, seq) of a [B, R, heads, 128] bf16 tensor with
 // 128-byte swizzled boxes of 64 elements x box_heads x box_rows.
 int encode_sw128_map(CUtensorMap* map, const void* base, int B, int R, int heads, int box_heads, int box_rows) {
@@ -160,9 +181,11 @@ int encode_sw128_map(CUtensorMap* map, const void* base, int B, int R, int heads
 
 int run_attention(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, const uint16_t* cache_k,
                   const uint16_t* cache_v, const int32_t* start_pos, int32_t max_kv_len_hint, float scale,
-                  uint16_t* out, void* workspace, size_t workspace_bytes, int32_t* dev_status,
-                  kvattn_stream_t stream) {
+                  const kvattn_attn_mask* mask, uint16_t* out, void* workspace, size_t workspace_bytes,
+                  int32_t* dev_status, kvattn_stream_t stream) {
   int rc = check_dims(dims);
+  if (rc != KVATTN_OK) return rc;
+  rc = check_mask(mask);
   if (rc != KVATTN_OK) return rc;
   if (T < 1) return KVATTN_ERR_INVALID_ARG;
   if (!group_supported(dims->n_heads / dims->n_kv_heads)) return KVATTN_ERR_UNSUPPORTED;
@@ -181,7 +204,9 @@ int run_attention(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, con
   if (rc != KVATTN_OK) return rc;
   int kv_div = 1;
   const int groups = decode_groups(dims, &kv_div);
-  const kvattn::DecodePlan plan = kvattn::plan_decode(dims->batch, T, dims->n_heads, groups, hint, sms);
+  const kvattn::DecodePlan plan = kvattn::plan_decode(dims->batch, T, dims->n_heads, groups,
+                                                      visible_len_bound(hint, mask), sms,
+                                                      mask && mask->sink_logits);
   if (plan.ws_bytes > 0) {
     if (!workspace || workspace_bytes < plan.ws_bytes || !aligned16(workspace)) return KVATTN_ERR_WORKSPACE;
   }
@@ -210,6 +235,7 @@ int run_attention(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, con
   a.rows_per_split = plan.rows_per_split;
   a.max_splits = plan.max_splits;
   a.scale_log2 = scale * 1.4426950408889634f;
+  apply_mask(a, mask);
   a.q = q_rot;
   a.out = out;
   a.start_pos = start_pos;
@@ -222,8 +248,10 @@ int run_attention(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, con
 
 int run_prefill_tc(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, const uint16_t* cache_k,
                    const uint16_t* cache_v, const int32_t* start_pos, int32_t max_kv_len_hint, float scale,
-                   uint16_t* out, int32_t* dev_status, kvattn_stream_t stream) {
+                   const kvattn_attn_mask* mask, uint16_t* out, int32_t* dev_status, kvattn_stream_t stream) {
   int rc = check_dims(dims);
+  if (rc != KVATTN_OK) return rc;
+  rc = check_mask(mask);
   if (rc != KVATTN_OK) return rc;
   if (T < 1) return KVATTN_ERR_INVALID_ARG;
   const int G = dims->n_heads / dims->n_kv_heads;
@@ -260,6 +288,9 @@ int run_prefill_tc(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, co
   a.start_pos = start_pos;
   a.out = out;
   a.dev_status = dev_status;
+  a.window = mask ? mask->window : 0;
+  a.n_sink = (mask && mask->window > 0) ? mask->n_sink : 0;
+  a.sink_logits = mask ? mask->sink_logits : nullptr;
   return kvattn::launch_status(kvattn::launch_prefill(a, tq, tk, tv, (cudaStream_t)stream));
 }
 
@@ -311,7 +342,7 @@ size_t kvattn_decode_workspace_bytes(const kvattn_dims* dims, int32_t max_kv_len
 int kvattn_decode(const kvattn_dims* dims, const uint16_t* q_rot, const uint16_t* cache_k, const uint16_t* cache_v,
                   const int32_t* start_pos, int32_t max_kv_len_hint, float scale, uint16_t* out, void* workspace,
                   size_t workspace_bytes, int32_t* dev_status, kvattn_stream_t stream) {
-  return run_attention(dims, 1, q_rot, cache_k, cache_v, start_pos, max_kv_len_hint, scale, out, workspace,
+  return run_attention(dims, 1, q_rot, cache_k, cache_v, start_pos, max_kv_len_hint, scale, nullptr, out, workspace,
                        workspace_bytes, dev_status, stream);
 }
 
@@ -408,7 +439,38 @@ int kvattn_prefill_chunk(const kvattn_dims* dims, int32_t T, const uint16_t* q_r
                          kvattn_stream_t stream) {
   (void)workspace;
   (void)workspace_bytes;
-  return run_prefill_tc(dims, T, q_rot, cache_k, cache_v, start_pos, max_kv_len_hint, scale, out, dev_status,
+  return run_prefill_tc(dims, T, q_rot, cache_k, cache_v, start_pos, max_kv_len_hint, scale, nullptr, out, dev_status,
+                        stream);
+}
+
+size_t kvattn_decode_masked_workspace_bytes(const kvattn_dims* dims, int32_t max_kv_len_hint,
+                                            const kvattn_attn_mask* mask) {
+  if (check_dims(dims) != KVATTN_OK || check_mask(mask) != KVATTN_OK) return 0;
+  const int hint = hint_or_default(max_kv_len_hint, dims->max_seq_len);
+  if (hint > dims->max_seq_len || hint < 1) return 0;
+  int sms = 0;
+  if (current_sm_count(&sms) != KVATTN_OK) return 0;
+  int kv_div = 1;
+  return kvattn::plan_decode(dims->batch, 1, dims->n_heads, decode_groups(dims, &kv_div),
+                             visible_len_bound(hint, mask), sms, mask && mask->sink_logits)
+      .ws_bytes;
+}
+
+int kvattn_decode_masked(const kvattn_dims* dims, const uint16_t* q_rot, const uint16_t* cache_k,
+                         const uint16_t* cache_v, const int32_t* start_pos, int32_t max_kv_len_hint, float scale,
+                         const kvattn_attn_mask* mask, uint16_t* out, void* workspace, size_t workspace_bytes,
+                         int32_t* dev_status, kvattn_stream_t stream) {
+  return run_attention(dims, 1, q_rot, cache_k, cache_v, start_pos, max_kv_len_hint, scale, mask, out, workspace,
+                       workspace_bytes, dev_status, stream);
+}
+
+int kvattn_prefill_chunk_masked(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, const uint16_t* cache_k,
+                                const uint16_t* cache_v, const int32_t* start_pos, int32_t max_kv_len_hint,
+                                float scale, const kvattn_attn_mask* mask, uint16_t* out, void* workspace,
+                                size_t workspace_bytes, int32_t* dev_status, kvattn_stream_t stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  return run_prefill_tc(dims, T, q_rot, cache_k, cache_v, start_pos, max_kv_len_hint, scale, mask, out, dev_status,
                         stream);
 }
 

@@ -66,6 +66,12 @@ struct DecodeArgs {
   uint16_t* q_rot_out;    // [B, 1, H, d] or null
   int* exit_counter;      // CTAs that finished (counter reset by the last)
   int* merge_counter;     // [B, Hkv] splits finished per row set and KV head
+  // optional masks: window > 0 shows a token at position p the rows
+  // p - window < r <= p and the first n_sink rows; sink_logits (fp32 [H],
+  // score units, or null) adds e^{sink} to each head's softmax denominator
+  int window;
+  int n_sink;
+  const float* sink_logits;
 };
 
 // Group view of the decode kernels: G <= 16 query heads per KV head run as
@@ -88,7 +94,10 @@ struct DecodePlan {
 };
 
 // Split size, persistent grid and workspace for these shapes on this device.
-DecodePlan plan_decode(int B, int Tq, int H, int Hkv, int kv_len_hint, int sm_count);
+// always_partials: every row set writes split partials for the merge kernel
+// (learned sinks are applied there), so a workspace is needed even without
+// splits.
+DecodePlan plan_decode(int B, int Tq, int H, int Hkv, int kv_len_hint, int sm_count, bool always_partials = false);
 
 // G >= 8 runs the tensor-core decode, whose cache view is 128B-swizzled
 // boxes of 64 elements x 64 rows (else plain boxes of 128 elements x 32 rows).
@@ -113,6 +122,9 @@ struct PrefillArgs {
   const int32_t* start_pos;
   uint16_t* out;    // [B, T, H, d]
   int32_t* dev_status;
+  int window;       // > 0: token at position p sees keys p - window < k <= p and k < n_sink
+  int n_sink;
+  const float* sink_logits;  // fp32 [H] learned sink logits (score units), or null
 };
 
 // Tokens per 128-row M tile for group size G (128 / G).

@@ -243,6 +243,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const int t_last = min(t0 + TT, a.T) - 1;
   const int Lmax = sp + t_last + 1;          // keys the tile's last token sees
   const int n_kv = (Lmax + kBN - 1) / kBN;
+  // Key tiles the M tile reads: all of 0..n_kv-1, or with a window the tiles
+  // holding the attention sinks followed by the tiles from the one holding
+  // the first token's earliest window key (the union of the rows' windows).
+  int sink_tiles = 0, win_first = 0;
+  if (a.window > 0) {
+    win_first = max(0, sp + t0 - a.window + 1) / kBN;
+    sink_tiles = min((a.n_sink + kBN - 1) / kBN, win_first);
+  }
+  const int n_iter = sink_tiles + (n_kv - win_first);
+  auto key_tile = [&](int j) { return j < sink_tiles ? j : win_first + (j - sink_tiles); };
 
   if (tid == 0) {
     bar_init(bar(kBarQFull), 1);
@@ -280,17 +290,18 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       bar_expect_tx(bar(kBarQFull), 2 * kHalf);
       tma_load_4d_raw(sQ, &tmap_q, bar(kBarQFull), 0, kvh * G, t0, b);
       tma_load_4d_raw(sQ + kHalf, &tmap_q, bar(kBarQFull), 64, kvh * G, t0, b);
-      for (int j = 0; j < n_kv; ++j) {
+      for (int j = 0; j < n_iter; ++j) {
         const int s = j & 1;
         const uint32_t par = ((j >> 1) & 1) ^ 1;
+        const int key0 = key_tile(j) * kBN;
         if (!bar_wait(bar(kBarKEmpty + s), par, abort_addr, a.dev_status)) break;
         bar_expect_tx(bar(kBarKFull + s), 2 * kHalf);
-        tma_load_4d_raw(sK + (2 * s) * kHalf, &tmap_k, bar(kBarKFull + s), 0, kvh, j * kBN, b);
-        tma_load_4d_raw(sK + (2 * s + 1) * kHalf, &tmap_k, bar(kBarKFull + s), 64, kvh, j * kBN, b);
+        tma_load_4d_raw(sK + (2 * s) * kHalf, &tmap_k, bar(kBarKFull + s), 0, kvh, key0, b);
+        tma_load_4d_raw(sK + (2 * s + 1) * kHalf, &tmap_k, bar(kBarKFull + s), 64, kvh, key0, b);
         if (!bar_wait(bar(kBarVEmpty + s), par, abort_addr, a.dev_status)) break;
         bar_expect_tx(bar(kBarVFull + s), 2 * kHalf);
-        tma_load_4d_raw(sV + (2 * s) * kHalf, &tmap_v, bar(kBarVFull + s), 0, kvh, j * kBN, b);
-        tma_load_4d_raw(sV + (2 * s + 1) * kHalf, &tmap_v, bar(kBarVFull + s), 64, kvh, j * kBN, b);
+        tma_load_4d_raw(sV + (2 * s) * kHalf, &tmap_v, bar(kBarVFull + s), 0, kvh, key0, b);
+        tma_load_4d_raw(sV + (2 * s + 1) * kHalf, &tmap_v, bar(kBarVFull + s), 64, kvh, key0, b);
       }
     }
   } else if (warp == 1) {
@@ -317,8 +328,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         return true;
       };
       if (ok) ok = issue_qk(0);
-      for (int j = 0; j < n_kv && ok; ++j) {
-        if (j + 1 < n_kv && !issue_qk(j + 1)) break;
+      for (int j = 0; j < n_iter && ok; ++j) {
+        if (j + 1 < n_iter && !issue_qk(j + 1)) break;
         const int s = j & 1;
         if (!bar_wait(bar(kBarPFull + s), (j >> 1) & 1, abort_addr, a.dev_status, kMmaSuspend)) break;
         if (!bar_wait(bar(kBarVFull + s), (j >> 1) & 1, abort_addr, a.dev_status, kMmaSuspend)) break;
@@ -347,6 +358,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int tok = t0 + m / G;
     const int head = kvh * G + (m % G);
     const int lim = sp + min(tok, a.T - 1);  // last visible key (rows past T borrow the last token's)
+    // with a window: keys n_sink <= k < lo_vis are hidden as well
+    const int lo_vis = a.window > 0 ? lim - a.window + 1 : 0;
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * quarter) << 16);
     const int st = tid - 64;              // 0..255 among the softmax threads
     const uint32_t xmax_mine = base + kOffXmax + (uint32_t)(ch * 128 + m) * 4;
@@ -355,8 +368,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     float m_ref = -INFINITY;
     float l = 0.f;                        // sum over this thread's column half
 
-    for (int j = 0; j < n_kv; ++j) {
+    for (int j = 0; j < n_iter; ++j) {
       const int s = j & 1;
+      const int jt = key_tile(j);
       bar_wait(bar(kBarSFull + s), (j >> 1) & 1, abort_addr, a.dev_status);
       tc_fence_after();
       // this thread's 64 columns of the S row: two 32-column loads, one wait
@@ -370,11 +384,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 
       // mask (raw scores; the scale is folded into the exponent below) and
       // partial row max over eight independent accumulators
-      const int kbase = j * kBN + 64 * ch;
-      if (kbase + 63 > lim) {
+      const int kbase = jt * kBN + 64 * ch;
+      if (kbase + 63 > lim || (kbase < lo_vis && kbase + 63 >= a.n_sink)) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (kbase + c > lim) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+        for (int c = 0; c < 64; ++c) {
+          const int k = kbase + c;
+          if (k > lim || (k < lo_vis && k >= a.n_sink)) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+        }
       }
       float mx8[8];
 #pragma unroll
@@ -441,11 +457,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         bar_wait(bar(kBarPVDone + s), ((j >> 1) - 1) & 1, abort_addr, a.dev_status);
         tc_fence_after();
       }
-      if (j == n_kv - 1 && Lmax < j * kBN + kBN) {
+      if (j == n_iter - 1 && Lmax < jt * kBN + kBN) {
         // rows of the last V tile past the last visible key may hold any bits;
         // zero them so that 0 * (garbage) cannot reach O
         bar_wait(bar(kBarVFull + s), (j >> 1) & 1, abort_addr, a.dev_status);
-        const int first_bad = Lmax - j * kBN;
+        const int first_bad = Lmax - jt * kBN;
         const int nchunks = (kBN - first_bad) * 16;  // 16-byte chunks over both halves
         for (int c = st; c < nchunks; c += kSoftmaxWarps * 32) {
           const int r = first_bad + (c >> 4);
@@ -470,9 +486,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     named_bar_sync(pair_bar, 64);
     float l_other;
     asm volatile("ld.shared.f32 %0, [%1];" : "=f"(l_other) : "r"(xsum_other) : "memory");
-    bar_wait(bar(kBarPVDone + ((n_kv - 1) & 1)), ((n_kv - 1) >> 1) & 1, abort_addr, a.dev_status);
+    bar_wait(bar(kBarPVDone + ((n_iter - 1) & 1)), ((n_iter - 1) >> 1) & 1, abort_addr, a.dev_status);
     tc_fence_after();
-    const float inv_l = 1.f / (l + l_other);
+    float inv_l = 1.f / (l + l_other);
+    if (a.sink_logits) {
+      // learned sink: e^{sink} joins the denominator (log2 units, reference m_ref)
+      const float s2 = __ldg(a.sink_logits + head) * 1.4426950408889634f;
+      const float mn = fmaxf(m_ref, s2);
+      const float f = (m_ref == -INFINITY) ? 0.f : fast_exp2(m_ref - mn);
+      inv_l = f / ((l + l_other) * f + fast_exp2(s2 - mn));
+    }
     const bool store = tok < a.T;
     uint16_t* dst = a.out + (((size_t)b * a.T + (store ? tok : 0)) * a.H + head) * kHeadDim + 64 * ch;
 #pragma unroll

@@ -163,6 +163,50 @@ KVATTN_API int kvattn_decode(const kvattn_dims* dims, const uint16_t* q_rot, con
 KVATTN_API int kvattn_decode_plan(const kvattn_dims* dims, int32_t max_kv_len_hint, int32_t* rows_per_split,
                                   int32_t* max_splits, int32_t* grid, int32_t* ctas_per_sm);
 
+/* Optional attention masks of "The Modern Decoder Block" (modules L7.5 and
+ * L7.7: sliding window, StreamingLLM attention sinks, learned sinks).  The
+ * page names them without defining them; the readings taken are the plain
+ * ones of the works it cites:
+ *  - window W > 0: the token at position p sees cache rows p - W < r <= p
+ *    (W = 0: every row 0..p);
+ *  - n_sink (with a window): rows 0..n_sink-1 stay visible as well; positions
+ *    stay absolute (RoPE is applied at the true position, rows are
+ *    positions);
+ *  - sink_logits: device fp32 [H] or NULL, one learned logit sigma_h per query
+ *    head in the units of the scaled score: e^{sigma_h} joins the head's
+ *    softmax denominator and carries no value,
+ *    out = sum_r e^{s_r} V_r / (e^{sigma_h} + sum_r e^{s_r}).
+ * A NULL mask pointer means none of these. */
+typedef struct kvattn_attn_mask {
+  int32_t window;
+  int32_t n_sink;
+  const float* sink_logits;
+} kvattn_attn_mask;
+
+/* kvattn_decode with a mask (mask may be NULL).  Only the visible rows are
+ * read from HBM: the sink rows and the window rows (each rounded out to
+ * 64-row boundaries).  Workspace: kvattn_decode_masked_workspace_bytes() for
+ * the same mask (with learned sinks every sequence writes split partials and
+ * the merge kernel adds the sink term, so a workspace is needed even when no
+ * sequence is split).
+ * Host errors: those of kvattn_decode, and INVALID_ARG for a negative window
+ * or n_sink or a misaligned sink_logits. */
+KVATTN_API size_t kvattn_decode_masked_workspace_bytes(const kvattn_dims* dims, int32_t max_kv_len_hint,
+                                                       const kvattn_attn_mask* mask);
+KVATTN_API int kvattn_decode_masked(const kvattn_dims* dims, const uint16_t* q_rot, const uint16_t* cache_k,
+                                    const uint16_t* cache_v, const int32_t* start_pos, int32_t max_kv_len_hint,
+                                    float scale, const kvattn_attn_mask* mask, uint16_t* out, void* workspace,
+                                    size_t workspace_bytes, int32_t* dev_status, kvattn_stream_t stream);
+
+/* kvattn_prefill_chunk with a mask (mask may be NULL): each token applies its
+ * own window; key tiles outside every row's window and the sinks are not
+ * read. */
+KVATTN_API int kvattn_prefill_chunk_masked(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot,
+                                           const uint16_t* cache_k, const uint16_t* cache_v,
+                                           const int32_t* start_pos, int32_t max_kv_len_hint, float scale,
+                                           const kvattn_attn_mask* mask, uint16_t* out, void* workspace,
+                                           size_t workspace_bytes, int32_t* dev_status, kvattn_stream_t stream);
+
 /* Bytes of device workspace kvattn_decode_fused needs for these dims and
  * max_kv_len_hint on the CURRENT device (0: none needed, or invalid
  * arguments). */

@@ -151,3 +151,15 @@ def test_fused_decode_rejects_bad_args(lib):
     # hint beyond the cache
     assert lib.kvattn_decode_fused(ctypes.byref(d), ctypes.byref(rope), FAKE, None, *P7[:5], 65, 0.0, FAKE, None, 0,
                                    None, None) == 3
+
+
+def test_masked_entry_points_validate_the_mask(lib):
+    d = _dims()
+    P = [FAKE] * 4
+    for bad in (kv.kvattn_attn_mask(-1, 0, None), kv.kvattn_attn_mask(8, -2, None),
+                kv.kvattn_attn_mask(8, 0, 0x10002)):
+        assert lib.kvattn_decode_masked(ctypes.byref(d), *P, 0, 0.0, ctypes.byref(bad), FAKE, None, 0, None,
+                                        None) == 1
+        assert lib.kvattn_prefill_chunk_masked(ctypes.byref(d), 1, *P, 0, 0.0, ctypes.byref(bad), FAKE, None, 0,
+                                               None, None) == 1
+        assert lib.kvattn_decode_masked_workspace_bytes(ctypes.byref(d), 0, ctypes.byref(bad)) == 0
