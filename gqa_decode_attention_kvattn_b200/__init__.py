@@ -237,13 +237,13 @@ def kvattn_decode_plan(batch, n_heads, n_kv_heads, max_seq_len, max_kv_len_hint=
     lib = _load()
     fn = lib.kvattn_decode_plan
     fn.restype = ctypes.c_int
-    fn.argtypes = [ctypes.POINTER(kvattn_dims), ctypes.c_int32] + [ctypes.POINTER(ctypes.c_int32)] * 4
+    fn.argtypes = [ctypes.POINTER(kvattn_dims), ctypes.c_int32] + [ctypes.POINTER(ctypes.c_int32)] * 5
     dims = kvattn_dims(batch, n_heads, n_kv_heads, head_dim, max_seq_len)
-    out = [ctypes.c_int32() for _ in range(4)]
+    out = [ctypes.c_int32() for _ in range(5)]
     rc = fn(ctypes.byref(dims), int(max_kv_len_hint), *[ctypes.byref(o) for o in out])
     _check_status(rc, "kvattn_decode_plan")
     return dict(rows_per_split=out[0].value, max_splits=out[1].value, grid=out[2].value,
-                ctas_per_sm=out[3].value)
+                ctas_per_sm=out[3].value, tensor_cores=bool(out[4].value))
 
 
 def kvattn_prefill_workspace_bytes(batch, n_heads, n_kv_heads, max_seq_len, T, max_kv_len_hint=0,

@@ -845,6 +845,11 @@ __global__ void __launch_bounds__(kHeadDim) decode_merge_kernel(const DecodeArgs
 // online softmax rescales O without any exchange between lanes.  K and V
 // arrive by TMA as 128B-swizzled 64-element halves, read with ldmatrix.
 constexpr int kMmaTileRows = 64;
+// G = 4 calls with at least this many (row, KV head) pairs run on the
+// tensor-core decode (its 64-row tiles and 2 CTAs per SM pay off once the
+// call streams tens of MB; a single short sequence is latency-bound and runs
+// faster on the CUDA-core kernel's 32-row tiles and 3 CTAs per SM)
+constexpr long long kMmaMinWork = 1ll << 18;
 constexpr int kMmaStages = 2;
 constexpr uint32_t kMmaHalfBytes = kMmaTileRows * 64 * 2;  // 8 KB
 
@@ -897,7 +902,7 @@ template <int G, bool FUSED, bool WINDOW>
 __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(
     const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
     const DecodeArgs a, const int evict_first, const __grid_constant__ RopeTable tab) {
-  static_assert(G == 8 || G == 16, "tensor-core decode handles G = 8 or 16");
+  static_assert(G == 1 || G == 2 || G == 4 || G == 8 || G == 16, "tensor-core decode handles G <= 16");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   SmemMma<G>& sm = *reinterpret_cast<SmemMma<G>*>(smem_raw);
   // the 128B-swizzled tiles need a 1024-byte aligned base; refuse otherwise
@@ -1003,8 +1008,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const int col = 8 * kk + c4;  // word index of dims 16kk + 2*c4
-          qa[kk][0] = qw[g * 64 + col];
-          qa[kk][2] = qw[g * 64 + col + 4];
+          // rows g >= G pad the 16-row MMA tile with zeros
+          qa[kk][0] = (G >= 8 || g < G) ? qw[g * 64 + col] : 0u;
+          qa[kk][2] = (G >= 8 || g < G) ? qw[g * 64 + col + 4] : 0u;
           if constexpr (G == 16) {
             qa[kk][1] = qw[(g + 8) * 64 + col];
             qa[kk][3] = qw[(g + 8) * 64 + col + 4];
@@ -1126,14 +1132,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(
       float lsum = l_run[hh];
       lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
       lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
-      if (c4 == 0) {
-        sm.merge_m[warp][g + 8 * hh] = m_run[hh];
-        sm.merge_l[warp][g + 8 * hh] = lsum;
-      }
+      if (G >= 8 || g < G) {  // padding rows carry no head
+        if (c4 == 0) {
+          sm.merge_m[warp][g + 8 * hh] = m_run[hh];
+          sm.merge_l[warp][g + 8 * hh] = lsum;
+        }
 #pragma unroll
-      for (int dt = 0; dt < 16; ++dt)
-        *reinterpret_cast<float2*>(&sm.merge_o[warp][g + 8 * hh][8 * dt + 2 * c4]) =
-            make_float2(o[dt][2 * hh], o[dt][2 * hh + 1]);
+        for (int dt = 0; dt < 16; ++dt)
+          *reinterpret_cast<float2*>(&sm.merge_o[warp][g + 8 * hh][8 * dt + 2 * c4]) =
+              make_float2(o[dt][2 * hh], o[dt][2 * hh + 1]);
+      }
     }
     cons_sync();
     {
@@ -1181,23 +1189,25 @@ size_t smem_bytes() {
   return sizeof(Smem<G>);
 }
 
-template <int G, bool FUSED, bool WINDOW>
+// G >= 8 always runs the tensor-core kernel; G = 4 has both (MMA when the
+// call is large enough, see decode_use_mma); G <= 2 the CUDA-core kernel.
+template <int G, bool FUSED, bool WINDOW, bool MMA>
 auto decode_kernel() {
-  if constexpr (G >= 8) return decode_mma_kernel<G, FUSED, WINDOW>;
+  if constexpr (MMA) return decode_mma_kernel<G, FUSED, WINDOW>;
   else return decode_splitk_kernel<G, FUSED, WINDOW>;
 }
 
-template <int G>
+template <int G, bool MMA>
 size_t decode_smem_bytes() {
-  if constexpr (G >= 8) return smem_bytes_mma<G>();
+  if constexpr (MMA) return smem_bytes_mma<G>();
   else return smem_bytes<G>();
 }
 
-template <int G, bool FUSED, bool WINDOW>
+template <int G, bool FUSED, bool WINDOW, bool MMA>
 cudaError_t launch_g(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, const RopeTable& tab,
                      cudaStream_t st) {
-  auto kernel = decode_kernel<G, FUSED, WINDOW>();
-  const size_t smem = decode_smem_bytes<G>();
+  auto kernel = decode_kernel<G, FUSED, WINDOW, MMA>();
+  const size_t smem = decode_smem_bytes<G, MMA>();
   static bool configured[64] = {false};
   int dev = 0;
   cudaError_t e0 = cudaGetDevice(&dev);
@@ -1228,20 +1238,35 @@ cudaError_t launch_g(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorM
 template <int G>
 cudaError_t launch_g(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st,
                      const RopeTable* fused) {
-  if (fused) return launch_g<G, true, false>(a, tk, tv, *fused, st);
   RopeTable unused{};
-  if (a.window > 0) return launch_g<G, false, true>(a, tk, tv, unused, st);
-  return launch_g<G, false, false>(a, tk, tv, unused, st);
+  if constexpr (G >= 8) {
+    if (fused) return launch_g<G, true, false, true>(a, tk, tv, *fused, st);
+    if (a.window > 0) return launch_g<G, false, true, true>(a, tk, tv, unused, st);
+    return launch_g<G, false, false, true>(a, tk, tv, unused, st);
+  } else if constexpr (G == 4) {
+    if (a.mma) {
+      if (fused) return launch_g<G, true, false, true>(a, tk, tv, *fused, st);
+      if (a.window > 0) return launch_g<G, false, true, true>(a, tk, tv, unused, st);
+      return launch_g<G, false, false, true>(a, tk, tv, unused, st);
+    }
+    if (fused) return launch_g<G, true, false, false>(a, tk, tv, *fused, st);
+    if (a.window > 0) return launch_g<G, false, true, false>(a, tk, tv, unused, st);
+    return launch_g<G, false, false, false>(a, tk, tv, unused, st);
+  } else {
+    if (fused) return launch_g<G, true, false, false>(a, tk, tv, *fused, st);
+    if (a.window > 0) return launch_g<G, false, true, false>(a, tk, tv, unused, st);
+    return launch_g<G, false, false, false>(a, tk, tv, unused, st);
+  }
 }
 
 }  // namespace
 
 // Resident CTAs per SM of the decode kernel for group size G (occupancy
 // query: registers and shared memory both count).
-template <int G, bool FUSED, bool WINDOW>
+template <int G, bool FUSED, bool WINDOW, bool MMA>
 int resident_ctas_of() {
-  auto kernel = decode_kernel<G, FUSED, WINDOW>();
-  const size_t smem = decode_smem_bytes<G>();
+  auto kernel = decode_kernel<G, FUSED, WINDOW, MMA>();
+  const size_t smem = decode_smem_bytes<G, MMA>();
   int n = 0;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess ||
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kThreads, smem) != cudaSuccess || n < 1)
@@ -1250,25 +1275,26 @@ int resident_ctas_of() {
 }
 
 // the persistent grid serves the unfused, the fused and the window kernels
-template <int G>
+template <int G, bool MMA>
 int resident_ctas() {
-  return std::min(std::min(resident_ctas_of<G, false, false>(), resident_ctas_of<G, true, false>()),
-                  resident_ctas_of<G, false, true>());
+  return std::min(std::min(resident_ctas_of<G, false, false, MMA>(), resident_ctas_of<G, true, false, MMA>()),
+                  resident_ctas_of<G, false, true, MMA>());
 }
 
-int resident_ctas_for(int G) {
-  static int cached[64][5] = {};  // [device][log2 G], 0 = not yet queried
+int resident_ctas_for(int G, bool mma) {
+  static int cached[64][6] = {};  // [device][kernel], 0 = not yet queried
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
-  const int gi = G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : G == 8 ? 3 : 4;
+  const int gi = G == 1 ? 0 : G == 2 ? 1 : G == 4 ? (mma ? 5 : 2) : G == 8 ? 3 : 4;
   int n = __atomic_load_n(&cached[dev][gi], __ATOMIC_RELAXED);
   if (n == 0) {
-    switch (G) {
-      case 1: n = resident_ctas<1>(); break;
-      case 2: n = resident_ctas<2>(); break;
-      case 4: n = resident_ctas<4>(); break;
-      case 8: n = resident_ctas<8>(); break;
-      default: n = resident_ctas<16>(); break;
+    switch (gi) {
+      case 0: n = resident_ctas<1, false>(); break;
+      case 1: n = resident_ctas<2, false>(); break;
+      case 2: n = resident_ctas<4, false>(); break;
+      case 5: n = resident_ctas<4, true>(); break;
+      case 3: n = resident_ctas<8, true>(); break;
+      default: n = resident_ctas<16, true>(); break;
     }
     __atomic_store_n(&cached[dev][gi], n, __ATOMIC_RELAXED);
   }
@@ -1278,7 +1304,8 @@ int resident_ctas_for(int G) {
 DecodePlan plan_decode(int B, int Tq, int H, int Hkv, int kv_len_hint, int sm_count, bool always_partials) {
   DecodePlan p;
   const int G = H / Hkv;
-  const int ctas_per_sm = resident_ctas_for(G);
+  p.mma = decode_use_mma(G, (long long)B * Tq * Hkv * kv_len_hint);
+  const int ctas_per_sm = resident_ctas_for(G, p.mma);
   p.ctas_per_sm = ctas_per_sm;
   const int slots = sm_count * ctas_per_sm;
   const long long row_sets = (long long)B * Tq;
@@ -1347,6 +1374,6 @@ cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tk, const CUte
   }
 }
 
-bool decode_uses_tensor_cores(int G) { return G >= 8; }
+bool decode_use_mma(int G, long long work_rows) { return G >= 8 || (G == 4 && work_rows >= kMmaMinWork); }
 
 }  // namespace kvattn

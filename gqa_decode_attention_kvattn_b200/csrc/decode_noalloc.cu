@@ -133,7 +133,7 @@ extern "C" KVATTN_API int kvattn_decode_noalloc(const kvattn_dims* dims, const u
     if (rc != KVATTN_OK) return rc;
   }
   CUtensorMap tk, tv;
-  const bool swizzled = kvattn::decode_uses_tensor_cores(G);
+  const bool swizzled = plan.mma;
   rc = cache_map(&tk, cache_k, dims->batch, dims->max_seq_len, dims->n_kv_heads, swizzled);
   if (rc != KVATTN_OK) return rc;
   rc = cache_map(&tv, cache_v, dims->batch, dims->max_seq_len, dims->n_kv_heads, swizzled);
@@ -157,5 +157,6 @@ extern "C" KVATTN_API int kvattn_decode_noalloc(const kvattn_dims* dims, const u
   kvattn::bind_decode_workspace(a, plan, scratch);
   a.dev_status = dev_status;
   a.grid = plan.grid;
+  a.mma = plan.mma ? 1 : 0;
   return kvattn::launch_status(kvattn::launch_decode(a, tk, tv, (cudaStream_t)stream));
 }

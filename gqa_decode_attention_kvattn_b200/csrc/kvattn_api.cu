@@ -212,7 +212,7 @@ int run_attention(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, con
   }
 
   CUtensorMap tk, tv;
-  if (kvattn::decode_uses_tensor_cores(dims->n_heads / dims->n_kv_heads)) {
+  if (plan.mma) {
     rc = encode_sw128_map(&tk, cache_k, dims->batch, dims->max_seq_len, dims->n_kv_heads, 1, 64);
     if (rc != KVATTN_OK) return rc;
     rc = encode_sw128_map(&tv, cache_v, dims->batch, dims->max_seq_len, dims->n_kv_heads, 1, 64);
@@ -242,6 +242,7 @@ int run_attention(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, con
   kvattn::bind_decode_workspace(a, plan, workspace);
   a.dev_status = dev_status;
   a.grid = plan.grid;
+  a.mma = plan.mma ? 1 : 0;
   return kvattn::launch_status(kvattn::launch_decode(a, tk, tv, (cudaStream_t)stream));
 }
 
@@ -389,7 +390,7 @@ int kvattn_decode_fused(const kvattn_dims* dims, const kvattn_rope_params* rope,
     if (!workspace || workspace_bytes < plan.fused_ws_bytes || !aligned16(workspace)) return KVATTN_ERR_WORKSPACE;
   }
   CUtensorMap tk, tv;
-  if (kvattn::decode_uses_tensor_cores(dims->n_heads / dims->n_kv_heads)) {
+  if (plan.mma) {
     rc = encode_sw128_map(&tk, cache_k, dims->batch, dims->max_seq_len, dims->n_kv_heads, 1, 64);
     if (rc != KVATTN_OK) return rc;
     rc = encode_sw128_map(&tv, cache_v, dims->batch, dims->max_seq_len, dims->n_kv_heads, 1, 64);
@@ -418,6 +419,7 @@ int kvattn_decode_fused(const kvattn_dims* dims, const kvattn_rope_params* rope,
   kvattn::bind_decode_workspace(a, plan, workspace, true);
   a.dev_status = dev_status;
   a.grid = plan.grid;
+  a.mma = plan.mma ? 1 : 0;
   a.k_new = k_new;
   a.v_new = v_new;
   a.cache_k = cache_k;
@@ -475,7 +477,7 @@ int kvattn_prefill_chunk_masked(const kvattn_dims* dims, int32_t T, const uint16
 }
 
 int kvattn_decode_plan(const kvattn_dims* dims, int32_t max_kv_len_hint, int32_t* rows_per_split,
-                       int32_t* max_splits, int32_t* grid, int32_t* ctas_per_sm) {
+                       int32_t* max_splits, int32_t* grid, int32_t* ctas_per_sm, int32_t* tensor_cores) {
   int rc = check_dims(dims);
   if (rc != KVATTN_OK) return rc;
   if (!group_supported(dims->n_heads / dims->n_kv_heads)) return KVATTN_ERR_UNSUPPORTED;
@@ -490,6 +492,7 @@ int kvattn_decode_plan(const kvattn_dims* dims, int32_t max_kv_len_hint, int32_t
   if (max_splits) *max_splits = p.max_splits;
   if (grid) *grid = p.grid;
   if (ctas_per_sm) *ctas_per_sm = p.ctas_per_sm;
+  if (tensor_cores) *tensor_cores = p.mma ? 1 : 0;
   return KVATTN_OK;
 }
 

@@ -72,6 +72,7 @@ struct DecodeArgs {
   int window;
   int n_sink;
   const float* sink_logits;
+  int mma;       // 1: the tensor-core kernel (its 128B-swizzled 64-row cache view)
 };
 
 // Group view of the decode kernels: G <= 16 query heads per KV head run as
@@ -89,6 +90,7 @@ struct DecodePlan {
   int max_splits;
   int grid;
   int ctas_per_sm;
+  bool mma;               // tensor-core decode (else the CUDA-core kernel)
   size_t ws_bytes;        // partials + work counter (unfused decode)
   size_t fused_ws_bytes;  // partials + the counters of the fused decode
 };
@@ -99,9 +101,10 @@ struct DecodePlan {
 // splits.
 DecodePlan plan_decode(int B, int Tq, int H, int Hkv, int kv_len_hint, int sm_count, bool always_partials = false);
 
-// G >= 8 runs the tensor-core decode, whose cache view is 128B-swizzled
-// boxes of 64 elements x 64 rows (else plain boxes of 128 elements x 32 rows).
-bool decode_uses_tensor_cores(int G);
+// Whether a call of G heads per KV head over work_rows (row, KV head) pairs
+// runs on the tensor-core decode, whose cache view is 128B-swizzled boxes of
+// 64 elements x 64 rows (else plain boxes of 128 elements x 32 rows).
+bool decode_use_mma(int G, long long work_rows);
 
 // Points ws_o / ws_ml / counter (and, when `fused`, the fused decode's
 // counters) of `a` into a workspace of plan.ws_bytes (plan.fused_ws_bytes).

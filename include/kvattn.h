@@ -157,11 +157,13 @@ KVATTN_API int kvattn_decode(const kvattn_dims* dims, const uint16_t* q_rot, con
 
 /* How kvattn_decode will split the work for these dims and max_kv_len_hint
  * on the CURRENT device: rows per split (C), the most splits a sequence can
- * have, the persistent grid (CTAs) and the CTAs resident per SM.  Any output
- * pointer may be NULL.  Returns a kvattn_status (host-side only, launches
- * nothing). */
+ * have, the persistent grid (CTAs), the CTAs resident per SM, and whether the
+ * tensor-core decode runs (1; G >= 8 always, G = 4 for calls of at least
+ * 2^18 (row, KV head) pairs) or the CUDA-core one (0).  Any output pointer
+ * may be NULL.  Returns a kvattn_status (host-side only, launches nothing). */
 KVATTN_API int kvattn_decode_plan(const kvattn_dims* dims, int32_t max_kv_len_hint, int32_t* rows_per_split,
-                                  int32_t* max_splits, int32_t* grid, int32_t* ctas_per_sm);
+                                  int32_t* max_splits, int32_t* grid, int32_t* ctas_per_sm,
+                                  int32_t* tensor_cores);
 
 /* Optional attention masks of "The Modern Decoder Block" (modules L7.5 and
  * L7.7: sliding window, StreamingLLM attention sinks, learned sinks).  The

@@ -57,6 +57,7 @@ def _check_step(seed, B, T, H, Hkv, S, sp, rope, kind, hint=0, in_place=False):
     (5, 64, 8, 520, [1, 127, 128, 511, 519], kv.LLAMA3),  # G = 8 (tensor cores)
     (3, 32, 2, 700, [0, 63, 64, 699][:3], kv.LLAMA3),     # G = 16 (tensor cores)
     (4, 64, 8, 3000, [2999, 64, 65, 1000], kv.LLAMA3_1),  # G = 8, several splits
+    (8, 32, 8, 8192, [8191, 0, 63, 64, 4000, 777, 5000, 12], kv.LLAMA3),  # G = 4 on the tensor-core kernel
     (3, 32, 1, 2500, [0, 1000, 2499], kv.LLAMA3),       # G = 32 (MQA): two 16-head groups per KV head
     (2, 64, 2, 1500, [1499, 700], kv.LLAMA3),           # G = 32 with two KV heads
     (2, 64, 1, 900, [899, 33], kv.LLAMA3_1),            # G = 64 (MQA, 64 heads)
@@ -271,3 +272,12 @@ def test_rope_layouts_and_partial_rotary(layout, rotary_dim, scaled, kind, T):
     assert st == 0
     r = rotary_dim or 128
     assert np.array_equal(g_qrot[..., r:], q[..., r:])
+
+
+def test_decode_kernel_choice():
+    """G = 4 runs on the tensor-core decode for large calls and on the
+    CUDA-core kernel for small ones; G >= 8 always on tensor cores."""
+    assert kv.kvattn_decode_plan(8, 32, 8, 8192)["tensor_cores"]
+    assert not kv.kvattn_decode_plan(1, 32, 8, 8192, max_kv_len_hint=1001)["tensor_cores"]
+    assert kv.kvattn_decode_plan(1, 64, 8, 4096)["tensor_cores"]
+    assert not kv.kvattn_decode_plan(64, 16, 8, 8192)["tensor_cores"]
