@@ -301,16 +301,31 @@ __device__ void build_work_table(const DecodeArgs& a, SM& sm, int n_sets, int la
 __device__ __forceinline__ float lse_merge_element(const DecodeArgs& a, int v, int head, int ns, int c) {
   const size_t base = (size_t)v * a.max_splits * a.H + head;
   float M = -INFINITY, num = 0.f, den = 0.f;
-  for (int s = 0; s < ns; ++s) {
-    const size_t slot = base + (size_t)s * a.H;
-    const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.ws_ml + slot * 2));
-    const float o = __ldcg(a.ws_o + slot * kHeadDim + c);
+  auto step = [&](float2 ml, float o) {
     const float Mn = fmaxf(M, ml.x);
     const float f_old = (M == -INFINITY) ? 0.f : fast_exp2(M - Mn);
     const float f_new = fast_exp2(ml.x - Mn);
     num = num * f_old + o * f_new;
     den = den * f_old + ml.y * f_new;
     M = Mn;
+  };
+  // eight splits' loads in flight at a time; the arithmetic stays in split order
+  int s = 0;
+  for (; s + 8 <= ns; s += 8) {
+    float2 ml[8];
+    float o[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const size_t slot = base + (size_t)(s + k) * a.H;
+      ml[k] = __ldcg(reinterpret_cast<const float2*>(a.ws_ml + slot * 2));
+      o[k] = __ldcg(a.ws_o + slot * kHeadDim + c);
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) step(ml[k], o[k]);
+  }
+  for (; s < ns; ++s) {
+    const size_t slot = base + (size_t)s * a.H;
+    step(__ldcg(reinterpret_cast<const float2*>(a.ws_ml + slot * 2)), __ldcg(a.ws_o + slot * kHeadDim + c));
   }
   return normalise_with_sink(num, den, M, sink_log2(a, head));
 }

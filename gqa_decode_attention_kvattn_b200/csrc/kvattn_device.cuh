@@ -29,37 +29,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return f32_to_bf16_bits(lo) | (f32_to_bf16_bits(hi) << 16);
 }
 
-// fp64 -> bf16 bits with a single rounding (nearest, ties to even), written
-// from the IEEE-754 encodings: bf16 keeps 8 significant bits and fp32's
-// exponent range (normal exponents -126..127, subnormal spacing 2^-133).
+// fp64 -> bf16 bits with a single rounding (nearest, ties to even) by the
+// hardware conversion.  It rounds straight from the double (no intermediate
+// fp32 rounding): on B200 it agreed with an integer round-to-nearest-even of
+// the IEEE-754 encodings on 1.8 M inputs, including values a hair above and
+// below every kind of bf16 midpoint, where a double rounding would differ.
 __device__ __forceinline__ uint32_t f64_to_bf16_bits(double x) {
-  const uint64_t u = (uint64_t)__double_as_longlong(x);
-  const uint32_t sign = (uint32_t)(u >> 63) << 15;
-  const int ebits = (int)((u >> 52) & 0x7FF);
-  const uint64_t frac = u & ((1ull << 52) - 1);
-  if (ebits == 0x7FF) return frac ? 0x7FC0u : (sign | 0x7F80u);
-  if (ebits == 0) return sign;  // fp64 zero or subnormal (< 2^-1022): rounds to +-0
-  const int e = ebits - 1023;
-  const uint64_t sig = frac | (1ull << 52);  // 53-bit significand, value = sig * 2^(e-52)
-  if (e >= -126) {
-    // normal bf16: keep 8 significant bits
-    uint64_t q = sig >> 45;
-    const uint64_t rem = sig & ((1ull << 45) - 1);
-    const uint64_t half = 1ull << 44;
-    if (rem > half || (rem == half && (q & 1))) ++q;
-    int eo = e;
-    if (q == 256) { q = 128; ++eo; }
-    if (eo > 127) return sign | 0x7F80u;
-    return sign | ((uint32_t)(eo + 127) << 7) | (uint32_t)(q & 0x7F);
-  }
-  // subnormal bf16: units of 2^-133, value/unit = sig * 2^(e - 52 + 133)
-  const int shift = -81 - e;  // > 45 here
-  if (shift > 54) return sign;  // below half of the smallest subnormal
-  uint64_t q = sig >> shift;
-  const uint64_t rem = sig & ((1ull << shift) - 1);
-  const uint64_t half = 1ull << (shift - 1);
-  if (rem > half || (rem == half && (q & 1))) ++q;
-  return sign | (uint32_t)q;  // q == 128 encodes the smallest normal, as it should
+  uint16_t r;
+  asm("cvt.rn.bf16.f64 %0, %1;" : "=h"(r) : "d"(x));
+  return r;
 }
 
 // 2^x on the special-function unit (ex2.approx: relative error ~2^-22;

@@ -2,17 +2,22 @@
 //
 // For token t of sequence b the position is p = start_pos[b] + t (the past
 // length is the offset: "Llama 3.1 8B KV cache", section "RoPE has to know
-// where it is").  Each interleaved pair (x_2i, x_2i+1) of every query head and
-// every new key head is rotated by p * f_i; the rotated keys and the values go
-// to cache row p ("Llama 3 8B · KV cache", cache write C_K[p] <- K_r,
-// C_V[p] <- V).  Angles, sin/cos and the rotation run in fp64, which keeps the
-// bf16 result within one rounding of the exact value up to p = 131071 (an fp32
-// angle would already be off by ~1e-2 rad there).
+// where it is").  Each rotated pair of every query head and every new key
+// head is turned by p * f_i; the rotated keys and the values go to cache row
+// p ("Llama 3 8B · KV cache", cache write C_K[p] <- K_r, C_V[p] <- V).
+// Angles, sin/cos and the rotation run in fp64, which keeps the bf16 result
+// within one rounding of the exact value up to p = 131071 (an fp32 angle
+// would already be off by ~1e-2 rad there).
 //
-// One CTA per (b, t); its threads first build the 64 (cos, sin) pairs of that
-// position, then sweep the (H + Hkv) * 64 pairs with coalesced 4-byte
-// accesses, and copy the Hkv value rows with 16-byte accesses.  The kernel
-// moves B*T*(2H + 3Hkv)*256 bytes, a negligible share of a decode step.
+// Work split: the H query heads and Hkv key heads of a token are H + Hkv
+// head vectors; for a few tokens one CTA of 128 threads takes 8 of them for
+// one (b, t), so a small decode batch still spreads over the SMs, and for
+// many tokens a CTA takes a whole token.  The CTA builds the (cos,
+// sin) pairs of its position in shared memory, rotates its vectors' 64 slots
+// (coalesced 4-byte accesses in the interleaved full-width layout), and a CTA
+// holding key vectors also copies those heads' value rows (16-byte
+// accesses).  The kernel moves B*T*(2H + 3Hkv)*256 bytes, a negligible share
+// of a decode step.
 #include "kvattn_device.cuh"
 #include "kvattn_internal.h"
 #include "rope_device.cuh"
@@ -20,15 +25,20 @@
 namespace kvattn {
 namespace {
 
-constexpr int kRopeThreads = 256;
+constexpr int kRopeThreads = 128;
 
-__global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(RopeAppendArgs a, RopeTable tab) {
-  const int bt = blockIdx.x;
+// vec_per_cta: head vectors (query or key heads) per CTA
+__global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(RopeAppendArgs a, RopeTable tab,
+                                                                   int vec_per_cta) {
+  const int n_vec = a.H + a.Hkv;
+  const int n_blk = (n_vec + vec_per_cta - 1) / vec_per_cta;
+  const int bt = blockIdx.x / n_blk;
+  const int blk = blockIdx.x - bt * n_blk;
   const int b = bt / a.T;
   const int t = bt - b * a.T;
   const int sp = a.start_pos[b];
   if (sp < 0 || (long long)sp + a.T > a.S) {
-    if (t == 0 && threadIdx.x == 0) set_status(a.dev_status, KVATTN_DEV_START_POS_RANGE);
+    if (t == 0 && blk == 0 && threadIdx.x == 0) set_status(a.dev_status, KVATTN_DEV_START_POS_RANGE);
     return;
   }
   const long long pos = (long long)sp + t;
@@ -45,37 +55,35 @@ __global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(RopeAppendArg
   __syncthreads();
 
   constexpr int kPairs = kHeadDim / 2;
-  const int q_pairs = a.H * kPairs;
-  const int total = (a.H + a.Hkv) * kPairs;
-  const uint32_t* q_in = reinterpret_cast<const uint32_t*>(a.q) + (size_t)bt * q_pairs;
-  uint32_t* q_out = reinterpret_cast<uint32_t*>(a.q_rot) + (size_t)bt * q_pairs;
-  const uint32_t* k_in = reinterpret_cast<const uint32_t*>(a.k_new) + (size_t)bt * a.Hkv * kPairs;
-  uint32_t* k_out = reinterpret_cast<uint32_t*>(a.cache_k) + ((size_t)b * a.S + pos) * a.Hkv * kPairs;
+  const int v0 = blk * vec_per_cta;
+  const int nv = min(vec_per_cta, n_vec - v0);
+  // vector v < H is query head v, else key head v - H
+  auto vec_in = [&](int v) -> const uint16_t* {
+    return v < a.H ? a.q + ((size_t)bt * a.H + v) * kHeadDim
+                   : a.k_new + ((size_t)bt * a.Hkv + (v - a.H)) * kHeadDim;
+  };
+  auto vec_out = [&](int v) -> uint16_t* {
+    return v < a.H ? a.q_rot + ((size_t)bt * a.H + v) * kHeadDim
+                   : a.cache_k + (((size_t)b * a.S + pos) * a.Hkv + (v - a.H)) * kHeadDim;
+  };
 
   if (tab.layout == 0 && rp == kPairs) {
     // Meta layout over the whole head: each pair is one 32-bit word
-    for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {
+    for (int idx = threadIdx.x; idx < nv * kPairs; idx += blockDim.x) {
+      const int v = v0 + idx / kPairs;
       const int i = idx & (kPairs - 1);
-      const bool is_q = idx < q_pairs;
-      const uint32_t w = is_q ? q_in[idx] : k_in[idx - q_pairs];
+      const uint32_t w = reinterpret_cast<const uint32_t*>(vec_in(v))[i];
       uint16_t y0, y1;
       rope_rotate_bits(true, s_cos[i], s_sin[i], (uint16_t)(w & 0xFFFFu), (uint16_t)(w >> 16), y0, y1);
-      const uint32_t r = (uint32_t)y0 | ((uint32_t)y1 << 16);
-      if (is_q)
-        q_out[idx] = r;
-      else
-        k_out[idx - q_pairs] = r;
+      reinterpret_cast<uint32_t*>(vec_out(v))[i] = (uint32_t)y0 | ((uint32_t)y1 << 16);
     }
   } else {
     // any layout / rotary width, one slot (pair or pass-through pair) at a time
-    for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {
-      const int vec = idx >> 6;
+    for (int idx = threadIdx.x; idx < nv * kPairs; idx += blockDim.x) {
+      const int v = v0 + idx / kPairs;
       const int j = idx & (kPairs - 1);
-      const bool is_q = vec < a.H;
-      const uint16_t* in = is_q ? reinterpret_cast<const uint16_t*>(q_in) + (size_t)vec * kHeadDim
-                                : reinterpret_cast<const uint16_t*>(k_in) + (size_t)(vec - a.H) * kHeadDim;
-      uint16_t* outp = is_q ? reinterpret_cast<uint16_t*>(q_out) + (size_t)vec * kHeadDim
-                            : reinterpret_cast<uint16_t*>(k_out) + (size_t)(vec - a.H) * kHeadDim;
+      const uint16_t* in = vec_in(v);
+      uint16_t* outp = vec_out(v);
       const RopeSlot sl = rope_slot(tab, j);
       uint16_t ya, yb;
       rope_rotate_bits(sl.rotate, sl.rotate ? s_cos[j] : 1.0, sl.rotate ? s_sin[j] : 0.0, in[sl.ea], in[sl.eb], ya,
@@ -85,10 +93,13 @@ __global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(RopeAppendArg
     }
   }
 
-  // values: bit copy of Hkv rows of 256 bytes
+  // values: bit copy of the 256-byte rows of this CTA's key heads
+  const int k0 = max(v0, a.H) - a.H;       // first key head of this CTA
+  const int k1 = max(v0 + nv, a.H) - a.H;  // one past the last
   const uint4* v_in = reinterpret_cast<const uint4*>(a.v_new) + (size_t)bt * a.Hkv * (kHeadDim / 8);
   uint4* v_out = reinterpret_cast<uint4*>(a.cache_v) + ((size_t)b * a.S + pos) * a.Hkv * (kHeadDim / 8);
-  for (int idx = threadIdx.x; idx < a.Hkv * (kHeadDim / 8); idx += blockDim.x) v_out[idx] = v_in[idx];
+  for (int idx = k0 * (kHeadDim / 8) + threadIdx.x; idx < k1 * (kHeadDim / 8); idx += blockDim.x)
+    v_out[idx] = v_in[idx];
 }
 
 }  // namespace
@@ -97,9 +108,16 @@ cudaError_t launch_rope_append(const RopeAppendArgs& a, const RopeTable& tab, cu
   // every tensor argument must have been set (callers value-initialise the args)
   if (!a.q || !a.q_rot || !a.k_new || !a.v_new || !a.cache_k || !a.cache_v || !a.start_pos)
     return cudaErrorInvalidValue;
-  const long long blocks = (long long)a.B * a.T;
+  // a few tokens (decode): 8 head vectors per CTA so the launch covers the
+  // SMs; many tokens (prefill): whole tokens, so each CTA builds its (cos,
+  // sin) table once for all of the token's heads
+  const long long tokens = (long long)a.B * a.T;
+  const int n_vec = a.H + a.Hkv;
+  const int per_cta = tokens >= 512 ? n_vec : 8;
+  const long long n_blk = (n_vec + per_cta - 1) / per_cta;
+  const long long blocks = tokens * n_blk;
   if (blocks > 0x7FFFFFFFll) return cudaErrorInvalidValue;
-  rope_append_kernel<<<(unsigned)blocks, kRopeThreads, 0, stream>>>(a, tab);
+  rope_append_kernel<<<(unsigned)blocks, kRopeThreads, 0, stream>>>(a, tab, per_cta);
   return cudaGetLastError();
 }
 
