@@ -6,8 +6,9 @@
 One "step" is one pass of the whole hot path over one batch: for every layer,
 RoPE + cache append (kvattn_rope_append) then attention (kvattn_decode: the
 split-K kernel and its LSE merge kernel, or kvattn_prefill_chunk for the
-prefill workload), each layer with its own cache.  --path fused times the
-single-launch kvattn_decode_fused instead.  The default workload is batched ragged decode: B=64 sequences, 32
+prefill workload), each layer with its own cache.  Small, latency-bound
+decode workloads (the single sequence at p=1000) run the single-launch
+kvattn_decode_fused instead (--path auto; --path split|fused forces one).  The default workload is batched ragged decode: B=64 sequences, 32
 layers with separate [64, 8192, 8, 128] bf16 caches (64 GiB in HBM, far
 larger than L2, so every step streams its K/V rows from HBM), start positions
 uniform in [512, 8191].
@@ -194,7 +195,7 @@ class Layer:
     pass
 
 
-def build_state(w, seed, device, path="split"):
+def build_state(w, seed, device, path="auto"):
     import torch
     import gqa_decode_attention_kvattn_b200 as kv
     sp = w.start_pos(seed)
@@ -216,6 +217,8 @@ def build_state(w, seed, device, path="split"):
         L.q_rot = torch.empty_like(L.q)
         L.out = torch.empty_like(L.q)
         layers.append(L)
+    if path == "auto":
+        path = "fused" if w.B * w.Hkv * w.kv_len_hint < (1 << 18) else "split"
     fused = w.kind == "decode" and path == "fused"
     if fused:
         ws_bytes = kv.kvattn_decode_fused_workspace_bytes(w.B, w.H, w.Hkv, w.S, w.kv_len_hint)
@@ -595,9 +598,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=HEADLINE)
     ap.add_argument("--seed", type=int, default=ks.DEFAULT_SEED)
-    ap.add_argument("--path", choices=["fused", "split"], default="split",
-                    help="decode entry points: rope_append + decode (+ merge kernel), the faster on B200 today, "
-                         "or one kvattn_decode_fused launch per layer")
+    ap.add_argument("--path", choices=["auto", "fused", "split"], default="auto",
+                    help="decode entry points: rope_append + decode (+ merge kernel), or one kvattn_decode_fused "
+                         "launch per layer; auto takes the fused launch for small, latency-bound calls (fewer than "
+                         "2^18 (row, KV head) pairs per layer) and the split path otherwise")
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

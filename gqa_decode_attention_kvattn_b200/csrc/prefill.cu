@@ -42,8 +42,16 @@ namespace {
 constexpr int kBM = 128;            // query rows per tile
 constexpr int kBN = 128;            // key rows per tile
 constexpr int kHalf = 128 * 64 * 2; // one 128-row x 64-element bf16 half tile (16 KB)
-constexpr int kPrefillThreads = 320;  // 10 warps
-constexpr int kSoftmaxWarps = 8;
+#ifndef KVATTN_PREFILL_COL_GROUPS
+#define KVATTN_PREFILL_COL_GROUPS 2
+#endif
+// softmax warps per TMEM lane quarter: each takes 128 / kColGroups columns of
+// its 32 rows (more warps hide more of the softmax's latency)
+constexpr int kColGroups = KVATTN_PREFILL_COL_GROUPS;
+constexpr int kCols = 128 / kColGroups;  // S / O columns per softmax thread
+constexpr int kSoftmaxWarps = 4 * kColGroups;
+constexpr int kPrefillThreads = 64 + 32 * kSoftmaxWarps;
+static_assert(kColGroups == 2 || kColGroups == 4, "column groups");
 constexpr uint32_t kTmemCols = 512; // S0 [0,128), S1 [128,256), O [256,384), P0 [384,448), P1 [448,512)
 constexpr uint32_t kColO = 256;
 constexpr uint32_t kColP = 384;     // bf16 P, two per 32-bit column: 64 columns per buffer
@@ -60,9 +68,9 @@ constexpr uint32_t kBarQFull = 0, kBarKFull = 1, kBarKEmpty = 3, kBarVFull = 5, 
                    kBarSEmpty = 11, kBarPFull = 13, kBarPVDone = 15, kBarMmaDone = 17, kNumBars = 18;
 constexpr uint32_t kOffTmemSlot = kOffBar + 8 * kNumBars;
 constexpr uint32_t kOffAbort = kOffTmemSlot + 8;
-constexpr uint32_t kOffXmax = kOffAbort + 8;        // [2 column halves][128 rows] fp32
-constexpr uint32_t kOffXsum = kOffXmax + 2 * 128 * 4;
-constexpr uint32_t kPrefillSmemBytes = kOffXsum + 2 * 128 * 4 + 1024;  // + alignment slack
+constexpr uint32_t kOffXmax = kOffAbort + 8;        // [column groups][128 rows] fp32
+constexpr uint32_t kOffXsum = kOffXmax + kColGroups * 128 * 4;
+constexpr uint32_t kPrefillSmemBytes = kOffXsum + kColGroups * 128 * 4 + 1024;  // + alignment slack
 
 // ------------------------------------------------------------ raw smem helpers
 __device__ __forceinline__ void bar_init(uint32_t a, uint32_t count) {
@@ -200,6 +208,14 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,"
       "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
       KV_W32(r)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
@@ -353,7 +369,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   } else {
     // ================================================================ softmax / epilogue
     const int quarter = warp & 3;         // TMEM lanes 32*quarter .. +31
-    const int ch = (warp - 2) >> 2;       // column half: S/O columns 64*ch .. +63
+    const int cg = (warp - 2) >> 2;       // column group: S/O columns kCols*cg .. +kCols-1
     const int m = 32 * quarter + lane;    // query row of this thread
     const int tok = t0 + m / G;
     const int head = kvh * G + (m % G);
@@ -361,22 +377,23 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     // with a window: keys n_sink <= k < lo_vis are hidden as well
     const int lo_vis = a.window > 0 ? lim - a.window + 1 : 0;
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * quarter) << 16);
-    const int st = tid - 64;              // 0..255 among the softmax threads
-    const uint32_t xmax_mine = base + kOffXmax + (uint32_t)(ch * 128 + m) * 4;
-    const uint32_t xmax_other = base + kOffXmax + (uint32_t)((1 - ch) * 128 + m) * 4;
-    const int pair_bar = 1 + quarter;     // named barrier of the two warps sharing these rows
+    const int st = tid - 64;              // index among the softmax threads
+    const uint32_t xmax_row = base + kOffXmax + (uint32_t)m * 4;  // + g * 512 for group g
+    const int row_bar = 1 + quarter;      // named barrier of the warps sharing these rows
+    constexpr int kRowThreads = 32 * kColGroups;
     float m_ref = -INFINITY;
-    float l = 0.f;                        // sum over this thread's column half
+    float l = 0.f;                        // sum over this thread's columns
 
     for (int j = 0; j < n_iter; ++j) {
       const int s = j & 1;
       const int jt = key_tile(j);
       bar_wait(bar(kBarSFull + s), (j >> 1) & 1, abort_addr, a.dev_status);
       tc_fence_after();
-      // this thread's 64 columns of the S row: two 32-column loads, one wait
-      uint32_t sr[2][32];
+      // this thread's kCols columns of the S row
+      uint32_t sr[kCols / 32][32];
 #pragma unroll
-      for (int c2 = 0; c2 < 2; ++c2) tmem_ld32(lane_addr + (uint32_t)s * 128u + 64u * ch + 32u * c2, sr[c2]);
+      for (int c2 = 0; c2 < kCols / 32; ++c2)
+        tmem_ld32(lane_addr + (uint32_t)s * 128u + (uint32_t)(kCols * cg) + 32u * c2, sr[c2]);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
@@ -384,10 +401,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 
       // mask (raw scores; the scale is folded into the exponent below) and
       // partial row max over eight independent accumulators
-      const int kbase = jt * kBN + 64 * ch;
-      if (kbase + 63 > lim || (kbase < lo_vis && kbase + 63 >= a.n_sink)) {
+      const int kbase = jt * kBN + kCols * cg;
+      if (kbase + kCols - 1 > lim || (kbase < lo_vis && kbase + kCols - 1 >= a.n_sink)) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
+        for (int c = 0; c < kCols; ++c) {
           const int k = kbase + c;
           if (k > lim || (k < lo_vis && k >= a.n_sink)) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
         }
@@ -396,19 +413,24 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll
       for (int k = 0; k < 8; ++k) mx8[k] = __uint_as_float(sr[0][k]);
 #pragma unroll
-      for (int c = 8; c < 64; c += 8)
+      for (int c = 8; c < kCols; c += 8)
 #pragma unroll
         for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], __uint_as_float(sr[c >> 5][(c & 31) + k]));
-      const float mx_half = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+      const float mx_part = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      // combine with the other column half: both threads of a row take the
+      // combine the column groups of the row: every thread of a row takes the
       // same decisions from the same numbers
-      asm volatile("st.shared.f32 [%0], %1;" ::"r"(xmax_mine), "f"(mx_half) : "memory");
-      named_bar_sync(pair_bar, 64);
-      float mx_other;
-      asm volatile("ld.shared.f32 %0, [%1];" : "=f"(mx_other) : "r"(xmax_other) : "memory");
-      named_bar_sync(pair_bar, 64);  // both read before either writes the next tile's value
-      const float mx = fmaxf(mx_half, mx_other) * a.scale_log2;
+      asm volatile("st.shared.f32 [%0], %1;" ::"r"(xmax_row + (uint32_t)cg * 512u), "f"(mx_part) : "memory");
+      named_bar_sync(row_bar, kRowThreads);
+      float mx_row = -INFINITY;
+#pragma unroll
+      for (int g2 = 0; g2 < kColGroups; ++g2) {
+        float v;
+        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(xmax_row + (uint32_t)g2 * 512u) : "memory");
+        mx_row = fmaxf(mx_row, v);
+      }
+      named_bar_sync(row_bar, kRowThreads);  // all read before any writes the next tile's value
+      const float mx = mx_row * a.scale_log2;
       const bool move = mx > m_ref + 8.f;
       const float m_new = move ? mx : m_ref;
       const float alpha = move ? fast_exp2(m_ref - m_new) : 1.f;
@@ -418,10 +440,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       const float neg_m = (m_new == -INFINITY) ? 0.f : -m_new;
       const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2);
       const uint64_t nm2 = f2_pack(neg_m, neg_m);
-      uint32_t pk[32];
+      uint32_t pk[kCols / 2];
       uint64_t sum2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) {
+      for (int c = 0; c < kCols; c += 2) {
         const uint64_t sv = ((uint64_t)sr[c >> 5][(c & 31) + 1] << 32) | sr[c >> 5][c & 31];
         float x0, x1;
         f2_unpack(f2_fma(sv, sc2, nm2), x0, x1);
@@ -441,13 +463,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         tc_fence_after();
         {
 #pragma unroll
-          for (int c2 = 0; c2 < 2; ++c2) {
+          for (int c2 = 0; c2 < kCols / 32; ++c2) {
             uint32_t r[32];
-            tmem_ld32(lane_addr + kColO + 64u * ch + 32u * c2, r);
+            tmem_ld32(lane_addr + kColO + (uint32_t)(kCols * cg) + 32u * c2, r);
             tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
-            tmem_st32(lane_addr + kColO + 64u * ch + 32u * c2, r);
+            tmem_st32(lane_addr + kColO + (uint32_t)(kCols * cg) + 32u * c2, r);
           }
           tmem_wait_st();
         }
@@ -470,8 +492,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           st_shared_v4(sV + (2 * s + half) * kHalf + r * 128 + cc * 16, 0u, 0u, 0u, 0u);
         }
       }
-      // P row m, keys 64*ch .. +63: columns 32*ch .. +31 of P buffer j%2
-      tmem_st32(lane_addr + kColP + 64u * (uint32_t)s + 32u * ch, pk);
+      // P row m, keys kCols*cg .. +kCols-1: columns kCols/2*cg .. of P buffer j%2
+      if constexpr (kCols == 64) {
+        tmem_st32(lane_addr + kColP + 64u * (uint32_t)s + 32u * cg, *reinterpret_cast<const uint32_t(*)[32]>(pk));
+      } else {
+        tmem_st16(lane_addr + kColP + 64u * (uint32_t)s + 16u * cg, *reinterpret_cast<const uint32_t(*)[16]>(pk));
+      }
       tmem_wait_st();
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the zeroed V rows, if any
       tc_fence_before();
@@ -479,29 +505,33 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       if (lane == 0) bar_arrive(bar(kBarPFull + s));
     }
 
-    // ---- epilogue: O / l -> bf16 rows (this thread's 64 columns)
-    const uint32_t xsum_mine = base + kOffXsum + (uint32_t)(ch * 128 + m) * 4;
-    const uint32_t xsum_other = base + kOffXsum + (uint32_t)((1 - ch) * 128 + m) * 4;
-    asm volatile("st.shared.f32 [%0], %1;" ::"r"(xsum_mine), "f"(l) : "memory");
-    named_bar_sync(pair_bar, 64);
-    float l_other;
-    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(l_other) : "r"(xsum_other) : "memory");
+    // ---- epilogue: O / l -> bf16 rows (this thread's kCols columns)
+    const uint32_t xsum_row = base + kOffXsum + (uint32_t)m * 4;
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(xsum_row + (uint32_t)cg * 512u), "f"(l) : "memory");
+    named_bar_sync(row_bar, kRowThreads);
+    float l_row = 0.f;
+#pragma unroll
+    for (int g2 = 0; g2 < kColGroups; ++g2) {
+      float v;
+      asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(xsum_row + (uint32_t)g2 * 512u) : "memory");
+      l_row += v;
+    }
     bar_wait(bar(kBarPVDone + ((n_iter - 1) & 1)), ((n_iter - 1) >> 1) & 1, abort_addr, a.dev_status);
     tc_fence_after();
-    float inv_l = 1.f / (l + l_other);
+    float inv_l = 1.f / l_row;
     if (a.sink_logits) {
       // learned sink: e^{sink} joins the denominator (log2 units, reference m_ref)
       const float s2 = __ldg(a.sink_logits + head) * 1.4426950408889634f;
       const float mn = fmaxf(m_ref, s2);
       const float f = (m_ref == -INFINITY) ? 0.f : fast_exp2(m_ref - mn);
-      inv_l = f / ((l + l_other) * f + fast_exp2(s2 - mn));
+      inv_l = f / (l_row * f + fast_exp2(s2 - mn));
     }
     const bool store = tok < a.T;
-    uint16_t* dst = a.out + (((size_t)b * a.T + (store ? tok : 0)) * a.H + head) * kHeadDim + 64 * ch;
+    uint16_t* dst = a.out + (((size_t)b * a.T + (store ? tok : 0)) * a.H + head) * kHeadDim + kCols * cg;
 #pragma unroll
-    for (int c2 = 0; c2 < 2; ++c2) {
+    for (int c2 = 0; c2 < kCols / 32; ++c2) {
       uint32_t r[32];
-      tmem_ld32(lane_addr + kColO + 64u * ch + 32u * c2, r);
+      tmem_ld32(lane_addr + kColO + (uint32_t)(kCols * cg) + 32u * c2, r);
       tmem_wait_ld();
       if (store) {
 #pragma unroll
