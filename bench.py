@@ -228,7 +228,7 @@ def build_state(w, seed, device, path="auto"):
             ws_bytes = kv.kvattn_decode_workspace_bytes(w.B, w.H, w.Hkv, w.S, w.kv_len_hint)
         else:
             ws_bytes = kv.kvattn_prefill_workspace_bytes(w.B, w.H, w.Hkv, w.S, w.T, w.kv_len_hint)
-        ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=device)
+        ws = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device=device)  # counters start at zero
     status = torch.zeros(1, dtype=torch.int32, device=device)
     torch.cuda.synchronize(device)
     return dict(sp=sp, dsp=dsp, rope=rope, layers=layers, ws=ws, ws_bytes=ws_bytes, status=status, fused=fused)

@@ -253,8 +253,10 @@ def kvattn_prefill_workspace_bytes(batch, n_heads, n_kv_heads, max_seq_len, T, m
 
 
 def alloc_workspace(nbytes: int, device=None):
+    """A zeroed decode workspace (its work counter must start at zero; every
+    completed call leaves it zero)."""
     import torch
-    return torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device or "cuda")
+    return torch.zeros(max(nbytes, 16), dtype=torch.uint8, device=device or "cuda")
 
 
 def _mask(window, n_sink, sink_logits):

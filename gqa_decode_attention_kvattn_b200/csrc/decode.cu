@@ -512,6 +512,8 @@ __global__ void __launch_bounds__(kThreads, Shape<G>::MIN_BLOCKS) decode_splitk_
   // the compiler, so accesses through `sm` become LDS/STS
   extern __shared__ __align__(128) unsigned char smem_raw[];
   Smem<G>& sm = *reinterpret_cast<Smem<G>*>(smem_raw);
+  pdl_wait();  // the previous kernel in the stream (rope_append, say) has finished
+  pdl_launch_dependents();
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -835,6 +837,10 @@ __global__ void __launch_bounds__(kThreads, Shape<G>::MIN_BLOCKS) decode_splitk_
 // K3: log-sum-exp merge of the split partials.  One CTA per (head, row set),
 // one thread per output element; one pass with a running maximum.
 __global__ void __launch_bounds__(kHeadDim) decode_merge_kernel(const DecodeArgs a) {
+  pdl_wait();  // the split-K kernel has finished and its partials are visible
+  pdl_launch_dependents();
+  // the split-K kernel is done with the work counter: leave it zero for the next call
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0 && a.counter) *a.counter = 0;
   const int head = blockIdx.x;
   const int v = blockIdx.y;
   const int L = set_length<true>(a, v);
@@ -920,6 +926,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(
   static_assert(G == 1 || G == 2 || G == 4 || G == 8 || G == 16, "tensor-core decode handles G <= 16");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   SmemMma<G>& sm = *reinterpret_cast<SmemMma<G>*>(smem_raw);
+  pdl_wait();  // the previous kernel in the stream (rope_append, say) has finished
+  pdl_launch_dependents();
   // the 128B-swizzled tiles need a 1024-byte aligned base; refuse otherwise
   if ((smem_u32(smem_raw) & 1023u) != 0) {
     if (threadIdx.x == 0) set_status(a.dev_status, KVATTN_DEV_INTERNAL);
@@ -1234,18 +1242,12 @@ cudaError_t launch_g(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorM
     configured[dev] = true;
   }
   const int evict_first = a.Tq == 1 ? 1 : 0;
-  if (!FUSED && a.counter) {
-    // the fused kernel leaves its counters at zero itself
-    cudaError_t e1 = cudaMemsetAsync(a.counter, 0, sizeof(int), st);
-    if (e1 != cudaSuccess) return e1;
-  }
-  kernel<<<a.grid, kThreads, smem, st>>>(tk, tv, a, evict_first, tab);
-  cudaError_t e = cudaGetLastError();
+  // The work counter starts at zero: the merge kernel (unfused) or the last
+  // CTA to finish (fused) resets it after every call.
+  cudaError_t e = launch_pdl(kernel, dim3(a.grid), dim3(kThreads), smem, st, tk, tv, a, evict_first, tab);
   if (e != cudaSuccess) return e;
   if (!FUSED && (a.max_splits > 1 || a.sink_logits)) {
-    dim3 grid(a.H, a.B * a.Tq);
-    decode_merge_kernel<<<grid, kHeadDim, 0, st>>>(a);
-    e = cudaGetLastError();
+    e = launch_pdl(decode_merge_kernel, dim3(a.H, a.B * a.Tq), dim3(kHeadDim), 0, st, a);
   }
   return e;
 }
@@ -1341,14 +1343,20 @@ DecodePlan plan_decode(int B, int Tq, int H, int Hkv, int kv_len_hint, int sm_co
   if (p.grid < 1) p.grid = 1;
   // partial (o, max, sum) per (row set, split, head), then the work counter
   p.ws_bytes = (p.max_splits > 1 || always_partials)
-                   ? (size_t)row_sets * p.max_splits * H * (kHeadDim + 2) * sizeof(float) + 16
+                   ? 16 + (size_t)row_sets * p.max_splits * H * (kHeadDim + 2) * sizeof(float)
                    : 0;
-  // fused: the same, then (work, exit) counters and one merge counter per
-  // (row set, KV head), padded to 16 bytes
+  // fused: the same plus one merge counter per (row set, KV-head group),
+  // padded to 16 bytes (see bind_decode_workspace)
   p.fused_ws_bytes = p.max_splits > 1 ? p.ws_bytes + (((size_t)row_sets * Hkv * sizeof(int) + 15) & ~(size_t)15) : 0;
   return p;
 }
 
+// Workspace layout: a 16-byte header (work counter; exit counter of the fused
+// decode), the fused decode's merge counters (one per row set and KV-head
+// group, padded to 16 bytes), then the partial o [row sets, splits, H, d] and
+// (max, sum) [row sets, splits, H, 2].  The counters sit at fixed offsets, so
+// calls of any shape can share one workspace; every completed call leaves them
+// zero, and they must be zero before the first call.
 void bind_decode_workspace(DecodeArgs& a, const DecodePlan& plan, void* workspace, bool fused) {
   a.exit_counter = nullptr;
   a.merge_counter = nullptr;
@@ -1359,14 +1367,16 @@ void bind_decode_workspace(DecodeArgs& a, const DecodePlan& plan, void* workspac
     return;
   }
   const size_t n_slots = (size_t)a.B * a.Tq * plan.max_splits * a.H;
-  float* ws = static_cast<float*>(workspace);
-  a.ws_o = ws;
-  a.ws_ml = ws + n_slots * kHeadDim;
-  a.counter = reinterpret_cast<int*>(ws + n_slots * (kHeadDim + 2));
+  unsigned char* base = static_cast<unsigned char*>(workspace);
+  a.counter = reinterpret_cast<int*>(base);
+  size_t off = 16;
   if (fused) {
     a.exit_counter = a.counter + 1;
-    a.merge_counter = a.counter + 4;
+    a.merge_counter = reinterpret_cast<int*>(base + off);
+    off += ((size_t)a.B * a.Tq * a.Hkv * sizeof(int) + 15) & ~(size_t)15;
   }
+  a.ws_o = reinterpret_cast<float*>(base + off);
+  a.ws_ml = a.ws_o + n_slots * kHeadDim;
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st,

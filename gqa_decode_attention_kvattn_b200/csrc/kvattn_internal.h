@@ -9,6 +9,26 @@
 
 namespace kvattn {
 
+// Launch `kernel` with programmatic stream serialization: it may be scheduled
+// while the previous kernel in the stream is finishing, and waits for it
+// (pdl_wait) before it touches any input.  Every kernel of the library starts
+// that way, so any of them may follow any other.
+template <class... KArgs, class... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 // Maps a launch result to a kvattn_status (KVATTN_OK or KVATTN_ERR_CUDA) and
 // remembers a failure for kvattn_last_cuda_error() on this host thread.
 int launch_status(cudaError_t e);

@@ -232,6 +232,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_v, const PrefillArgs a) {
   constexpr int TT = kBM / G;  // tokens per M tile
+  pdl_wait();  // the previous kernel in the stream (rope_append, say) has finished
+  pdl_launch_dependents();
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const uint32_t sQ = base + kOffQ, sK = base + kOffK, sV = base + kOffV;
@@ -571,8 +573,8 @@ cudaError_t launch_prefill_g(const PrefillArgs& a, const CUtensorMap& tq, const 
   }
   const long long grid = (long long)a.n_mtiles * a.Hkv * a.B;
   if (grid <= 0 || grid > 0x7FFFFFFFll) return cudaErrorInvalidValue;
-  prefill_tc_kernel<G><<<(unsigned)grid, kPrefillThreads, kPrefillSmemBytes, st>>>(tq, tk, tv, a);
-  return cudaGetLastError();
+  return launch_pdl(prefill_tc_kernel<G>, dim3((unsigned)grid), dim3(kPrefillThreads), kPrefillSmemBytes, st, tq, tk,
+                    tv, a);
 }
 
 }  // namespace

@@ -30,6 +30,8 @@ constexpr int kRopeThreads = 128;
 // vec_per_cta: head vectors (query or key heads) per CTA
 __global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(RopeAppendArgs a, RopeTable tab,
                                                                    int vec_per_cta) {
+  pdl_wait();  // the previous kernel in the stream has finished
+  pdl_launch_dependents();
   const int n_vec = a.H + a.Hkv;
   const int n_blk = (n_vec + vec_per_cta - 1) / vec_per_cta;
   const int bt = blockIdx.x / n_blk;
@@ -117,8 +119,7 @@ cudaError_t launch_rope_append(const RopeAppendArgs& a, const RopeTable& tab, cu
   const long long n_blk = (n_vec + per_cta - 1) / per_cta;
   const long long blocks = tokens * n_blk;
   if (blocks > 0x7FFFFFFFll) return cudaErrorInvalidValue;
-  rope_append_kernel<<<(unsigned)blocks, kRopeThreads, 0, stream>>>(a, tab, per_cta);
-  return cudaGetLastError();
+  return launch_pdl(rope_append_kernel, dim3((unsigned)blocks), dim3(kRopeThreads), 0, stream, a, tab, per_cta);
 }
 
 }  // namespace kvattn

@@ -147,8 +147,14 @@ KVATTN_API size_t kvattn_decode_workspace_bytes(const kvattn_dims* dims, int32_t
  * workspace.  A sequence above the hint or outside the cache leaves its
  * output untouched and sets a KVATTN_DEV_* bit.  out is bf16 [B,1,H,d].
  * workspace: device memory of kvattn_decode_workspace_bytes() bytes, 16-byte
- * aligned, owned by the caller, contents need no initialisation; calls that
- * share a workspace must be ordered on one stream.
+ * aligned, owned by the caller.  Its first 16 bytes hold a work counter that
+ * must be ZERO before the first call (e.g. cudaMemset once after
+ * allocation); every call leaves it zero again (the merge kernel resets it),
+ * so one workspace serves calls of any shape with no memset between them.
+ * Calls that share a workspace must be ordered on one stream.
+ * Every kernel of the library is launched with programmatic stream
+ * serialization and waits for the previous kernel in the stream before it
+ * reads anything, so consecutive calls may overlap their launch and tail.
  * Host errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
 KVATTN_API int kvattn_decode(const kvattn_dims* dims, const uint16_t* q_rot, const uint16_t* cache_k,
                   const uint16_t* cache_v, const int32_t* start_pos, int32_t max_kv_len_hint,
@@ -258,7 +264,8 @@ KVATTN_API int kvattn_decode_fused(const kvattn_dims* dims, const kvattn_rope_pa
  *    device; make that first call before any stream capture.
  *  - Every call shares the one array: calls whose kernels overlap on the GPU
  *    (other streams, other host threads) race and must be serialised by the
- *    caller.  Nothing in the array needs to start at zero.
+ *    caller.  The array starts zeroed and each call leaves its work counter
+ *    zero again.
  *  - Shapes whose partials need more than the array (see
  *    kvattn_decode_workspace_bytes) return KVATTN_ERR_WORKSPACE and launch
  *    nothing. */

@@ -281,3 +281,26 @@ def test_decode_kernel_choice():
     assert not kv.kvattn_decode_plan(1, 32, 8, 8192, max_kv_len_hint=1001)["tensor_cores"]
     assert kv.kvattn_decode_plan(1, 64, 8, 4096)["tensor_cores"]
     assert not kv.kvattn_decode_plan(64, 16, 8, 8192)["tensor_cores"]
+
+
+def test_decode_workspace_shared_across_shapes_and_left_zeroed():
+    """One workspace serves calls of different shapes in a row: its work
+    counter sits at a fixed offset and every call leaves it zero."""
+    ws = kv.alloc_workspace(kv.kvattn_decode_workspace_bytes(8, 32, 8, 8192))
+    for seed, (B, H, Hkv, S, sp) in enumerate([(8, 32, 8, 8192, [8191, 0, 63, 64, 4000, 777, 5000, 12]),
+                                               (4, 32, 8, 4096, [1499, 700, 64, 1000]),
+                                               (3, 64, 8, 3000, [2999, 5, 1500])]):
+        q, k, v, ck, cv = U.host_inputs(70 + seed, B, 1, H, Hkv, S, sp)
+        dq, dk, dv, dck, dcv = (U.to_dev(x) for x in (q, k, v, ck, cv))
+        dsp = torch.from_numpy(np.asarray(sp, np.int32)).cuda()
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        q_rot = kv.kvattn_rope_append(dq, dk, dv, dck, dcv, dsp, dev_status=st)
+        need = kv.kvattn_decode_workspace_bytes(B, H, Hkv, S)
+        out = kv.kvattn_decode(q_rot, dck, dcv, dsp, workspace=ws[:max(need, 16)], dev_status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        assert int(ws[:16].view(torch.int32).abs().sum().item()) == 0
+        o_ck, o_cv = ck.copy(), cv.copy()
+        _, ref, rc = oracle.step(q, k, v, o_ck, o_cv, np.asarray(sp, np.int32), U.oracle_freqs(kv.LLAMA3))
+        assert rc == 0
+        U.assert_attention_close(U.to_host(out), ref, f"shape {B},{H},{Hkv},{S}")
