@@ -11,26 +11,33 @@
 //
 // Tiling.  The G query heads of one KV head and 128/G consecutive tokens form
 // one 128-row M tile (row m = token * G + head), so the grouped heads share
-// every K/V tile without a materialised repeat.  One CTA owns one (M tile, KV
-// head, sequence) and walks the key rows in 128-row tiles up to the last key
-// its last token sees.  Per KV tile j:
-//   S_j = Q K_j^T        tcgen05.mma M=128 N=128 K=16 x8, bf16 -> fp32 in TMEM
-//   P_j = softmax part   8 warps, each row split over two threads, read S
-//                        from TMEM, mask, exponentiate (log2 units), write
-//                        bf16 P back into TMEM
-//   O  += P_j V_j        tcgen05.mma with P read from TMEM and V from shared
+// every K/V tile without a materialised repeat.  One CTA owns two consecutive
+// M tiles of one (KV head, sequence) and walks the key rows in 128-row tiles
+// up to the last key its last token sees; each K/V tile it loads serves both
+// Q tiles, which halves the K/V bytes the SMs pull from L2 per MMA (with one
+// Q tile per CTA the kernel was bound by that traffic).  Per KV tile j and Q
+// tile g:
+//   S_g = Q_g K_j^T      tcgen05.mma M=128 N=128 K=16 x8, bf16 -> fp32 in TMEM
+//   P_g = softmax part   one thread per row reads its 128 scores from TMEM,
+//                        masks, exponentiates (log2 units) and writes the
+//                        bf16 P row back over the S columns it has read
+//   O_g += P_g V_j       tcgen05.mma with P read from TMEM and V from shared
 //                        memory as an MN-major operand, fp32 in TMEM
-// S and P are double buffered in TMEM so that S_{j+1} = Q K_{j+1}^T runs on
-// the tensor cores while the softmax warps work on S_j; O stays in TMEM.  P
-// never touches shared memory, which leaves shared-memory bandwidth to the
-// TMA writes and the Q, K, V operand reads.  The
-// reference max of a row only moves when a tile's max exceeds it by more than
-// 8 (probabilities stay <= 2^8), so O is rescaled rarely.
+// TMEM holds S_0, S_1, O_0 and O_1 (512 columns).  The MMA thread ping-pongs
+// between the Q tiles, QK_0(j), PV_1(j-1), QK_1(j), PV_0(j), so the tensor
+// cores run one tile's MMAs while the softmax warps of the other work, and
+// QK_g(j+1) waits for PV_g(j) to finish reading P_g(j) out of the columns it
+// overwrites.  P never touches shared memory, which leaves shared-memory
+// bandwidth to the TMA writes and the Q, K, V operand reads.
+//
+// The softmax reference.  A row's reference max only moves when a tile's max
+// exceeds it by more than 8 (probabilities stay <= 2^8), so O is rescaled
+// rarely; when it moves, the row's thread rescales O_g itself (PV_g(j-1) has
+// finished by the time S_g(j) exists).
 //
 // Warps: 0 = TMA producer, 1 = TMEM owner and MMA issuer (one thread),
 // 2..9 = softmax and epilogue: warp w reads TMEM lanes 32*(w%4)..+31 and
-// takes column half (w-2)/4 of every S and O row; the two warps that share
-// rows exchange their partial row maxima through shared memory.
+// works on Q tile (w-2)/4.
 #include "kvattn_device.cuh"
 #include "kvattn_internal.h"
 
@@ -42,35 +49,32 @@ namespace {
 constexpr int kBM = 128;            // query rows per tile
 constexpr int kBN = 128;            // key rows per tile
 constexpr int kHalf = 128 * 64 * 2; // one 128-row x 64-element bf16 half tile (16 KB)
-#ifndef KVATTN_PREFILL_COL_GROUPS
-#define KVATTN_PREFILL_COL_GROUPS 2
-#endif
-// softmax warps per TMEM lane quarter: each takes 128 / kColGroups columns of
-// its 32 rows (more warps hide more of the softmax's latency)
-constexpr int kColGroups = KVATTN_PREFILL_COL_GROUPS;
-constexpr int kCols = 128 / kColGroups;  // S / O columns per softmax thread
-constexpr int kSoftmaxWarps = 4 * kColGroups;
+// two softmax groups of four warps (one warp per TMEM lane quarter each), one
+// per Q tile
+constexpr int kGroupWarps = 4;
+constexpr int kGroupThreads = 32 * kGroupWarps;
+constexpr int kSoftmaxWarps = 2 * kGroupWarps;
 constexpr int kPrefillThreads = 64 + 32 * kSoftmaxWarps;
-static_assert(kColGroups == 2 || kColGroups == 4, "column groups");
-constexpr uint32_t kTmemCols = 512; // S0 [0,128), S1 [128,256), O [256,384), P0 [384,448), P1 [448,512)
+// TMEM: S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512); bf16 P_g is
+// written over the first 64 columns of S_g (two per 32-bit column)
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0;
 constexpr uint32_t kColO = 256;
-constexpr uint32_t kColP = 384;     // bf16 P, two per 32-bit column: 64 columns per buffer
 
 // shared memory layout (offsets from a 1024-byte aligned base)
-constexpr uint32_t kOffQ = 0;                       // 2 halves
-constexpr uint32_t kOffK = kOffQ + 2 * kHalf;       // [stage 2][half 2]
+constexpr uint32_t kOffQ = 0;                       // [Q tile 2][half 2]
+constexpr uint32_t kOffK = kOffQ + 4 * kHalf;       // [stage 2][half 2]
 constexpr uint32_t kOffV = kOffK + 4 * kHalf;       // [stage 2][half 2]
 constexpr uint32_t kOffBar = kOffV + 4 * kHalf;
-// barrier slots (8 bytes each)
+// barrier slots (8 bytes each): K/V per stage, S/P/PV per Q tile
 // (every pipeline barrier exists once per buffer, so a waiter is never more
 // than one phase behind the barrier it waits on)
 constexpr uint32_t kBarQFull = 0, kBarKFull = 1, kBarKEmpty = 3, kBarVFull = 5, kBarVEmpty = 7, kBarSFull = 9,
-                   kBarSEmpty = 11, kBarPFull = 13, kBarPVDone = 15, kBarMmaDone = 17, kNumBars = 18;
+                   kBarPFull = 11, kBarPVDone = 13, kBarMmaDone = 15, kNumBars = 16;
 constexpr uint32_t kOffTmemSlot = kOffBar + 8 * kNumBars;
 constexpr uint32_t kOffAbort = kOffTmemSlot + 8;
-constexpr uint32_t kOffXmax = kOffAbort + 8;        // [column groups][128 rows] fp32
-constexpr uint32_t kOffXsum = kOffXmax + kColGroups * 128 * 4;
-constexpr uint32_t kPrefillSmemBytes = kOffXsum + kColGroups * 128 * 4 + 1024;  // + alignment slack
+constexpr uint32_t kPrefillSmemBytes = kOffAbort + 8 + 1024;  // + alignment slack
+static_assert(kPrefillSmemBytes <= 227 * 1024, "shared memory per CTA");
 
 // ------------------------------------------------------------ raw smem helpers
 __device__ __forceinline__ void bar_init(uint32_t a, uint32_t count) {
@@ -82,9 +86,6 @@ __device__ __forceinline__ void bar_arrive(uint32_t a) {
 __device__ __forceinline__ void bar_expect_tx(uint32_t a, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(a), "r"(bytes) : "memory");
 }
-#ifndef KVATTN_PREFILL_SPIN_MMA
-#define KVATTN_PREFILL_SPIN_MMA 0
-#endif
 #ifndef KVATTN_PREFILL_SPIN_ALL
 #define KVATTN_PREFILL_SPIN_ALL 1
 #endif
@@ -244,24 +245,26 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
-  // heaviest M tiles (latest tokens, most keys) first
-  const int per_tile = a.Hkv * a.B;
-  const int mtile = a.n_mtiles - 1 - (int)(blockIdx.x / per_tile);
-  const int rem = (int)(blockIdx.x % per_tile);
+  // heaviest M tile pairs (latest tokens, most keys) first
+  const int per_pair = a.Hkv * a.B;
+  const int n_pairs = (a.n_mtiles + 1) / 2;
+  const int pair = n_pairs - 1 - (int)(blockIdx.x / per_pair);
+  const int rem = (int)(blockIdx.x % per_pair);
   const int kvh = rem % a.Hkv;
   const int b = rem / a.Hkv;
   const int sp = a.start_pos[b];
   if (sp < 0 || (long long)sp + a.T > a.S || (long long)sp + a.T > a.kv_len_hint) {
-    if (mtile == 0 && kvh == 0 && tid == 0)
+    if (pair == 0 && kvh == 0 && tid == 0)
       set_status(a.dev_status, (sp < 0 || (long long)sp + a.T > a.S) ? KVATTN_DEV_START_POS_RANGE
                                                                     : KVATTN_DEV_KV_LEN_HINT);
     return;
   }
-  const int t0 = mtile * TT;
-  const int t_last = min(t0 + TT, a.T) - 1;
-  const int Lmax = sp + t_last + 1;          // keys the tile's last token sees
+  // Q tile g holds tokens t0 + g*TT ..; the second exists when it starts before T
+  const int t0 = pair * 2 * TT;
+  const int n_q = (t0 + TT < a.T) ? 2 : 1;
+  const int Lmax = sp + min(t0 + n_q * TT, a.T);  // keys the pair's last token sees
   const int n_kv = (Lmax + kBN - 1) / kBN;
-  // Key tiles the M tile reads: all of 0..n_kv-1, or with a window the tiles
+  // Key tiles the pair reads: all of 0..n_kv-1, or with a window the tiles
   // holding the attention sinks followed by the tiles from the one holding
   // the first token's earliest window key (the union of the rows' windows).
   int sink_tiles = 0, win_first = 0;
@@ -271,6 +274,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   }
   const int n_iter = sink_tiles + (n_kv - win_first);
   auto key_tile = [&](int j) { return j < sink_tiles ? j : win_first + (j - sink_tiles); };
+  // Q tile 0 stops at the key tile of its own last token (at most one short)
+  const int n_kv0 = (sp + min(t0 + TT, a.T) + kBN - 1) / kBN;
+  const int n_it0 = sink_tiles + (n_kv0 - win_first);
+  auto active = [&](int g, int j) { return g < n_q && j < (g == 0 ? n_it0 : n_iter); };
 
   if (tid == 0) {
     bar_init(bar(kBarQFull), 1);
@@ -280,8 +287,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       bar_init(bar(kBarVFull + s), 1);
       bar_init(bar(kBarVEmpty + s), 1);
       bar_init(bar(kBarSFull + s), 1);
-      bar_init(bar(kBarSEmpty + s), kSoftmaxWarps);
-      bar_init(bar(kBarPFull + s), kSoftmaxWarps);
+      bar_init(bar(kBarPFull + s), kGroupWarps);
       bar_init(bar(kBarPVDone + s), 1);
     }
     bar_init(bar(kBarMmaDone), 1);
@@ -305,9 +311,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       prefetch_tensormap(&tmap_q);
       prefetch_tensormap(&tmap_k);
       prefetch_tensormap(&tmap_v);
-      bar_expect_tx(bar(kBarQFull), 2 * kHalf);
-      tma_load_4d_raw(sQ, &tmap_q, bar(kBarQFull), 0, kvh * G, t0, b);
-      tma_load_4d_raw(sQ + kHalf, &tmap_q, bar(kBarQFull), 64, kvh * G, t0, b);
+      bar_expect_tx(bar(kBarQFull), (uint32_t)n_q * 2u * kHalf);
+      for (int g = 0; g < n_q; ++g) {
+        tma_load_4d_raw(sQ + (2 * g) * kHalf, &tmap_q, bar(kBarQFull), 0, kvh * G, t0 + g * TT, b);
+        tma_load_4d_raw(sQ + (2 * g + 1) * kHalf, &tmap_q, bar(kBarQFull), 64, kvh * G, t0 + g * TT, b);
+      }
       for (int j = 0; j < n_iter; ++j) {
         const int s = j & 1;
         const uint32_t par = ((j >> 1) & 1) ^ 1;
@@ -327,42 +335,58 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_m128_n128(false);
       constexpr uint32_t idesc_pv = idesc_bf16_m128_n128(true);
-      constexpr bool kMmaSuspend = !(KVATTN_PREFILL_SPIN_MMA || KVATTN_PREFILL_SPIN_ALL);
       bool ok = bar_wait(bar(kBarQFull), 0, abort_addr, a.dev_status);
       tc_fence_after();
-      auto issue_qk = [&](int j) {
-        const int s = j & 1;
-        if (!bar_wait(bar(kBarKFull + s), (j >> 1) & 1, abort_addr, a.dev_status, kMmaSuspend)) return false;
-        if (!bar_wait(bar(kBarSEmpty + s), ((j >> 1) & 1) ^ 1, abort_addr, a.dev_status, kMmaSuspend)) return false;
+      // S_g = Q_g K_j^T into S buffer g, once PV_g(j-1) has read P_g(j-1)
+      // out of the same columns
+      auto qk = [&](int g, int j) {
+        if (j > 0 && !bar_wait(bar(kBarPVDone + g), (uint32_t)(j - 1) & 1u, abort_addr, a.dev_status)) return false;
         tc_fence_after();
+        const int s = j & 1;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t da = sw128_desc(sQ + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024);
+          const uint64_t da = sw128_desc(sQ + (2 * g + (kk >> 2)) * kHalf + (kk & 3) * 32, 16, 1024);
           const uint64_t db = sw128_desc(sK + (2 * s + (kk >> 2)) * kHalf + (kk & 3) * 32, 16, 1024);
-          tc_mma(tmem + (uint32_t)s * 128u, da, db, idesc_qk, kk > 0 ? 1u : 0u);
+          tc_mma(tmem + kColS + 128u * (uint32_t)g, da, db, idesc_qk, kk > 0 ? 1u : 0u);
         }
-        tc_commit(bar(kBarSFull + s));
-        tc_commit(bar(kBarKEmpty + s));
+        tc_commit(bar(kBarSFull + g));
         return true;
       };
-      if (ok) ok = issue_qk(0);
-      for (int j = 0; j < n_iter && ok; ++j) {
-        if (j + 1 < n_iter && !issue_qk(j + 1)) break;
+      // O_g += P_g(j) V_j once the softmax has published P_g(j)
+      auto pv = [&](int g, int j) {
         const int s = j & 1;
-        if (!bar_wait(bar(kBarPFull + s), (j >> 1) & 1, abort_addr, a.dev_status, kMmaSuspend)) break;
-        if (!bar_wait(bar(kBarVFull + s), (j >> 1) & 1, abort_addr, a.dev_status, kMmaSuspend)) break;
+        if (!bar_wait(bar(kBarVFull + s), (uint32_t)(j >> 1) & 1u, abort_addr, a.dev_status)) return false;
+        if (!bar_wait(bar(kBarPFull + g), (uint32_t)j & 1u, abort_addr, a.dev_status)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          // P_j from TMEM: keys 16kk..16kk+15 are columns 8kk..8kk+7 of its buffer
-          const uint32_t pa = tmem + kColP + 64u * (uint32_t)s + 8u * kk;
+          // P_g from TMEM: keys 16kk..16kk+15 are columns 8kk..8kk+7 of S buffer g
+          const uint32_t pa = tmem + kColS + 128u * (uint32_t)g + 8u * kk;
           // V tile as B = [keys x dims], dims contiguous: 64-dim atoms one half
           // apart (LBO), 8-key groups 1 KB apart (SBO); 16 keys per step
           const uint64_t db = sw128_desc(sV + (2 * s) * kHalf + kk * 2048, kHalf, 1024);
-          tc_mma_ts(tmem + kColO, pa, db, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_ts(tmem + kColO + 128u * (uint32_t)g, pa, db, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(bar(kBarVEmpty + s));
-        tc_commit(bar(kBarPVDone + s));
+        tc_commit(bar(kBarPVDone + g));
+        return true;
+      };
+      // Ping-pong: the tensor cores run Q tile 1's MMAs while the softmax
+      // works on tile 0's scores and the other way round.  Per key tile j:
+      //   QK_0(j), PV_1(j-1), QK_1(j), PV_0(j)
+      for (int j = 0; j <= n_iter && ok; ++j) {
+        if (j < n_iter) {
+          if (!bar_wait(bar(kBarKFull + (j & 1)), (uint32_t)(j >> 1) & 1u, abort_addr, a.dev_status)) break;
+          if (active(0, j) && !qk(0, j)) break;
+        }
+        if (j > 0) {
+          if (active(1, j - 1) && !pv(1, j - 1)) break;
+          tc_commit(bar(kBarVEmpty + ((j - 1) & 1)));  // both PVs of tile j-1 issued
+        }
+        if (j < n_iter) {
+          if (active(1, j) && !qk(1, j)) break;
+          tc_commit(bar(kBarKEmpty + (j & 1)));  // both QKs of tile j issued
+          if (active(0, j) && !pv(0, j)) break;
+        }
       }
       tc_commit(bar(kBarMmaDone));
       // every MMA issued above has finished once this completes
@@ -371,42 +395,37 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   } else {
     // ================================================================ softmax / epilogue
     const int quarter = warp & 3;         // TMEM lanes 32*quarter .. +31
-    const int cg = (warp - 2) >> 2;       // column group: S/O columns kCols*cg .. +kCols-1
-    const int m = 32 * quarter + lane;    // query row of this thread
-    const int tok = t0 + m / G;
+    const int grp = (warp - 2) >> 2;      // Q tile of this warp
+    const int m = 32 * quarter + lane;    // query row of this thread within its Q tile
+    const int tok = t0 + grp * TT + m / G;
     const int head = kvh * G + (m % G);
     const int lim = sp + min(tok, a.T - 1);  // last visible key (rows past T borrow the last token's)
     // with a window: keys n_sink <= k < lo_vis are hidden as well
     const int lo_vis = a.window > 0 ? lim - a.window + 1 : 0;
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * quarter) << 16);
-    const int st = tid - 64;              // index among the softmax threads
-    const uint32_t xmax_row = base + kOffXmax + (uint32_t)m * 4;  // + g * 512 for group g
-    const int row_bar = 1 + quarter;      // named barrier of the warps sharing these rows
-    constexpr int kRowThreads = 32 * kColGroups;
-    float m_ref = -INFINITY;
-    float l = 0.f;                        // sum over this thread's columns
+    const uint32_t col_s = kColS + 128u * (uint32_t)grp;  // S, then P over its first 64 columns
+    const uint32_t col_o = kColO + 128u * (uint32_t)grp;
+    const int gt = tid - 64 - kGroupThreads * grp;  // index within the group
+    const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2);
+    float ref = -INFINITY;   // reference max (log2 units) of the row
+    float l = 0.f;           // row sum in units of 2^ref
 
-    for (int j = 0; j < n_iter; ++j) {
-      const int s = j & 1;
+    for (int j = 0; active(grp, j); ++j) {
       const int jt = key_tile(j);
-      bar_wait(bar(kBarSFull + s), (j >> 1) & 1, abort_addr, a.dev_status);
+      bar_wait(bar(kBarSFull + grp), (uint32_t)j & 1u, abort_addr, a.dev_status);
       tc_fence_after();
-      // this thread's kCols columns of the S row
-      uint32_t sr[kCols / 32][32];
+      // the thread's whole S row
+      uint32_t sr[4][32];
 #pragma unroll
-      for (int c2 = 0; c2 < kCols / 32; ++c2)
-        tmem_ld32(lane_addr + (uint32_t)s * 128u + (uint32_t)(kCols * cg) + 32u * c2, sr[c2]);
+      for (int c2 = 0; c2 < 4; ++c2) tmem_ld32(lane_addr + col_s + 32u * c2, sr[c2]);
       tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) bar_arrive(bar(kBarSEmpty + s));
 
       // mask (raw scores; the scale is folded into the exponent below) and
-      // partial row max over eight independent accumulators
-      const int kbase = jt * kBN + kCols * cg;
-      if (kbase + kCols - 1 > lim || (kbase < lo_vis && kbase + kCols - 1 >= a.n_sink)) {
+      // row max over eight independent accumulators
+      const int kbase = jt * kBN;
+      if (kbase + kBN - 1 > lim || (kbase < lo_vis && kbase + kBN - 1 >= a.n_sink)) {
 #pragma unroll
-        for (int c = 0; c < kCols; ++c) {
+        for (int c = 0; c < kBN; ++c) {
           const int k = kbase + c;
           if (k > lim || (k < lo_vis && k >= a.n_sink)) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
         }
@@ -415,125 +434,94 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll
       for (int k = 0; k < 8; ++k) mx8[k] = __uint_as_float(sr[0][k]);
 #pragma unroll
-      for (int c = 8; c < kCols; c += 8)
+      for (int c = 8; c < kBN; c += 8)
 #pragma unroll
         for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], __uint_as_float(sr[c >> 5][(c & 31) + k]));
-      const float mx_part = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                  fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      // combine the column groups of the row: every thread of a row takes the
-      // same decisions from the same numbers
-      asm volatile("st.shared.f32 [%0], %1;" ::"r"(xmax_row + (uint32_t)cg * 512u), "f"(mx_part) : "memory");
-      named_bar_sync(row_bar, kRowThreads);
-      float mx_row = -INFINITY;
-#pragma unroll
-      for (int g2 = 0; g2 < kColGroups; ++g2) {
-        float v;
-        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(xmax_row + (uint32_t)g2 * 512u) : "memory");
-        mx_row = fmaxf(mx_row, v);
-      }
-      named_bar_sync(row_bar, kRowThreads);  // all read before any writes the next tile's value
-      const float mx = mx_row * a.scale_log2;
-      const bool move = mx > m_ref + 8.f;
-      const float m_new = move ? mx : m_ref;
-      const float alpha = move ? fast_exp2(m_ref - m_new) : 1.f;
-      m_ref = m_new;
-      // p = 2^(s * scale_log2 - m): packed FMA for two scores, one ex2 each,
-      // packed sums in four accumulators
-      const float neg_m = (m_new == -INFINITY) ? 0.f : -m_new;
-      const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2);
-      const uint64_t nm2 = f2_pack(neg_m, neg_m);
-      uint32_t pk[kCols / 2];
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) *
+                       a.scale_log2;
+      const bool move = mx > ref + 8.f;
+      const float ref_new = move ? mx : ref;
+      const float alpha = move ? fast_exp2(ref - ref_new) : 1.f;
+      ref = ref_new;
+      // p = 2^(s * scale_log2 - ref): packed FMA for two scores, one ex2 each,
+      // packed sums in four accumulators; 32 keys (16 P columns) at a time,
+      // written over the S columns already read
+      const float neg_ref = (ref == -INFINITY) ? 0.f : -ref;
+      const uint64_t nr2 = f2_pack(neg_ref, neg_ref);
       uint64_t sum2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-      for (int c = 0; c < kCols; c += 2) {
-        const uint64_t sv = ((uint64_t)sr[c >> 5][(c & 31) + 1] << 32) | sr[c >> 5][c & 31];
-        float x0, x1;
-        f2_unpack(f2_fma(sv, sc2, nm2), x0, x1);
-        const float p0 = fast_exp2(x0);
-        const float p1 = fast_exp2(x1);
-        sum2[(c >> 1) & 3] = f2_add(sum2[(c >> 1) & 3], f2_pack(p0, p1));
-        pk[c >> 1] = pack_bf16x2_rn(p0, p1);
+      for (int c2 = 0; c2 < 4; ++c2) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          const uint64_t sv = ((uint64_t)sr[c2][c + 1] << 32) | sr[c2][c];
+          float x0, x1;
+          f2_unpack(f2_fma(sv, sc2, nr2), x0, x1);
+          const float p0 = fast_exp2(x0);
+          const float p1 = fast_exp2(x1);
+          sum2[(c >> 1) & 3] = f2_add(sum2[(c >> 1) & 3], f2_pack(p0, p1));
+          pk[c >> 1] = pack_bf16x2_rn(p0, p1);
+        }
+        tmem_st16(lane_addr + col_s + 16u * c2, pk);
       }
       float sa, sb;
       f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), sa, sb);
-      const float sum = sa + sb;
-      l = l * alpha + sum;
+      l = l * alpha + (sa + sb);
 
       if (j > 0 && __any_sync(0xffffffffu, move)) {
-        // a row's reference moved: rescale its O once PV_{j-1} has finished
-        bar_wait(bar(kBarPVDone + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort_addr, a.dev_status);
-        tc_fence_after();
-        {
+        // a row's reference moved: rescale its O (PV_g(j-1) has finished:
+        // QK_g(j) was issued after it)
 #pragma unroll
-          for (int c2 = 0; c2 < kCols / 32; ++c2) {
-            uint32_t r[32];
-            tmem_ld32(lane_addr + kColO + (uint32_t)(kCols * cg) + 32u * c2, r);
-            tmem_wait_ld();
+        for (int c2 = 0; c2 < 4; ++c2) {
+          uint32_t r[32];
+          tmem_ld32(lane_addr + col_o + 32u * c2, r);
+          tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
-            tmem_st32(lane_addr + kColO + (uint32_t)(kCols * cg) + 32u * c2, r);
-          }
-          tmem_wait_st();
+          for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
+          tmem_st32(lane_addr + col_o + 32u * c2, r);
         }
-      }
-      if (j >= 2) {
-        // P buffer j%2 is free once PV_{j-2} has read it
-        bar_wait(bar(kBarPVDone + s), ((j >> 1) - 1) & 1, abort_addr, a.dev_status);
-        tc_fence_after();
       }
       if (j == n_iter - 1 && Lmax < jt * kBN + kBN) {
         // rows of the last V tile past the last visible key may hold any bits;
-        // zero them so that 0 * (garbage) cannot reach O
-        bar_wait(bar(kBarVFull + s), (j >> 1) & 1, abort_addr, a.dev_status);
+        // zero them so that 0 * (garbage) cannot reach O (both Q tiles' groups
+        // write the same zeros before their own P goes out)
+        const int s = j & 1;
+        bar_wait(bar(kBarVFull + s), (uint32_t)(j >> 1) & 1u, abort_addr, a.dev_status);
         const int first_bad = Lmax - jt * kBN;
         const int nchunks = (kBN - first_bad) * 16;  // 16-byte chunks over both halves
-        for (int c = st; c < nchunks; c += kSoftmaxWarps * 32) {
+        for (int c = gt; c < nchunks; c += kGroupThreads) {
           const int r = first_bad + (c >> 4);
           const int half = (c >> 3) & 1;
           const int cc = c & 7;
           st_shared_v4(sV + (2 * s + half) * kHalf + r * 128 + cc * 16, 0u, 0u, 0u, 0u);
         }
       }
-      // P row m, keys kCols*cg .. +kCols-1: columns kCols/2*cg .. of P buffer j%2
-      if constexpr (kCols == 64) {
-        tmem_st32(lane_addr + kColP + 64u * (uint32_t)s + 32u * cg, *reinterpret_cast<const uint32_t(*)[32]>(pk));
-      } else {
-        tmem_st16(lane_addr + kColP + 64u * (uint32_t)s + 16u * cg, *reinterpret_cast<const uint32_t(*)[16]>(pk));
-      }
       tmem_wait_st();
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the zeroed V rows, if any
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) bar_arrive(bar(kBarPFull + s));
+      if (lane == 0) bar_arrive(bar(kBarPFull + grp));
     }
 
-    // ---- epilogue: O / l -> bf16 rows (this thread's kCols columns)
-    const uint32_t xsum_row = base + kOffXsum + (uint32_t)m * 4;
-    asm volatile("st.shared.f32 [%0], %1;" ::"r"(xsum_row + (uint32_t)cg * 512u), "f"(l) : "memory");
-    named_bar_sync(row_bar, kRowThreads);
-    float l_row = 0.f;
-#pragma unroll
-    for (int g2 = 0; g2 < kColGroups; ++g2) {
-      float v;
-      asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(xsum_row + (uint32_t)g2 * 512u) : "memory");
-      l_row += v;
-    }
-    bar_wait(bar(kBarPVDone + ((n_iter - 1) & 1)), ((n_iter - 1) >> 1) & 1, abort_addr, a.dev_status);
+    // ---- epilogue: O / l -> bf16 rows
+    // (the MMA-done barrier completes once, after the last PV has finished)
+    bar_wait(bar(kBarMmaDone), 0, abort_addr, a.dev_status);
     tc_fence_after();
-    float inv_l = 1.f / l_row;
+    float inv_l = 1.f / l;
     if (a.sink_logits) {
-      // learned sink: e^{sink} joins the denominator (log2 units, reference m_ref)
+      // learned sink: e^{sink} joins the denominator (log2 units, reference ref)
       const float s2 = __ldg(a.sink_logits + head) * 1.4426950408889634f;
-      const float mn = fmaxf(m_ref, s2);
-      const float f = (m_ref == -INFINITY) ? 0.f : fast_exp2(m_ref - mn);
-      inv_l = f / (l_row * f + fast_exp2(s2 - mn));
+      const float mn = fmaxf(ref, s2);
+      const float f = (ref == -INFINITY) ? 0.f : fast_exp2(ref - mn);
+      inv_l = f / (l * f + fast_exp2(s2 - mn));
     }
-    const bool store = tok < a.T;
-    uint16_t* dst = a.out + (((size_t)b * a.T + (store ? tok : 0)) * a.H + head) * kHeadDim + kCols * cg;
+    const bool store = grp < n_q && tok < a.T;
+    uint16_t* dst = a.out + (((size_t)b * a.T + (store ? tok : 0)) * a.H + head) * kHeadDim;
 #pragma unroll
-    for (int c2 = 0; c2 < kCols / 32; ++c2) {
+    for (int c2 = 0; c2 < 4; ++c2) {
       uint32_t r[32];
-      tmem_ld32(lane_addr + kColO + (uint32_t)(kCols * cg) + 32u * c2, r);
+      tmem_ld32(lane_addr + col_o + 32u * c2, r);
       tmem_wait_ld();
       if (store) {
 #pragma unroll
@@ -571,7 +559,7 @@ cudaError_t launch_prefill_g(const PrefillArgs& a, const CUtensorMap& tq, const 
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
-  const long long grid = (long long)a.n_mtiles * a.Hkv * a.B;
+  const long long grid = (long long)((a.n_mtiles + 1) / 2) * a.Hkv * a.B;  // one CTA per M tile pair
   if (grid <= 0 || grid > 0x7FFFFFFFll) return cudaErrorInvalidValue;
   return launch_pdl(prefill_tc_kernel<G>, dim3((unsigned)grid), dim3(kPrefillThreads), kPrefillSmemBytes, st, tq, tk,
                     tv, a);
