@@ -25,9 +25,9 @@
 //                        memory as an MN-major operand, fp32 in TMEM
 // TMEM holds S_0, S_1, O_0 and O_1 (512 columns).  The MMA thread ping-pongs
 // between the Q tiles, QK_0(j), PV_1(j-1), QK_1(j), PV_0(j), so the tensor
-// cores run one tile's MMAs while the softmax warps of the other work, and
-// QK_g(j+1) waits for PV_g(j) to finish reading P_g(j) out of the columns it
-// overwrites.  P never touches shared memory, which leaves shared-memory
+// cores run one tile's MMAs while the softmax warps of the other work.
+// QK_g(j+1) overwrites the columns PV_g(j) reads P_g(j) from; it is issued
+// after PV_g(j) by the same thread, and one thread's MMAs run in issue order.  P never touches shared memory, which leaves shared-memory
 // bandwidth to the TMA writes and the Q, K, V operand reads.
 //
 // The softmax reference.  A row's reference max only moves when a tile's max
@@ -66,11 +66,11 @@ constexpr uint32_t kOffQ = 0;                       // [Q tile 2][half 2]
 constexpr uint32_t kOffK = kOffQ + 4 * kHalf;       // [stage 2][half 2]
 constexpr uint32_t kOffV = kOffK + 4 * kHalf;       // [stage 2][half 2]
 constexpr uint32_t kOffBar = kOffV + 4 * kHalf;
-// barrier slots (8 bytes each): K/V per stage, S/P/PV per Q tile
+// barrier slots (8 bytes each): K/V per stage, S/P per Q tile
 // (every pipeline barrier exists once per buffer, so a waiter is never more
 // than one phase behind the barrier it waits on)
 constexpr uint32_t kBarQFull = 0, kBarKFull = 1, kBarKEmpty = 3, kBarVFull = 5, kBarVEmpty = 7, kBarSFull = 9,
-                   kBarPFull = 11, kBarPVDone = 13, kBarMmaDone = 15, kNumBars = 16;
+                   kBarPFull = 11, kBarMmaDone = 13, kNumBars = 14;
 constexpr uint32_t kOffTmemSlot = kOffBar + 8 * kNumBars;
 constexpr uint32_t kOffAbort = kOffTmemSlot + 8;
 constexpr uint32_t kPrefillSmemBytes = kOffAbort + 8 + 1024;  // + alignment slack
@@ -288,7 +288,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       bar_init(bar(kBarVEmpty + s), 1);
       bar_init(bar(kBarSFull + s), 1);
       bar_init(bar(kBarPFull + s), kGroupWarps);
-      bar_init(bar(kBarPVDone + s), 1);
     }
     bar_init(bar(kBarMmaDone), 1);
     st_shared_i32(abort_addr, 0);
@@ -337,10 +336,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       constexpr uint32_t idesc_pv = idesc_bf16_m128_n128(true);
       bool ok = bar_wait(bar(kBarQFull), 0, abort_addr, a.dev_status);
       tc_fence_after();
-      // S_g = Q_g K_j^T into S buffer g, once PV_g(j-1) has read P_g(j-1)
-      // out of the same columns
+      // S_g = Q_g K_j^T into S buffer g.  It is issued right after PV_g(j-1),
+      // which reads P_g(j-1) out of the same columns: MMAs issued by one
+      // thread run in issue order, so the PV has read its operand before this
+      // QK writes the accumulator.
       auto qk = [&](int g, int j) {
-        if (j > 0 && !bar_wait(bar(kBarPVDone + g), (uint32_t)(j - 1) & 1u, abort_addr, a.dev_status)) return false;
         tc_fence_after();
         const int s = j & 1;
 #pragma unroll
@@ -367,7 +367,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           const uint64_t db = sw128_desc(sV + (2 * s) * kHalf + kk * 2048, kHalf, 1024);
           tc_mma_ts(tmem + kColO + 128u * (uint32_t)g, pa, db, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(bar(kBarPVDone + g));
         return true;
       };
       // Ping-pong: the tensor cores run Q tile 1's MMAs while the softmax
