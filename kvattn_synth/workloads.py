@@ -58,6 +58,12 @@ WORKLOADS = {
     "decode_mqa_g32_b64": Workload(
         "decode_mqa_g32_b64", B=64, T=1, H=32, Hkv=1, S=32768, sp_lo=4096, sp_hi=32767,
         note="multi-query attention: all 32 query heads share one KV head"),
+    "decode_mha_g1_b16": Workload(
+        "decode_mha_g1_b16", B=16, T=1, H=32, Hkv=32, S=8192, sp_lo=512, sp_hi=8191,
+        note="multi-head attention: one KV head per query head (G = 1)"),
+    "decode_g2_b64": Workload(
+        "decode_g2_b64", B=64, T=1, H=16, Hkv=8, S=8192, sp_lo=512, sp_hi=8191,
+        note="16 query heads over 8 KV heads (G = 2, the Qwen3-0.6B layout)"),
 }
 
 # the workload the headline metric is quoted on

@@ -49,6 +49,8 @@ def _sample(w, sp):
     ("decode_long_scaled_b8", 0),
     ("decode_wide_g8_b128", 0),
     ("decode_mqa_g32_b64", 0),
+    ("decode_mha_g1_b16", 0),
+    ("decode_g2_b64", 0),
 ])
 def test_workload_full_size(name, layer):
     w = WORKLOADS[name]
