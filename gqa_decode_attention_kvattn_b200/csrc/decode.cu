@@ -1401,4 +1401,10 @@ cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tk, const CUte
 
 bool decode_use_mma(int G, long long work_rows) { return G >= 8 || (G == 4 && work_rows >= kMmaMinWork); }
 
+cudaError_t launch_decode_merge(const DecodeArgs& a, cudaStream_t st) {
+  if (!a.ws_o || !a.ws_ml || !a.out || !a.start_pos || a.rows_per_split < 1 || a.max_splits < 1)
+    return cudaErrorInvalidValue;
+  return launch_pdl(decode_merge_kernel, dim3(a.H, a.B * a.Tq), dim3(kHeadDim), 0, st, a);
+}
+
 }  // namespace kvattn

@@ -1,6 +1,7 @@
 // C-ABI layer of libkvattn.so: host-side validation, the RoPE frequency
 // table, TMA descriptors for the caches, and the launches.  Declared in
 // include/kvattn.h, which states each call's contract.
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -243,6 +244,52 @@ int run_attention(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, con
   a.dev_status = dev_status;
   a.grid = plan.grid;
   a.mma = plan.mma ? 1 : 0;
+
+  // One new token per sequence with all 32 query heads on one KV head (G = 32,
+  // multi-query): the 32 heads fill one 128-row tcgen05 M tile, so the
+  // tensor-core prefill kernel in split mode runs the contraction (the warp
+  // MMAs of the decode kernels top out near 100 TFLOP/s, a third of what
+  // this shape needs at HBM speed), then the same LSE merge.
+  const bool masked = mask && (mask->window > 0 || mask->sink_logits);
+  if (dims->n_heads == 32 * dims->n_kv_heads && T == 1 && !masked && plan.mma && plan.max_splits > 1 &&
+      plan.ws_bytes > 0) {
+    const int tiles_per_seq = (hint + 127) / 128;
+    // about four CTAs per SM over the call's key tiles, at least four tiles
+    // each, and no more splits per sequence than the workspace has slots for
+    const long long tiles = (long long)dims->batch * dims->n_kv_heads * tiles_per_seq;
+    long long st = std::max<long long>(4, (tiles + 4LL * sms - 1) / (4LL * sms));
+    st = std::max<long long>(st, (tiles_per_seq + plan.max_splits - 1) / plan.max_splits);
+    const int split_tiles = (int)std::min<long long>(st, tiles_per_seq);
+    const int split_grid = (tiles_per_seq + split_tiles - 1) / split_tiles;
+    CUtensorMap tq, tk2, tv2;
+    rc = encode_sw128_map(&tq, q_rot, dims->batch, 1, dims->n_heads, 32, kvattn::prefill_tokens_per_tile(32));
+    if (rc != KVATTN_OK) return rc;
+    rc = encode_sw128_map(&tk2, cache_k, dims->batch, dims->max_seq_len, dims->n_kv_heads, 1, 128);
+    if (rc != KVATTN_OK) return rc;
+    rc = encode_sw128_map(&tv2, cache_v, dims->batch, dims->max_seq_len, dims->n_kv_heads, 1, 128);
+    if (rc != KVATTN_OK) return rc;
+    kvattn::PrefillArgs p{};
+    p.B = dims->batch;
+    p.T = 1;
+    p.H = dims->n_heads;
+    p.Hkv = dims->n_kv_heads;
+    p.S = dims->max_seq_len;
+    p.kv_len_hint = hint;
+    p.n_mtiles = 1;
+    p.scale_log2 = a.scale_log2;
+    p.start_pos = start_pos;
+    p.out = out;
+    p.dev_status = dev_status;
+    p.split_tiles = split_tiles;
+    p.split_grid = split_grid;
+    p.part_splits = plan.max_splits;
+    p.part_o = a.ws_o;
+    p.part_ml = a.ws_ml;
+    a.rows_per_split = split_tiles * 128;
+    const cudaError_t e = kvattn::launch_prefill(p, tq, tk2, tv2, (cudaStream_t)stream);
+    if (e != cudaSuccess) return kvattn::launch_status(e);
+    return kvattn::launch_status(kvattn::launch_decode_merge(a, (cudaStream_t)stream));
+  }
   return kvattn::launch_status(kvattn::launch_decode(a, tk, tv, (cudaStream_t)stream));
 }
 
@@ -277,7 +324,7 @@ int run_prefill_tc(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, co
   rc = encode_sw128_map(&tv, cache_v, dims->batch, dims->max_seq_len, dims->n_kv_heads, 1, 128);
   if (rc != KVATTN_OK) return rc;
 
-  kvattn::PrefillArgs a;
+  kvattn::PrefillArgs a{};
   a.B = dims->batch;
   a.T = T;
   a.H = dims->n_heads;

@@ -148,6 +148,17 @@ struct PrefillArgs {
   int window;       // > 0: token at position p sees keys p - window < k <= p and k < n_sink
   int n_sink;
   const float* sink_logits;  // fp32 [H] learned sink logits (score units), or null
+  // Split mode (split_tiles > 0; no window, no learned sinks): CTA
+  // (unit, split) takes key tiles [split * split_tiles, +split_tiles) of its
+  // (sequence, KV head); split_grid splits per unit are launched.  A row set
+  // with more than one split writes its unnormalised O and (max in log2
+  // units, sum) to part_o [B*T, part_splits, H, d] / part_ml [.., 2], the
+  // layout the decode's LSE merge reads; one with a single split writes out.
+  int split_tiles;
+  int split_grid;
+  int part_splits;
+  float* part_o;
+  float* part_ml;
 };
 
 // Tokens per 128-row M tile for group size G (128 / G).
@@ -155,5 +166,9 @@ int prefill_tokens_per_tile(int G);
 
 cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& tmap_q, const CUtensorMap& tmap_k,
                            const CUtensorMap& tmap_v, cudaStream_t stream);
+
+// The decode's LSE merge of split partials (a.ws_o / a.ws_ml, a.rows_per_split
+// rows per split, a.max_splits slots per row set) into a.out.
+cudaError_t launch_decode_merge(const DecodeArgs& a, cudaStream_t stream);
 
 }  // namespace kvattn

@@ -245,16 +245,20 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
-  // heaviest M tile pairs (latest tokens, most keys) first
+  // heaviest M tile pairs (latest tokens, most keys) first; in split mode
+  // each (pair, KV head, sequence) unit has split_grid consecutive CTAs
+  const int n_split_grid = a.split_tiles > 0 ? a.split_grid : 1;
+  const int unit = (int)(blockIdx.x / n_split_grid);
+  const int split = (int)(blockIdx.x - (unsigned)unit * n_split_grid);
   const int per_pair = a.Hkv * a.B;
   const int n_pairs = (a.n_mtiles + 1) / 2;
-  const int pair = n_pairs - 1 - (int)(blockIdx.x / per_pair);
-  const int rem = (int)(blockIdx.x % per_pair);
+  const int pair = n_pairs - 1 - unit / per_pair;
+  const int rem = unit % per_pair;
   const int kvh = rem % a.Hkv;
   const int b = rem / a.Hkv;
   const int sp = a.start_pos[b];
   if (sp < 0 || (long long)sp + a.T > a.S || (long long)sp + a.T > a.kv_len_hint) {
-    if (pair == 0 && kvh == 0 && tid == 0)
+    if (pair == 0 && kvh == 0 && split == 0 && tid == 0)
       set_status(a.dev_status, (sp < 0 || (long long)sp + a.T > a.S) ? KVATTN_DEV_START_POS_RANGE
                                                                     : KVATTN_DEV_KV_LEN_HINT);
     return;
@@ -272,11 +276,21 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     win_first = max(0, sp + t0 - a.window + 1) / kBN;
     sink_tiles = min((a.n_sink + kBN - 1) / kBN, win_first);
   }
-  const int n_iter = sink_tiles + (n_kv - win_first);
-  auto key_tile = [&](int j) { return j < sink_tiles ? j : win_first + (j - sink_tiles); };
+  const int n_all = sink_tiles + (n_kv - win_first);
+  // this CTA's key tiles: j0 .. j0 + n_iter - 1 of the n_all (all of them
+  // unless in split mode); the loops below count j from 0
+  const int j0 = a.split_tiles > 0 ? split * a.split_tiles : 0;
+  const int n_iter = a.split_tiles > 0 ? min(a.split_tiles, n_all - j0) : n_all;
+  const int n_splits_here = a.split_tiles > 0 ? (n_all + a.split_tiles - 1) / a.split_tiles : 1;
+  if (n_iter <= 0) return;  // a shorter row set: no work in this split (before anything shared)
+  auto key_tile = [&](int j) {
+    const int jj = j0 + j;
+    return jj < sink_tiles ? jj : win_first + (jj - sink_tiles);
+  };
+  const bool last_split = j0 + n_iter == n_all;  // holds the row set's last key tile
   // Q tile 0 stops at the key tile of its own last token (at most one short)
   const int n_kv0 = (sp + min(t0 + TT, a.T) + kBN - 1) / kBN;
-  const int n_it0 = sink_tiles + (n_kv0 - win_first);
+  const int n_it0 = min(n_iter, sink_tiles + (n_kv0 - win_first) - j0);
   auto active = [&](int g, int j) { return g < n_q && j < (g == 0 ? n_it0 : n_iter); };
 
   if (tid == 0) {
@@ -481,7 +495,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           tmem_st32(lane_addr + col_o + 32u * c2, r);
         }
       }
-      if (j == n_iter - 1 && Lmax < jt * kBN + kBN) {
+      if (last_split && j == n_iter - 1 && Lmax < jt * kBN + kBN) {
         // rows of the last V tile past the last visible key may hold any bits;
         // zero them so that 0 * (garbage) cannot reach O (both Q tiles' groups
         // write the same zeros before their own P goes out)
@@ -516,6 +530,28 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       inv_l = f / (l * f + fast_exp2(s2 - mn));
     }
     const bool store = grp < n_q && tok < a.T;
+    if (a.split_tiles > 0 && n_splits_here > 1) {
+      // this split's partial: unnormalised O and (max, sum), both relative
+      // to 2^ref (a group without key tiles here contributes nothing)
+      const bool any = active(grp, 0);
+      const size_t slot = (((size_t)b * a.T + (store ? tok : 0)) * a.part_splits + split) * a.H + head;
+      float* po = a.part_o + slot * kHeadDim;
+#pragma unroll
+      for (int c2 = 0; c2 < 4; ++c2) {
+        uint32_t r[32];
+        tmem_ld32(lane_addr + col_o + 32u * c2, r);
+        tmem_wait_ld();
+        if (store) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 4)
+            *reinterpret_cast<float4*>(po + 32 * c2 + c) =
+                any ? make_float4(__uint_as_float(r[c]), __uint_as_float(r[c + 1]), __uint_as_float(r[c + 2]),
+                                  __uint_as_float(r[c + 3]))
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+      if (store) *reinterpret_cast<float2*>(a.part_ml + slot * 2) = make_float2(any ? ref : -INFINITY, any ? l : 0.f);
+    } else {
     uint16_t* dst = a.out + (((size_t)b * a.T + (store ? tok : 0)) * a.H + head) * kHeadDim;
 #pragma unroll
     for (int c2 = 0; c2 < 4; ++c2) {
@@ -533,6 +569,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           *reinterpret_cast<uint4*>(dst + 32 * c2 + c) = w;
         }
       }
+    }
     }
   }
 
@@ -558,7 +595,8 @@ cudaError_t launch_prefill_g(const PrefillArgs& a, const CUtensorMap& tq, const 
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
-  const long long grid = (long long)((a.n_mtiles + 1) / 2) * a.Hkv * a.B;  // one CTA per M tile pair
+  // one CTA per M tile pair (times split_grid in split mode)
+  const long long grid = (long long)((a.n_mtiles + 1) / 2) * a.Hkv * a.B * (a.split_tiles > 0 ? a.split_grid : 1);
   if (grid <= 0 || grid > 0x7FFFFFFFll) return cudaErrorInvalidValue;
   return launch_pdl(prefill_tc_kernel<G>, dim3((unsigned)grid), dim3(kPrefillThreads), kPrefillSmemBytes, st, tq, tk,
                     tv, a);

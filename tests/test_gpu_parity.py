@@ -58,7 +58,8 @@ def _check_step(seed, B, T, H, Hkv, S, sp, rope, kind, hint=0, in_place=False):
     (3, 32, 2, 700, [0, 63, 64, 699][:3], kv.LLAMA3),     # G = 16 (tensor cores)
     (4, 64, 8, 3000, [2999, 64, 65, 1000], kv.LLAMA3_1),  # G = 8, several splits
     (8, 32, 8, 8192, [8191, 0, 63, 64, 4000, 777, 5000, 12], kv.LLAMA3),  # G = 4 on the tensor-core kernel
-    (3, 32, 1, 2500, [0, 1000, 2499], kv.LLAMA3),       # G = 32 (MQA): two 16-head groups per KV head
+    (3, 32, 1, 2500, [0, 1000, 2499], kv.LLAMA3),       # G = 32 (MQA): tcgen05 split path, 1 / 2 / 5 splits
+    (6, 32, 1, 6000, [5999, 127, 128, 129, 3000, 4095], kv.LLAMA3_1),  # G = 32 at key-tile edges
     (2, 64, 2, 1500, [1499, 700], kv.LLAMA3),           # G = 32 with two KV heads
     (2, 64, 1, 900, [899, 33], kv.LLAMA3_1),            # G = 64 (MQA, 64 heads)
 ])
@@ -289,7 +290,8 @@ def test_decode_workspace_shared_across_shapes_and_left_zeroed():
     ws = kv.alloc_workspace(kv.kvattn_decode_workspace_bytes(8, 32, 8, 8192))
     for seed, (B, H, Hkv, S, sp) in enumerate([(8, 32, 8, 8192, [8191, 0, 63, 64, 4000, 777, 5000, 12]),
                                                (4, 32, 8, 4096, [1499, 700, 64, 1000]),
-                                               (3, 64, 8, 3000, [2999, 5, 1500])]):
+                                               (3, 64, 8, 3000, [2999, 5, 1500]),
+                                               (2, 32, 1, 3000, [2999, 100])]):
         q, k, v, ck, cv = U.host_inputs(70 + seed, B, 1, H, Hkv, S, sp)
         dq, dk, dv, dck, dcv = (U.to_dev(x) for x in (q, k, v, ck, cv))
         dsp = torch.from_numpy(np.asarray(sp, np.int32)).cuda()
