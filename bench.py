@@ -58,6 +58,8 @@ def measured_peaks():
 
 KERNEL_SOURCES = {
     "decode_splitk": ("decode.cu", "kvattn_device.cuh"),
+    # multi-query decode (G = 32): the tcgen05 kernel in split mode + the LSE merge
+    "decode_tc": ("prefill.cu", "decode.cu", "kvattn_device.cuh"),
     "decode_fused": ("decode.cu", "kvattn_device.cuh", "rope_device.cuh"),
     "prefill_chunk": ("prefill.cu", "kvattn_device.cuh"),
 }
@@ -429,9 +431,12 @@ def run_ours(args, w, rank, world, device):
         achieved = kv_bytes_layer / (attn_avg_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                 "frac": round(achieved / hbm_peak, 4),
-                "traffic": profiled_traffic("decode_fused" if st["fused"] else "decode_splitk", w.name),
+                "traffic": profiled_traffic("decode_fused" if st["fused"] else
+                                            "decode_tc" if w.H == 32 * w.Hkv else "decode_splitk", w.name),
                 "kernel": ("kvattn_decode_fused (rope + append + split-K attention + LSE merge, one kernel)"
-                           if st["fused"] else "kvattn_decode (split-K kernel + LSE merge kernel)"),
+                           if st["fused"] else
+                           "kvattn_decode (tcgen05 split kernel + LSE merge kernel)" if w.H == 32 * w.Hkv else
+                           "kvattn_decode (split-K kernel + LSE merge kernel)"),
                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback 6650 GB/s",
                 "avg_launch_ms": round(attn_avg_ms, 5), "launches_timed": nl,
                 "bytes_per_launch": kv_bytes_layer}

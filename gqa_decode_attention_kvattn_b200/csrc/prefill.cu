@@ -247,11 +247,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 
   // heaviest M tile pairs (latest tokens, most keys) first; in split mode
   // each (pair, KV head, sequence) unit has split_grid consecutive CTAs
+  const int per_pair = a.Hkv * a.B;
+  const int n_pairs = (a.n_mtiles + 1) / 2;
   const int n_split_grid = a.split_tiles > 0 ? a.split_grid : 1;
   const int unit = (int)(blockIdx.x / n_split_grid);
   const int split = (int)(blockIdx.x - (unsigned)unit * n_split_grid);
-  const int per_pair = a.Hkv * a.B;
-  const int n_pairs = (a.n_mtiles + 1) / 2;
   const int pair = n_pairs - 1 - unit / per_pair;
   const int rem = unit % per_pair;
   const int kvh = rem % a.Hkv;
