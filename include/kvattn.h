@@ -138,10 +138,15 @@ KVATTN_API size_t kvattn_decode_workspace_bytes(const kvattn_dims* dims, int32_t
  * The cache rows 0..start_pos[b] must already hold the sequence (row
  * start_pos[b] written by kvattn_rope_append earlier on the same stream).
  * The rows of each (sequence, KV head) are streamed from HBM once and serve
- * all G query heads (G = 32, 64, 128, e.g. multi-query attention, run as
- * G/16 groups of 16 heads over the same rows, scheduled side by side so the
- * repeat reads are served by L2); long rows are split across CTAs and the partial
- * (o, max, sum) triples are merged by log-sum-exp in a second kernel.
+ * all G query heads.  At G = 32 (e.g. multi-query attention with 32 heads) a
+ * call with more than one split runs on the 5th-generation tensor cores: the
+ * 32 heads form one 128-row MMA tile and each CTA takes a range of 128-row
+ * key tiles.  G = 64, 128 (and masked G = 32 calls) run as G/16 groups of 16
+ * heads over the same rows, scheduled side by side so the repeat reads are
+ * served by L2.  Long rows are split across CTAs and the partial
+ * (o, max, sum) triples are merged by log-sum-exp in a second kernel; the
+ * tensor-core G = 32 path uses the same workspace layout and merge, with its
+ * own split size (a multiple of 128 rows, never more splits than the plan's).
  * scale <= 0 selects 1/sqrt(d).  max_kv_len_hint (<= 0: max_seq_len) is a
  * host upper bound on start_pos[b] + 1; it sizes the splits and the
  * workspace.  A sequence above the hint or outside the cache leaves its
