@@ -98,7 +98,9 @@ struct DecodeArgs {
 // Group view of the decode kernels: G <= 16 query heads per KV head run as
 // one group; G = 32, 64, 128 run as G/16 groups of 16 heads that read the
 // same KV head (neighbouring work items, so the second read of a row is
-// normally served by L2).
+// normally served by L2).  (Unmasked multi-split G = 32 calls do not reach
+// these kernels: the decode entry runs them on the tcgen05 prefill kernel in
+// split mode.)
 inline void decode_group_view(int H, int Hkv, int* groups, int* kv_div) {
   const int G = H / Hkv;
   *kv_div = G > 16 ? G / 16 : 1;
