@@ -228,7 +228,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
   return r;
 }
 
-template <int G>
+// DUAL: split mode (a.split_tiles > 0), see the mapping below
+template <int G, bool DUAL>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_v, const PrefillArgs a) {
@@ -245,13 +246,17 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
-  // heaviest M tile pairs (latest tokens, most keys) first; in split mode
-  // each (pair, KV head, sequence) unit has split_grid consecutive CTAs
+  // heaviest M tile pairs (latest tokens, most keys) first.  In split mode
+  // (`dual`) the two Q tiles of a CTA are the same token's heads over two
+  // consecutive splits 2c, 2c + 1 of the row set, each with its own K/V
+  // stream (stage g), so one split's MMAs overlap the other's softmax; each
+  // (pair, KV head, sequence) unit then has ceil(split_grid / 2) CTAs.
+  constexpr bool dual = DUAL;
   const int per_pair = a.Hkv * a.B;
   const int n_pairs = (a.n_mtiles + 1) / 2;
-  const int n_split_grid = a.split_tiles > 0 ? a.split_grid : 1;
+  const int n_split_grid = dual ? (a.split_grid + 1) / 2 : 1;
   const int unit = (int)(blockIdx.x / n_split_grid);
-  const int split = (int)(blockIdx.x - (unsigned)unit * n_split_grid);
+  const int split = (int)(blockIdx.x - (unsigned)unit * n_split_grid);  // split pair c in split mode
   const int pair = n_pairs - 1 - unit / per_pair;
   const int rem = unit % per_pair;
   const int kvh = rem % a.Hkv;
@@ -277,21 +282,27 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     sink_tiles = min((a.n_sink + kBN - 1) / kBN, win_first);
   }
   const int n_all = sink_tiles + (n_kv - win_first);
-  // this CTA's key tiles: j0 .. j0 + n_iter - 1 of the n_all (all of them
-  // unless in split mode); the loops below count j from 0
-  const int j0 = a.split_tiles > 0 ? split * a.split_tiles : 0;
-  const int n_iter = a.split_tiles > 0 ? min(a.split_tiles, n_all - j0) : n_all;
-  const int n_splits_here = a.split_tiles > 0 ? (n_all + a.split_tiles - 1) / a.split_tiles : 1;
-  if (n_iter <= 0) return;  // a shorter row set: no work in this split (before anything shared)
-  auto key_tile = [&](int j) {
-    const int jj = j0 + j;
+  // Q tile g's key tiles: j0g[g] .. j0g[g] + ntg[g] - 1 of the n_all (all of
+  // them unless in split mode); the loops below count j from 0
+  const int n_splits_here = dual ? (n_all + a.split_tiles - 1) / a.split_tiles : 1;
+  // Q tile 0 stops at the key tile of its own last token (at most one short)
+  const int j00 = dual ? 2 * split * a.split_tiles : 0;
+  const int j01 = dual ? j00 + a.split_tiles : 0;
+  const int nt0 = dual ? max(0, min(a.split_tiles, n_all - j00))
+                       : sink_tiles + ((sp + min(t0 + TT, a.T) + kBN - 1) / kBN - win_first);
+  const int nt1 = dual ? max(0, min(a.split_tiles, n_all - j01)) : (n_q > 1 ? n_all : 0);
+  const int n_iter = max(nt0, nt1);
+  if (n_iter <= 0) return;  // a shorter row set: no work in this split pair (before anything shared)
+  auto first_tile = [&](int g) { return g == 0 ? j00 : j01; };
+  auto key_tile = [&](int g, int j) {
+    const int jj = first_tile(g) + j;
     return jj < sink_tiles ? jj : win_first + (jj - sink_tiles);
   };
-  const bool last_split = j0 + n_iter == n_all;  // holds the row set's last key tile
-  // Q tile 0 stops at the key tile of its own last token (at most one short)
-  const int n_kv0 = (sp + min(t0 + TT, a.T) + kBN - 1) / kBN;
-  const int n_it0 = min(n_iter, sink_tiles + (n_kv0 - win_first) - j0);
-  auto active = [&](int g, int j) { return g < n_q && j < (g == 0 ? n_it0 : n_iter); };
+  auto active = [&](int g, int j) { return j < (g == 0 ? nt0 : nt1); };
+  // K/V stage and phase parity of key tile j: a shared two-stage stream, or
+  // in split mode one stage per Q tile's stream
+  auto kv_stage = [&](int g, int j) { return dual ? g : (j & 1); };
+  auto kv_par = [&](int j) { return dual ? (uint32_t)(j & 1) : (uint32_t)((j >> 1) & 1); };
 
   if (tid == 0) {
     bar_init(bar(kBarQFull), 1);
@@ -329,18 +340,23 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         tma_load_4d_raw(sQ + (2 * g) * kHalf, &tmap_q, bar(kBarQFull), 0, kvh * G, t0 + g * TT, b);
         tma_load_4d_raw(sQ + (2 * g + 1) * kHalf, &tmap_q, bar(kBarQFull), 64, kvh * G, t0 + g * TT, b);
       }
-      for (int j = 0; j < n_iter; ++j) {
-        const int s = j & 1;
-        const uint32_t par = ((j >> 1) & 1) ^ 1;
-        const int key0 = key_tile(j) * kBN;
-        if (!bar_wait(bar(kBarKEmpty + s), par, abort_addr, a.dev_status)) break;
-        bar_expect_tx(bar(kBarKFull + s), 2 * kHalf);
-        tma_load_4d_raw(sK + (2 * s) * kHalf, &tmap_k, bar(kBarKFull + s), 0, kvh, key0, b);
-        tma_load_4d_raw(sK + (2 * s + 1) * kHalf, &tmap_k, bar(kBarKFull + s), 64, kvh, key0, b);
-        if (!bar_wait(bar(kBarVEmpty + s), par, abort_addr, a.dev_status)) break;
-        bar_expect_tx(bar(kBarVFull + s), 2 * kHalf);
-        tma_load_4d_raw(sV + (2 * s) * kHalf, &tmap_v, bar(kBarVFull + s), 0, kvh, key0, b);
-        tma_load_4d_raw(sV + (2 * s + 1) * kHalf, &tmap_v, bar(kBarVFull + s), 64, kvh, key0, b);
+      bool go = true;
+      for (int j = 0; j < n_iter && go; ++j) {
+        // the shared stream loads key tile j once; split mode loads it per Q tile
+        for (int g = 0; g < (dual ? 2 : 1) && go; ++g) {
+          if (dual && !active(g, j)) continue;
+          const int s = kv_stage(g, j);
+          const uint32_t par = kv_par(j) ^ 1u;
+          const int key0 = key_tile(g, j) * kBN;
+          if (!bar_wait(bar(kBarKEmpty + s), par, abort_addr, a.dev_status)) { go = false; break; }
+          bar_expect_tx(bar(kBarKFull + s), 2 * kHalf);
+          tma_load_4d_raw(sK + (2 * s) * kHalf, &tmap_k, bar(kBarKFull + s), 0, kvh, key0, b);
+          tma_load_4d_raw(sK + (2 * s + 1) * kHalf, &tmap_k, bar(kBarKFull + s), 64, kvh, key0, b);
+          if (!bar_wait(bar(kBarVEmpty + s), par, abort_addr, a.dev_status)) { go = false; break; }
+          bar_expect_tx(bar(kBarVFull + s), 2 * kHalf);
+          tma_load_4d_raw(sV + (2 * s) * kHalf, &tmap_v, bar(kBarVFull + s), 0, kvh, key0, b);
+          tma_load_4d_raw(sV + (2 * s + 1) * kHalf, &tmap_v, bar(kBarVFull + s), 64, kvh, key0, b);
+        }
       }
     }
   } else if (warp == 1) {
@@ -354,22 +370,27 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       // which reads P_g(j-1) out of the same columns: MMAs issued by one
       // thread run in issue order, so the PV has read its operand before this
       // QK writes the accumulator.
+      // (in split mode both Q tiles read Q slot 0, the one token's heads, and
+      // K tile j of Q tile g's own stream, released per stream)
       auto qk = [&](int g, int j) {
+        const int s = kv_stage(g, j);
+        if (dual && !bar_wait(bar(kBarKFull + s), kv_par(j), abort_addr, a.dev_status)) return false;
         tc_fence_after();
-        const int s = j & 1;
+        const int qs = dual ? 0 : g;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t da = sw128_desc(sQ + (2 * g + (kk >> 2)) * kHalf + (kk & 3) * 32, 16, 1024);
+          const uint64_t da = sw128_desc(sQ + (2 * qs + (kk >> 2)) * kHalf + (kk & 3) * 32, 16, 1024);
           const uint64_t db = sw128_desc(sK + (2 * s + (kk >> 2)) * kHalf + (kk & 3) * 32, 16, 1024);
           tc_mma(tmem + kColS + 128u * (uint32_t)g, da, db, idesc_qk, kk > 0 ? 1u : 0u);
         }
         tc_commit(bar(kBarSFull + g));
+        if (dual) tc_commit(bar(kBarKEmpty + s));
         return true;
       };
       // O_g += P_g(j) V_j once the softmax has published P_g(j)
       auto pv = [&](int g, int j) {
-        const int s = j & 1;
-        if (!bar_wait(bar(kBarVFull + s), (uint32_t)(j >> 1) & 1u, abort_addr, a.dev_status)) return false;
+        const int s = kv_stage(g, j);
+        if (!bar_wait(bar(kBarVFull + s), kv_par(j), abort_addr, a.dev_status)) return false;
         if (!bar_wait(bar(kBarPFull + g), (uint32_t)j & 1u, abort_addr, a.dev_status)) return false;
         tc_fence_after();
 #pragma unroll
@@ -381,6 +402,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           const uint64_t db = sw128_desc(sV + (2 * s) * kHalf + kk * 2048, kHalf, 1024);
           tc_mma_ts(tmem + kColO + 128u * (uint32_t)g, pa, db, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
+        if (dual) tc_commit(bar(kBarVEmpty + s));
         return true;
       };
       // Ping-pong: the tensor cores run Q tile 1's MMAs while the softmax
@@ -388,16 +410,17 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       //   QK_0(j), PV_1(j-1), QK_1(j), PV_0(j)
       for (int j = 0; j <= n_iter && ok; ++j) {
         if (j < n_iter) {
-          if (!bar_wait(bar(kBarKFull + (j & 1)), (uint32_t)(j >> 1) & 1u, abort_addr, a.dev_status)) break;
+          if (!dual && !bar_wait(bar(kBarKFull + (j & 1)), (uint32_t)(j >> 1) & 1u, abort_addr, a.dev_status))
+            break;
           if (active(0, j) && !qk(0, j)) break;
         }
         if (j > 0) {
           if (active(1, j - 1) && !pv(1, j - 1)) break;
-          tc_commit(bar(kBarVEmpty + ((j - 1) & 1)));  // both PVs of tile j-1 issued
+          if (!dual) tc_commit(bar(kBarVEmpty + ((j - 1) & 1)));  // both PVs of tile j-1 issued
         }
         if (j < n_iter) {
           if (active(1, j) && !qk(1, j)) break;
-          tc_commit(bar(kBarKEmpty + (j & 1)));  // both QKs of tile j issued
+          if (!dual) tc_commit(bar(kBarKEmpty + (j & 1)));  // both QKs of tile j issued
           if (active(0, j) && !pv(0, j)) break;
         }
       }
@@ -410,7 +433,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int quarter = warp & 3;         // TMEM lanes 32*quarter .. +31
     const int grp = (warp - 2) >> 2;      // Q tile of this warp
     const int m = 32 * quarter + lane;    // query row of this thread within its Q tile
-    const int tok = t0 + grp * TT + m / G;
+    const int tok = t0 + (dual ? 0 : grp * TT) + m / G;  // split mode: both Q tiles are one token
     const int head = kvh * G + (m % G);
     const int lim = sp + min(tok, a.T - 1);  // last visible key (rows past T borrow the last token's)
     // with a window: keys n_sink <= k < lo_vis are hidden as well
@@ -424,7 +447,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     float l = 0.f;           // row sum in units of 2^ref
 
     for (int j = 0; active(grp, j); ++j) {
-      const int jt = key_tile(j);
+      const int jt = key_tile(grp, j);
       bar_wait(bar(kBarSFull + grp), (uint32_t)j & 1u, abort_addr, a.dev_status);
       tc_fence_after();
       // the thread's whole S row
@@ -495,12 +518,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           tmem_st32(lane_addr + col_o + 32u * c2, r);
         }
       }
-      if (last_split && j == n_iter - 1 && Lmax < jt * kBN + kBN) {
+      if (first_tile(grp) + j == n_all - 1 && Lmax < jt * kBN + kBN) {
         // rows of the last V tile past the last visible key may hold any bits;
         // zero them so that 0 * (garbage) cannot reach O (both Q tiles' groups
         // write the same zeros before their own P goes out)
-        const int s = j & 1;
-        bar_wait(bar(kBarVFull + s), (uint32_t)(j >> 1) & 1u, abort_addr, a.dev_status);
+        const int s = kv_stage(grp, j);
+        bar_wait(bar(kBarVFull + s), kv_par(j), abort_addr, a.dev_status);
         const int first_bad = Lmax - jt * kBN;
         const int nchunks = (kBN - first_bad) * 16;  // 16-byte chunks over both halves
         for (int c = gt; c < nchunks; c += kGroupThreads) {
@@ -529,12 +552,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       const float f = (ref == -INFINITY) ? 0.f : fast_exp2(ref - mn);
       inv_l = f / (l * f + fast_exp2(s2 - mn));
     }
-    const bool store = grp < n_q && tok < a.T;
+    const bool store = (dual ? active(grp, 0) : grp < n_q) && tok < a.T;
     if (a.split_tiles > 0 && n_splits_here > 1) {
       // this split's partial: unnormalised O and (max, sum), both relative
       // to 2^ref (a group without key tiles here contributes nothing)
       const bool any = active(grp, 0);
-      const size_t slot = (((size_t)b * a.T + (store ? tok : 0)) * a.part_splits + split) * a.H + head;
+      const size_t slot =
+          (((size_t)b * a.T + (store ? tok : 0)) * a.part_splits + (2 * split + grp)) * a.H + head;
       float* po = a.part_o + slot * kHeadDim;
 #pragma unroll
       for (int c2 = 0; c2 < 4; ++c2) {
@@ -581,25 +605,36 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   }
 }
 
-template <int G>
-cudaError_t launch_prefill_g(const PrefillArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
-                             const CUtensorMap& tv, cudaStream_t st) {
+template <int G, bool DUAL>
+cudaError_t launch_prefill_gd(const PrefillArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
+                              const CUtensorMap& tv, cudaStream_t st) {
   static bool configured[64] = {false};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!configured[dev]) {
-    e = cudaFuncSetAttribute(prefill_tc_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(prefill_tc_kernel<G, DUAL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kPrefillSmemBytes);
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
-  // one CTA per M tile pair (times split_grid in split mode)
-  const long long grid = (long long)((a.n_mtiles + 1) / 2) * a.Hkv * a.B * (a.split_tiles > 0 ? a.split_grid : 1);
+  // one CTA per M tile pair (times ceil(split_grid / 2) in split mode)
+  const long long grid = (long long)((a.n_mtiles + 1) / 2) * a.Hkv * a.B * (DUAL ? (a.split_grid + 1) / 2 : 1);
   if (grid <= 0 || grid > 0x7FFFFFFFll) return cudaErrorInvalidValue;
-  return launch_pdl(prefill_tc_kernel<G>, dim3((unsigned)grid), dim3(kPrefillThreads), kPrefillSmemBytes, st, tq, tk,
-                    tv, a);
+  return launch_pdl(prefill_tc_kernel<G, DUAL>, dim3((unsigned)grid), dim3(kPrefillThreads), kPrefillSmemBytes, st,
+                    tq, tk, tv, a);
+}
+
+template <int G>
+cudaError_t launch_prefill_g(const PrefillArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
+                             const CUtensorMap& tv, cudaStream_t st) {
+  if constexpr (G == 32) {  // split mode serves the multi-query decode (G = 32) only
+    if (a.split_tiles > 0) return launch_prefill_gd<G, true>(a, tq, tk, tv, st);
+  } else {
+    if (a.split_tiles > 0) return cudaErrorInvalidValue;
+  }
+  return launch_prefill_gd<G, false>(a, tq, tk, tv, st);
 }
 
 }  // namespace
