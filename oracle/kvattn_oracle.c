@@ -66,9 +66,11 @@
  * only on the relative offset, rotates (1,0) by 90 degrees to (0,1) at angle
  * pi/2, composes additively; the unscaled frequency table has f_0 = 1,
  * f_{d/4} = 1/sqrt(theta) and a constant ratio; the scaled table keeps the
- * high frequencies, divides the low ones by the factor exactly and is
- * continuous at both cutoffs (its interior blend values are pinned only by
- * that continuity); attention is checked against MHA with repeated KV
+ * high frequencies, divides the low ones by the factor exactly, is
+ * continuous at both cutoffs, gives the blend weights of pairs 29..34 worked
+ * out by hand from the rule, and blends linearly in L0/wavelength (a pair
+ * placed at wavelength L0/2.5 gets exactly 0.5625 f); attention is checked
+ * against MHA with repeated KV
  * heads, MQA, single-row and uniform-weight closed forms, a planted-row
  * index test, prefill-vs-stepwise schedule equivalence, and a brute-force
  * complex-number / direct-softmax formula written separately in Python.

@@ -119,6 +119,18 @@ def test_rope_append_large_positions_scaled():
         row = U.to_host(dck[b, sp[b]:sp[b] + T])
         assert U.ulp_distance(row, ck[0, sp[b]:]).max() <= 1
         assert np.array_equal(U.to_host(dcv[b, sp[b]:sp[b] + T]), cv[0, sp[b]:])
+        # Pairs 29..34 (elements 58..69) are the ones the Llama-3.1 rule
+        # blends; at these positions a misread blend would turn them by far
+        # more than one ulp.  Checked on their own, and shown to be sensitive:
+        # the unscaled rotation differs there.
+        blend = slice(58, 70)
+        assert U.ulp_distance(g_q[b][..., blend], qr[0][..., blend]).max() <= 1
+        assert U.ulp_distance(row[..., blend], ck[0, sp[b]:][..., blend]).max() <= 1
+        ck0 = np.zeros_like(ck)
+        qr0, rc = oracle.rope_append(q[b:b + 1].copy(), k[b:b + 1].copy(), v[b:b + 1].copy(), ck0,
+                                     np.zeros_like(ck0), np.array([sp[b]], np.int32), U.oracle_freqs(kv.LLAMA3))
+        assert rc == 0
+        assert np.mean(U.ulp_distance(g_q[b][..., blend], qr0[0][..., blend]) > 1) > 0.5
 
 
 @pytest.mark.parametrize("kind,T", [("decode", 1), ("prefill", 4)])

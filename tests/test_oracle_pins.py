@@ -78,6 +78,37 @@ def test_scaled_freqs_regions():
     assert np.allclose(oracle.rope_freqs(128, 500000.0, True, factor=1.0), base, rtol=1e-15)
 
 
+# Blend weights s_i of pairs 29..34 at d = 128, theta = 500000, L0 = 8192,
+# low = 1, high = 4, worked out by hand from the public Llama-3.1 rule
+# (wavelength 2*pi/f_i, s = (L0/wavelength - low) / (high - low)) and written
+# to three decimals; the rule itself is only named on the pages
+# ("Llama 3.1 8B · Repeat heads", sku_list excerpt with use_scaled_rope True;
+# "Llama 3.1 8B KV cache", section "Training details that matter": the 8x
+# factor and the low and high frequency cutoffs).
+BLEND_S = {29: 0.804, 30: 0.593, 31: 0.421, 32: 0.281, 33: 0.167, 34: 0.074}
+
+
+def test_scaled_freqs_blend_interior_values():
+    base = oracle.rope_freqs(128, 500000.0)
+    sc = oracle.rope_freqs(128, 500000.0, use_scaled=True)
+    for i, s in BLEND_S.items():
+        # scaled f_i = ((1 - s)/8 + s) f_i, so s = (f'/f - 1/8) * 8/7
+        s_oracle = (sc[i] / base[i] - 1.0 / 8.0) * 8.0 / 7.0
+        assert abs(s_oracle - s) <= 1e-3, (i, s_oracle, s)
+
+
+def test_scaled_freqs_blend_is_linear_in_inverse_wavelength():
+    # Put pair i's wavelength at L0/2.5: the rule blends linearly in
+    # L0/wavelength, so s = (2.5 - 1)/(4 - 1) = 1/2 and the scaled frequency
+    # is exactly (1/16 + 1/2) f = 0.5625 f.  A blend linear in the wavelength
+    # itself would give (L0/2.5 - L0/4)/(L0 - L0/4) = 0.2 and 0.825 f.
+    for i in (29, 31, 40, 60):
+        f = oracle.rope_freqs(128, 500000.0)[i]
+        L0 = 2.5 * (2 * math.pi / f)
+        got = oracle.rope_freqs(128, 500000.0, True, 8.0, 1.0, 4.0, L0)[i]
+        assert abs(got / f - 0.5625) <= 1e-12, (i, got / f)
+
+
 @pytest.mark.parametrize("cut", ["short", "long"])
 def test_scaled_freqs_continuous_at_cutoffs(cut):
     # Move the original context L0 so that the wavelength of pair i sits just
