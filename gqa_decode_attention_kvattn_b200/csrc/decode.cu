@@ -12,10 +12,13 @@
 // heads of that group from the same tiles (no materialised repeat_kv).  Items
 // are numbered with the KV head fastest, so CTAs that run side by side read
 // the same cache rows of neighbouring heads.  A persistent grid of
-// (SMs x CTAs per SM) walks the items round-robin.
+// (SMs x CTAs per SM) takes the items from a per-call atomic work counter
+// (full splits first, then the last splits largest first), so the tail of a
+// ragged batch ends with the smallest pieces; a call with no workspace (no
+// splits, no counter) hands item i to CTA i mod grid.
 //
 // Inside a CTA: one producer warp issues TMA tensor loads of 32-row K and V
-// tiles (32 x 256 B each, row stride Hkv*256 B) into a 4-stage shared-memory
+// tiles (32 x 256 B each, row stride Hkv*256 B) into a 3-stage shared-memory
 // ring; four consumer warps each take 8 rows of every tile.  Sixteen lanes
 // share one cache row, each holding 8 of its 128 elements, so a half-warp
 // reads a row's 256 bytes from shared memory conflict-free.  Partial dot
@@ -834,15 +837,15 @@ __global__ void __launch_bounds__(kThreads, Shape<G>::MIN_BLOCKS) decode_splitk_
   }
 }
 
-// K3: log-sum-exp merge of the split partials.  One CTA per (head, row set),
+// K3: log-sum-exp merge of the split partials.  One CTA per (row set, head),
 // one thread per output element; one pass with a running maximum.
 __global__ void __launch_bounds__(kHeadDim) decode_merge_kernel(const DecodeArgs a) {
   pdl_wait();  // the split-K kernel has finished and its partials are visible
   pdl_launch_dependents();
   // the split-K kernel is done with the work counter: leave it zero for the next call
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0 && a.counter) *a.counter = 0;
-  const int head = blockIdx.x;
-  const int v = blockIdx.y;
+  const int v = blockIdx.x;     // row set (up to 2^24 of them: the grid's x extent)
+  const int head = blockIdx.y;  // query head (at most 65535: the y extent)
   const int L = set_length<true>(a, v);
   const int ns = (L + a.rows_per_split - 1) / a.rows_per_split;
   if (L == 0 || (ns <= 1 && !a.sink_logits)) return;  // invalid, or written directly by K2
@@ -1247,7 +1250,7 @@ cudaError_t launch_g(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorM
   cudaError_t e = launch_pdl(kernel, dim3(a.grid), dim3(kThreads), smem, st, tk, tv, a, evict_first, tab);
   if (e != cudaSuccess) return e;
   if (!FUSED && (a.max_splits > 1 || a.sink_logits)) {
-    e = launch_pdl(decode_merge_kernel, dim3(a.H, a.B * a.Tq), dim3(kHeadDim), 0, st, a);
+    e = launch_pdl(decode_merge_kernel, dim3(a.B * a.Tq, a.H), dim3(kHeadDim), 0, st, a);
   }
   return e;
 }
@@ -1326,8 +1329,8 @@ DecodePlan plan_decode(int B, int Tq, int H, int Hkv, int kv_len_hint, int sm_co
   p.ctas_per_sm = ctas_per_sm;
   const int slots = sm_count * ctas_per_sm;
   const long long row_sets = (long long)B * Tq;
-  // Aim for ~16 items per resident CTA so the round-robin stays balanced when
-  // lengths are ragged; never split below 64 rows, and do not split at all
+  // Aim for ~16 items per resident CTA so the work counter's tail stays
+  // balanced when lengths are ragged; never split below 64 rows, and do not split at all
   // when the (b, t, head) units alone already give that much parallelism.
   long long want = (row_sets * Hkv * (long long)kv_len_hint) / (16LL * slots);
   int C = 64;
@@ -1404,7 +1407,7 @@ bool decode_use_mma(int G, long long work_rows) { return G >= 8 || (G == 4 && wo
 cudaError_t launch_decode_merge(const DecodeArgs& a, cudaStream_t st) {
   if (!a.ws_o || !a.ws_ml || !a.out || !a.start_pos || a.rows_per_split < 1 || a.max_splits < 1)
     return cudaErrorInvalidValue;
-  return launch_pdl(decode_merge_kernel, dim3(a.H, a.B * a.Tq), dim3(kHeadDim), 0, st, a);
+  return launch_pdl(decode_merge_kernel, dim3(a.B * a.Tq, a.H), dim3(kHeadDim), 0, st, a);
 }
 
 }  // namespace kvattn

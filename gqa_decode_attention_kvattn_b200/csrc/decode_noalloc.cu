@@ -16,9 +16,17 @@
 // first time the entry point runs on it (so that first call should come
 // before any stream capture).  All calls share the array: two calls whose
 // kernels overlap on the GPU (different streams, or different host threads on
-// one device) race on it.  The decode kernels write every partial before
-// reading it, so nothing in the array has to start at zero and leftovers from
-// an earlier call do no harm.
+// one device) race on it.
+//
+// What the array keeps between calls.  Its first 16 bytes are the split
+// kernel's work counter, which must be zero when a call starts: the array
+// starts zeroed, and every call whose kernels were launched leaves the
+// counter zero again (the merge kernel clears it after the split kernel has
+// finished, also when a pipeline wait in that kernel gave up).  If the merge
+// launch fails after the split kernel was launched, the entry point queues a
+// clear of those 16 bytes itself, because the caller has no way to reach
+// them.  The partials after the header are written before they are read, so
+// leftovers there do no harm.
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -114,6 +122,8 @@ extern "C" KVATTN_API int kvattn_decode_noalloc(const kvattn_dims* dims, const u
   if (!aligned16(q_rot) || !aligned16(cache_k) || !aligned16(cache_v) || !aligned16(out) ||
       (reinterpret_cast<uintptr_t>(start_pos) & 3u))
     return KVATTN_ERR_INVALID_ARG;
+  // the merge kernel's grid is (sequences, heads)
+  if (dims->batch > (1 << 24) || dims->n_heads > 65535) return KVATTN_ERR_UNSUPPORTED;
   const int hint = max_kv_len_hint <= 0 ? dims->max_seq_len : max_kv_len_hint;
   if (hint > dims->max_seq_len || hint < 1) return KVATTN_ERR_OUT_OF_RANGE;
   if (!(scale > 0.f)) scale = 1.0f / std::sqrt((float)kHeadDim);
@@ -158,5 +168,11 @@ extern "C" KVATTN_API int kvattn_decode_noalloc(const kvattn_dims* dims, const u
   a.dev_status = dev_status;
   a.grid = plan.grid;
   a.mma = plan.mma ? 1 : 0;
-  return kvattn::launch_status(kvattn::launch_decode(a, tk, tv, (cudaStream_t)stream));
+  const cudaError_t e = kvattn::launch_decode(a, tk, tv, (cudaStream_t)stream);
+  if (e != cudaSuccess && a.counter) {
+    // the split kernel may have run without the merge that clears its
+    // counter: clear it here (best effort; no allocation)
+    (void)cudaMemsetAsync(a.counter, 0, 16, (cudaStream_t)stream);
+  }
+  return kvattn::launch_status(e);
 }

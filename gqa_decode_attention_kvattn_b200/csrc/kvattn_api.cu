@@ -198,7 +198,9 @@ int run_attention(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, con
   if (hint > dims->max_seq_len || hint < T) return KVATTN_ERR_OUT_OF_RANGE;
   if (!(scale > 0.f)) scale = 1.0f / std::sqrt((float)kHeadDim);
   if (!std::isfinite(scale)) return KVATTN_ERR_INVALID_ARG;
-  if ((long long)dims->batch * T > (1LL << 24)) return KVATTN_ERR_UNSUPPORTED;
+  // the merge kernel's grid is (row sets, heads): at most 2^24 row sets and
+  // 65535 heads, checked before anything is launched
+  if ((long long)dims->batch * T > (1LL << 24) || dims->n_heads > 65535) return KVATTN_ERR_UNSUPPORTED;
 
   int sms = 0;
   rc = current_sm_count(&sms);
@@ -428,7 +430,7 @@ int kvattn_decode_fused(const kvattn_dims* dims, const kvattn_rope_params* rope,
   if (hint > dims->max_seq_len || hint < 1) return KVATTN_ERR_OUT_OF_RANGE;
   if (!(scale > 0.f)) scale = 1.0f / std::sqrt((float)kHeadDim);
   if (!std::isfinite(scale)) return KVATTN_ERR_INVALID_ARG;
-  if ((long long)dims->batch > (1LL << 24)) return KVATTN_ERR_UNSUPPORTED;
+  if ((long long)dims->batch > (1LL << 24) || dims->n_heads > 65535) return KVATTN_ERR_UNSUPPORTED;
 
   int sms = 0;
   rc = current_sm_count(&sms);

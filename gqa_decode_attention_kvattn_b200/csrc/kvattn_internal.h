@@ -150,10 +150,13 @@ struct PrefillArgs {
   int window;       // > 0: token at position p sees keys p - window < k <= p and k < n_sink
   int n_sink;
   const float* sink_logits;  // fp32 [H] learned sink logits (score units), or null
-  // Split mode (split_tiles > 0; no window, no learned sinks): CTA
-  // (unit, split) takes key tiles [split * split_tiles, +split_tiles) of its
-  // (sequence, KV head); split_grid splits per unit are launched.  A row set
-  // with more than one split writes its unnormalised O and (max in log2
+  // Split mode (split_tiles > 0; no window, no learned sinks; the
+  // multi-query decode): the key tiles of a (sequence, KV head) are cut into
+  // split_grid splits of split_tiles tiles, and CTA c of the unit takes the
+  // two consecutive splits 2c and 2c + 1 as its two Q tiles (both hold the
+  // same token's heads, each with its own K/V stream), so ceil(split_grid / 2)
+  // CTAs run per unit.  Q tile g of CTA c writes partial slot 2c + g.  A row
+  // set with more than one split writes its unnormalised O and (max in log2
   // units, sum) to part_o [B*T, part_splits, H, d] / part_ml [.., 2], the
   // layout the decode's LSE merge reads; one with a single split writes out.
   int split_tiles;

@@ -520,8 +520,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       }
       if (first_tile(grp) + j == n_all - 1 && Lmax < jt * kBN + kBN) {
         // rows of the last V tile past the last visible key may hold any bits;
-        // zero them so that 0 * (garbage) cannot reach O (both Q tiles' groups
-        // write the same zeros before their own P goes out)
+        // zero them so that 0 * (garbage) cannot reach O.  On the shared
+        // stream both Q tiles' groups write the same zeros into the one stage
+        // before their own P goes out; in split mode only the group whose
+        // split holds key tile n_all - 1 gets here, and it zeroes its own stage
         const int s = kv_stage(grp, j);
         bar_wait(bar(kBarVFull + s), kv_par(j), abort_addr, a.dev_status);
         const int first_bad = Lmax - jt * kBN;

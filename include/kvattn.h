@@ -140,8 +140,9 @@ KVATTN_API size_t kvattn_decode_workspace_bytes(const kvattn_dims* dims, int32_t
  * The rows of each (sequence, KV head) are streamed from HBM once and serve
  * all G query heads.  At G = 32 (e.g. multi-query attention with 32 heads) a
  * call with more than one split runs on the 5th-generation tensor cores: the
- * 32 heads form one 128-row MMA tile and each CTA takes a range of 128-row
- * key tiles.  G = 64, 128 (and masked G = 32 calls) run as G/16 groups of 16
+ * 32 heads form one 128-row MMA tile, the rows of a (sequence, KV head) are
+ * cut into splits of whole 128-row key tiles, and each CTA takes two
+ * consecutive splits, one per tensor-memory accumulator.  G = 64, 128 (and masked G = 32 calls) run as G/16 groups of 16
  * heads over the same rows, scheduled side by side so the repeat reads are
  * served by L2.  Long rows are split across CTAs and the partial
  * (o, max, sum) triples are merged by log-sum-exp in a second kernel; the
@@ -154,8 +155,10 @@ KVATTN_API size_t kvattn_decode_workspace_bytes(const kvattn_dims* dims, int32_t
  * workspace: device memory of kvattn_decode_workspace_bytes() bytes, 16-byte
  * aligned, owned by the caller.  Its first 16 bytes hold a work counter that
  * must be ZERO before the first call (e.g. cudaMemset once after
- * allocation); every call leaves it zero again (the merge kernel resets it),
- * so one workspace serves calls of any shape with no memset between them.
+ * allocation); every call leaves it zero again (the merge kernel resets it,
+ * also after a pipeline wait gave up), so one workspace serves calls of any
+ * shape with no memset between them.  After a call that returned
+ * KVATTN_ERR_CUDA, zero those 16 bytes again before the next call.
  * Calls that share a workspace must be ordered on one stream.
  * Every kernel of the library is launched with programmatic stream
  * serialization and waits for the previous kernel in the stream before it
@@ -270,7 +273,10 @@ KVATTN_API int kvattn_decode_fused(const kvattn_dims* dims, const kvattn_rope_pa
  *  - Every call shares the one array: calls whose kernels overlap on the GPU
  *    (other streams, other host threads) race and must be serialised by the
  *    caller.  The array starts zeroed and each call leaves its work counter
- *    zero again.
+ *    zero again, also a call that set KVATTN_DEV_WAIT_TIMEOUT (its merge
+ *    kernel clears the counter after the split kernel ends) and a call whose
+ *    merge launch failed (the entry point then queues the clear itself), so
+ *    the caller never has to reset anything.
  *  - Shapes whose partials need more than the array (see
  *    kvattn_decode_workspace_bytes) return KVATTN_ERR_WORKSPACE and launch
  *    nothing. */

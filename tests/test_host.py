@@ -163,3 +163,21 @@ def test_masked_entry_points_validate_the_mask(lib):
         assert lib.kvattn_prefill_chunk_masked(ctypes.byref(d), 1, *P, 0, 0.0, ctypes.byref(bad), FAKE, None, 0,
                                                None, None) == 1
         assert lib.kvattn_decode_masked_workspace_bytes(ctypes.byref(d), 0, ctypes.byref(bad)) == 0
+
+
+def test_merge_grid_limits_refused_before_launch(lib):
+    # The split-K merge runs one CTA per (row set, head): row sets on the
+    # grid's x extent (B*T at most 2^24 here), heads on its y extent (at most
+    # 65535).  Larger calls are refused on the host, before the split kernel
+    # could be launched without the merge that clears its work counter.
+    P = [FAKE] * 4
+    big_b = _dims(batch=(1 << 24) + 1)
+    assert lib.kvattn_decode(ctypes.byref(big_b), *P, 0, 0.0, FAKE, None, 0, None, None) == 2
+    many_heads = _dims(n_heads=65536 * 2, n_kv_heads=65536 * 2 // 4)
+    assert lib.kvattn_decode(ctypes.byref(many_heads), *P, 0, 0.0, FAKE, None, 0, None, None) == 2
+    noalloc = kv._load_noalloc()
+    assert noalloc(ctypes.byref(many_heads), *P, 0, 0.0, FAKE, None, None) == 2
+    assert noalloc(ctypes.byref(big_b), *P, 0, 0.0, FAKE, None, None) == 2
+    rope = kv.LLAMA3.as_c()
+    assert lib.kvattn_decode_fused(ctypes.byref(many_heads), ctypes.byref(rope), FAKE, None, *[FAKE] * 5, 0, 0.0,
+                                   FAKE, None, 0, None, None) == 2
