@@ -197,28 +197,59 @@ class Layer:
     pass
 
 
-def build_state(w, seed, device, path="auto"):
+def l2_bytes(device) -> int:
+    import torch
+    try:
+        return int(torch.cuda.get_device_properties(device).L2_cache_size)
+    except Exception:
+        return 126 << 20
+
+
+def rotation_sets(w, kv_bytes_layer, device, rotate=0) -> int:
+    """How many distinct copies of the step's caches to rotate through so that
+    consecutive uses of one copy are more than twice the L2 size apart (a
+    cold L2 for every step); a small latency-bound step (under 16 MB of K/V)
+    rotates over at least 64 caches.  rotate > 0 forces a count."""
+    if rotate > 0:
+        return rotate
+    step_bytes = max(1, w.layers * kv_bytes_layer)
+    need = math.ceil(2 * l2_bytes(device) / step_bytes)
+    if need <= 1:
+        return 1
+    if step_bytes < (16 << 20):
+        need = max(need, math.ceil(64 / w.layers))
+    return need
+
+
+def build_state(w, seed, device, path="auto", sets=1):
+    """Device state of the step: `sets` copies of the step's layers (each
+    layer with its own caches and new q/k/v), the start positions, the
+    workspace and the status word."""
     import torch
     import gqa_decode_attention_kvattn_b200 as kv
     sp = w.start_pos(seed)
     dsp = torch.from_numpy(sp).to(device)
     rope = kv.LLAMA3_1 if w.scaled_rope else kv.LLAMA3
-    layers = []
-    for l in range(w.layers):
-        L = Layer()
-        L.q = torch.empty((w.B, w.T, w.H, 128), dtype=torch.bfloat16, device=device)
-        L.k = torch.empty((w.B, w.T, w.Hkv, 128), dtype=torch.bfloat16, device=device)
-        L.v = torch.empty_like(L.k)
-        ks.device_normal_bf16(seed, ks.layer_stream(ks.STREAM_Q, l), L.q)
-        ks.device_normal_bf16(seed, ks.layer_stream(ks.STREAM_K_NEW, l), L.k)
-        ks.device_normal_bf16(seed, ks.layer_stream(ks.STREAM_V_NEW, l), L.v)
-        L.ck = torch.empty((w.B, w.S, w.Hkv, 128), dtype=torch.bfloat16, device=device)
-        L.cv = torch.empty_like(L.ck)
-        ks.device_cache_fill(seed, ks.layer_stream(ks.STREAM_CACHE_K, l), L.ck, dsp)
-        ks.device_cache_fill(seed, ks.layer_stream(ks.STREAM_CACHE_V, l), L.cv, dsp)
-        L.q_rot = torch.empty_like(L.q)
-        L.out = torch.empty_like(L.q)
-        layers.append(L)
+    layer_sets = []
+    for r in range(sets):
+        layers = []
+        for l in range(w.layers):
+            g = r * w.layers + l   # distinct synthetic data per copy and layer
+            L = Layer()
+            L.q = torch.empty((w.B, w.T, w.H, 128), dtype=torch.bfloat16, device=device)
+            L.k = torch.empty((w.B, w.T, w.Hkv, 128), dtype=torch.bfloat16, device=device)
+            L.v = torch.empty_like(L.k)
+            ks.device_normal_bf16(seed, ks.layer_stream(ks.STREAM_Q, g), L.q)
+            ks.device_normal_bf16(seed, ks.layer_stream(ks.STREAM_K_NEW, g), L.k)
+            ks.device_normal_bf16(seed, ks.layer_stream(ks.STREAM_V_NEW, g), L.v)
+            L.ck = torch.empty((w.B, w.S, w.Hkv, 128), dtype=torch.bfloat16, device=device)
+            L.cv = torch.empty_like(L.ck)
+            ks.device_cache_fill(seed, ks.layer_stream(ks.STREAM_CACHE_K, g), L.ck, dsp)
+            ks.device_cache_fill(seed, ks.layer_stream(ks.STREAM_CACHE_V, g), L.cv, dsp)
+            L.q_rot = torch.empty_like(L.q)
+            L.out = torch.empty_like(L.q)
+            layers.append(L)
+        layer_sets.append(layers)
     if path == "auto":
         path = "fused" if w.B * w.Hkv * w.kv_len_hint < (1 << 18) else "split"
     fused = w.kind == "decode" and path == "fused"
@@ -233,12 +264,14 @@ def build_state(w, seed, device, path="auto"):
         ws = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device=device)  # counters start at zero
     status = torch.zeros(1, dtype=torch.int32, device=device)
     torch.cuda.synchronize(device)
-    return dict(sp=sp, dsp=dsp, rope=rope, layers=layers, ws=ws, ws_bytes=ws_bytes, status=status, fused=fused)
+    return dict(sp=sp, dsp=dsp, rope=rope, sets=layer_sets, layers=layer_sets[0], ws=ws, ws_bytes=ws_bytes,
+                status=status, fused=fused)
 
 
 def run_layer(w, st, L, ev=None):
-    """One layer of the step on the current stream; `ev` = (before, after)
-    events around the attention call."""
+    """One layer of the step on the current stream; `ev` = three events:
+    before the rope call, between rope and attention, after attention (the
+    fused path records the first and the last)."""
     import gqa_decode_attention_kvattn_b200 as kv
     if st["fused"]:
         # one launch: rope + append + split-K attention + merge
@@ -248,12 +281,14 @@ def run_layer(w, st, L, ev=None):
                                max_kv_len_hint=w.kv_len_hint, out=L.out, workspace=st["ws"],
                                dev_status=st["status"])
         if ev is not None:
-            ev[1].record()
+            ev[2].record()
         return
+    if ev is not None:
+        ev[0].record()
     kv.kvattn_rope_append(L.q, L.k, L.v, L.ck, L.cv, st["dsp"], rope=st["rope"], q_rot=L.q_rot,
                           dev_status=st["status"])
     if ev is not None:
-        ev[0].record()
+        ev[1].record()
     if w.kind == "decode":
         kv.kvattn_decode(L.q_rot, L.ck, L.cv, st["dsp"], max_kv_len_hint=w.kv_len_hint, out=L.out,
                          workspace=st["ws"], dev_status=st["status"])
@@ -261,11 +296,11 @@ def run_layer(w, st, L, ev=None):
         kv.kvattn_prefill_chunk(L.q_rot, L.ck, L.cv, st["dsp"], max_kv_len_hint=w.kv_len_hint, out=L.out,
                                 workspace=st["ws"], dev_status=st["status"])
     if ev is not None:
-        ev[1].record()
+        ev[2].record()
 
 
-def run_step(w, st, events=None):
-    for i, L in enumerate(st["layers"]):
+def run_step(w, st, layers, events=None):
+    for i, L in enumerate(layers):
         run_layer(w, st, L, None if events is None else events[i])
 
 
@@ -354,48 +389,80 @@ def cpu_baseline_leg(w, st, seed, target_s=12.0):
 
 
 # ----------------------------------------------------------------- arms
+def kernel_tag(w, st):
+    """Which attention kernel the step runs: the profile file name's prefix."""
+    import gqa_decode_attention_kvattn_b200 as kv
+    if w.kind != "decode":
+        return "prefill_chunk", "kvattn_prefill_chunk (tcgen05 prefill kernel)"
+    if st["fused"]:
+        return "decode_fused", "kvattn_decode_fused (rope + append + split-K attention + LSE merge, one kernel)"
+    if w.H == 32 * w.Hkv:
+        return "decode_tc", "kvattn_decode (tcgen05 split kernel + LSE merge kernel)"
+    plan = kv.kvattn_decode_plan(w.B, w.H, w.Hkv, w.S, w.kv_len_hint)
+    if plan["tensor_cores"]:
+        return "decode_mma", "kvattn_decode (warp-MMA split-K kernel + LSE merge kernel)"
+    return "decode_splitk", "kvattn_decode (CUDA-core split-K kernel + LSE merge kernel)"
+
+
+def spread(samples_ms):
+    """median, p10, p90 of a list of milliseconds."""
+    a = np.sort(np.asarray(samples_ms, np.float64))
+    return float(np.median(a)), float(np.percentile(a, 10)), float(np.percentile(a, 90))
+
+
 def run_ours(args, w, rank, world, device):
     import torch
-    import torch.distributed as dist
     import gqa_decode_attention_kvattn_b200 as kv
 
-    st = build_state(w, args.seed, device, args.path)
-    nl = len(st["layers"])
-    kv_bytes_layer, flops_layer = work_units(w, st["sp"])
+    sp = w.start_pos(args.seed)
+    kv_bytes_layer, flops_layer = work_units(w, sp)
+    n_sets = rotation_sets(w, kv_bytes_layer, device, args.rotate)
+    st = build_state(w, args.seed, device, args.path, n_sets)
+    nl = w.layers
     merge = 1 if st["ws_bytes"] > 0 else 0
     launches_per_layer = 1 if st["fused"] else 2 + merge
 
-    # warm-up, eager
-    for _ in range(args.warmup):
-        run_step(w, st)
+    # warm-up, eager, over every copy of the caches
+    for k in range(max(args.warmup, n_sets)):
+        run_step(w, st, st["sets"][k % n_sets])
     torch.cuda.synchronize(device)
     if int(st["status"].item()) != 0:
         raise RuntimeError(f"device status {st['status'].item()} after warm-up")
 
-    # capture one step (every layer) twice: as it runs, and with timing events
-    # around each attention call.  Event nodes between the kernels would cut
-    # the programmatic launch overlap, so the timed region replays the plain
-    # graph and then the event graph once, for the last step.
-    events = [(torch.cuda.Event(enable_timing=True, external=True),
-               torch.cuda.Event(enable_timing=True, external=True)) for _ in range(nl)]
-    graph = graph_ev = None
+    # Capture each copy's step twice: as it runs, and with timing events
+    # around each rope and attention call.  Event nodes between the kernels
+    # cut the programmatic launch overlap, so the timed region replays the
+    # plain graphs and the per-kernel times come from separate replays of the
+    # event graphs afterwards.
+    events = [[tuple(torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)) for _ in range(nl)]
+              for _ in range(n_sets)]
+    graphs, graphs_ev = [], []
     if not args.no_graph:
         stream = torch.cuda.Stream(device)
         stream.wait_stream(torch.cuda.current_stream(device))
         with torch.cuda.stream(stream):
-            run_step(w, st)  # one more warm-up on the capture stream
+            run_step(w, st, st["sets"][0])  # one more warm-up on the capture stream
         torch.cuda.current_stream(device).wait_stream(stream)
         torch.cuda.synchronize(device)
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            run_step(w, st)
-        graph_ev = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph_ev):
-            run_step(w, st, events)
-        for _ in range(max(1, args.warmup)):
-            graph.replay()
-        graph_ev.replay()
+        for r in range(n_sets):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                run_step(w, st, st["sets"][r])
+            ge = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(ge):
+                run_step(w, st, st["sets"][r], events[r])
+            graphs.append(g)
+            graphs_ev.append(ge)
+        for k in range(max(args.warmup, n_sets)):
+            graphs[k % n_sets].replay()
         torch.cuda.synchronize(device)
+
+    def step(k, timed_events=False):
+        r = k % n_sets
+        if graphs:
+            (graphs_ev if timed_events else graphs)[r].replay()
+        else:
+            run_step(w, st, st["sets"][r], events[r] if timed_events else None)
 
     # ---------------- timed region
     barrier(world)
@@ -407,56 +474,75 @@ def run_ours(args, w, rank, world, device):
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record()
     for k in range(args.steps):
-        last = k == args.steps - 1
-        if graph is not None:
-            (graph_ev if last else graph).replay()
-        else:
-            run_step(w, st, events if last else None)
+        step(k)
     t1.record()
     torch.cuda.synchronize(device)
     clocks = sampler.stop()
     barrier(world)
     ms = t0.elapsed_time(t1)
-    attn_ms = [a.elapsed_time(b) for a, b in events]   # the last step's attention calls
     ms = max_over_ranks(ms, world, device)
     status = int(st["status"].item())
+
+    # ---------------- per-kernel times: at least 50 event-carrying replays
+    attn_ms, rope_ms = [], []
+    reps = max(50, n_sets)
+    for k in range(reps):
+        step(k, timed_events=True)
+        torch.cuda.synchronize(device)
+        for e0, e1, e2 in events[k % n_sets]:
+            if st["fused"]:
+                attn_ms.append(e0.elapsed_time(e2))
+            else:
+                rope_ms.append(e0.elapsed_time(e1))
+                attn_ms.append(e1.elapsed_time(e2))
+    a_med, a_p10, a_p90 = spread(attn_ms)
 
     secs = ms / 1e3
     ms_per_step = ms / args.steps
     hbm_peak, tf_peak, peak_src = measured_peaks()
-    attn_avg_ms = float(np.mean(attn_ms))
+    tag, kname = kernel_tag(w, st)
+    stats = {"avg_launch_ms": round(a_med, 5), "median_ms": round(a_med, 5), "p10_ms": round(a_p10, 5),
+             "p90_ms": round(a_p90, 5), "samples": len(attn_ms), "replays": reps}
     if w.kind == "decode":
         value = job_throughput(nl * kv_bytes_layer, args.steps, world, ms) / 1e9
         unit = "GB/s"
-        achieved = kv_bytes_layer / (attn_avg_ms / 1e3) / 1e9
+        achieved = kv_bytes_layer / (a_med / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                 "frac": round(achieved / hbm_peak, 4),
-                "traffic": profiled_traffic("decode_fused" if st["fused"] else
-                                            "decode_tc" if w.H == 32 * w.Hkv else "decode_splitk", w.name),
-                "kernel": ("kvattn_decode_fused (rope + append + split-K attention + LSE merge, one kernel)"
-                           if st["fused"] else
-                           "kvattn_decode (tcgen05 split kernel + LSE merge kernel)" if w.H == 32 * w.Hkv else
-                           "kvattn_decode (split-K kernel + LSE merge kernel)"),
-                "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback 6650 GB/s",
-                "avg_launch_ms": round(attn_avg_ms, 5), "launches_timed": nl,
-                "bytes_per_launch": kv_bytes_layer}
+                "traffic": profiled_traffic(tag, w.name), "kernel": kname,
+                "peak_source": (f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else
+                                f"fallback {FALLBACK_HBM_GBS:.0f} GB/s"),
+                **stats, "bytes_per_launch": kv_bytes_layer,
+                "achieved_p10_p90": [round(kv_bytes_layer / (a_p90 / 1e3) / 1e9, 1),
+                                     round(kv_bytes_layer / (a_p10 / 1e3) / 1e9, 1)]}
     else:
         value = job_throughput(nl * flops_layer, args.steps, world, ms) / 1e12
         unit = "TFLOP/s"
-        achieved = flops_layer / (attn_avg_ms / 1e3) / 1e12
+        achieved = flops_layer / (a_med / 1e3) / 1e12
         roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": tf_peak, "unit": "TFLOP/s",
                 "frac": round(achieved / tf_peak, 4),
-                "traffic": profiled_traffic("prefill_chunk", w.name),
-                "kernel": "kvattn_prefill_chunk",
-                "peak_source": f"{peak_src} (MEASURED_PEAKS.json bf16_tflops)",
-                "avg_launch_ms": round(attn_avg_ms, 5), "launches_timed": nl,
-                "flops_per_launch": flops_layer}
+                "traffic": profiled_traffic(tag, w.name), "kernel": kname,
+                "peak_source": (f"{peak_src} (MEASURED_PEAKS.json bf16_tflops)" if peak_src == "measured" else
+                                f"fallback {FALLBACK_BF16_TFLOPS:.0f} TFLOP/s"),
+                **stats, "flops_per_launch": flops_layer,
+                "achieved_p10_p90": [round(flops_layer / (a_p90 / 1e3) / 1e12, 2),
+                                     round(flops_layer / (a_p10 / 1e3) / 1e12, 2)]}
+    rope = None
+    if rope_ms:
+        r_med, r_p10, r_p90 = spread(rope_ms)
+        # bytes one rope_append call moves: q in, q_rot out, k_new and v_new in,
+        # the new K and V rows out
+        rope_bytes = w.B * w.T * (2 * w.H + 4 * w.Hkv) * 128 * 2
+        rope = {"kernel": "kvattn_rope_append", "median_ms": round(r_med, 5), "p10_ms": round(r_p10, 5),
+                "p90_ms": round(r_p90, 5), "samples": len(rope_ms), "bytes_per_launch": rope_bytes,
+                "achieved_gbs": round(rope_bytes / (r_med / 1e3) / 1e9, 1)}
 
     # ---------------- end to end with host buffers
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, w, st, device, kv_bytes_layer, flops_layer, world)
 
+    step_bytes = nl * kv_bytes_layer
     line = {
         "metric": METRIC if w.kind == "decode" else "GQA chunked prefill: attention TFLOP/s (% of bf16 tensor peak)",
         "value": round(value, 2), "unit": unit, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -466,19 +552,24 @@ def run_ours(args, w, rank, world, device):
                    "head_dim": 128, "cache_rows": w.S, "layers": nl,
                    "start_pos": f"uniform [{w.sp_lo}, {w.sp_hi}] seed {args.seed}" if w.sp_lo != w.sp_hi else w.sp_lo,
                    "rope": "llama3.1 scaled, theta 500000" if w.scaled_rope else "theta 500000",
-                   "l2": "inputs larger than L2" if nl * w.B * w.S * w.Hkv * 512 > 256e6 else
-                         "inputs smaller than L2 (latency-bound case)",
-                   "graph": graph is not None,
+                   "l2": (f"inputs larger than L2 ({step_bytes / 1e6:.0f} MB of K/V per step)" if n_sets == 1 else
+                          f"cold L2: {n_sets} copies of the step's caches rotated, "
+                          f"{n_sets * step_bytes / 1e6:.0f} MB of K/V between reuses"),
+                   "cache_copies": n_sets,
+                   "graph": bool(graphs),
                    "path": "fused" if st["fused"] else "rope_append + " + ("decode" if w.kind == "decode" else "prefill"),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "pct_of_hbm_peak": round(100 * (value / world) / hbm_peak, 2) if w.kind == "decode" else None,
         "layer_steps_per_s": round(world * args.steps * nl / secs, 1),
+        "us_per_layer": round(1e3 * ms_per_step / nl, 3),
         "steps_per_s": round(world * args.steps / secs, 2),
         "roofline": roof,
         "gpu_launches": args.steps * nl * launches_per_layer,
         "clocks": clocks,
         "device_status": status,
     }
+    if rope is not None:
+        line["rope_append"] = rope
     if e2e is not None:
         line["e2e"] = e2e
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -644,6 +735,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=0,
                     help="override the workload's layer count (small profiling cases)")
+    ap.add_argument("--rotate", type=int, default=0,
+                    help="copies of the step's caches to rotate through (0: enough for a cold L2 each step)")
+    ap.add_argument("--all", action="store_true",
+                    help="run every workload (each with these options) and print one JSON line per workload")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -671,14 +766,21 @@ def main():
     torch.cuda.set_device(device)
     if world > 1:
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+    names = sorted(WORKLOADS) if args.all else [w.name]
     try:
-        line = run_ours(args, w, rank, world, device)
+        for name in names:
+            wl = WORKLOADS[name] if args.all else w
+            if args.all and args.layers > 0:
+                import dataclasses
+                wl = dataclasses.replace(wl, layers=args.layers)
+            line = run_ours(args, wl, rank, world, device)
+            if rank == 0:
+                print(json.dumps(line), flush=True)
+            torch.cuda.empty_cache()
     finally:
         if world > 1:
             dist.barrier()
             dist.destroy_process_group()
-    if rank == 0:
-        print(json.dumps(line), flush=True)
     return 0
 
 

@@ -134,6 +134,8 @@ def _load():
     lib.kvattn_last_cuda_error_string.argtypes = []
     lib.kvattn_version.restype = ctypes.c_int
     lib.kvattn_version.argtypes = []
+    lib.kvattn_set_wait_policy.restype = ctypes.c_int
+    lib.kvattn_set_wait_policy.argtypes = [ctypes.c_uint64, P]
     _lib = lib
     return lib
 
@@ -156,6 +158,19 @@ def kvattn_version() -> int:
 
 def kvattn_status_string(status: int) -> str:
     return _load().kvattn_status_string(int(status)).decode()
+
+
+def kvattn_set_wait_policy(limit_ns: int = 0, gate=None) -> None:
+    """Limit of every in-kernel pipeline wait for later launches (0: one
+    second) and an optional gate (a one-element int32 CUDA tensor) that the
+    pipelined kernels wait on before issuing any copy; a gate that stays zero
+    makes them give up after the limit and set KVATTN_DEV_WAIT_TIMEOUT (see
+    include/kvattn.h).  kvattn_set_wait_policy() restores the defaults."""
+    if gate is not None:
+        import torch
+        if gate.dtype != torch.int32 or not gate.is_cuda or gate.numel() < 1:
+            raise ValueError("gate must be an int32 CUDA tensor")
+    _check_status(_load().kvattn_set_wait_policy(int(limit_ns), _ptr(gate)), "kvattn_set_wait_policy")
 
 
 # ------------------------------------------------------------------ helpers

@@ -382,9 +382,18 @@ __device__ __forceinline__ void produce(const DecodeArgs& a, const RopeTable& ta
     if constexpr (FUSED) return __shfl_sync(0xffffffffu, x, 0);
     else return x;
   };
+  const uint64_t wlim = wait_limit(a.wait_ns);
   int stage = 0;
   uint32_t phase = 0;
   int next_static = blockIdx.x;
+  // stages whose full barrier this warp has armed, and the phase parity each
+  // was armed on last (to wait for copies still in flight after an abort)
+  uint32_t armed = 0, armed_par = 0;
+  auto arm = [&](int st) {
+    armed |= 1u << st;
+    armed_par = (armed_par & ~(1u << st)) | (phase << st);
+  };
+  if (leader && !gate_wait(a.gate, wlim)) abort_pipeline(&sm.abort, a.dev_status);
   for (;;) {
     int i = 0, stop = 0;
     if (leader) {
@@ -397,8 +406,9 @@ __device__ __forceinline__ void produce(const DecodeArgs& a, const RopeTable& ta
     if (stop) {
       // hand the consumers the end marker through the next stage
       if (leader) {
-        if (mbar_wait(&sm.empty[stage], phase ^ 1, &sm.abort)) {
+        if (mbar_wait(&sm.empty[stage], phase ^ 1, &sm.abort, wlim)) {
           sm.stage_item[stage] = -1;
+          arm(stage);  // (a phase with no copy: it completes on this arrival)
           mbar_arrive(&sm.full[stage]);
         } else {
           abort_pipeline(&sm.abort, a.dev_status);
@@ -411,7 +421,7 @@ __device__ __forceinline__ void produce(const DecodeArgs& a, const RopeTable& ta
     if (it.nsplit == 0) continue;  // invalid row set: nothing to stream
     for (int row = it.r0; row < it.r1; row += TILE_ROWS) {
       int ok = 1;
-      if (leader) ok = mbar_wait(&sm.empty[stage], phase ^ 1, &sm.abort) ? 1 : 0;
+      if (leader) ok = mbar_wait(&sm.empty[stage], phase ^ 1, &sm.abort, wlim) ? 1 : 0;
       ok = bcast(ok);
       if (!ok) {
         if (leader) abort_pipeline(&sm.abort, a.dev_status);
@@ -421,6 +431,7 @@ __device__ __forceinline__ void produce(const DecodeArgs& a, const RopeTable& ta
       if (!FUSED || !first) {
         if (leader) {
           sm.stage_item[stage] = i;
+          arm(stage);
           mbar_arrive_expect_tx(&sm.full[stage], tile_bytes + (first ? kQBytes : 0u));
           if (first) {
             const uint16_t* qsrc = a.q + (((size_t)it.b * a.Tq + it.t) * a.H + (size_t)it.kvh * G) * kHeadDim;
@@ -456,6 +467,7 @@ __device__ __forceinline__ void produce(const DecodeArgs& a, const RopeTable& ta
         }
         if (leader) {
           sm.stage_item[stage] = i;
+          arm(stage);
           mbar_expect_tx(&sm.full[stage], tile_bytes);
           load(stage, it, item_row(it, row));
         }
@@ -485,12 +497,21 @@ __device__ __forceinline__ void produce(const DecodeArgs& a, const RopeTable& ta
   if (!leader) return;
   // Leave only once every copy into this CTA's shared memory has landed:
   // wait (bounded) until the consumers have released every stage.
-  for (int s = 0; s < STAGES; ++s) {
-    if (!mbar_wait(&sm.empty[stage], phase ^ 1, nullptr)) {
-      abort_pipeline(&sm.abort, a.dev_status);
-      break;
+  if (!sm.abort) {
+    for (int s = 0; s < STAGES; ++s) {
+      if (!mbar_wait(&sm.empty[stage], phase ^ 1, &sm.abort, wlim)) {
+        abort_pipeline(&sm.abort, a.dev_status);
+        break;
+      }
+      if (++stage == STAGES) { stage = 0; phase ^= 1; }
     }
-    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+  }
+  if (sm.abort) {
+    // a wait gave up and the consumers may have left without waiting for
+    // their tiles: wait (bounded, regardless of the abort) for the last
+    // copies issued into every stage to land before the CTA can exit
+    for (int s = 0; s < STAGES; ++s)
+      if ((armed >> s) & 1u) mbar_wait(&sm.full[s], (armed_par >> s) & 1u, nullptr, wlim);
   }
   if constexpr (FUSED) {
     // the last CTA to finish leaves the work counter at zero for the next call
@@ -522,6 +543,7 @@ __global__ void __launch_bounds__(kThreads, Shape<G>::MIN_BLOCKS) decode_splitk_
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const int n_sets = a.B * a.Tq;
+  const uint64_t wlim = wait_limit(a.wait_ns);
 
   // ---- work table and barriers
   if (warp == 0) {
@@ -596,7 +618,7 @@ __global__ void __launch_bounds__(kThreads, Shape<G>::MIN_BLOCKS) decode_splitk_
   auto cons_sync = [&]() {
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.cons);
-    mbar_wait(&sm.cons, cons_phase, &sm.abort);
+    mbar_wait(&sm.cons, cons_phase, &sm.abort, wlim);
     cons_phase ^= 1;
     __syncwarp();
   };
@@ -604,7 +626,7 @@ __global__ void __launch_bounds__(kThreads, Shape<G>::MIN_BLOCKS) decode_splitk_
   // Every consumer warp reads the same item sequence from the stages the
   // producer fills.  After an aborted wait the warps stop at their next item.
   for (;;) {
-    if (!mbar_wait(&sm.full[stage], phase, &sm.abort)) abort_pipeline(&sm.abort, a.dev_status);
+    if (!mbar_wait(&sm.full[stage], phase, &sm.abort, wlim)) abort_pipeline(&sm.abort, a.dev_status);
     const int i = sm.stage_item[stage];
     if (i < 0 || sm.abort) {
       __syncwarp();
@@ -622,7 +644,7 @@ __global__ void __launch_bounds__(kThreads, Shape<G>::MIN_BLOCKS) decode_splitk_
     float l_run = 0.f;        // running sum of my slots
 
     for (int row = it.r0; row < it.r1; row += kTileRows) {
-      if (row != it.r0 && !mbar_wait(&sm.full[stage], phase, &sm.abort)) abort_pipeline(&sm.abort, a.dev_status);
+      if (row != it.r0 && !mbar_wait(&sm.full[stage], phase, &sm.abort, wlim)) abort_pipeline(&sm.abort, a.dev_status);
       if (row == it.r0) {
 #pragma unroll
         for (int h = 0; h < G; ++h) {
@@ -941,6 +963,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const int n_sets = a.B * a.Tq;
+  const uint64_t wlim = wait_limit(a.wait_ns);
 
   if (warp == 0) {
     if (a.max_splits == 1) {
@@ -1002,13 +1025,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(
   auto cons_sync = [&]() {
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.cons);
-    mbar_wait(&sm.cons, cons_phase, &sm.abort);
+    mbar_wait(&sm.cons, cons_phase, &sm.abort, wlim);
     cons_phase ^= 1;
     __syncwarp();
   };
 
   for (;;) {
-    if (!mbar_wait(&sm.full[stage], phase, &sm.abort)) abort_pipeline(&sm.abort, a.dev_status);
+    if (!mbar_wait(&sm.full[stage], phase, &sm.abort, wlim)) abort_pipeline(&sm.abort, a.dev_status);
     const int i = sm.stage_item[stage];
     if (i < 0 || sm.abort) {
       __syncwarp();
@@ -1028,7 +1051,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(
     float l_run[2] = {0.f, 0.f};
 
     for (int row = it.r0; row < it.r1; row += kMmaTileRows) {
-      if (row != it.r0 && !mbar_wait(&sm.full[stage], phase, &sm.abort)) abort_pipeline(&sm.abort, a.dev_status);
+      if (row != it.r0 && !mbar_wait(&sm.full[stage], phase, &sm.abort, wlim)) abort_pipeline(&sm.abort, a.dev_status);
       if (row == it.r0) {
         const uint32_t* qw = reinterpret_cast<const uint32_t*>(&sm.q[stage][0][0]);
 #pragma unroll

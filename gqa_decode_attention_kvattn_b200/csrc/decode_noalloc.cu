@@ -168,6 +168,7 @@ extern "C" KVATTN_API int kvattn_decode_noalloc(const kvattn_dims* dims, const u
   a.dev_status = dev_status;
   a.grid = plan.grid;
   a.mma = plan.mma ? 1 : 0;
+  kvattn::apply_wait_policy(a);
   const cudaError_t e = kvattn::launch_decode(a, tk, tv, (cudaStream_t)stream);
   if (e != cudaSuccess && a.counter) {
     // the split kernel may have run without the merge that clears its

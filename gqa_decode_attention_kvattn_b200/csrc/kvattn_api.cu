@@ -2,6 +2,7 @@
 // table, TMA descriptors for the caches, and the launches.  Declared in
 // include/kvattn.h, which states each call's contract.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -23,6 +24,30 @@ int launch_status(cudaError_t e) {
   if (e == cudaSuccess) return KVATTN_OK;
   t_last_cuda_error = (int)e;
   return KVATTN_ERR_CUDA;
+}
+
+namespace {
+// kvattn_set_wait_policy: in-kernel wait limit (0: the kernels' default of
+// one second) and the diagnostics gate, read by every later launch
+std::atomic<uint64_t> g_wait_ns{0};
+std::atomic<const int32_t*> g_gate{nullptr};
+}  // namespace
+
+void apply_wait_policy(DecodeArgs& a) {
+  a.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
+  a.gate = g_gate.load(std::memory_order_relaxed);
+}
+
+void apply_wait_policy(PrefillArgs& a) {
+  a.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
+  a.gate = g_gate.load(std::memory_order_relaxed);
+}
+
+int set_wait_policy(uint64_t limit_ns, const int32_t* gate) {
+  if (reinterpret_cast<uintptr_t>(gate) & 3u) return KVATTN_ERR_INVALID_ARG;
+  g_wait_ns.store(limit_ns, std::memory_order_relaxed);
+  g_gate.store(gate, std::memory_order_relaxed);
+  return KVATTN_OK;
 }
 
 }  // namespace kvattn
@@ -246,6 +271,7 @@ int run_attention(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, con
   a.dev_status = dev_status;
   a.grid = plan.grid;
   a.mma = plan.mma ? 1 : 0;
+  kvattn::apply_wait_policy(a);
 
   // One new token per sequence with all 32 query heads on one KV head (G = 32,
   // multi-query): the 32 heads fill one 128-row tcgen05 M tile, so the
@@ -290,6 +316,7 @@ int run_attention(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, con
     p.part_splits = plan.max_splits;
     p.part_o = a.ws_o;
     p.part_ml = a.ws_ml;
+    kvattn::apply_wait_policy(p);
     a.rows_per_split = split_tiles * 128;
     const cudaError_t e = kvattn::launch_prefill(p, tq, tk2, tv2, (cudaStream_t)stream);
     if (e != cudaSuccess) return kvattn::launch_status(e);
@@ -344,6 +371,7 @@ int run_prefill_tc(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, co
   a.window = mask ? mask->window : 0;
   a.n_sink = (mask && mask->window > 0) ? mask->n_sink : 0;
   a.sink_logits = mask ? mask->sink_logits : nullptr;
+  kvattn::apply_wait_policy(a);
   return kvattn::launch_status(kvattn::launch_prefill(a, tq, tk, tv, (cudaStream_t)stream));
 }
 
@@ -477,6 +505,7 @@ int kvattn_decode_fused(const kvattn_dims* dims, const kvattn_rope_params* rope,
   a.cache_k = cache_k;
   a.cache_v = cache_v;
   a.q_rot_out = q_rot;
+  kvattn::apply_wait_policy(a);
   return kvattn::launch_status(kvattn::launch_decode(a, tk, tv, (cudaStream_t)stream, &tab));
 }
 
@@ -567,5 +596,7 @@ const char* kvattn_last_cuda_error_string(void) {
 }
 
 int kvattn_version(void) { return 100; }
+
+int kvattn_set_wait_policy(uint64_t limit_ns, const int32_t* gate) { return kvattn::set_wait_policy(limit_ns, gate); }
 
 }  // extern "C"

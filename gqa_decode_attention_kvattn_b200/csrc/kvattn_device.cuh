@@ -89,9 +89,13 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// Upper bound of any single pipeline wait.  A legitimate wait is microseconds;
-// one second means the pipeline is broken, and the waiter gives up.
-constexpr uint64_t kWaitLimitNs = 1000000000ull;
+// Default upper bound of any single pipeline wait.  A legitimate wait is
+// microseconds; one second means the pipeline is broken, and the waiter gives
+// up.  (kvattn_set_wait_policy changes it for later launches.)
+constexpr uint64_t kDefaultWaitLimitNs = 1000000000ull;
+
+// The wait limit a launch was given (0: the default).
+__device__ __forceinline__ uint64_t wait_limit(uint64_t ns) { return ns ? ns : kDefaultWaitLimitNs; }
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
@@ -135,16 +139,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity, ui
   return ok != 0;
 }
 // Wait for the phase with the given parity.  Returns false when it did not
-// complete within kWaitLimitNs, or at once when *abort (shared memory, may be
+// complete within limit_ns, or at once when *abort (shared memory, may be
 // null) is set by another warp that already gave up.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const volatile int* abort,
+                                          uint64_t limit_ns) {
   if (abort && *abort) return false;
   if (mbar_try_wait(bar, parity, 1u << 20)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (;;) {
     if (mbar_try_wait(bar, parity, 1u << 20)) return true;
     if (abort && *abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
+// Diagnostics gate (kvattn_set_wait_policy): with a gate, wait until *gate
+// is non-zero, at most limit_ns.  True when there is no gate or it opened.
+__device__ __forceinline__ bool gate_wait(const int32_t* gate, uint64_t limit_ns) {
+  if (!gate) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    int32_t v;
+    asm volatile("ld.volatile.global.b32 %0, [%1];" : "=r"(v) : "l"(gate) : "memory");
+    if (v != 0) return true;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+    __nanosleep(1000);
   }
 }
 

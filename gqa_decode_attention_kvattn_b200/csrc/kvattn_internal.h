@@ -93,6 +93,10 @@ struct DecodeArgs {
   int n_sink;
   const float* sink_logits;
   int mma;       // 1: the tensor-core kernel (its 128B-swizzled 64-row cache view)
+  // limit of each in-kernel wait (0: one second) and the diagnostics gate
+  // (kvattn_set_wait_policy; null: none)
+  uint64_t wait_ns;
+  const int32_t* gate;
 };
 
 // Group view of the decode kernels: G <= 16 query heads per KV head run as
@@ -164,7 +168,15 @@ struct PrefillArgs {
   int part_splits;
   float* part_o;
   float* part_ml;
+  uint64_t wait_ns;     // limit of each in-kernel wait (0: one second)
+  const int32_t* gate;  // diagnostics gate (null: none)
 };
+
+// The process's wait policy (kvattn_set_wait_policy) copied into launch
+// arguments.
+void apply_wait_policy(DecodeArgs& a);
+void apply_wait_policy(PrefillArgs& a);
+int set_wait_policy(uint64_t limit_ns, const int32_t* gate);
 
 // Tokens per 128-row M tile for group size G (128 / G).
 int prefill_tokens_per_tile(int G);

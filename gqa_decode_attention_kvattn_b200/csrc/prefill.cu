@@ -54,7 +54,10 @@ constexpr int kHalf = 128 * 64 * 2; // one 128-row x 64-element bf16 half tile (
 constexpr int kGroupWarps = 4;
 constexpr int kGroupThreads = 32 * kGroupWarps;
 constexpr int kSoftmaxWarps = 2 * kGroupWarps;
-constexpr int kPrefillThreads = 64 + 32 * kSoftmaxWarps;
+// warp 0: TMA producer; warp 1: TMEM owner and MMA issuer of Q tile 0; warps
+// 2..9: softmax; warp 10: MMA issuer of Q tile 1
+constexpr int kMmaWarp1 = 2 + kSoftmaxWarps;
+constexpr int kPrefillThreads = 32 * (kMmaWarp1 + 1);
 // TMEM: S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512); bf16 P_g is
 // written over the first 64 columns of S_g (two per 32-bit column)
 constexpr uint32_t kTmemCols = 512;
@@ -70,7 +73,7 @@ constexpr uint32_t kOffBar = kOffV + 4 * kHalf;
 // (every pipeline barrier exists once per buffer, so a waiter is never more
 // than one phase behind the barrier it waits on)
 constexpr uint32_t kBarQFull = 0, kBarKFull = 1, kBarKEmpty = 3, kBarVFull = 5, kBarVEmpty = 7, kBarSFull = 9,
-                   kBarPFull = 11, kBarMmaDone = 13, kNumBars = 14;
+                   kBarPFull = 11, kBarMmaDone = 13, kNumBars = 15;  // MMA done: one per Q tile's issuer
 constexpr uint32_t kOffTmemSlot = kOffBar + 8 * kNumBars;
 constexpr uint32_t kOffAbort = kOffTmemSlot + 8;
 constexpr uint32_t kPrefillSmemBytes = kOffAbort + 8 + 1024;  // + alignment slack
@@ -88,6 +91,15 @@ __device__ __forceinline__ void bar_expect_tx(uint32_t a, uint32_t bytes) {
 }
 #ifndef KVATTN_PREFILL_SPIN_ALL
 #define KVATTN_PREFILL_SPIN_ALL 1
+#endif
+// waits of the producer and the MMA issuers: suspend (1) or spin
+#ifndef KVATTN_PREFILL_ISSUER_SUSPEND
+#define KVATTN_PREFILL_ISSUER_SUSPEND 0
+#endif
+// softmax exponentiates against the current reference while loading (1), or
+// loads the whole row and takes its max first (0)
+#ifndef KVATTN_PREFILL_OPTIMISTIC
+#define KVATTN_PREFILL_OPTIMISTIC 1
 #endif
 // One try of a phase wait.  With `suspend` the thread sleeps in hardware
 // until the phase completes (or ~1 ms passes); without it the call returns at
@@ -120,18 +132,28 @@ __device__ __forceinline__ void st_shared_i32(uint32_t a, int v) {
 // Bounded wait (see kWaitLimitNs); gives up at once when the CTA's abort flag
 // is set, and sets it (plus the status bit) when it gives up itself.
 __device__ __forceinline__ bool bar_wait(uint32_t a, uint32_t parity, uint32_t abort_addr, int32_t* dev_status,
-                                         bool suspend = !KVATTN_PREFILL_SPIN_ALL) {
+                                         uint64_t limit_ns, bool suspend = !KVATTN_PREFILL_SPIN_ALL) {
   if (ld_shared_i32(abort_addr)) return false;
   if (bar_try_wait(a, parity, suspend)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (;;) {
     if (bar_try_wait(a, parity, suspend)) return true;
     if (ld_shared_i32(abort_addr)) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       st_shared_i32(abort_addr, 1);
       if (dev_status) atomicOr(dev_status, KVATTN_DEV_WAIT_TIMEOUT);
       return false;
     }
+  }
+}
+// Bounded wait that does not give up when the abort flag is set: for the
+// completion of work already handed to the tensor cores or the copy engine.
+__device__ __forceinline__ bool bar_wait_all(uint32_t a, uint32_t parity, uint64_t limit_ns) {
+  if (bar_try_wait(a, parity, false)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    if (bar_try_wait(a, parity, true)) return true;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
   }
 }
 __device__ __forceinline__ void tma_load_4d_raw(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1,
@@ -245,6 +267,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
+  const uint64_t wlim = wait_limit(a.wait_ns);
 
   // heaviest M tile pairs (latest tokens, most keys) first.  In split mode
   // (`dual`) the two Q tiles of a CTA are the same token's heads over two
@@ -304,17 +327,21 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   auto kv_stage = [&](int g, int j) { return dual ? g : (j & 1); };
   auto kv_par = [&](int j) { return dual ? (uint32_t)(j & 1) : (uint32_t)((j >> 1) & 1); };
 
+  // a K/V stage is released by a commit of every issuer that reads it: the
+  // shared stream's stages by both Q tiles' issuers (one if the pair has a
+  // single Q tile), a split-mode stage by its own Q tile's issuer
+  const uint32_t kv_readers = dual ? 1u : (uint32_t)n_q;
   if (tid == 0) {
     bar_init(bar(kBarQFull), 1);
     for (int s = 0; s < 2; ++s) {
       bar_init(bar(kBarKFull + s), 1);
-      bar_init(bar(kBarKEmpty + s), 1);
+      bar_init(bar(kBarKEmpty + s), kv_readers);
       bar_init(bar(kBarVFull + s), 1);
-      bar_init(bar(kBarVEmpty + s), 1);
+      bar_init(bar(kBarVEmpty + s), kv_readers);
       bar_init(bar(kBarSFull + s), 1);
       bar_init(bar(kBarPFull + s), kGroupWarps);
+      bar_init(bar(kBarMmaDone + s), 1);
     }
-    bar_init(bar(kBarMmaDone), 1);
     st_shared_i32(abort_addr, 0);
     fence_barrier_init();
   }
@@ -329,18 +356,29 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   tc_fence_after();
   const uint32_t tmem = (uint32_t)ld_shared_i32(base + kOffTmemSlot);
 
+  // producer state kept to the end of the kernel: whether the gate opened
+  // (the Q tiles were loaded) and the key tile last loaded into each K and V
+  // stage (-1: none), to wait for copies still in flight after an abort
+  bool gate_open = false;
+  int last_k[2] = {-1, -1}, last_v[2] = {-1, -1};
   if (warp == 0) {
     // ================================================================ producer
     if (lane == 0) {
       prefetch_tensormap(&tmap_q);
       prefetch_tensormap(&tmap_k);
       prefetch_tensormap(&tmap_v);
-      bar_expect_tx(bar(kBarQFull), (uint32_t)n_q * 2u * kHalf);
-      for (int g = 0; g < n_q; ++g) {
-        tma_load_4d_raw(sQ + (2 * g) * kHalf, &tmap_q, bar(kBarQFull), 0, kvh * G, t0 + g * TT, b);
-        tma_load_4d_raw(sQ + (2 * g + 1) * kHalf, &tmap_q, bar(kBarQFull), 64, kvh * G, t0 + g * TT, b);
+      gate_open = gate_wait(a.gate, wlim);
+      bool go = gate_open;
+      if (!go) {
+        st_shared_i32(abort_addr, 1);
+        set_status(a.dev_status, KVATTN_DEV_WAIT_TIMEOUT);
+      } else {
+        bar_expect_tx(bar(kBarQFull), (uint32_t)n_q * 2u * kHalf);
+        for (int g = 0; g < n_q; ++g) {
+          tma_load_4d_raw(sQ + (2 * g) * kHalf, &tmap_q, bar(kBarQFull), 0, kvh * G, t0 + g * TT, b);
+          tma_load_4d_raw(sQ + (2 * g + 1) * kHalf, &tmap_q, bar(kBarQFull), 64, kvh * G, t0 + g * TT, b);
+        }
       }
-      bool go = true;
       for (int j = 0; j < n_iter && go; ++j) {
         // the shared stream loads key tile j once; split mode loads it per Q tile
         for (int g = 0; g < (dual ? 2 : 1) && go; ++g) {
@@ -348,85 +386,79 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           const int s = kv_stage(g, j);
           const uint32_t par = kv_par(j) ^ 1u;
           const int key0 = key_tile(g, j) * kBN;
-          if (!bar_wait(bar(kBarKEmpty + s), par, abort_addr, a.dev_status)) { go = false; break; }
+          if (!bar_wait(bar(kBarKEmpty + s), par, abort_addr, a.dev_status, wlim, KVATTN_PREFILL_ISSUER_SUSPEND || !KVATTN_PREFILL_SPIN_ALL)) { go = false; break; }
           bar_expect_tx(bar(kBarKFull + s), 2 * kHalf);
+          last_k[s] = j;
           tma_load_4d_raw(sK + (2 * s) * kHalf, &tmap_k, bar(kBarKFull + s), 0, kvh, key0, b);
           tma_load_4d_raw(sK + (2 * s + 1) * kHalf, &tmap_k, bar(kBarKFull + s), 64, kvh, key0, b);
-          if (!bar_wait(bar(kBarVEmpty + s), par, abort_addr, a.dev_status)) { go = false; break; }
+          if (!bar_wait(bar(kBarVEmpty + s), par, abort_addr, a.dev_status, wlim, KVATTN_PREFILL_ISSUER_SUSPEND || !KVATTN_PREFILL_SPIN_ALL)) { go = false; break; }
           bar_expect_tx(bar(kBarVFull + s), 2 * kHalf);
+          last_v[s] = j;
           tma_load_4d_raw(sV + (2 * s) * kHalf, &tmap_v, bar(kBarVFull + s), 0, kvh, key0, b);
           tma_load_4d_raw(sV + (2 * s + 1) * kHalf, &tmap_v, bar(kBarVFull + s), 64, kvh, key0, b);
         }
       }
     }
-  } else if (warp == 1) {
-    // ================================================================ MMA issuer
+  } else if (warp == 1 || warp == kMmaWarp1) {
+    // ================================================================ MMA issuers
+    // One thread per Q tile issues that tile's MMAs (a single issuing thread
+    // cannot feed the tensor core one 128x128x16 MMA per 64 cycles; two can).
+    // Per key tile j of Q tile g, in issue order:
+    //   O_g += P_g(j-1) V_{j-1}   once the softmax has published P_g(j-1)
+    //   S_g  = Q_g K_j^T          into the same TMEM columns P_g(j-1) is read from:
+    //                             one thread's MMAs run in issue order, so the
+    //                             PV has read its operand before the QK writes
+    // so the tensor cores run one Q tile's MMAs while the other tile's softmax
+    // works.  (In split mode both Q tiles read Q slot 0, the one token's
+    // heads, and K/V tile j of Q tile g's own stream.)
     if (lane == 0) {
+      const int g = warp == 1 ? 0 : 1;
+      const int nt = g == 0 ? nt0 : nt1;
       constexpr uint32_t idesc_qk = idesc_bf16_m128_n128(false);
       constexpr uint32_t idesc_pv = idesc_bf16_m128_n128(true);
-      bool ok = bar_wait(bar(kBarQFull), 0, abort_addr, a.dev_status);
+      const uint32_t d_s = tmem + kColS + 128u * (uint32_t)g;
+      const uint32_t d_o = tmem + kColO + 128u * (uint32_t)g;
+      // operand descriptors of k-step 0; k-step kk adds (byte offset) >> 4
+      const uint64_t q_desc = sw128_desc(sQ + (dual ? 0u : 2u * (uint32_t)g) * kHalf, 16, 1024);
+      bool ok = nt > 0 && bar_wait(bar(kBarQFull), 0, abort_addr, a.dev_status, wlim, KVATTN_PREFILL_ISSUER_SUSPEND || !KVATTN_PREFILL_SPIN_ALL);
       tc_fence_after();
-      // S_g = Q_g K_j^T into S buffer g.  It is issued right after PV_g(j-1),
-      // which reads P_g(j-1) out of the same columns: MMAs issued by one
-      // thread run in issue order, so the PV has read its operand before this
-      // QK writes the accumulator.
-      // (in split mode both Q tiles read Q slot 0, the one token's heads, and
-      // K tile j of Q tile g's own stream, released per stream)
-      auto qk = [&](int g, int j) {
+      auto pv = [&](int j) {
         const int s = kv_stage(g, j);
-        if (dual && !bar_wait(bar(kBarKFull + s), kv_par(j), abort_addr, a.dev_status)) return false;
+        if (!bar_wait(bar(kBarVFull + s), kv_par(j), abort_addr, a.dev_status, wlim, KVATTN_PREFILL_ISSUER_SUSPEND || !KVATTN_PREFILL_SPIN_ALL)) return false;
+        if (!bar_wait(bar(kBarPFull + g), (uint32_t)j & 1u, abort_addr, a.dev_status, wlim, KVATTN_PREFILL_ISSUER_SUSPEND || !KVATTN_PREFILL_SPIN_ALL)) return false;
         tc_fence_after();
-        const int qs = dual ? 0 : g;
+        // V tile as B = [keys x dims], dims contiguous: 64-dim atoms one half
+        // apart (LBO), 8-key groups 1 KB apart (SBO); 16 keys (2 KB) per step;
+        // P_g from TMEM: keys 16kk..16kk+15 are columns 8kk..8kk+7 of S_g
+        const uint64_t v_desc = sw128_desc(sV + 2u * (uint32_t)s * kHalf, kHalf, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc_mma_ts(d_o, d_s + 8u * kk, v_desc + (uint64_t)(kk * 2048 / 16), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(bar(kBarVEmpty + s));
+        return true;
+      };
+      for (int j = 0; ok && j < nt; ++j) {
+        if (j > 0 && !pv(j - 1)) { ok = false; break; }
+        const int s = kv_stage(g, j);
+        if (!bar_wait(bar(kBarKFull + s), kv_par(j), abort_addr, a.dev_status, wlim, KVATTN_PREFILL_ISSUER_SUSPEND || !KVATTN_PREFILL_SPIN_ALL)) { ok = false; break; }
+        tc_fence_after();
+        const uint64_t k_desc = sw128_desc(sK + 2u * (uint32_t)s * kHalf, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t da = sw128_desc(sQ + (2 * qs + (kk >> 2)) * kHalf + (kk & 3) * 32, 16, 1024);
-          const uint64_t db = sw128_desc(sK + (2 * s + (kk >> 2)) * kHalf + (kk & 3) * 32, 16, 1024);
-          tc_mma(tmem + kColS + 128u * (uint32_t)g, da, db, idesc_qk, kk > 0 ? 1u : 0u);
+          const uint64_t off = (uint64_t)(((kk >> 2) * kHalf + (kk & 3) * 32) >> 4);
+          tc_mma(d_s, q_desc + off, k_desc + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
         tc_commit(bar(kBarSFull + g));
-        if (dual) tc_commit(bar(kBarKEmpty + s));
-        return true;
-      };
-      // O_g += P_g(j) V_j once the softmax has published P_g(j)
-      auto pv = [&](int g, int j) {
-        const int s = kv_stage(g, j);
-        if (!bar_wait(bar(kBarVFull + s), kv_par(j), abort_addr, a.dev_status)) return false;
-        if (!bar_wait(bar(kBarPFull + g), (uint32_t)j & 1u, abort_addr, a.dev_status)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          // P_g from TMEM: keys 16kk..16kk+15 are columns 8kk..8kk+7 of S buffer g
-          const uint32_t pa = tmem + kColS + 128u * (uint32_t)g + 8u * kk;
-          // V tile as B = [keys x dims], dims contiguous: 64-dim atoms one half
-          // apart (LBO), 8-key groups 1 KB apart (SBO); 16 keys per step
-          const uint64_t db = sw128_desc(sV + (2 * s) * kHalf + kk * 2048, kHalf, 1024);
-          tc_mma_ts(tmem + kColO + 128u * (uint32_t)g, pa, db, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        if (dual) tc_commit(bar(kBarVEmpty + s));
-        return true;
-      };
-      // Ping-pong: the tensor cores run Q tile 1's MMAs while the softmax
-      // works on tile 0's scores and the other way round.  Per key tile j:
-      //   QK_0(j), PV_1(j-1), QK_1(j), PV_0(j)
-      for (int j = 0; j <= n_iter && ok; ++j) {
-        if (j < n_iter) {
-          if (!dual && !bar_wait(bar(kBarKFull + (j & 1)), (uint32_t)(j >> 1) & 1u, abort_addr, a.dev_status))
-            break;
-          if (active(0, j) && !qk(0, j)) break;
-        }
-        if (j > 0) {
-          if (active(1, j - 1) && !pv(1, j - 1)) break;
-          if (!dual) tc_commit(bar(kBarVEmpty + ((j - 1) & 1)));  // both PVs of tile j-1 issued
-        }
-        if (j < n_iter) {
-          if (active(1, j) && !qk(1, j)) break;
-          if (!dual) tc_commit(bar(kBarKEmpty + (j & 1)));  // both QKs of tile j issued
-          if (active(0, j) && !pv(0, j)) break;
-        }
+        tc_commit(bar(kBarKEmpty + s));
       }
-      tc_commit(bar(kBarMmaDone));
-      // every MMA issued above has finished once this completes
-      bar_wait(bar(kBarMmaDone), 0, abort_addr, nullptr);
+      if (ok && nt > 0) pv(nt - 1);
+      // (Q tile 0 may stop one key tile short of the shared stream's last
+      // tile; nothing waits for that stage to be released again)
+      tc_commit(bar(kBarMmaDone + g));
+      // every MMA this thread issued has finished once this completes; wait
+      // for it even after an abort (bounded), so TMEM and shared memory stay
+      // in use until the tensor cores are done with them
+      bar_wait_all(bar(kBarMmaDone + g), 0, wlim);
     }
   } else {
     // ================================================================ softmax / epilogue
@@ -448,46 +480,42 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 
     for (int j = 0; active(grp, j); ++j) {
       const int jt = key_tile(grp, j);
-      bar_wait(bar(kBarSFull + grp), (uint32_t)j & 1u, abort_addr, a.dev_status);
+      if (!bar_wait(bar(kBarSFull + grp), (uint32_t)j & 1u, abort_addr, a.dev_status, wlim)) break;
       tc_fence_after();
-      // the thread's whole S row
+      // the thread's whole S row, 32 columns (one TMEM load) at a time
       uint32_t sr[4][32];
-#pragma unroll
-      for (int c2 = 0; c2 < 4; ++c2) tmem_ld32(lane_addr + col_s + 32u * c2, sr[c2]);
-      tmem_wait_ld();
-
-      // mask (raw scores; the scale is folded into the exponent below) and
-      // row max over eight independent accumulators
+      // mask (raw scores; the scale is folded into the exponent below)
       const int kbase = jt * kBN;
-      if (kbase + kBN - 1 > lim || (kbase < lo_vis && kbase + kBN - 1 >= a.n_sink)) {
+      const bool need_mask = kbase + kBN - 1 > lim || (kbase < lo_vis && kbase + kBN - 1 >= a.n_sink);
+      auto mask_chunk = [&](int c2) {
+        if (need_mask) {
 #pragma unroll
-        for (int c = 0; c < kBN; ++c) {
-          const int k = kbase + c;
-          if (k > lim || (k < lo_vis && k >= a.n_sink)) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+          for (int c = 0; c < 32; ++c) {
+            const int k = kbase + 32 * c2 + c;
+            if (k > lim || (k < lo_vis && k >= a.n_sink)) sr[c2][c] = __float_as_uint(-INFINITY);
+          }
         }
-      }
+      };
+      // row max over eight independent accumulators
       float mx8[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) mx8[k] = __uint_as_float(sr[0][k]);
+      for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
+      auto max_chunk = [&](int c2) {
 #pragma unroll
-      for (int c = 8; c < kBN; c += 8)
+        for (int c = 0; c < 32; c += 8)
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], __uint_as_float(sr[c >> 5][(c & 31) + k]));
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) *
-                       a.scale_log2;
-      const bool move = mx > ref + 8.f;
-      const float ref_new = move ? mx : ref;
-      const float alpha = move ? fast_exp2(ref - ref_new) : 1.f;
-      ref = ref_new;
+          for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], __uint_as_float(sr[c2][c + k]));
+      };
+      auto row_max = [&]() {
+        return fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                     fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) *
+               a.scale_log2;
+      };
       // p = 2^(s * scale_log2 - ref): packed FMA for two scores, one ex2 each,
       // packed sums in four accumulators; 32 keys (16 P columns) at a time,
       // written over the S columns already read
-      const float neg_ref = (ref == -INFINITY) ? 0.f : -ref;
-      const uint64_t nr2 = f2_pack(neg_ref, neg_ref);
       uint64_t sum2[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-      for (int c2 = 0; c2 < 4; ++c2) {
+      auto exp_chunk = [&](int c2, uint64_t nr2) {
         uint32_t pk[16];
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
@@ -500,6 +528,65 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           pk[c >> 1] = pack_bf16x2_rn(p0, p1);
         }
         tmem_st16(lane_addr + col_s + 16u * c2, pk);
+      };
+      auto neg_ref2 = [&]() {
+        const float nr = (ref == -INFINITY) ? 0.f : -ref;
+        return f2_pack(nr, nr);
+      };
+      bool move;
+      float alpha = 1.f;
+#if KVATTN_PREFILL_OPTIMISTIC
+      if (ref != -INFINITY) {
+        // The row's reference rarely moves (only when a tile's max exceeds it
+        // by more than 8), so exponentiate each 32-column chunk against the
+        // current reference as soon as it is loaded, with the next chunk's
+        // load in flight, and track the max alongside.  If the reference does
+        // have to move, redo the tile's exponentials from the scores still in
+        // registers: the same values as exponentiating after the max.
+        tmem_ld32(lane_addr + col_s, sr[0]);
+        tmem_wait_ld();
+        const uint64_t nr2 = neg_ref2();
+#pragma unroll
+        for (int c2 = 0; c2 < 4; ++c2) {
+          if (c2 < 3) tmem_ld32(lane_addr + col_s + 32u * (c2 + 1), sr[c2 + 1]);
+          mask_chunk(c2);
+          max_chunk(c2);
+          exp_chunk(c2, nr2);
+          if (c2 < 3) tmem_wait_ld();
+        }
+        const float mx = row_max();
+        move = mx > ref + 8.f;
+        if (move) {
+          alpha = fast_exp2(ref - mx);
+          ref = mx;
+          tmem_wait_st();  // the first P stores land before they are overwritten
+#pragma unroll
+          for (int k = 0; k < 4; ++k) sum2[k] = 0ull;
+          const uint64_t nr2m = neg_ref2();
+#pragma unroll
+          for (int c2 = 0; c2 < 4; ++c2) exp_chunk(c2, nr2m);
+        }
+      } else
+#endif
+      {
+        // (first tile of the row, or the plain order) load the row, take its
+        // max, then exponentiate
+#pragma unroll
+        for (int c2 = 0; c2 < 4; ++c2) tmem_ld32(lane_addr + col_s + 32u * c2, sr[c2]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c2 = 0; c2 < 4; ++c2) {
+          mask_chunk(c2);
+          max_chunk(c2);
+        }
+        const float mx = row_max();
+        move = mx > ref + 8.f;
+        const float ref_new = move ? mx : ref;
+        alpha = move ? fast_exp2(ref - ref_new) : 1.f;
+        ref = ref_new;
+        const uint64_t nr2 = neg_ref2();
+#pragma unroll
+        for (int c2 = 0; c2 < 4; ++c2) exp_chunk(c2, nr2);
       }
       float sa, sb;
       f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), sa, sb);
@@ -525,7 +612,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         // before their own P goes out; in split mode only the group whose
         // split holds key tile n_all - 1 gets here, and it zeroes its own stage
         const int s = kv_stage(grp, j);
-        bar_wait(bar(kBarVFull + s), kv_par(j), abort_addr, a.dev_status);
+        bar_wait(bar(kBarVFull + s), kv_par(j), abort_addr, a.dev_status, wlim);
         const int first_bad = Lmax - jt * kBN;
         const int nchunks = (kBN - first_bad) * 16;  // 16-byte chunks over both halves
         for (int c = gt; c < nchunks; c += kGroupThreads) {
@@ -544,7 +631,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 
     // ---- epilogue: O / l -> bf16 rows
     // (the MMA-done barrier completes once, after the last PV has finished)
-    bar_wait(bar(kBarMmaDone), 0, abort_addr, a.dev_status);
+    bar_wait(bar(kBarMmaDone + grp), 0, abort_addr, a.dev_status, wlim);
     tc_fence_after();
     float inv_l = 1.f / l;
     if (a.sink_logits) {
@@ -604,6 +691,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+  }
+  if (tid == 0 && ld_shared_i32(abort_addr)) {
+    // a wait gave up somewhere in the CTA, so some tiles may never have been
+    // waited for: before the CTA exits, wait (bounded, regardless of the
+    // abort) until every copy issued into its shared memory has landed
+    if (gate_open) bar_wait_all(bar(kBarQFull), 0, wlim);
+    for (int s = 0; s < 2; ++s) {
+      if (last_k[s] >= 0) bar_wait_all(bar(kBarKFull + s), kv_par(last_k[s]), wlim);
+      if (last_v[s] >= 0) bar_wait_all(bar(kBarVFull + s), kv_par(last_v[s]), wlim);
+    }
   }
 }
 

@@ -317,6 +317,28 @@ KVATTN_API const char* kvattn_last_cuda_error_string(void);
 /* Library version, major*10000 + minor*100 + patch. */
 KVATTN_API int kvattn_version(void);
 
+/* Failure-path diagnostics (no counterpart on the pages).  Every in-kernel
+ * pipeline wait of the library is bounded: when it does not complete within
+ * the limit, the CTA sets KVATTN_DEV_WAIT_TIMEOUT in *dev_status, stops
+ * waiting, lets the copies and tensor-core work it already issued finish,
+ * frees its tensor memory and exits; the call's outputs are then undefined
+ * (a fused decode may also leave its new cache row unwritten).  This sets,
+ * for every launch made afterwards by this process:
+ *  - limit_ns: the limit of each wait in nanoseconds (0: the default, one
+ *    second);
+ *  - gate: NULL, or a 4-byte aligned device int32 that the pipelined kernels
+ *    (kvattn_decode, kvattn_decode_masked, kvattn_decode_fused,
+ *    kvattn_decode_noalloc, kvattn_prefill_chunk(_masked)) wait on, within
+ *    the limit, until it is non-zero, before they issue any copy.  A gate
+ *    that stays zero makes every such launch give up after the limit, which
+ *    is how the failure path is tested without breaking any kernel.
+ * Recovery after a call that set KVATTN_DEV_WAIT_TIMEOUT: kvattn_decode,
+ * kvattn_decode_masked and kvattn_decode_noalloc leave their work counter
+ * zero and need nothing; zero a kvattn_decode_fused workspace again.
+ * Process-wide; change it only while no other thread launches library work.
+ * Returns KVATTN_OK, or INVALID_ARG for a misaligned gate. */
+KVATTN_API int kvattn_set_wait_policy(uint64_t limit_ns, const int32_t* gate);
+
 #ifdef __cplusplus
 }
 #endif
