@@ -7,8 +7,8 @@ One "step" is one pass of the whole hot path over one batch: for every layer,
 RoPE + cache append (kvattn_rope_append) then attention (kvattn_decode: the
 split-K kernel and its LSE merge kernel, or kvattn_prefill_chunk for the
 prefill workload), each layer with its own cache.  Small, latency-bound
-decode workloads (the single sequence at p=1000) run the single-launch
-kvattn_decode_fused instead (--path auto; --path split|fused forces one).  The default workload is batched ragged decode: B=64 sequences, 32
+decode workloads can run the single-launch kvattn_decode_fused instead
+(--path fused; the default split path measured faster at every size).  The default workload is batched ragged decode: B=64 sequences, 32
 layers with separate [64, 8192, 8, 128] bf16 caches (64 GiB in HBM, far
 larger than L2, so every step streams its K/V rows from HBM), start positions
 uniform in [512, 8191].
@@ -58,6 +58,7 @@ def measured_peaks():
 
 KERNEL_SOURCES = {
     "decode_splitk": ("decode.cu", "kvattn_device.cuh"),
+    "decode_mma": ("decode.cu", "kvattn_device.cuh"),
     # multi-query decode (G = 32): the tcgen05 kernel in split mode + the LSE merge
     "decode_tc": ("prefill.cu", "decode.cu", "kvattn_device.cuh"),
     "decode_fused": ("decode.cu", "kvattn_device.cuh", "rope_device.cuh"),
@@ -251,7 +252,11 @@ def build_state(w, seed, device, path="auto", sets=1):
             layers.append(L)
         layer_sets.append(layers)
     if path == "auto":
-        path = "fused" if w.B * w.Hkv * w.kv_len_hint < (1 << 18) else "split"
+        # the split path (rope_append, decode, merge: three launches chained by
+        # programmatic dependent launch) measured faster than the one-launch
+        # fused decode at every size, the single sequence at p=1000 included
+        # (14.4 against 20.3 us per layer in a 32-layer graph with a cold L2)
+        path = "split"
     fused = w.kind == "decode" and path == "fused"
     if fused:
         ws_bytes = kv.kvattn_decode_fused_workspace_bytes(w.B, w.H, w.Hkv, w.S, w.kv_len_hint)
@@ -728,8 +733,7 @@ def main():
     ap.add_argument("--seed", type=int, default=ks.DEFAULT_SEED)
     ap.add_argument("--path", choices=["auto", "fused", "split"], default="auto",
                     help="decode entry points: rope_append + decode (+ merge kernel), or one kvattn_decode_fused "
-                         "launch per layer; auto takes the fused launch for small, latency-bound calls (fewer than "
-                         "2^18 (row, KV head) pairs per layer) and the split path otherwise")
+                         "launch per layer; auto takes the split path (measured faster at every size)")
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -54,10 +54,8 @@ constexpr int kHalf = 128 * 64 * 2; // one 128-row x 64-element bf16 half tile (
 constexpr int kGroupWarps = 4;
 constexpr int kGroupThreads = 32 * kGroupWarps;
 constexpr int kSoftmaxWarps = 2 * kGroupWarps;
-// warp 0: TMA producer; warp 1: TMEM owner and MMA issuer of Q tile 0; warps
-// 2..9: softmax; warp 10: MMA issuer of Q tile 1
-constexpr int kMmaWarp1 = 2 + kSoftmaxWarps;
-constexpr int kPrefillThreads = 32 * (kMmaWarp1 + 1);
+// warp 0: TMA producer; warp 1: TMEM owner and MMA issuer; warps 2..9: softmax
+constexpr int kPrefillThreads = 64 + 32 * kSoftmaxWarps;
 // TMEM: S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512); bf16 P_g is
 // written over the first 64 columns of S_g (two per 32-bit column)
 constexpr uint32_t kTmemCols = 512;
@@ -73,7 +71,7 @@ constexpr uint32_t kOffBar = kOffV + 4 * kHalf;
 // (every pipeline barrier exists once per buffer, so a waiter is never more
 // than one phase behind the barrier it waits on)
 constexpr uint32_t kBarQFull = 0, kBarKFull = 1, kBarKEmpty = 3, kBarVFull = 5, kBarVEmpty = 7, kBarSFull = 9,
-                   kBarPFull = 11, kBarMmaDone = 13, kNumBars = 15;  // MMA done: one per Q tile's issuer
+                   kBarPFull = 11, kBarMmaDone = 13, kNumBars = 15;  // MMA done: one per Q tile's softmax group
 constexpr uint32_t kOffTmemSlot = kOffBar + 8 * kNumBars;
 constexpr uint32_t kOffAbort = kOffTmemSlot + 8;
 constexpr uint32_t kPrefillSmemBytes = kOffAbort + 8 + 1024;  // + alignment slack
@@ -99,7 +97,25 @@ __device__ __forceinline__ void bar_expect_tx(uint32_t a, uint32_t bytes) {
 // softmax exponentiates against the current reference while loading (1), or
 // loads the whole row and takes its max first (0)
 #ifndef KVATTN_PREFILL_OPTIMISTIC
-#define KVATTN_PREFILL_OPTIMISTIC 1
+#define KVATTN_PREFILL_OPTIMISTIC 0
+#endif
+// of every four pairs of scores, how many are exponentiated by polynomial on
+// the FMA pipes instead of the special-function unit (0..4)
+#ifndef KVATTN_PREFILL_POLY_PAIRS
+#define KVATTN_PREFILL_POLY_PAIRS 1
+#endif
+// P to bf16 on the integer pipes (1) or with the conversion instruction (0)
+#ifndef KVATTN_PREFILL_INT_PACK
+#define KVATTN_PREFILL_INT_PACK 1
+#endif
+// softmax reads each S chunk twice from TMEM (max, then exponentials) instead
+// of holding the 128-column row in registers
+#ifndef KVATTN_PREFILL_TWO_PASS
+#define KVATTN_PREFILL_TWO_PASS 0
+#endif
+// row max with three-input max instructions
+#ifndef KVATTN_PREFILL_MAX3
+#define KVATTN_PREFILL_MAX3 1
 #endif
 // One try of a phase wait.  With `suspend` the thread sleeps in hardware
 // until the phase completes (or ~1 ms passes); without it the call returns at
@@ -244,6 +260,58 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// 2^x of two fp32 values on the FMA pipes, to take part of the softmax's
+// exponentials off the special-function unit.  Cody and Waite's argument
+// reduction: x = n + f with n = round(x) (adding 1.5 * 2^23 leaves round(x) in
+// the low mantissa bits) and f in [-1/2, 1/2]; 2^f by a cubic fitted to it on
+// that interval by a Remez exchange on the relative error (max relative error
+// 7.5e-5, far below the bf16 rounding of P); 2^n by adding n to the exponent
+// field.  x is clamped to >= -125 (2^-125, a normal number); a caller that
+// needs 2^-inf = 0 selects it.
+constexpr float kExp2C0 = 9.999280572e-01f, kExp2C1 = 6.932609677e-01f, kExp2C2 = 2.426111251e-01f,
+                kExp2C3 = 5.517166853e-02f;
+__device__ __forceinline__ void exp2_poly_x2(float x0, float x1, float& p0, float& p1) {
+  x0 = fmaxf(x0, -125.f);
+  x1 = fmaxf(x1, -125.f);
+  const uint64_t x = f2_pack(x0, x1);
+  const uint64_t t = f2_add(x, f2_pack(12582912.f, 12582912.f));  // 1.5 * 2^23 + round(x)
+  const uint64_t n = f2_add(t, f2_pack(-12582912.f, -12582912.f));
+  const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), x);
+  uint64_t q = f2_fma(f2_pack(kExp2C3, kExp2C3), f, f2_pack(kExp2C2, kExp2C2));
+  q = f2_fma(q, f, f2_pack(kExp2C1, kExp2C1));
+  q = f2_fma(q, f, f2_pack(kExp2C0, kExp2C0));
+  float q0, q1, t0, t1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(t, t0, t1);
+  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
+// Two non-negative finite fp32 values (softmax probabilities) to packed bf16
+// on the integer pipes: add half a bf16 ulp, keep the upper 16 bits of each
+// (round to nearest, ties away from zero; ties of the fp32 inputs are rare
+// and the result is within half an ulp either way).  The conversion
+// instruction would run on the special-function pipe that the exponentials
+// already saturate.
+__device__ __forceinline__ uint32_t pack_bf16x2_p(float lo, float hi) {
+#if KVATTN_PREFILL_INT_PACK
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(r) : "r"(__float_as_uint(lo) + 0x8000u), "r"(__float_as_uint(hi) + 0x8000u));
+  return r;
+#else
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+#endif
+}
+
+// max(a, b, c) in one instruction (NaN inputs are ignored, as by fmaxf)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
@@ -327,17 +395,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   auto kv_stage = [&](int g, int j) { return dual ? g : (j & 1); };
   auto kv_par = [&](int j) { return dual ? (uint32_t)(j & 1) : (uint32_t)((j >> 1) & 1); };
 
-  // a K/V stage is released by a commit of every issuer that reads it: the
-  // shared stream's stages by both Q tiles' issuers (one if the pair has a
-  // single Q tile), a split-mode stage by its own Q tile's issuer
-  const uint32_t kv_readers = dual ? 1u : (uint32_t)n_q;
   if (tid == 0) {
     bar_init(bar(kBarQFull), 1);
     for (int s = 0; s < 2; ++s) {
       bar_init(bar(kBarKFull + s), 1);
-      bar_init(bar(kBarKEmpty + s), kv_readers);
+      bar_init(bar(kBarKEmpty + s), 1);
       bar_init(bar(kBarVFull + s), 1);
-      bar_init(bar(kBarVEmpty + s), kv_readers);
+      bar_init(bar(kBarVEmpty + s), 1);
       bar_init(bar(kBarSFull + s), 1);
       bar_init(bar(kBarPFull + s), kGroupWarps);
       bar_init(bar(kBarMmaDone + s), 1);
@@ -399,66 +463,85 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
       }
     }
-  } else if (warp == 1 || warp == kMmaWarp1) {
-    // ================================================================ MMA issuers
-    // One thread per Q tile issues that tile's MMAs (a single issuing thread
-    // cannot feed the tensor core one 128x128x16 MMA per 64 cycles; two can).
-    // Per key tile j of Q tile g, in issue order:
-    //   O_g += P_g(j-1) V_{j-1}   once the softmax has published P_g(j-1)
-    //   S_g  = Q_g K_j^T          into the same TMEM columns P_g(j-1) is read from:
-    //                             one thread's MMAs run in issue order, so the
-    //                             PV has read its operand before the QK writes
+  } else if (warp == 1) {
+    // ================================================================ MMA issuer
+    // One thread issues every MMA, in an order that keeps the two Q tiles half
+    // a period apart: per key tile j,
+    //   QK_0(j), PV_1(j-1), QK_1(j), PV_0(j)
     // so the tensor cores run one Q tile's MMAs while the other tile's softmax
-    // works.  (In split mode both Q tiles read Q slot 0, the one token's
-    // heads, and K/V tile j of Q tile g's own stream.)
+    // works.  S_g = Q_g K_j^T goes into TMEM columns that PV_g(j-1) reads
+    // P_g(j-1) from; it is issued after that PV by the same thread, and one
+    // thread's MMAs run in issue order, so the PV has read its operand first.
+    // (A single thread issues an MMA every ~90 cycles; a 128x128x16 MMA takes
+    // 64.  Two issuing threads, one per Q tile, reach the tensor core's rate
+    // but drift into lockstep: both softmaxes then share the exponential unit
+    // and the tensor cores idle meanwhile, which measured slower.)
+    // In split mode both Q tiles read Q slot 0, the one token's heads, and K/V
+    // tile j of Q tile g's own stream, released per stream.
     if (lane == 0) {
-      const int g = warp == 1 ? 0 : 1;
-      const int nt = g == 0 ? nt0 : nt1;
+      constexpr bool kSusp = KVATTN_PREFILL_ISSUER_SUSPEND || !KVATTN_PREFILL_SPIN_ALL;
       constexpr uint32_t idesc_qk = idesc_bf16_m128_n128(false);
       constexpr uint32_t idesc_pv = idesc_bf16_m128_n128(true);
-      const uint32_t d_s = tmem + kColS + 128u * (uint32_t)g;
-      const uint32_t d_o = tmem + kColO + 128u * (uint32_t)g;
-      // operand descriptors of k-step 0; k-step kk adds (byte offset) >> 4
-      const uint64_t q_desc = sw128_desc(sQ + (dual ? 0u : 2u * (uint32_t)g) * kHalf, 16, 1024);
-      bool ok = nt > 0 && bar_wait(bar(kBarQFull), 0, abort_addr, a.dev_status, wlim, KVATTN_PREFILL_ISSUER_SUSPEND || !KVATTN_PREFILL_SPIN_ALL);
+      bool ok = bar_wait(bar(kBarQFull), 0, abort_addr, a.dev_status, wlim, kSusp);
       tc_fence_after();
-      auto pv = [&](int j) {
+      // operand descriptors of k-step 0; k-step kk adds (byte offset) >> 4
+      auto qk = [&](int g, int j) {
         const int s = kv_stage(g, j);
-        if (!bar_wait(bar(kBarVFull + s), kv_par(j), abort_addr, a.dev_status, wlim, KVATTN_PREFILL_ISSUER_SUSPEND || !KVATTN_PREFILL_SPIN_ALL)) return false;
-        if (!bar_wait(bar(kBarPFull + g), (uint32_t)j & 1u, abort_addr, a.dev_status, wlim, KVATTN_PREFILL_ISSUER_SUSPEND || !KVATTN_PREFILL_SPIN_ALL)) return false;
+        if (dual && !bar_wait(bar(kBarKFull + s), kv_par(j), abort_addr, a.dev_status, wlim, kSusp)) return false;
         tc_fence_after();
-        // V tile as B = [keys x dims], dims contiguous: 64-dim atoms one half
-        // apart (LBO), 8-key groups 1 KB apart (SBO); 16 keys (2 KB) per step;
-        // P_g from TMEM: keys 16kk..16kk+15 are columns 8kk..8kk+7 of S_g
-        const uint64_t v_desc = sw128_desc(sV + 2u * (uint32_t)s * kHalf, kHalf, 1024);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          tc_mma_ts(d_o, d_s + 8u * kk, v_desc + (uint64_t)(kk * 2048 / 16), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(bar(kBarVEmpty + s));
-        return true;
-      };
-      for (int j = 0; ok && j < nt; ++j) {
-        if (j > 0 && !pv(j - 1)) { ok = false; break; }
-        const int s = kv_stage(g, j);
-        if (!bar_wait(bar(kBarKFull + s), kv_par(j), abort_addr, a.dev_status, wlim, KVATTN_PREFILL_ISSUER_SUSPEND || !KVATTN_PREFILL_SPIN_ALL)) { ok = false; break; }
-        tc_fence_after();
+        const uint64_t q_desc = sw128_desc(sQ + (dual ? 0u : 2u * (uint32_t)g) * kHalf, 16, 1024);
         const uint64_t k_desc = sw128_desc(sK + 2u * (uint32_t)s * kHalf, 16, 1024);
+        const uint32_t d_s = tmem + kColS + 128u * (uint32_t)g;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t off = (uint64_t)(((kk >> 2) * kHalf + (kk & 3) * 32) >> 4);
           tc_mma(d_s, q_desc + off, k_desc + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
         tc_commit(bar(kBarSFull + g));
-        tc_commit(bar(kBarKEmpty + s));
+        if (dual) tc_commit(bar(kBarKEmpty + s));
+        return true;
+      };
+      // O_g += P_g(j) V_j once the softmax has published P_g(j)
+      auto pv = [&](int g, int j) {
+        const int s = kv_stage(g, j);
+        if (!bar_wait(bar(kBarVFull + s), kv_par(j), abort_addr, a.dev_status, wlim, kSusp)) return false;
+        if (!bar_wait(bar(kBarPFull + g), (uint32_t)j & 1u, abort_addr, a.dev_status, wlim, kSusp)) return false;
+        tc_fence_after();
+        // V tile as B = [keys x dims], dims contiguous: 64-dim atoms one half
+        // apart (LBO), 8-key groups 1 KB apart (SBO); 16 keys (2 KB) per step;
+        // P_g from TMEM: keys 16kk..16kk+15 are columns 8kk..8kk+7 of S_g
+        const uint64_t v_desc = sw128_desc(sV + 2u * (uint32_t)s * kHalf, kHalf, 1024);
+        const uint32_t d_s = tmem + kColS + 128u * (uint32_t)g;
+        const uint32_t d_o = tmem + kColO + 128u * (uint32_t)g;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc_mma_ts(d_o, d_s + 8u * kk, v_desc + (uint64_t)(kk * 2048 / 16), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        if (dual) tc_commit(bar(kBarVEmpty + s));
+        return true;
+      };
+      for (int j = 0; j <= n_iter && ok; ++j) {
+        if (j < n_iter) {
+          if (!dual && !bar_wait(bar(kBarKFull + (j & 1)), (uint32_t)(j >> 1) & 1u, abort_addr, a.dev_status, wlim,
+                                 kSusp))
+            break;
+          if (active(0, j) && !qk(0, j)) break;
+        }
+        if (j > 0) {
+          if (active(1, j - 1) && !pv(1, j - 1)) break;
+          if (!dual) tc_commit(bar(kBarVEmpty + ((j - 1) & 1)));  // both PVs of tile j-1 issued
+        }
+        if (j < n_iter) {
+          if (active(1, j) && !qk(1, j)) break;
+          if (!dual) tc_commit(bar(kBarKEmpty + (j & 1)));  // both QKs of tile j issued
+          if (active(0, j) && !pv(0, j)) break;
+        }
       }
-      if (ok && nt > 0) pv(nt - 1);
-      // (Q tile 0 may stop one key tile short of the shared stream's last
-      // tile; nothing waits for that stage to be released again)
-      tc_commit(bar(kBarMmaDone + g));
-      // every MMA this thread issued has finished once this completes; wait
-      // for it even after an abort (bounded), so TMEM and shared memory stay
-      // in use until the tensor cores are done with them
-      bar_wait_all(bar(kBarMmaDone + g), 0, wlim);
+      tc_commit(bar(kBarMmaDone));
+      tc_commit(bar(kBarMmaDone + 1));
+      // every MMA issued above has finished once this completes; wait for it
+      // even after an abort (bounded), so TMEM and shared memory stay in use
+      // until the tensor cores are done with them
+      bar_wait_all(bar(kBarMmaDone), 0, wlim);
     }
   } else {
     // ================================================================ softmax / epilogue
@@ -487,25 +570,36 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       // mask (raw scores; the scale is folded into the exponent below)
       const int kbase = jt * kBN;
       const bool need_mask = kbase + kBN - 1 > lim || (kbase < lo_vis && kbase + kBN - 1 >= a.n_sink);
-      auto mask_chunk = [&](int c2) {
+      auto mask_regs = [&](uint32_t (&r)[32], int c2) {
         if (need_mask) {
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
             const int k = kbase + 32 * c2 + c;
-            if (k > lim || (k < lo_vis && k >= a.n_sink)) sr[c2][c] = __float_as_uint(-INFINITY);
+            if (k > lim || (k < lo_vis && k >= a.n_sink)) r[c] = __float_as_uint(-INFINITY);
           }
         }
       };
+      auto mask_chunk = [&](int c2) { mask_regs(sr[c2], c2); };
       // row max over eight independent accumulators
       float mx8[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
-      auto max_chunk = [&](int c2) {
+      auto max_regs = [&](const uint32_t (&r)[32]) {
+#if KVATTN_PREFILL_MAX3
+        // three-input max: half the instructions of a pairwise reduction
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          mx8[k] = fmax3(mx8[k], __uint_as_float(r[k]), __uint_as_float(r[k + 8]));
+          mx8[k] = fmax3(mx8[k], __uint_as_float(r[k + 16]), __uint_as_float(r[k + 24]));
+        }
+#else
 #pragma unroll
         for (int c = 0; c < 32; c += 8)
 #pragma unroll
-          for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], __uint_as_float(sr[c2][c + k]));
+          for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], __uint_as_float(r[c + k]));
+#endif
       };
+      auto max_chunk = [&](int c2) { max_regs(sr[c2]); };
       auto row_max = [&]() {
         return fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                      fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) *
@@ -515,20 +609,31 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       // packed sums in four accumulators; 32 keys (16 P columns) at a time,
       // written over the S columns already read
       uint64_t sum2[4] = {0ull, 0ull, 0ull, 0ull};
-      auto exp_chunk = [&](int c2, uint64_t nr2) {
+      auto exp_regs = [&](const uint32_t (&r)[32], int c2, uint64_t nr2) {
         uint32_t pk[16];
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
-          const uint64_t sv = ((uint64_t)sr[c2][c + 1] << 32) | sr[c2][c];
+          const uint64_t sv = ((uint64_t)r[c + 1] << 32) | r[c];
           float x0, x1;
           f2_unpack(f2_fma(sv, sc2, nr2), x0, x1);
-          const float p0 = fast_exp2(x0);
-          const float p1 = fast_exp2(x1);
+          float p0, p1;
+          if (((c >> 1) & 3) < 4 - KVATTN_PREFILL_POLY_PAIRS) {
+            p0 = fast_exp2(x0);
+            p1 = fast_exp2(x1);
+          } else {
+            // this pair on the FMA pipes (masked scores are -inf: 2^-inf = 0)
+            exp2_poly_x2(x0, x1, p0, p1);
+            if (need_mask) {
+              p0 = x0 == -INFINITY ? 0.f : p0;
+              p1 = x1 == -INFINITY ? 0.f : p1;
+            }
+          }
           sum2[(c >> 1) & 3] = f2_add(sum2[(c >> 1) & 3], f2_pack(p0, p1));
-          pk[c >> 1] = pack_bf16x2_rn(p0, p1);
+          pk[c >> 1] = pack_bf16x2_p(p0, p1);
         }
         tmem_st16(lane_addr + col_s + 16u * c2, pk);
       };
+      auto exp_chunk = [&](int c2, uint64_t nr2) { exp_regs(sr[c2], c2, nr2); };
       auto neg_ref2 = [&]() {
         const float nr = (ref == -INFINITY) ? 0.f : -ref;
         return f2_pack(nr, nr);
@@ -568,6 +673,40 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
       } else
 #endif
+#if KVATTN_PREFILL_TWO_PASS
+      {
+        // Two passes over TMEM, 32 columns at a time with the next chunk's
+        // load in flight: the row max, then the exponentials from a second
+        // load of each chunk (a TMEM reload is cheaper than keeping the whole
+        // 128-column row in registers).  P chunk c2 goes to columns
+        // 16c2 .. 16c2+15, which the second pass has already read.
+        uint32_t cb[2][32];
+        tmem_ld32(lane_addr + col_s, cb[0]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c2 = 0; c2 < 4; ++c2) {
+          if (c2 < 3) tmem_ld32(lane_addr + col_s + 32u * (c2 + 1), cb[(c2 + 1) & 1]);
+          mask_regs(cb[c2 & 1], c2);
+          max_regs(cb[c2 & 1]);
+          if (c2 < 3) tmem_wait_ld();
+        }
+        const float mx = row_max();
+        move = mx > ref + 8.f;
+        const float ref_new = move ? mx : ref;
+        alpha = move ? fast_exp2(ref - ref_new) : 1.f;
+        ref = ref_new;
+        const uint64_t nr2 = neg_ref2();
+        tmem_ld32(lane_addr + col_s, cb[0]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c2 = 0; c2 < 4; ++c2) {
+          if (c2 < 3) tmem_ld32(lane_addr + col_s + 32u * (c2 + 1), cb[(c2 + 1) & 1]);
+          mask_regs(cb[c2 & 1], c2);
+          exp_regs(cb[c2 & 1], c2, nr2);
+          if (c2 < 3) tmem_wait_ld();
+        }
+      }
+#else
       {
         // (first tile of the row, or the plain order) load the row, take its
         // max, then exponentiate
@@ -588,6 +727,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll
         for (int c2 = 0; c2 < 4; ++c2) exp_chunk(c2, nr2);
       }
+#endif
       float sa, sb;
       f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), sa, sb);
       l = l * alpha + (sa + sb);
