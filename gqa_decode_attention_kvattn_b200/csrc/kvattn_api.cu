@@ -282,10 +282,11 @@ int run_attention(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, con
   if (dims->n_heads == 32 * dims->n_kv_heads && T == 1 && !masked && plan.mma && plan.max_splits > 1 &&
       plan.ws_bytes > 0) {
     const int tiles_per_seq = (hint + 127) / 128;
-    // about eight CTAs per SM over the call's key tiles (measured: 2, 4, 8,
-    // 12, 16, 24 per SM on a 64-sequence multi-query call; 8 is fastest), at
-    // least four tiles each, and no more splits per sequence than the
-    // workspace has slots for
+    // splits sized for about eight per SM over the call's key tiles (each CTA
+    // takes two), at least four tiles each, and no more splits per sequence
+    // than the workspace has slots for.  Measured on a 64-sequence
+    // multi-query call (4k-32k rows) with two splits per CTA: 4, 8, 16, 32
+    // per SM gave 168.9, 151.6, 156.7, 178.4 us
     constexpr long long kCtasPerSm = 8;
     const long long tiles = (long long)dims->batch * dims->n_kv_heads * tiles_per_seq;
     long long st = std::max<long long>(4, (tiles + kCtasPerSm * sms - 1) / (kCtasPerSm * sms));

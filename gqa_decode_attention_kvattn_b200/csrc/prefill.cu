@@ -437,10 +437,17 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         st_shared_i32(abort_addr, 1);
         set_status(a.dev_status, KVATTN_DEV_WAIT_TIMEOUT);
       } else {
-        bar_expect_tx(bar(kBarQFull), (uint32_t)n_q * 2u * kHalf);
-        for (int g = 0; g < n_q; ++g) {
-          tma_load_4d_raw(sQ + (2 * g) * kHalf, &tmap_q, bar(kBarQFull), 0, kvh * G, t0 + g * TT, b);
-          tma_load_4d_raw(sQ + (2 * g + 1) * kHalf, &tmap_q, bar(kBarQFull), 64, kvh * G, t0 + g * TT, b);
+        // Q tile g: tokens t0 + g*TT ..; in split mode both Q tiles hold the
+        // one token, tile 1 loaded from token coordinate -1 so that its rows
+        // sit 32 TMEM lanes lower (rows of token -1 and of tokens past T are
+        // the copy's zero fill): the two splits' softmax rows then belong to
+        // warps on different SM sub-partitions
+        const int n_slots = dual ? 2 : n_q;
+        bar_expect_tx(bar(kBarQFull), (uint32_t)n_slots * 2u * kHalf);
+        for (int g = 0; g < n_slots; ++g) {
+          const int tq0 = dual ? t0 - g : t0 + g * TT;
+          tma_load_4d_raw(sQ + (2 * g) * kHalf, &tmap_q, bar(kBarQFull), 0, kvh * G, tq0, b);
+          tma_load_4d_raw(sQ + (2 * g + 1) * kHalf, &tmap_q, bar(kBarQFull), 64, kvh * G, tq0, b);
         }
       }
       for (int j = 0; j < n_iter && go; ++j) {
@@ -476,8 +483,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     // 64.  Two issuing threads, one per Q tile, reach the tensor core's rate
     // but drift into lockstep: both softmaxes then share the exponential unit
     // and the tensor cores idle meanwhile, which measured slower.)
-    // In split mode both Q tiles read Q slot 0, the one token's heads, and K/V
-    // tile j of Q tile g's own stream, released per stream.
+    // In split mode Q tile g reads Q slot g (the one token's heads, 32g rows
+    // down in slot 1) and K/V tile j of its own stream, released per stream.
     if (lane == 0) {
       constexpr bool kSusp = KVATTN_PREFILL_ISSUER_SUSPEND || !KVATTN_PREFILL_SPIN_ALL;
       constexpr uint32_t idesc_qk = idesc_bf16_m128_n128(false);
@@ -489,7 +496,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const int s = kv_stage(g, j);
         if (dual && !bar_wait(bar(kBarKFull + s), kv_par(j), abort_addr, a.dev_status, wlim, kSusp)) return false;
         tc_fence_after();
-        const uint64_t q_desc = sw128_desc(sQ + (dual ? 0u : 2u * (uint32_t)g) * kHalf, 16, 1024);
+        const uint64_t q_desc = sw128_desc(sQ + 2u * (uint32_t)g * kHalf, 16, 1024);
         const uint64_t k_desc = sw128_desc(sK + 2u * (uint32_t)s * kHalf, 16, 1024);
         const uint32_t d_s = tmem + kColS + 128u * (uint32_t)g;
 #pragma unroll
@@ -548,7 +555,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int quarter = warp & 3;         // TMEM lanes 32*quarter .. +31
     const int grp = (warp - 2) >> 2;      // Q tile of this warp
     const int m = 32 * quarter + lane;    // query row of this thread within its Q tile
-    const int tok = t0 + (dual ? 0 : grp * TT) + m / G;  // split mode: both Q tiles are one token
+    // token of this row (split mode: the one token, 32 rows down in Q tile 1)
+    const int tok = t0 + (dual ? m / G - grp : grp * TT + m / G);
     const int head = kvh * G + (m % G);
     const int lim = sp + min(tok, a.T - 1);  // last visible key (rows past T borrow the last token's)
     // with a window: keys n_sink <= k < lo_vis are hidden as well
@@ -560,11 +568,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2);
     float ref = -INFINITY;   // reference max (log2 units) of the row
     float l = 0.f;           // row sum in units of 2^ref
+    // a warp whose 32 rows are all padding (tokens before 0 or past T) only
+    // keeps the barriers moving; its rows of P and O are never stored
+    const bool idle = __all_sync(0xffffffffu, tok < 0 || tok >= a.T);
 
     for (int j = 0; active(grp, j); ++j) {
       const int jt = key_tile(grp, j);
       if (!bar_wait(bar(kBarSFull + grp), (uint32_t)j & 1u, abort_addr, a.dev_status, wlim)) break;
       tc_fence_after();
+      if (!idle) {
       // the thread's whole S row, 32 columns (one TMEM load) at a time
       uint32_t sr[4][32];
       // mask (raw scores; the scale is folded into the exponent below)
@@ -745,6 +757,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           tmem_st32(lane_addr + col_o + 32u * c2, r);
         }
       }
+      }  // !idle
       if (first_tile(grp) + j == n_all - 1 && Lmax < jt * kBN + kBN) {
         // rows of the last V tile past the last visible key may hold any bits;
         // zero them so that 0 * (garbage) cannot reach O.  On the shared
@@ -781,7 +794,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       const float f = (ref == -INFINITY) ? 0.f : fast_exp2(ref - mn);
       inv_l = f / (l * f + fast_exp2(s2 - mn));
     }
-    const bool store = (dual ? active(grp, 0) : grp < n_q) && tok < a.T;
+    const bool store = (dual ? active(grp, 0) : grp < n_q) && tok >= 0 && tok < a.T;
     if (a.split_tiles > 0 && n_splits_here > 1) {
       // this split's partial: unnormalised O and (max, sum), both relative
       // to 2^ref (a group without key tiles here contributes nothing)
