@@ -69,39 +69,83 @@ __global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(RopeAppendArg
                    : a.cache_k + (((size_t)b * a.S + pos) * a.Hkv + (v - a.H)) * kHeadDim;
   };
 
+  // Each thread loads a batch of its words before it stores any: q_rot may be
+  // q itself, so the compiler cannot move a load above an earlier store, and
+  // one word at a time would pay a full memory latency per word.  Every word
+  // is read and written by the same thread, so rotating in place is safe.
+  constexpr int kBatch = 8;
+  const int n_slots = nv * kPairs;
   if (tab.layout == 0 && rp == kPairs) {
     // Meta layout over the whole head: each pair is one 32-bit word
-    for (int idx = threadIdx.x; idx < nv * kPairs; idx += blockDim.x) {
-      const int v = v0 + idx / kPairs;
-      const int i = idx & (kPairs - 1);
-      const uint32_t w = reinterpret_cast<const uint32_t*>(vec_in(v))[i];
-      uint16_t y0, y1;
-      rope_rotate_bits(true, s_cos[i], s_sin[i], (uint16_t)(w & 0xFFFFu), (uint16_t)(w >> 16), y0, y1);
-      reinterpret_cast<uint32_t*>(vec_out(v))[i] = (uint32_t)y0 | ((uint32_t)y1 << 16);
+    for (int base_idx = threadIdx.x; base_idx < n_slots; base_idx += blockDim.x * kBatch) {
+      uint32_t w[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int idx = base_idx + u * blockDim.x;
+        w[u] = idx < n_slots ? reinterpret_cast<const uint32_t*>(vec_in(v0 + idx / kPairs))[idx & (kPairs - 1)] : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int idx = base_idx + u * blockDim.x;
+        if (idx < n_slots) {
+          const int i = idx & (kPairs - 1);
+          uint16_t y0, y1;
+          rope_rotate_bits(true, s_cos[i], s_sin[i], (uint16_t)(w[u] & 0xFFFFu), (uint16_t)(w[u] >> 16), y0, y1);
+          reinterpret_cast<uint32_t*>(vec_out(v0 + idx / kPairs))[i] = (uint32_t)y0 | ((uint32_t)y1 << 16);
+        }
+      }
     }
   } else {
     // any layout / rotary width, one slot (pair or pass-through pair) at a time
-    for (int idx = threadIdx.x; idx < nv * kPairs; idx += blockDim.x) {
-      const int v = v0 + idx / kPairs;
-      const int j = idx & (kPairs - 1);
-      const uint16_t* in = vec_in(v);
-      uint16_t* outp = vec_out(v);
-      const RopeSlot sl = rope_slot(tab, j);
-      uint16_t ya, yb;
-      rope_rotate_bits(sl.rotate, sl.rotate ? s_cos[j] : 1.0, sl.rotate ? s_sin[j] : 0.0, in[sl.ea], in[sl.eb], ya,
-                       yb);
-      outp[sl.ea] = ya;
-      outp[sl.eb] = yb;
+    for (int base_idx = threadIdx.x; base_idx < n_slots; base_idx += blockDim.x * kBatch) {
+      uint16_t xa[kBatch], xb[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int idx = base_idx + u * blockDim.x;
+        xa[u] = xb[u] = 0;
+        if (idx < n_slots) {
+          const uint16_t* in = vec_in(v0 + idx / kPairs);
+          const RopeSlot sl = rope_slot(tab, idx & (kPairs - 1));
+          xa[u] = in[sl.ea];
+          xb[u] = in[sl.eb];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int idx = base_idx + u * blockDim.x;
+        if (idx < n_slots) {
+          const int j = idx & (kPairs - 1);
+          uint16_t* outp = vec_out(v0 + idx / kPairs);
+          const RopeSlot sl = rope_slot(tab, j);
+          uint16_t ya, yb;
+          rope_rotate_bits(sl.rotate, sl.rotate ? s_cos[j] : 1.0, sl.rotate ? s_sin[j] : 0.0, xa[u], xb[u], ya, yb);
+          outp[sl.ea] = ya;
+          outp[sl.eb] = yb;
+        }
+      }
     }
   }
 
-  // values: bit copy of the 256-byte rows of this CTA's key heads
+  // values: bit copy of the 256-byte rows of this CTA's key heads (a batch of
+  // 16-byte loads before the stores, as above)
   const int k0 = max(v0, a.H) - a.H;       // first key head of this CTA
   const int k1 = max(v0 + nv, a.H) - a.H;  // one past the last
   const uint4* v_in = reinterpret_cast<const uint4*>(a.v_new) + (size_t)bt * a.Hkv * (kHeadDim / 8);
   uint4* v_out = reinterpret_cast<uint4*>(a.cache_v) + ((size_t)b * a.S + pos) * a.Hkv * (kHeadDim / 8);
-  for (int idx = k0 * (kHeadDim / 8) + threadIdx.x; idx < k1 * (kHeadDim / 8); idx += blockDim.x)
-    v_out[idx] = v_in[idx];
+  const int c_end = k1 * (kHeadDim / 8);
+  for (int base_idx = k0 * (kHeadDim / 8) + threadIdx.x; base_idx < c_end; base_idx += blockDim.x * 4) {
+    uint4 t[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int idx = base_idx + u * blockDim.x;
+      if (idx < c_end) t[u] = v_in[idx];
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int idx = base_idx + u * blockDim.x;
+      if (idx < c_end) v_out[idx] = t[u];
+    }
+  }
 }
 
 }  // namespace
