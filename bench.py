@@ -59,10 +59,10 @@ def measured_peaks():
 KERNEL_SOURCES = {
     "decode_splitk": ("decode.cu", "kvattn_device.cuh"),
     "decode_mma": ("decode.cu", "kvattn_device.cuh"),
-    # multi-query decode (G = 32): the tcgen05 kernel in split mode + the LSE merge
-    "decode_tc": ("prefill.cu", "decode.cu", "kvattn_device.cuh"),
+    # multi-query decode (G = 32): the tcgen05 multi-query kernel + the LSE merge
+    "decode_tc": ("mqa_decode.cu", "tc_device.cuh", "decode.cu", "kvattn_device.cuh"),
     "decode_fused": ("decode.cu", "kvattn_device.cuh", "rope_device.cuh"),
-    "prefill_chunk": ("prefill.cu", "kvattn_device.cuh"),
+    "prefill_chunk": ("prefill.cu", "tc_device.cuh", "kvattn_device.cuh"),
 }
 
 
@@ -402,7 +402,7 @@ def kernel_tag(w, st):
     if st["fused"]:
         return "decode_fused", "kvattn_decode_fused (rope + append + split-K attention + LSE merge, one kernel)"
     if w.H == 32 * w.Hkv:
-        return "decode_tc", "kvattn_decode (tcgen05 split kernel + LSE merge kernel)"
+        return "decode_tc", "kvattn_decode (tcgen05 multi-query kernel + LSE merge kernel)"
     plan = kv.kvattn_decode_plan(w.B, w.H, w.Hkv, w.S, w.kv_len_hint)
     if plan["tensor_cores"]:
         return "decode_mma", "kvattn_decode (warp-MMA split-K kernel + LSE merge kernel)"

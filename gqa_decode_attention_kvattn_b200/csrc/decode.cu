@@ -869,8 +869,15 @@ __global__ void __launch_bounds__(kHeadDim) decode_merge_kernel(const DecodeArgs
   const int v = blockIdx.x;     // row set (up to 2^24 of them: the grid's x extent)
   const int head = blockIdx.y;  // query head (at most 65535: the y extent)
   const int L = set_length<true>(a, v);
-  const int ns = (L + a.rows_per_split - 1) / a.rows_per_split;
-  if (L == 0 || (ns <= 1 && !a.sink_logits)) return;  // invalid, or written directly by K2
+  if (L == 0) return;  // invalid row set
+  int ns;
+  if (a.unit_splits) {
+    // the multi-query tcgen05 decode: every unit's pieces are partials
+    ns = __ldcg(a.unit_splits + (size_t)v * a.Hkv_phys + head / (a.H / a.Hkv_phys));
+  } else {
+    ns = (L + a.rows_per_split - 1) / a.rows_per_split;
+    if (ns <= 1 && !a.sink_logits) return;  // written directly by K2
+  }
   const int b = v / a.Tq, t = v - b * a.Tq;
   const int c = threadIdx.x;
   const float r = lse_merge_element(a, v, head, ns, c);
@@ -1367,22 +1374,24 @@ DecodePlan plan_decode(int B, int Tq, int H, int Hkv, int kv_len_hint, int sm_co
   const long long items_bound = row_sets * Hkv * p.max_splits;
   p.grid = (int)std::min<long long>(items_bound, slots);
   if (p.grid < 1) p.grid = 1;
-  // partial (o, max, sum) per (row set, split, head), then the work counter
-  p.ws_bytes = (p.max_splits > 1 || always_partials)
-                   ? 16 + (size_t)row_sets * p.max_splits * H * (kHeadDim + 2) * sizeof(float)
-                   : 0;
-  // fused: the same plus one merge counter per (row set, KV-head group),
-  // padded to 16 bytes (see bind_decode_workspace)
-  p.fused_ws_bytes = p.max_splits > 1 ? p.ws_bytes + (((size_t)row_sets * Hkv * sizeof(int) + 15) & ~(size_t)15) : 0;
+  // the work counter's 16-byte header, one int per (row set, KV-head group)
+  // padded to 16 bytes (see bind_decode_workspace), then the partial (o, max,
+  // sum) per (row set, split, head)
+  const size_t bytes = 16 + (((size_t)row_sets * Hkv * sizeof(int) + 15) & ~(size_t)15) +
+                       (size_t)row_sets * p.max_splits * H * (kHeadDim + 2) * sizeof(float);
+  p.ws_bytes = (p.max_splits > 1 || always_partials) ? bytes : 0;
+  p.fused_ws_bytes = p.max_splits > 1 ? bytes : 0;
   return p;
 }
 
 // Workspace layout: a 16-byte header (work counter; exit counter of the fused
-// decode), the fused decode's merge counters (one per row set and KV-head
-// group, padded to 16 bytes), then the partial o [row sets, splits, H, d] and
-// (max, sum) [row sets, splits, H, 2].  The counters sit at fixed offsets, so
-// calls of any shape can share one workspace; every completed call leaves them
-// zero, and they must be zero before the first call.
+// decode), one int per row set and KV-head group padded to 16 bytes (the
+// fused decode's merge counters; the multi-query tcgen05 decode's slot counts
+// per unit, written before they are read), then the partial o [row sets,
+// splits, H, d] and (max, sum) [row sets, splits, H, 2].  The counters sit at
+// fixed offsets, so calls of any shape can share one workspace; every
+// completed call leaves them zero, and they must be zero before the first
+// call.
 void bind_decode_workspace(DecodeArgs& a, const DecodePlan& plan, void* workspace, bool fused) {
   a.exit_counter = nullptr;
   a.merge_counter = nullptr;
@@ -1399,8 +1408,8 @@ void bind_decode_workspace(DecodeArgs& a, const DecodePlan& plan, void* workspac
   if (fused) {
     a.exit_counter = a.counter + 1;
     a.merge_counter = reinterpret_cast<int*>(base + off);
-    off += ((size_t)a.B * a.Tq * a.Hkv * sizeof(int) + 15) & ~(size_t)15;
   }
+  off += ((size_t)a.B * a.Tq * a.Hkv * sizeof(int) + 15) & ~(size_t)15;
   a.ws_o = reinterpret_cast<float*>(base + off);
   a.ws_ml = a.ws_o + n_slots * kHeadDim;
 }

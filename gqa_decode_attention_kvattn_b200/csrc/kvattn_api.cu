@@ -43,6 +43,11 @@ void apply_wait_policy(PrefillArgs& a) {
   a.gate = g_gate.load(std::memory_order_relaxed);
 }
 
+void apply_wait_policy(MqaDecodeArgs& a) {
+  a.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
+  a.gate = g_gate.load(std::memory_order_relaxed);
+}
+
 int set_wait_policy(uint64_t limit_ns, const int32_t* gate) {
   if (reinterpret_cast<uintptr_t>(gate) & 3u) return KVATTN_ERR_INVALID_ARG;
   g_wait_ns.store(limit_ns, std::memory_order_relaxed);
@@ -274,53 +279,46 @@ int run_attention(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, con
   kvattn::apply_wait_policy(a);
 
   // One new token per sequence with all 32 query heads on one KV head (G = 32,
-  // multi-query): the 32 heads fill one 128-row tcgen05 M tile, so the
-  // tensor-core prefill kernel in split mode runs the contraction (the warp
-  // MMAs of the decode kernels top out near 100 TFLOP/s, a third of what
-  // this shape needs at HBM speed), then the same LSE merge.
+  // multi-query): the 32 heads are 32 rows of a 128-row tcgen05 M tile (the
+  // warp MMAs of the decode kernels top out near 100 TFLOP/s, a third of what
+  // this shape needs at HBM speed).  The multi-query kernel cuts the call's
+  // key tiles evenly over one CTA per SM, then the same LSE merge combines
+  // the pieces.
   const bool masked = mask && (mask->window > 0 || mask->sink_logits);
+  const long long units = (long long)dims->batch * dims->n_kv_heads;
+  const long long tiles_per_unit = (hint + 127) / 128;
   if (dims->n_heads == 32 * dims->n_kv_heads && T == 1 && !masked && plan.mma && plan.max_splits > 1 &&
-      plan.ws_bytes > 0) {
-    const int tiles_per_seq = (hint + 127) / 128;
-    // splits sized for about eight per SM over the call's key tiles (each CTA
-    // takes two), at least four tiles each, and no more splits per sequence
-    // than the workspace has slots for.  Measured on a 64-sequence
-    // multi-query call (4k-32k rows) with two splits per CTA: 4, 8, 16, 32
-    // per SM gave 168.9, 151.6, 156.7, 178.4 us
-    constexpr long long kCtasPerSm = 8;
-    const long long tiles = (long long)dims->batch * dims->n_kv_heads * tiles_per_seq;
-    long long st = std::max<long long>(4, (tiles + kCtasPerSm * sms - 1) / (kCtasPerSm * sms));
-    st = std::max<long long>(st, (tiles_per_seq + plan.max_splits - 1) / plan.max_splits);
-    const int split_tiles = (int)std::min<long long>(st, tiles_per_seq);
-    const int split_grid = (tiles_per_seq + split_tiles - 1) / split_tiles;
+      plan.ws_bytes > 0 && units <= (1 << 16) && units * tiles_per_unit < (1ll << 30)) {
     CUtensorMap tq, tk2, tv2;
-    rc = encode_sw128_map(&tq, q_rot, dims->batch, 1, dims->n_heads, 32, kvattn::prefill_tokens_per_tile(32));
+    // Q boxes: one token's 32 heads (32 rows of 128 bytes per 64-element half)
+    rc = encode_sw128_map(&tq, q_rot, dims->batch, 1, dims->n_heads, 32, 1);
     if (rc != KVATTN_OK) return rc;
     rc = encode_sw128_map(&tk2, cache_k, dims->batch, dims->max_seq_len, dims->n_kv_heads, 1, 128);
     if (rc != KVATTN_OK) return rc;
     rc = encode_sw128_map(&tv2, cache_v, dims->batch, dims->max_seq_len, dims->n_kv_heads, 1, 128);
     if (rc != KVATTN_OK) return rc;
-    kvattn::PrefillArgs p{};
-    p.B = dims->batch;
-    p.T = 1;
-    p.H = dims->n_heads;
-    p.Hkv = dims->n_kv_heads;
-    p.S = dims->max_seq_len;
-    p.kv_len_hint = hint;
-    p.n_mtiles = 1;
-    p.scale_log2 = a.scale_log2;
-    p.start_pos = start_pos;
-    p.out = out;
-    p.dev_status = dev_status;
-    p.split_tiles = split_tiles;
-    p.split_grid = split_grid;
-    p.part_splits = plan.max_splits;
-    p.part_o = a.ws_o;
-    p.part_ml = a.ws_ml;
-    kvattn::apply_wait_policy(p);
-    a.rows_per_split = split_tiles * 128;
-    const cudaError_t e = kvattn::launch_prefill(p, tq, tk2, tv2, (cudaStream_t)stream);
+    kvattn::MqaDecodeArgs m{};
+    m.B = dims->batch;
+    m.H = dims->n_heads;
+    m.Hkv = dims->n_kv_heads;
+    m.S = dims->max_seq_len;
+    m.kv_len_hint = hint;
+    m.part_splits = plan.max_splits;
+    // a unit of up to tiles_per_unit tiles spans at most
+    // ceil(tiles_per_unit / range) + 1 ranges: keep that within its slots
+    m.min_tiles = (int)std::max<long long>(1, (tiles_per_unit + plan.max_splits - 2) / (plan.max_splits - 1));
+    m.scale_log2 = a.scale_log2;
+    m.start_pos = start_pos;
+    m.part_o = a.ws_o;
+    m.part_ml = a.ws_ml;
+    // the per-unit slot counts sit where the fused decode keeps its merge counters
+    m.unit_splits = reinterpret_cast<int*>(static_cast<unsigned char*>(workspace) + 16);
+    m.dev_status = dev_status;
+    kvattn::apply_wait_policy(m);
+    const int grid = (int)std::min<long long>(sms, (units * tiles_per_unit + 1) / 2);
+    const cudaError_t e = kvattn::launch_mqa_decode(m, tq, tk2, tv2, grid, (cudaStream_t)stream);
     if (e != cudaSuccess) return kvattn::launch_status(e);
+    a.unit_splits = m.unit_splits;
     return kvattn::launch_status(kvattn::launch_decode_merge(a, (cudaStream_t)stream));
   }
   return kvattn::launch_status(kvattn::launch_decode(a, tk, tv, (cudaStream_t)stream));

@@ -86,6 +86,10 @@ struct DecodeArgs {
   uint16_t* q_rot_out;    // [B, 1, H, d] or null
   int* exit_counter;      // CTAs that finished (counter reset by the last)
   int* merge_counter;     // [B, Hkv] splits finished per row set and KV head
+  // multi-query decode on tcgen05 (Tq = 1): partial slots written per
+  // (sequence, KV head) of the caches, read by the merge instead of
+  // ceil(length / rows_per_split); null otherwise
+  const int* unit_splits;
   // optional masks: window > 0 shows a token at position p the rows
   // p - window < r <= p and the first n_sink rows; sink_logits (fp32 [H],
   // score units, or null) adds e^{sink} to each head's softmax denominator
@@ -172,10 +176,38 @@ struct PrefillArgs {
   const int32_t* gate;  // diagnostics gate (null: none)
 };
 
+// Multi-query decode (32 query heads per KV head, one new token) on tcgen05,
+// one CTA per SM: the key tiles of all (sequence, KV head) units, laid end to
+// end, are cut into 2 * grid equal contiguous ranges, two per CTA; each piece
+// of a unit that a range covers leaves one partial (unnormalised O and (max in
+// log2 units, sum)) in part_o [B, part_splits, H, d] / part_ml [.., 2], the
+// layout the decode's LSE merge reads, and unit_splits [B * Hkv] receives each
+// unit's slot count.  A unit spans at most ceil(tiles / range) + 1 ranges, so
+// ranges of at least min_tiles tiles, with
+// min_tiles >= ceil(ceil(kv_len_hint / 128) / (part_splits - 1)), fit its slots.
+struct MqaDecodeArgs {
+  int B, H, Hkv, S;
+  int kv_len_hint;  // upper bound on start_pos[b] + 1
+  int part_splits;  // partial slots per unit (>= 2)
+  int min_tiles;    // shortest range, in 128-row key tiles (>= 1)
+  float scale_log2; // softmax scale * log2(e)
+  const int32_t* start_pos;
+  float* part_o;
+  float* part_ml;
+  int* unit_splits;
+  int32_t* dev_status;
+  uint64_t wait_ns;     // limit of each in-kernel wait (0: one second)
+  const int32_t* gate;  // diagnostics gate (null: none)
+};
+
+cudaError_t launch_mqa_decode(const MqaDecodeArgs& a, const CUtensorMap& tmap_q, const CUtensorMap& tmap_k,
+                              const CUtensorMap& tmap_v, int grid, cudaStream_t stream);
+
 // The process's wait policy (kvattn_set_wait_policy) copied into launch
 // arguments.
 void apply_wait_policy(DecodeArgs& a);
 void apply_wait_policy(PrefillArgs& a);
+void apply_wait_policy(MqaDecodeArgs& a);
 int set_wait_policy(uint64_t limit_ns, const int32_t* gate);
 
 // Tokens per 128-row M tile for group size G (128 / G).

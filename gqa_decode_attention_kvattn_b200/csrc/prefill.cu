@@ -40,6 +40,7 @@
 // works on Q tile (w-2)/4.
 #include "kvattn_device.cuh"
 #include "kvattn_internal.h"
+#include "tc_device.cuh"
 
 #include <algorithm>
 
@@ -77,16 +78,6 @@ constexpr uint32_t kOffAbort = kOffTmemSlot + 8;
 constexpr uint32_t kPrefillSmemBytes = kOffAbort + 8 + 1024;  // + alignment slack
 static_assert(kPrefillSmemBytes <= 227 * 1024, "shared memory per CTA");
 
-// ------------------------------------------------------------ raw smem helpers
-__device__ __forceinline__ void bar_init(uint32_t a, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(a), "r"(count) : "memory");
-}
-__device__ __forceinline__ void bar_arrive(uint32_t a) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(a) : "memory");
-}
-__device__ __forceinline__ void bar_expect_tx(uint32_t a, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(a), "r"(bytes) : "memory");
-}
 #ifndef KVATTN_PREFILL_SPIN_ALL
 #define KVATTN_PREFILL_SPIN_ALL 1
 #endif
@@ -104,10 +95,6 @@ __device__ __forceinline__ void bar_expect_tx(uint32_t a, uint32_t bytes) {
 #ifndef KVATTN_PREFILL_POLY_PAIRS
 #define KVATTN_PREFILL_POLY_PAIRS 1
 #endif
-// P to bf16 on the integer pipes (1) or with the conversion instruction (0)
-#ifndef KVATTN_PREFILL_INT_PACK
-#define KVATTN_PREFILL_INT_PACK 1
-#endif
 // softmax reads each S chunk twice from TMEM (max, then exponentials) instead
 // of holding the 128-column row in registers
 #ifndef KVATTN_PREFILL_TWO_PASS
@@ -117,206 +104,6 @@ __device__ __forceinline__ void bar_expect_tx(uint32_t a, uint32_t bytes) {
 #ifndef KVATTN_PREFILL_MAX3
 #define KVATTN_PREFILL_MAX3 1
 #endif
-// One try of a phase wait.  With `suspend` the thread sleeps in hardware
-// until the phase completes (or ~1 ms passes); without it the call returns at
-// once and the caller spins, which wakes sooner but costs issue slots.
-__device__ __forceinline__ bool bar_try_wait(uint32_t a, uint32_t parity, bool suspend) {
-  uint32_t ok;
-  if (suspend) {
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(a), "r"(parity), "r"(1u << 20)
-        : "memory");
-  } else {
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(a), "r"(parity)
-        : "memory");
-  }
-  return ok != 0;
-}
-__device__ __forceinline__ int ld_shared_i32(uint32_t a) {
-  int v;
-  asm volatile("ld.volatile.shared.b32 %0, [%1];" : "=r"(v) : "r"(a));
-  return v;
-}
-__device__ __forceinline__ void st_shared_i32(uint32_t a, int v) {
-  asm volatile("st.volatile.shared.b32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
-}
-// Bounded wait (see kWaitLimitNs); gives up at once when the CTA's abort flag
-// is set, and sets it (plus the status bit) when it gives up itself.
-__device__ __forceinline__ bool bar_wait(uint32_t a, uint32_t parity, uint32_t abort_addr, int32_t* dev_status,
-                                         uint64_t limit_ns, bool suspend = !KVATTN_PREFILL_SPIN_ALL) {
-  if (ld_shared_i32(abort_addr)) return false;
-  if (bar_try_wait(a, parity, suspend)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (;;) {
-    if (bar_try_wait(a, parity, suspend)) return true;
-    if (ld_shared_i32(abort_addr)) return false;
-    if (globaltimer_ns() - t0 > limit_ns) {
-      st_shared_i32(abort_addr, 1);
-      if (dev_status) atomicOr(dev_status, KVATTN_DEV_WAIT_TIMEOUT);
-      return false;
-    }
-  }
-}
-// Bounded wait that does not give up when the abort flag is set: for the
-// completion of work already handed to the tensor cores or the copy engine.
-__device__ __forceinline__ bool bar_wait_all(uint32_t a, uint32_t parity, uint64_t limit_ns) {
-  if (bar_try_wait(a, parity, false)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (;;) {
-    if (bar_try_wait(a, parity, true)) return true;
-    if (globaltimer_ns() - t0 > limit_ns) return false;
-  }
-}
-__device__ __forceinline__ void tma_load_4d_raw(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1,
-                                                int c2, int c3) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
-      "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ void st_shared_v4(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
-}
-
-// ------------------------------------------------------------ tcgen05 helpers
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// Shared-memory matrix descriptor (sm_100 UMMA format): start address,
-// leading / stride byte offsets (all >> 4), version 1, 128-byte swizzle.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
-  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFF) << 16) |
-         ((uint64_t)((sbo_bytes >> 4) & 0x3FFF) << 32) | (1ull << 46) | (2ull << 61);
-}
-
-// Instruction descriptor of kind::f16: bf16 A and B, fp32 D, M=128, N=128;
-// b_mn_major selects an N-contiguous B operand.
-__host__ __device__ constexpr uint32_t idesc_bf16_m128_n128(bool b_mn_major) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((128u >> 3) << 17) |
-         ((128u >> 4) << 24);
-}
-
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                       uint32_t accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// A operand from tensor memory (rows in lanes, two bf16 per column).
-__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                          uint32_t accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
-}
-
-#define KV_R32(r)                                                                                               \
-  "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),    \
-      "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),     \
-      "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),    \
-      "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-#define KV_W32(r)                                                                                                 \
-  "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),   \
-      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), \
-      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), \
-      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-
-// 32 consecutive 32-bit TMEM columns of this thread's lane (warp-collective).
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
-      "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : KV_R32(r)
-      : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,"
-      "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      KV_W32(r)
-      : "memory");
-}
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
-          taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
-      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
-}
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-// 2^x of two fp32 values on the FMA pipes, to take part of the softmax's
-// exponentials off the special-function unit.  Cody and Waite's argument
-// reduction: x = n + f with n = round(x) (adding 1.5 * 2^23 leaves round(x) in
-// the low mantissa bits) and f in [-1/2, 1/2]; 2^f by a cubic fitted to it on
-// that interval by a Remez exchange on the relative error (max relative error
-// 7.5e-5, far below the bf16 rounding of P); 2^n by adding n to the exponent
-// field.  x is clamped to >= -125 (2^-125, a normal number); a caller that
-// needs 2^-inf = 0 selects it.
-constexpr float kExp2C0 = 9.999280572e-01f, kExp2C1 = 6.932609677e-01f, kExp2C2 = 2.426111251e-01f,
-                kExp2C3 = 5.517166853e-02f;
-__device__ __forceinline__ void exp2_poly_x2(float x0, float x1, float& p0, float& p1) {
-  x0 = fmaxf(x0, -125.f);
-  x1 = fmaxf(x1, -125.f);
-  const uint64_t x = f2_pack(x0, x1);
-  const uint64_t t = f2_add(x, f2_pack(12582912.f, 12582912.f));  // 1.5 * 2^23 + round(x)
-  const uint64_t n = f2_add(t, f2_pack(-12582912.f, -12582912.f));
-  const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), x);
-  uint64_t q = f2_fma(f2_pack(kExp2C3, kExp2C3), f, f2_pack(kExp2C2, kExp2C2));
-  q = f2_fma(q, f, f2_pack(kExp2C1, kExp2C1));
-  q = f2_fma(q, f, f2_pack(kExp2C0, kExp2C0));
-  float q0, q1, t0, t1;
-  f2_unpack(q, q0, q1);
-  f2_unpack(t, t0, t1);
-  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
-  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
-}
-
-// Two non-negative finite fp32 values (softmax probabilities) to packed bf16
-// on the integer pipes: add half a bf16 ulp, keep the upper 16 bits of each
-// (round to nearest, ties away from zero; ties of the fp32 inputs are rare
-// and the result is within half an ulp either way).  The conversion
-// instruction would run on the special-function pipe that the exponentials
-// already saturate.
-__device__ __forceinline__ uint32_t pack_bf16x2_p(float lo, float hi) {
-#if KVATTN_PREFILL_INT_PACK
-  uint32_t r;
-  asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(r) : "r"(__float_as_uint(lo) + 0x8000u), "r"(__float_as_uint(hi) + 0x8000u));
-  return r;
-#else
-  uint32_t r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-#endif
-}
-
-// max(a, b, c) in one instruction (NaN inputs are ignored, as by fmaxf)
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
-  uint32_t r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
 
 // DUAL: split mode (a.split_tiles > 0), see the mapping below
 template <int G, bool DUAL>

@@ -10,7 +10,7 @@ import re
 import numpy as np
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-SRC = os.path.join(ROOT, "gqa_decode_attention_kvattn_b200", "csrc", "prefill.cu")
+SRC = os.path.join(ROOT, "gqa_decode_attention_kvattn_b200", "csrc", "tc_device.cuh")
 
 
 def _coefficients():

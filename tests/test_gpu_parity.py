@@ -61,6 +61,11 @@ def _check_step(seed, B, T, H, Hkv, S, sp, rope, kind, hint=0, in_place=False):
     (3, 32, 1, 2500, [0, 1000, 2499], kv.LLAMA3),       # G = 32 (MQA): tcgen05 split path, 1 / 2 / 5 splits
     (6, 32, 1, 6000, [5999, 127, 128, 129, 3000, 4095], kv.LLAMA3_1),  # G = 32 at key-tile edges
     (2, 64, 2, 1500, [1499, 700], kv.LLAMA3),           # G = 32 with two KV heads
+    # G = 32 with many short row sets: the multi-query kernel's even ranges of
+    # key tiles cross several sequences each (Q reloaded, one partial per piece)
+    (150, 32, 1, 2048, [int(x) for x in np.random.RandomState(7).randint(0, 2048, 150)], kv.LLAMA3),
+    (40, 64, 2, 700, [0, 127, 128, 699] + [int(x) for x in np.random.RandomState(8).randint(0, 700, 36)],
+     kv.LLAMA3_1),
     (2, 64, 1, 900, [899, 33], kv.LLAMA3_1),            # G = 64 (MQA, 64 heads)
 ])
 def test_decode_step_small(case):
@@ -196,6 +201,32 @@ def test_out_of_range_start_pos_is_flagged_and_skipped():
     # the valid sequence is still right
     qr, kr, ref = U.oracle_sequence(q[1], k[1], v[1], ck[1], cv[1], 10, T, kv.LLAMA3)
     U.assert_attention_close(o[1], ref, "valid sequence beside bad ones")
+
+
+def test_mqa_decode_bad_positions_flagged_and_skipped():
+    """Multi-query decode (32 heads per KV head, tcgen05): sequences whose
+    start position is outside the cache or not below the hint add no key tiles
+    to the call's plan, keep the caller's output and set the status bits; the
+    others match the oracle."""
+    B, H, Hkv, S, hint = 6, 32, 1, 3000, 2500
+    sp = np.array([2499, -1, 1200, 3000, 2600, 64], np.int32)
+    q, k, v, ck, cv = U.host_inputs(15, B, 1, H, Hkv, S, np.clip(sp, 0, S - 1))
+    assert kv.kvattn_decode_plan(B, H, Hkv, S, max_kv_len_hint=hint)["max_splits"] > 1
+    dsp = torch.from_numpy(sp).cuda()
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sentinel = torch.full((B, 1, H, 128), 3.0, dtype=torch.bfloat16, device="cuda")
+    out = kv.kvattn_decode(U.to_dev(q), U.to_dev(ck), U.to_dev(cv), dsp, max_kv_len_hint=hint, out=sentinel,
+                           dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() & kv.KVATTN_DEV_START_POS_RANGE
+    assert st.item() & kv.KVATTN_DEV_KV_LEN_HINT
+    o = U.to_host(out)
+    for b in (1, 3, 4):
+        assert np.all(ks.bf16_bits_to_f64(o[b]) == 3.0), b
+    good = [0, 2, 5]
+    ref, rc = oracle.attention(q[good].copy(), ck[good].copy(), cv[good].copy(), sp[good].copy())
+    assert rc == 0
+    U.assert_attention_close(o[good], ref, "valid multi-query sequences beside bad ones")
 
 
 def test_kv_len_hint_exceeded_is_flagged():
