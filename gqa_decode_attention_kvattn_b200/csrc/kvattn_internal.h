@@ -107,8 +107,8 @@ struct DecodeArgs {
 // one group; G = 32, 64, 128 run as G/16 groups of 16 heads that read the
 // same KV head (neighbouring work items, so the second read of a row is
 // normally served by L2).  (Unmasked multi-split G = 32 calls do not reach
-// these kernels: the decode entry runs them on the tcgen05 prefill kernel in
-// split mode.)
+// these kernels: the decode entry runs them on the tcgen05 multi-query
+// kernel.)
 inline void decode_group_view(int H, int Hkv, int* groups, int* kv_div) {
   const int G = H / Hkv;
   *kv_div = G > 16 ? G / 16 : 1;
@@ -158,20 +158,6 @@ struct PrefillArgs {
   int window;       // > 0: token at position p sees keys p - window < k <= p and k < n_sink
   int n_sink;
   const float* sink_logits;  // fp32 [H] learned sink logits (score units), or null
-  // Split mode (split_tiles > 0; no window, no learned sinks; the
-  // multi-query decode): the key tiles of a (sequence, KV head) are cut into
-  // split_grid splits of split_tiles tiles, and CTA c of the unit takes the
-  // two consecutive splits 2c and 2c + 1 as its two Q tiles (both hold the
-  // same token's heads, each with its own K/V stream), so ceil(split_grid / 2)
-  // CTAs run per unit.  Q tile g of CTA c writes partial slot 2c + g.  A row
-  // set with more than one split writes its unnormalised O and (max in log2
-  // units, sum) to part_o [B*T, part_splits, H, d] / part_ml [.., 2], the
-  // layout the decode's LSE merge reads; one with a single split writes out.
-  int split_tiles;
-  int split_grid;
-  int part_splits;
-  float* part_o;
-  float* part_ml;
   uint64_t wait_ns;     // limit of each in-kernel wait (0: one second)
   const int32_t* gate;  // diagnostics gate (null: none)
 };

@@ -105,8 +105,7 @@ static_assert(kPrefillSmemBytes <= 227 * 1024, "shared memory per CTA");
 #define KVATTN_PREFILL_MAX3 1
 #endif
 
-// DUAL: split mode (a.split_tiles > 0), see the mapping below
-template <int G, bool DUAL>
+template <int G>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_v, const PrefillArgs a) {
@@ -124,24 +123,17 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const int lane = tid & 31;
   const uint64_t wlim = wait_limit(a.wait_ns);
 
-  // heaviest M tile pairs (latest tokens, most keys) first.  In split mode
-  // (`dual`) the two Q tiles of a CTA are the same token's heads over two
-  // consecutive splits 2c, 2c + 1 of the row set, each with its own K/V
-  // stream (stage g), so one split's MMAs overlap the other's softmax; each
-  // (pair, KV head, sequence) unit then has ceil(split_grid / 2) CTAs.
-  constexpr bool dual = DUAL;
+  // heaviest M tile pairs (latest tokens, most keys) first
   const int per_pair = a.Hkv * a.B;
   const int n_pairs = (a.n_mtiles + 1) / 2;
-  const int n_split_grid = dual ? (a.split_grid + 1) / 2 : 1;
-  const int unit = (int)(blockIdx.x / n_split_grid);
-  const int split = (int)(blockIdx.x - (unsigned)unit * n_split_grid);  // split pair c in split mode
+  const int unit = (int)blockIdx.x;
   const int pair = n_pairs - 1 - unit / per_pair;
   const int rem = unit % per_pair;
   const int kvh = rem % a.Hkv;
   const int b = rem / a.Hkv;
   const int sp = a.start_pos[b];
   if (sp < 0 || (long long)sp + a.T > a.S || (long long)sp + a.T > a.kv_len_hint) {
-    if (pair == 0 && kvh == 0 && split == 0 && tid == 0)
+    if (pair == 0 && kvh == 0 && tid == 0)
       set_status(a.dev_status, (sp < 0 || (long long)sp + a.T > a.S) ? KVATTN_DEV_START_POS_RANGE
                                                                     : KVATTN_DEV_KV_LEN_HINT);
     return;
@@ -160,27 +152,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     sink_tiles = min((a.n_sink + kBN - 1) / kBN, win_first);
   }
   const int n_all = sink_tiles + (n_kv - win_first);
-  // Q tile g's key tiles: j0g[g] .. j0g[g] + ntg[g] - 1 of the n_all (all of
-  // them unless in split mode); the loops below count j from 0
-  const int n_splits_here = dual ? (n_all + a.split_tiles - 1) / a.split_tiles : 1;
-  // Q tile 0 stops at the key tile of its own last token (at most one short)
-  const int j00 = dual ? 2 * split * a.split_tiles : 0;
-  const int j01 = dual ? j00 + a.split_tiles : 0;
-  const int nt0 = dual ? max(0, min(a.split_tiles, n_all - j00))
-                       : sink_tiles + ((sp + min(t0 + TT, a.T) + kBN - 1) / kBN - win_first);
-  const int nt1 = dual ? max(0, min(a.split_tiles, n_all - j01)) : (n_q > 1 ? n_all : 0);
+  // Q tile g reads key tiles 0 .. nt_g - 1 of the n_all; Q tile 0 stops at
+  // the key tile of its own last token (at most one short)
+  const int nt0 = sink_tiles + ((sp + min(t0 + TT, a.T) + kBN - 1) / kBN - win_first);
+  const int nt1 = n_q > 1 ? n_all : 0;
   const int n_iter = max(nt0, nt1);
-  if (n_iter <= 0) return;  // a shorter row set: no work in this split pair (before anything shared)
-  auto first_tile = [&](int g) { return g == 0 ? j00 : j01; };
-  auto key_tile = [&](int g, int j) {
-    const int jj = first_tile(g) + j;
-    return jj < sink_tiles ? jj : win_first + (jj - sink_tiles);
-  };
+  auto key_tile = [&](int j) { return j < sink_tiles ? j : win_first + (j - sink_tiles); };
   auto active = [&](int g, int j) { return j < (g == 0 ? nt0 : nt1); };
-  // K/V stage and phase parity of key tile j: a shared two-stage stream, or
-  // in split mode one stage per Q tile's stream
-  auto kv_stage = [&](int g, int j) { return dual ? g : (j & 1); };
-  auto kv_par = [&](int j) { return dual ? (uint32_t)(j & 1) : (uint32_t)((j >> 1) & 1); };
+  // K/V stage and phase parity of key tile j (a two-stage stream)
+  auto kv_stage = [&](int j) { return j & 1; };
+  auto kv_par = [&](int j) { return (uint32_t)((j >> 1) & 1); };
 
   if (tid == 0) {
     bar_init(bar(kBarQFull), 1);
@@ -224,26 +205,21 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         st_shared_i32(abort_addr, 1);
         set_status(a.dev_status, KVATTN_DEV_WAIT_TIMEOUT);
       } else {
-        // Q tile g: tokens t0 + g*TT ..; in split mode both Q tiles hold the
-        // one token, tile 1 loaded from token coordinate -1 so that its rows
-        // sit 32 TMEM lanes lower (rows of token -1 and of tokens past T are
-        // the copy's zero fill): the two splits' softmax rows then belong to
-        // warps on different SM sub-partitions
-        const int n_slots = dual ? 2 : n_q;
-        bar_expect_tx(bar(kBarQFull), (uint32_t)n_slots * 2u * kHalf);
-        for (int g = 0; g < n_slots; ++g) {
-          const int tq0 = dual ? t0 - g : t0 + g * TT;
+        // Q tile g: tokens t0 + g*TT .. (rows of tokens past T are the copy's
+        // zero fill)
+        bar_expect_tx(bar(kBarQFull), (uint32_t)n_q * 2u * kHalf);
+        for (int g = 0; g < n_q; ++g) {
+          const int tq0 = t0 + g * TT;
           tma_load_4d_raw(sQ + (2 * g) * kHalf, &tmap_q, bar(kBarQFull), 0, kvh * G, tq0, b);
           tma_load_4d_raw(sQ + (2 * g + 1) * kHalf, &tmap_q, bar(kBarQFull), 64, kvh * G, tq0, b);
         }
       }
       for (int j = 0; j < n_iter && go; ++j) {
-        // the shared stream loads key tile j once; split mode loads it per Q tile
-        for (int g = 0; g < (dual ? 2 : 1) && go; ++g) {
-          if (dual && !active(g, j)) continue;
-          const int s = kv_stage(g, j);
+        // key tile j, loaded once for both Q tiles
+        {
+          const int s = kv_stage(j);
           const uint32_t par = kv_par(j) ^ 1u;
-          const int key0 = key_tile(g, j) * kBN;
+          const int key0 = key_tile(j) * kBN;
           if (!bar_wait(bar(kBarKEmpty + s), par, abort_addr, a.dev_status, wlim, KVATTN_PREFILL_ISSUER_SUSPEND || !KVATTN_PREFILL_SPIN_ALL)) { go = false; break; }
           bar_expect_tx(bar(kBarKFull + s), 2 * kHalf);
           last_k[s] = j;
@@ -270,8 +246,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     // 64.  Two issuing threads, one per Q tile, reach the tensor core's rate
     // but drift into lockstep: both softmaxes then share the exponential unit
     // and the tensor cores idle meanwhile, which measured slower.)
-    // In split mode Q tile g reads Q slot g (the one token's heads, 32g rows
-    // down in slot 1) and K/V tile j of its own stream, released per stream.
     if (lane == 0) {
       constexpr bool kSusp = KVATTN_PREFILL_ISSUER_SUSPEND || !KVATTN_PREFILL_SPIN_ALL;
       constexpr uint32_t idesc_qk = idesc_bf16_m128_n128(false);
@@ -280,8 +254,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       tc_fence_after();
       // operand descriptors of k-step 0; k-step kk adds (byte offset) >> 4
       auto qk = [&](int g, int j) {
-        const int s = kv_stage(g, j);
-        if (dual && !bar_wait(bar(kBarKFull + s), kv_par(j), abort_addr, a.dev_status, wlim, kSusp)) return false;
+        const int s = kv_stage(j);
         tc_fence_after();
         const uint64_t q_desc = sw128_desc(sQ + 2u * (uint32_t)g * kHalf, 16, 1024);
         const uint64_t k_desc = sw128_desc(sK + 2u * (uint32_t)s * kHalf, 16, 1024);
@@ -292,12 +265,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           tc_mma(d_s, q_desc + off, k_desc + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
         tc_commit(bar(kBarSFull + g));
-        if (dual) tc_commit(bar(kBarKEmpty + s));
         return true;
       };
       // O_g += P_g(j) V_j once the softmax has published P_g(j)
       auto pv = [&](int g, int j) {
-        const int s = kv_stage(g, j);
+        const int s = kv_stage(j);
         if (!bar_wait(bar(kBarVFull + s), kv_par(j), abort_addr, a.dev_status, wlim, kSusp)) return false;
         if (!bar_wait(bar(kBarPFull + g), (uint32_t)j & 1u, abort_addr, a.dev_status, wlim, kSusp)) return false;
         tc_fence_after();
@@ -310,23 +282,21 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           tc_mma_ts(d_o, d_s + 8u * kk, v_desc + (uint64_t)(kk * 2048 / 16), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-        if (dual) tc_commit(bar(kBarVEmpty + s));
         return true;
       };
       for (int j = 0; j <= n_iter && ok; ++j) {
         if (j < n_iter) {
-          if (!dual && !bar_wait(bar(kBarKFull + (j & 1)), (uint32_t)(j >> 1) & 1u, abort_addr, a.dev_status, wlim,
-                                 kSusp))
+          if (!bar_wait(bar(kBarKFull + (j & 1)), (uint32_t)(j >> 1) & 1u, abort_addr, a.dev_status, wlim, kSusp))
             break;
           if (active(0, j) && !qk(0, j)) break;
         }
         if (j > 0) {
           if (active(1, j - 1) && !pv(1, j - 1)) break;
-          if (!dual) tc_commit(bar(kBarVEmpty + ((j - 1) & 1)));  // both PVs of tile j-1 issued
+          tc_commit(bar(kBarVEmpty + ((j - 1) & 1)));  // both PVs of tile j-1 issued
         }
         if (j < n_iter) {
           if (active(1, j) && !qk(1, j)) break;
-          if (!dual) tc_commit(bar(kBarKEmpty + (j & 1)));  // both QKs of tile j issued
+          tc_commit(bar(kBarKEmpty + (j & 1)));  // both QKs of tile j issued
           if (active(0, j) && !pv(0, j)) break;
         }
       }
@@ -342,8 +312,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int quarter = warp & 3;         // TMEM lanes 32*quarter .. +31
     const int grp = (warp - 2) >> 2;      // Q tile of this warp
     const int m = 32 * quarter + lane;    // query row of this thread within its Q tile
-    // token of this row (split mode: the one token, 32 rows down in Q tile 1)
-    const int tok = t0 + (dual ? m / G - grp : grp * TT + m / G);
+    const int tok = t0 + grp * TT + m / G;  // token of this row
     const int head = kvh * G + (m % G);
     const int lim = sp + min(tok, a.T - 1);  // last visible key (rows past T borrow the last token's)
     // with a window: keys n_sink <= k < lo_vis are hidden as well
@@ -360,7 +329,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const bool idle = __all_sync(0xffffffffu, tok < 0 || tok >= a.T);
 
     for (int j = 0; active(grp, j); ++j) {
-      const int jt = key_tile(grp, j);
+      const int jt = key_tile(j);
       if (!bar_wait(bar(kBarSFull + grp), (uint32_t)j & 1u, abort_addr, a.dev_status, wlim)) break;
       tc_fence_after();
       if (!idle) {
@@ -545,13 +514,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
       }
       }  // !idle
-      if (first_tile(grp) + j == n_all - 1 && Lmax < jt * kBN + kBN) {
+      if (j == n_all - 1 && Lmax < jt * kBN + kBN) {
         // rows of the last V tile past the last visible key may hold any bits;
-        // zero them so that 0 * (garbage) cannot reach O.  On the shared
-        // stream both Q tiles' groups write the same zeros into the one stage
-        // before their own P goes out; in split mode only the group whose
-        // split holds key tile n_all - 1 gets here, and it zeroes its own stage
-        const int s = kv_stage(grp, j);
+        // zero them so that 0 * (garbage) cannot reach O (both Q tiles' groups
+        // write the same zeros into the one stage before their own P goes out)
+        const int s = kv_stage(j);
         bar_wait(bar(kBarVFull + s), kv_par(j), abort_addr, a.dev_status, wlim);
         const int first_bad = Lmax - jt * kBN;
         const int nchunks = (kBN - first_bad) * 16;  // 16-byte chunks over both halves
@@ -581,30 +548,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       const float f = (ref == -INFINITY) ? 0.f : fast_exp2(ref - mn);
       inv_l = f / (l * f + fast_exp2(s2 - mn));
     }
-    const bool store = (dual ? active(grp, 0) : grp < n_q) && tok >= 0 && tok < a.T;
-    if (a.split_tiles > 0 && n_splits_here > 1) {
-      // this split's partial: unnormalised O and (max, sum), both relative
-      // to 2^ref (a group without key tiles here contributes nothing)
-      const bool any = active(grp, 0);
-      const size_t slot =
-          (((size_t)b * a.T + (store ? tok : 0)) * a.part_splits + (2 * split + grp)) * a.H + head;
-      float* po = a.part_o + slot * kHeadDim;
-#pragma unroll
-      for (int c2 = 0; c2 < 4; ++c2) {
-        uint32_t r[32];
-        tmem_ld32(lane_addr + col_o + 32u * c2, r);
-        tmem_wait_ld();
-        if (store) {
-#pragma unroll
-          for (int c = 0; c < 32; c += 4)
-            *reinterpret_cast<float4*>(po + 32 * c2 + c) =
-                any ? make_float4(__uint_as_float(r[c]), __uint_as_float(r[c + 1]), __uint_as_float(r[c + 2]),
-                                  __uint_as_float(r[c + 3]))
-                    : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-      }
-      if (store) *reinterpret_cast<float2*>(a.part_ml + slot * 2) = make_float2(any ? ref : -INFINITY, any ? l : 0.f);
-    } else {
+    const bool store = grp < n_q && tok >= 0 && tok < a.T;
     uint16_t* dst = a.out + (((size_t)b * a.T + (store ? tok : 0)) * a.H + head) * kHeadDim;
 #pragma unroll
     for (int c2 = 0; c2 < 4; ++c2) {
@@ -622,7 +566,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           *reinterpret_cast<uint4*>(dst + 32 * c2 + c) = w;
         }
       }
-    }
     }
   }
 
@@ -644,36 +587,25 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   }
 }
 
-template <int G, bool DUAL>
-cudaError_t launch_prefill_gd(const PrefillArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
-                              const CUtensorMap& tv, cudaStream_t st) {
+template <int G>
+cudaError_t launch_prefill_g(const PrefillArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
+                             const CUtensorMap& tv, cudaStream_t st) {
   static bool configured[64] = {false};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!configured[dev]) {
-    e = cudaFuncSetAttribute(prefill_tc_kernel<G, DUAL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(prefill_tc_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kPrefillSmemBytes);
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
-  // one CTA per M tile pair (times ceil(split_grid / 2) in split mode)
-  const long long grid = (long long)((a.n_mtiles + 1) / 2) * a.Hkv * a.B * (DUAL ? (a.split_grid + 1) / 2 : 1);
+  // one CTA per M tile pair
+  const long long grid = (long long)((a.n_mtiles + 1) / 2) * a.Hkv * a.B;
   if (grid <= 0 || grid > 0x7FFFFFFFll) return cudaErrorInvalidValue;
-  return launch_pdl(prefill_tc_kernel<G, DUAL>, dim3((unsigned)grid), dim3(kPrefillThreads), kPrefillSmemBytes, st,
-                    tq, tk, tv, a);
-}
-
-template <int G>
-cudaError_t launch_prefill_g(const PrefillArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
-                             const CUtensorMap& tv, cudaStream_t st) {
-  if constexpr (G == 32) {  // split mode serves the multi-query decode (G = 32) only
-    if (a.split_tiles > 0) return launch_prefill_gd<G, true>(a, tq, tk, tv, st);
-  } else {
-    if (a.split_tiles > 0) return cudaErrorInvalidValue;
-  }
-  return launch_prefill_gd<G, false>(a, tq, tk, tv, st);
+  return launch_pdl(prefill_tc_kernel<G>, dim3((unsigned)grid), dim3(kPrefillThreads), kPrefillSmemBytes, st, tq,
+                    tk, tv, a);
 }
 
 }  // namespace

@@ -140,14 +140,16 @@ KVATTN_API size_t kvattn_decode_workspace_bytes(const kvattn_dims* dims, int32_t
  * The rows of each (sequence, KV head) are streamed from HBM once and serve
  * all G query heads.  At G = 32 (e.g. multi-query attention with 32 heads) a
  * call with more than one split runs on the 5th-generation tensor cores: the
- * 32 heads form one 128-row MMA tile, the rows of a (sequence, KV head) are
- * cut into splits of whole 128-row key tiles, and each CTA takes two
- * consecutive splits, one per tensor-memory accumulator.  G = 64, 128 (and masked G = 32 calls) run as G/16 groups of 16
- * heads over the same rows, scheduled side by side so the repeat reads are
- * served by L2.  Long rows are split across CTAs and the partial
- * (o, max, sum) triples are merged by log-sum-exp in a second kernel; the
- * tensor-core G = 32 path uses the same workspace layout and merge, with its
- * own split size (a multiple of 128 rows, never more splits than the plan's).
+ * 32 heads are 32 rows of a 128-row MMA tile, and the 128-row key tiles of
+ * all (sequence, KV head) pairs, laid end to end, are cut into equal
+ * contiguous ranges, two per SM (one per tensor-memory accumulator); each
+ * piece of a sequence within a range leaves one partial.  G = 64, 128 (and
+ * masked G = 32 calls) run as G/16 groups of 16 heads over the same rows,
+ * scheduled side by side so the repeat reads are served by L2.  Long rows
+ * are split across CTAs and the partial (o, max, sum) triples are merged by
+ * log-sum-exp in a second kernel; the tensor-core G = 32 path uses the same
+ * workspace layout and merge (never more partials per sequence than the
+ * plan's splits).
  * scale <= 0 selects 1/sqrt(d).  max_kv_len_hint (<= 0: max_seq_len) is a
  * host upper bound on start_pos[b] + 1; it sizes the splits and the
  * workspace.  A sequence above the hint or outside the cache leaves its

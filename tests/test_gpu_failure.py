@@ -58,7 +58,7 @@ def _oracle(host, sp, rope=kv.LLAMA3):
     # B, T, H, Hkv, S, start positions, entry
     (3, 1, 32, 8, 2000, [1999, 700, 64], "decode"),        # G = 4, CUDA-core split kernel + merge
     (4, 1, 64, 8, 3000, [2999, 5, 1000, 2500], "decode"),  # G = 8, warp-MMA kernel + merge
-    (2, 1, 32, 1, 3000, [2999, 1500], "decode"),           # G = 32, tcgen05 split path + merge
+    (2, 1, 32, 1, 3000, [2999, 1500], "decode"),           # G = 32, tcgen05 multi-query kernel + merge
     (3, 1, 32, 8, 2000, [1999, 700, 64], "noalloc"),
     (2, 1, 32, 8, 1500, [1499, 300], "window"),
     (2, 64, 32, 8, 600, [500, 17], "prefill"),

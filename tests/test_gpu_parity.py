@@ -58,7 +58,7 @@ def _check_step(seed, B, T, H, Hkv, S, sp, rope, kind, hint=0, in_place=False):
     (3, 32, 2, 700, [0, 63, 64, 699][:3], kv.LLAMA3),     # G = 16 (tensor cores)
     (4, 64, 8, 3000, [2999, 64, 65, 1000], kv.LLAMA3_1),  # G = 8, several splits
     (8, 32, 8, 8192, [8191, 0, 63, 64, 4000, 777, 5000, 12], kv.LLAMA3),  # G = 4 on the tensor-core kernel
-    (3, 32, 1, 2500, [0, 1000, 2499], kv.LLAMA3),       # G = 32 (MQA): tcgen05 split path, 1 / 2 / 5 splits
+    (3, 32, 1, 2500, [0, 1000, 2499], kv.LLAMA3),       # G = 32 (MQA): the tcgen05 multi-query kernel
     (6, 32, 1, 6000, [5999, 127, 128, 129, 3000, 4095], kv.LLAMA3_1),  # G = 32 at key-tile edges
     (2, 64, 2, 1500, [1499, 700], kv.LLAMA3),           # G = 32 with two KV heads
     # G = 32 with many short row sets: the multi-query kernel's even ranges of
