@@ -897,6 +897,14 @@ __global__ void __launch_bounds__(kHeadDim) decode_merge_kernel(const DecodeArgs
 // O values belong to the same head (lane/4, and lane/4+8 when G = 16), so the
 // online softmax rescales O without any exchange between lanes.  K and V
 // arrive by TMA as 128B-swizzled 64-element halves, read with ldmatrix.
+//
+// G = 8 runs transposed (kSwap), so no MMA row is padding: per warp and 16
+// rows, S^T = K q^T with the rows as M and the 8 heads as N (8 k-steps), then
+// O^T += V^T P^T with 16 head dims as M per MMA (8 MMAs), V^T read with
+// ldmatrix.trans and P^T made from the S^T accumulators by one movmatrix
+// transpose per 8 rows.  Half the MMAs of the padded form.  Each lane holds
+// S and O for the same two heads (2(lane%4), +1), so the softmax state that
+// rescales O is the lane's own after a max over the lanes that share them.
 constexpr int kMmaTileRows = 64;
 // G = 4 calls with at least this many (row, KV head) pairs run on the
 // tensor-core decode (its 64-row tiles and 2 CTAs per SM pay off once the
@@ -944,6 +952,13 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                : "r"(addr));
+}
+// Transpose of an 8x8 b16 matrix held one row pair per lane (lane l: row
+// l/4, columns 2(l%4), 2(l%4)+1) into the same layout.
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+  uint32_t r;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(r) : "r"(x));
+  return r;
 }
 // byte offset of the 16-byte chunk holding elements 8*chunk.. of `row` in a
 // 128B-swizzled [rows][64] half tile
@@ -1047,7 +1062,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(
     }
     const Item it = decode_item<WINDOW>(a, sm, n_sets, i);
 
-    // q as A fragments (rows = heads g and g+8, columns = head dims)
+    constexpr bool kSwap = (G == 8);
+    // q as A fragments (rows = heads g and g+8, columns = head dims), or
+    // (kSwap) as B fragments (head lane/4, dims 16kk + 2c4 .. and + 8)
     uint32_t qa[8][4];
     float o[16][4];
 #pragma unroll
@@ -1063,6 +1080,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(
         const uint32_t* qw = reinterpret_cast<const uint32_t*>(&sm.q[stage][0][0]);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
+          if constexpr (kSwap) {
+            qa[kk][0] = qw[g * 64 + 8 * kk + c4];
+            qa[kk][1] = qw[g * 64 + 8 * kk + 4 + c4];
+            qa[kk][2] = 0u;
+            qa[kk][3] = 0u;
+            continue;
+          }
           const int col = 8 * kk + c4;  // word index of dims 16kk + 2*c4
           // rows g >= G pad the 16-row MMA tile with zeros
           qa[kk][0] = (G >= 8 || g < G) ? qw[g * 64 + col] : 0u;
@@ -1097,6 +1121,75 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(
           }
         }
         __syncwarp();
+      }
+
+      if constexpr (kSwap) {
+        // ---- S^T = K q^T for the warp's 16 rows: lane holds rows wrow + g
+        // (st[0], st[1]: heads 2c4, 2c4+1) and wrow + g + 8 (st[2], st[3])
+        float st[4] = {0.f, 0.f, 0.f, 0.f};
+        const int r = wrow + (lane & 7) + 8 * ((lane >> 3) & 1);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          // matrices (rows wrow..+7 | wrow+8..+15) x (dims chunk 2kk | 2kk+1)
+          const int chunk = 2 * kk + (lane >> 4);
+          const uint32_t addr = kbase + (uint32_t)(chunk >> 3) * kMmaHalfBytes + sw128_off(r, chunk & 7);
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(addr, a0, a1, a2, a3);
+          mma_bf16_16816(st, a0, a1, a2, a3, qa[kk][0], qa[kk][1]);
+        }
+        // ---- online softmax per head: the lane's heads 2c4 (hh = 0) and
+        // 2c4 + 1 (hh = 1) over its two rows, then over the 8 lanes sharing them
+        float pt[4];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          float s0 = st[hh] * a.scale_log2, s1 = st[2 + hh] * a.scale_log2;
+          if (masked) {
+            if (hidden(wrow + g)) s0 = -INFINITY;
+            if (hidden(wrow + g + 8)) s1 = -INFINITY;
+          }
+          float tmax = fmaxf(s0, s1);
+          tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
+          tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 8));
+          tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
+          const bool move = tmax > m_run[hh] + 8.f;
+          const float m_new = move ? tmax : m_run[hh];
+          const float alpha = move ? fast_exp2(m_run[hh] - m_new) : 1.f;
+          m_run[hh] = m_new;
+          const float p0 = (m_new == -INFINITY) ? 0.f : fast_exp2(s0 - m_new);
+          const float p1 = (m_new == -INFINITY) ? 0.f : fast_exp2(s1 - m_new);
+          pt[hh] = p0;
+          pt[2 + hh] = p1;
+          l_run[hh] = l_run[hh] * alpha + (p0 + p1);  // this lane's rows only
+          if (alpha != 1.f) {
+#pragma unroll
+            for (int mb = 0; mb < 8; ++mb) {
+              o[mb][hh] *= alpha;
+              o[mb][2 + hh] *= alpha;
+            }
+          }
+        }
+        // P^T as the B fragment: rows (K) 2c4, 2c4+1 of head (N) g, from the
+        // S^T layout (row g, heads 2c4, 2c4+1) by an 8x8 transpose per 8 rows
+        const uint32_t pb0 = movmatrix_t(pack_bf16x2(pt[0], pt[1]));
+        const uint32_t pb1 = movmatrix_t(pack_bf16x2(pt[2], pt[3]));
+        // ---- O^T += V^T P^T: M block mb covers dims 16mb .. 16mb + 15
+#pragma unroll
+        for (int mb = 0; mb < 8; ++mb) {
+          // matrices (rows wrow..+7 | wrow+8..+15) x (dims chunk 2mb | 2mb+1),
+          // transposed: a0 dims 16mb.., rows 0-7; a1 dims +8, rows 0-7;
+          // a2 dims 16mb.., rows 8-15; a3 dims +8, rows 8-15
+          const int mi = lane >> 3;
+          const int rr = wrow + 8 * (mi >> 1) + (lane & 7);
+          const int chunk = 2 * mb + (mi & 1);
+          const uint32_t addr = vbase + (uint32_t)(chunk >> 3) * kMmaHalfBytes + sw128_off(rr, chunk & 7);
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_t(addr, a0, a1, a2, a3);
+          mma_bf16_16816(o[mb], a0, a1, a2, a3, pb0, pb1);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.empty[stage]);
+        if (++stage == kMmaStages) { stage = 0; phase ^= 1; }
+        continue;
       }
 
       // ---- S = q K^T for the warp's 16 rows: n-tile nt covers rows wrow+8nt..+7
@@ -1183,8 +1276,28 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(
     }
 
     // ---- merge the four warps' states of this item
+    if constexpr (kSwap) {
+      // o[mb]: dims 16mb + g (0, 1) and + 8 (2, 3), heads 2c4 + (0 | 1)
 #pragma unroll
-    for (int hh = 0; hh < (G == 16 ? 2 : 1); ++hh) {
+      for (int hh = 0; hh < 2; ++hh) {
+        float lsum = l_run[hh];
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, 4);
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, 8);
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
+        const int h = 2 * c4 + hh;
+        if (g == 0) {
+          sm.merge_m[warp][h] = m_run[hh];
+          sm.merge_l[warp][h] = lsum;
+        }
+#pragma unroll
+        for (int mb = 0; mb < 8; ++mb) {
+          sm.merge_o[warp][h][16 * mb + g] = o[mb][hh];
+          sm.merge_o[warp][h][16 * mb + g + 8] = o[mb][2 + hh];
+        }
+      }
+    }
+#pragma unroll
+    for (int hh = 0; hh < (G == 16 ? 2 : 1) && !kSwap; ++hh) {
       float lsum = l_run[hh];
       lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
       lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
