@@ -61,6 +61,7 @@ def _check_step(seed, B, T, H, Hkv, S, sp, rope, kind, hint=0, in_place=False):
     (3, 32, 1, 2500, [0, 1000, 2499], kv.LLAMA3),       # G = 32 (MQA): the tcgen05 multi-query kernel
     (6, 32, 1, 6000, [5999, 127, 128, 129, 3000, 4095], kv.LLAMA3_1),  # G = 32 at key-tile edges
     (2, 64, 2, 1500, [1499, 700], kv.LLAMA3),           # G = 32 with two KV heads
+    (6, 32, 1, 1000, [95, 96, 97, 191, 192, 999], kv.LLAMA3),  # G = 32, short row sets (96 to 1000 rows)
     # G = 32 with many short row sets: the multi-query kernel's even ranges of
     # key tiles cross several sequences each (Q reloaded, one partial per piece)
     (150, 32, 1, 2048, [int(x) for x in np.random.RandomState(7).randint(0, 2048, 150)], kv.LLAMA3),
