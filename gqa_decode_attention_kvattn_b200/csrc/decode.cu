@@ -68,7 +68,6 @@ template <int G>
 struct Shape {
   static constexpr int RB = (G >= 16) ? 1 : (G >= 8) ? 2 : 4;  // rows per half-warp batch
   static constexpr int NV = G * RB;                // partial dot products per lane
-  static constexpr int LOG2NV = ilog2(NV);
   static constexpr int REP = NV >= 16 ? 1 : 16 / NV;  // lanes that end up with the same score
   static constexpr int PASSES = kTileRows / (kHalfWarps * RB);
   // pipeline depth and resident CTAs per SM: G <= 4 fits three CTAs (about
@@ -971,12 +970,14 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(
     const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
     const DecodeArgs a, const int evict_first, const __grid_constant__ RopeTable tab) {
   static_assert(G == 1 || G == 2 || G == 4 || G == 8 || G == 16, "tensor-core decode handles G <= 16");
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
-  SmemMma<G>& sm = *reinterpret_cast<SmemMma<G>*>(smem_raw);
+  // (its own name: the CUDA-core kernel in this file declares the dynamic
+  // shared memory with a smaller alignment)
+  extern __shared__ __align__(1024) unsigned char smem_mma_raw[];
+  SmemMma<G>& sm = *reinterpret_cast<SmemMma<G>*>(smem_mma_raw);
   pdl_wait();  // the previous kernel in the stream (rope_append, say) has finished
   pdl_launch_dependents();
   // the 128B-swizzled tiles need a 1024-byte aligned base; refuse otherwise
-  if ((smem_u32(smem_raw) & 1023u) != 0) {
+  if ((smem_u32(smem_mma_raw) & 1023u) != 0) {
     if (threadIdx.x == 0) set_status(a.dev_status, KVATTN_DEV_INTERNAL);
     return;
   }
@@ -1186,12 +1187,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(
           ldsm_x4_t(addr, a0, a1, a2, a3);
           mma_bf16_16816(o[mb], a0, a1, a2, a3, pb0, pb1);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.empty[stage]);
-        if (++stage == kMmaStages) { stage = 0; phase ^= 1; }
-        continue;
-      }
-
+      } else {
       // ---- S = q K^T for the warp's 16 rows: n-tile nt covers rows wrow+8nt..+7
       float sacc[2][4];
 #pragma unroll
@@ -1270,6 +1266,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_mma_kernel(
         mma_bf16_16816(o[2 * dp], pa0, pa1, pa2, pa3, b0, b1);
         mma_bf16_16816(o[2 * dp + 1], pa0, pa1, pa2, pa3, b2, b3);
       }
+      }  // !kSwap
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.empty[stage]);
       if (++stage == kMmaStages) { stage = 0; phase ^= 1; }
