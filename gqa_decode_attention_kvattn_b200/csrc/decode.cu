@@ -1469,10 +1469,18 @@ DecodePlan plan_decode(int B, int Tq, int H, int Hkv, int kv_len_hint, int sm_co
   p.ctas_per_sm = ctas_per_sm;
   const int slots = sm_count * ctas_per_sm;
   const long long row_sets = (long long)B * Tq;
-  // Aim for ~16 items per resident CTA so the work counter's tail stays
-  // balanced when lengths are ragged; never split below 64 rows, and do not split at all
-  // when the (b, t, head) units alone already give that much parallelism.
-  long long want = (row_sets * Hkv * (long long)kv_len_hint) / (16LL * slots);
+  // Split size: aim for a few items per resident CTA at full length (the
+  // work counter hands them out, so ragged lengths still balance), as long
+  // as that keeps every item long enough that its epilogue (the warps' merge
+  // through shared memory and the partial writes) stays small beside its
+  // rows.  Measured on 1 GB calls: the tensor-core kernel is fastest at ~4
+  // items per CTA (64/8 heads: 173.7 -> 163.0 us from 16 items; 32/8 heads:
+  // 168.7 -> 164.3; 131k rows: 449.7 -> 426.0), the CUDA-core kernel at ~8
+  // (16/8 heads: 170.6 -> 166.8; 32/32 heads flat, 4 % slower at 4).  Never
+  // split below 64 rows, and do not split at all when the (b, t, head)
+  // units alone already give enough parallelism.
+  const long long items_per_cta = p.mma ? 4 : 8;
+  long long want = (row_sets * Hkv * (long long)kv_len_hint) / (items_per_cta * slots);
   int C = 64;
   while (C < 4096 && (long long)C * 2 <= want) C *= 2;
   if (row_sets > kMaxRowSets || row_sets * Hkv >= 16LL * slots || Tq > 1) C = kv_len_hint;

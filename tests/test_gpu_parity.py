@@ -331,11 +331,12 @@ def test_decode_kernel_choice():
 def test_decode_workspace_shared_across_shapes_and_left_zeroed():
     """One workspace serves calls of different shapes in a row: its work
     counter sits at a fixed offset and every call leaves it zero."""
-    ws = kv.alloc_workspace(kv.kvattn_decode_workspace_bytes(8, 32, 8, 8192))
-    for seed, (B, H, Hkv, S, sp) in enumerate([(8, 32, 8, 8192, [8191, 0, 63, 64, 4000, 777, 5000, 12]),
-                                               (4, 32, 8, 4096, [1499, 700, 64, 1000]),
-                                               (3, 64, 8, 3000, [2999, 5, 1500]),
-                                               (2, 32, 1, 3000, [2999, 100])]):
+    shapes = [(8, 32, 8, 8192, [8191, 0, 63, 64, 4000, 777, 5000, 12]),
+              (4, 32, 8, 4096, [1499, 700, 64, 1000]),
+              (3, 64, 8, 3000, [2999, 5, 1500]),
+              (2, 32, 1, 3000, [2999, 100])]
+    ws = kv.alloc_workspace(max(kv.kvattn_decode_workspace_bytes(B, H, Hkv, S) for B, H, Hkv, S, _ in shapes))
+    for seed, (B, H, Hkv, S, sp) in enumerate(shapes):
         q, k, v, ck, cv = U.host_inputs(70 + seed, B, 1, H, Hkv, S, sp)
         dq, dk, dv, dck, dcv = (U.to_dev(x) for x in (q, k, v, ck, cv))
         dsp = torch.from_numpy(np.asarray(sp, np.int32)).cuda()
