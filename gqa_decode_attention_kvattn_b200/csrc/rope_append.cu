@@ -45,17 +45,6 @@ __global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(RopeAppendArg
   }
   const long long pos = (long long)sp + t;
 
-  __shared__ double s_cos[kMaxRopePairs];
-  __shared__ double s_sin[kMaxRopePairs];
-  const int rp = tab.rotary_dim / 2;  // rotated pairs
-  for (int i = threadIdx.x; i < rp; i += blockDim.x) {
-    double s, c;
-    rope_cos_sin(tab, i, pos, c, s);
-    s_cos[i] = c;
-    s_sin[i] = s;
-  }
-  __syncthreads();
-
   constexpr int kPairs = kHeadDim / 2;
   const int v0 = blk * vec_per_cta;
   const int nv = min(vec_per_cta, n_vec - v0);
@@ -68,21 +57,60 @@ __global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(RopeAppendArg
     return v < a.H ? a.q_rot + ((size_t)bt * a.H + v) * kHeadDim
                    : a.cache_k + (((size_t)b * a.S + pos) * a.Hkv + (v - a.H)) * kHeadDim;
   };
+  const int rp = tab.rotary_dim / 2;  // rotated pairs
+  const bool full_meta = tab.layout == 0 && rp == kPairs;
 
   // Each thread loads a batch of its words before it stores any: q_rot may be
   // q itself, so the compiler cannot move a load above an earlier store, and
   // one word at a time would pay a full memory latency per word.  Every word
-  // is read and written by the same thread, so rotating in place is safe.
+  // is read and written by the same thread, so rotating in place is safe.  The
+  // first batch (the whole of a decode token's share) is loaded before the
+  // (cos, sin) table is built, so its latency overlaps the fp64 sincos.
   constexpr int kBatch = 8;
   const int n_slots = nv * kPairs;
-  if (tab.layout == 0 && rp == kPairs) {
+  auto load_batch = [&](int base_idx, uint32_t (&w)[kBatch]) {
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int idx = base_idx + u * blockDim.x;
+      w[u] = idx < n_slots ? reinterpret_cast<const uint32_t*>(vec_in(v0 + idx / kPairs))[idx & (kPairs - 1)] : 0u;
+    }
+  };
+  uint32_t w_first[kBatch];
+  if (full_meta) load_batch(threadIdx.x, w_first);
+  // values: bit copy of the 256-byte rows of this CTA's key heads, the first
+  // batch of 16-byte chunks also in flight before the table
+  const int k0 = max(v0, a.H) - a.H;       // first key head of this CTA
+  const int k1 = max(v0 + nv, a.H) - a.H;  // one past the last
+  const uint4* v_in = reinterpret_cast<const uint4*>(a.v_new) + (size_t)bt * a.Hkv * (kHeadDim / 8);
+  uint4* v_out = reinterpret_cast<uint4*>(a.cache_v) + ((size_t)b * a.S + pos) * a.Hkv * (kHeadDim / 8);
+  const int c_begin = k0 * (kHeadDim / 8) + threadIdx.x;
+  const int c_end = k1 * (kHeadDim / 8);
+  uint4 t_first[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int idx = c_begin + u * blockDim.x;
+    if (idx < c_end) t_first[u] = v_in[idx];
+  }
+
+  __shared__ double s_cos[kMaxRopePairs];
+  __shared__ double s_sin[kMaxRopePairs];
+  for (int i = threadIdx.x; i < rp; i += blockDim.x) {
+    double s, c;
+    rope_cos_sin(tab, i, pos, c, s);
+    s_cos[i] = c;
+    s_sin[i] = s;
+  }
+  __syncthreads();
+
+  if (full_meta) {
     // Meta layout over the whole head: each pair is one 32-bit word
     for (int base_idx = threadIdx.x; base_idx < n_slots; base_idx += blockDim.x * kBatch) {
       uint32_t w[kBatch];
+      if (base_idx == (int)threadIdx.x) {
 #pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int idx = base_idx + u * blockDim.x;
-        w[u] = idx < n_slots ? reinterpret_cast<const uint32_t*>(vec_in(v0 + idx / kPairs))[idx & (kPairs - 1)] : 0u;
+        for (int u = 0; u < kBatch; ++u) w[u] = w_first[u];
+      } else {
+        load_batch(base_idx, w);
       }
 #pragma unroll
       for (int u = 0; u < kBatch; ++u) {
@@ -126,19 +154,18 @@ __global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(RopeAppendArg
     }
   }
 
-  // values: bit copy of the 256-byte rows of this CTA's key heads (a batch of
-  // 16-byte loads before the stores, as above)
-  const int k0 = max(v0, a.H) - a.H;       // first key head of this CTA
-  const int k1 = max(v0 + nv, a.H) - a.H;  // one past the last
-  const uint4* v_in = reinterpret_cast<const uint4*>(a.v_new) + (size_t)bt * a.Hkv * (kHeadDim / 8);
-  uint4* v_out = reinterpret_cast<uint4*>(a.cache_v) + ((size_t)b * a.S + pos) * a.Hkv * (kHeadDim / 8);
-  const int c_end = k1 * (kHeadDim / 8);
-  for (int base_idx = k0 * (kHeadDim / 8) + threadIdx.x; base_idx < c_end; base_idx += blockDim.x * 4) {
+  // the value rows: the first batch is already in registers
+  for (int base_idx = c_begin; base_idx < c_end; base_idx += blockDim.x * 4) {
     uint4 t[4];
+    if (base_idx == c_begin) {
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int idx = base_idx + u * blockDim.x;
-      if (idx < c_end) t[u] = v_in[idx];
+      for (int u = 0; u < 4; ++u) t[u] = t_first[u];
+    } else {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int idx = base_idx + u * blockDim.x;
+        if (idx < c_end) t[u] = v_in[idx];
+      }
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
