@@ -204,6 +204,19 @@ def test_out_of_range_start_pos_is_flagged_and_skipped():
     U.assert_attention_close(o[1], ref, "valid sequence beside bad ones")
 
 
+@pytest.mark.parametrize("seed", [101, 102, 103, 104, 105, 106])
+def test_mqa_decode_random_shapes(seed):
+    # multi-query decode at seeded random shapes: the call's key tiles are cut
+    # into even ranges that start and end anywhere inside the sequences
+    rng = np.random.RandomState(seed)
+    Hkv = int(rng.choice([1, 2]))
+    B = int(rng.randint(1, 60))
+    S = int(rng.randint(300, 4000))
+    sp = [int(x) for x in rng.randint(0, S, B)]
+    assert kv.kvattn_decode_plan(B, 32 * Hkv, Hkv, S)["max_splits"] > 1  # the multi-query kernel runs
+    _check_step(seed, B, 1, 32 * Hkv, Hkv, S, sp, kv.LLAMA3, "decode")
+
+
 def test_mqa_decode_bad_positions_flagged_and_skipped():
     """Multi-query decode (32 heads per KV head, tcgen05): sequences whose
     start position is outside the cache or not below the hint add no key tiles
