@@ -85,11 +85,6 @@ static_assert(kPrefillSmemBytes <= 227 * 1024, "shared memory per CTA");
 #ifndef KVATTN_PREFILL_ISSUER_SUSPEND
 #define KVATTN_PREFILL_ISSUER_SUSPEND 0
 #endif
-// softmax exponentiates against the current reference while loading (1), or
-// loads the whole row and takes its max first (0)
-#ifndef KVATTN_PREFILL_OPTIMISTIC
-#define KVATTN_PREFILL_OPTIMISTIC 0
-#endif
 // of every four pairs of scores, how many are exponentiated by polynomial on
 // the FMA pipes instead of the special-function unit (0..4)
 #ifndef KVATTN_PREFILL_POLY_PAIRS
@@ -408,39 +403,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       };
       bool move;
       float alpha = 1.f;
-#if KVATTN_PREFILL_OPTIMISTIC
-      if (ref != -INFINITY) {
-        // The row's reference rarely moves (only when a tile's max exceeds it
-        // by more than 8), so exponentiate each 32-column chunk against the
-        // current reference as soon as it is loaded, with the next chunk's
-        // load in flight, and track the max alongside.  If the reference does
-        // have to move, redo the tile's exponentials from the scores still in
-        // registers: the same values as exponentiating after the max.
-        tmem_ld32(lane_addr + col_s, sr[0]);
-        tmem_wait_ld();
-        const uint64_t nr2 = neg_ref2();
-#pragma unroll
-        for (int c2 = 0; c2 < 4; ++c2) {
-          if (c2 < 3) tmem_ld32(lane_addr + col_s + 32u * (c2 + 1), sr[c2 + 1]);
-          mask_chunk(c2);
-          max_chunk(c2);
-          exp_chunk(c2, nr2);
-          if (c2 < 3) tmem_wait_ld();
-        }
-        const float mx = row_max();
-        move = mx > ref + 8.f;
-        if (move) {
-          alpha = fast_exp2(ref - mx);
-          ref = mx;
-          tmem_wait_st();  // the first P stores land before they are overwritten
-#pragma unroll
-          for (int k = 0; k < 4; ++k) sum2[k] = 0ull;
-          const uint64_t nr2m = neg_ref2();
-#pragma unroll
-          for (int c2 = 0; c2 < 4; ++c2) exp_chunk(c2, nr2m);
-        }
-      } else
-#endif
 #if KVATTN_PREFILL_TWO_PASS
       {
         // Two passes over TMEM, 32 columns at a time with the next chunk's
@@ -476,8 +438,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       }
 #else
       {
-        // (first tile of the row, or the plain order) load the row, take its
-        // max, then exponentiate
+        // load the row, take its max, then exponentiate
 #pragma unroll
         for (int c2 = 0; c2 < 4; ++c2) tmem_ld32(lane_addr + col_s + 32u * c2, sr[c2]);
         tmem_wait_ld();
