@@ -489,9 +489,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           const int cc = c & 7;
           st_shared_v4(sV + (2 * s + half) * kHalf + r * 128 + cc * 16, 0u, 0u, 0u, 0u);
         }
+        // the zeroed rows, written through the generic proxy, before the
+        // tensor cores read the stage (only this tile needs the fence)
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       }
       tmem_wait_st();
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the zeroed V rows, if any
       tc_fence_before();
       __syncwarp();
       if (lane == 0) bar_arrive(bar(kBarPFull + grp));
