@@ -27,8 +27,11 @@
 // between the Q tiles, QK_0(j), PV_1(j-1), QK_1(j), PV_0(j), so the tensor
 // cores run one tile's MMAs while the softmax warps of the other work.
 // QK_g(j+1) overwrites the columns PV_g(j) reads P_g(j) from; it is issued
-// after PV_g(j) by the same thread, and one thread's MMAs run in issue order.  P never touches shared memory, which leaves shared-memory
-// bandwidth to the TMA writes and the Q, K, V operand reads.
+// after PV_g(j) by the same thread, and one thread's MMAs run in issue order.
+// The softmax publishes P in parts (the first 64 keys, then the rest), so the
+// first P.V steps run while the rest of P is computed.  P never touches
+// shared memory, which leaves shared-memory bandwidth to the TMA writes and
+// the Q, K, V operand reads.
 //
 // The softmax reference.  A row's reference max only moves when a tile's max
 // exceeds it by more than 8 (probabilities stay <= 2^8), so O is rescaled
@@ -71,8 +74,11 @@ constexpr uint32_t kOffBar = kOffV + 4 * kHalf;
 // barrier slots (8 bytes each): K/V per stage, S/P per Q tile
 // (every pipeline barrier exists once per buffer, so a waiter is never more
 // than one phase behind the barrier it waits on)
+// (P part k of Q tile g, slot kBarPPart + 3g + k: the P columns of the first
+// k+1 parts are in TMEM, the issuer may start P.V on them)
 constexpr uint32_t kBarQFull = 0, kBarKFull = 1, kBarKEmpty = 3, kBarVFull = 5, kBarVEmpty = 7, kBarSFull = 9,
-                   kBarPFull = 11, kBarMmaDone = 13, kNumBars = 15;  // MMA done: one per Q tile's softmax group
+                   kBarPFull = 11, kBarMmaDone = 13, kBarPPart = 15,
+                   kNumBars = 21;  // MMA done: one per Q tile's softmax group
 constexpr uint32_t kOffTmemSlot = kOffBar + 8 * kNumBars;
 constexpr uint32_t kOffAbort = kOffTmemSlot + 8;
 constexpr uint32_t kPrefillSmemBytes = kOffAbort + 8 + 1024;  // + alignment slack
@@ -90,11 +96,20 @@ static_assert(kPrefillSmemBytes <= 227 * 1024, "shared memory per CTA");
 #ifndef KVATTN_PREFILL_POLY_PAIRS
 #define KVATTN_PREFILL_POLY_PAIRS 1
 #endif
-// softmax reads each S chunk twice from TMEM (max, then exponentials) instead
-// of holding the 128-column row in registers
-#ifndef KVATTN_PREFILL_TWO_PASS
-#define KVATTN_PREFILL_TWO_PASS 0
+// P is published to the MMA issuer in parts, so P.V starts on the first part
+// while the rest is computed: 1 (all 128 keys), 2 (64 + 64), 3 (64 + 32 + 32)
+// or 4 (32 each); part h holds the 32-key chunks p_begin(h) .. p_begin(h+1)-1.
+// On the 4 x 512-token prefill over 3584 cached rows: 149.0 us in one part,
+// 144.5 in two, 147.0 in three, 158 in four (each signal costs the softmax a
+// TMEM store wait, and four parts spill).
+#ifndef KVATTN_PREFILL_P_PARTS
+#define KVATTN_PREFILL_P_PARTS 2
 #endif
+constexpr int kPParts = KVATTN_PREFILL_P_PARTS;
+static_assert(kPParts >= 1 && kPParts <= 4, "P parts");
+__host__ __device__ constexpr int p_begin(int h) {
+  return h >= kPParts ? 4 : kPParts == 1 ? 0 : kPParts == 2 ? 2 * h : kPParts == 3 ? (h == 0 ? 0 : h + 1) : h;
+}
 // row max with three-input max instructions
 #ifndef KVATTN_PREFILL_MAX3
 #define KVATTN_PREFILL_MAX3 1
@@ -167,6 +182,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       bar_init(bar(kBarVEmpty + s), 1);
       bar_init(bar(kBarSFull + s), 1);
       bar_init(bar(kBarPFull + s), kGroupWarps);
+      for (int k = 0; k < 3; ++k) bar_init(bar(kBarPPart + 3 * s + k), kGroupWarps);
       bar_init(bar(kBarMmaDone + s), 1);
     }
     st_shared_i32(abort_addr, 0);
@@ -262,21 +278,27 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         tc_commit(bar(kBarSFull + g));
         return true;
       };
-      // O_g += P_g(j) V_j once the softmax has published P_g(j)
+      // O_g += P_g(j) V_j, part by part as the softmax publishes P_g(j)
       auto pv = [&](int g, int j) {
         const int s = kv_stage(j);
         if (!bar_wait(bar(kBarVFull + s), kv_par(j), abort_addr, a.dev_status, wlim, kSusp)) return false;
-        if (!bar_wait(bar(kBarPFull + g), (uint32_t)j & 1u, abort_addr, a.dev_status, wlim, kSusp)) return false;
-        tc_fence_after();
         // V tile as B = [keys x dims], dims contiguous: 64-dim atoms one half
         // apart (LBO), 8-key groups 1 KB apart (SBO); 16 keys (2 KB) per step;
-        // P_g from TMEM: keys 16kk..16kk+15 are columns 8kk..8kk+7 of S_g
+        // P_g from TMEM: keys 16kk..16kk+15 are columns 8kk..8kk+7 of S_g.
+        // The steps of each part of P go out once the softmax has published
+        // that part.
         const uint64_t v_desc = sw128_desc(sV + 2u * (uint32_t)s * kHalf, kHalf, 1024);
         const uint32_t d_s = tmem + kColS + 128u * (uint32_t)g;
         const uint32_t d_o = tmem + kColO + 128u * (uint32_t)g;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          tc_mma_ts(d_o, d_s + 8u * kk, v_desc + (uint64_t)(kk * 2048 / 16), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        for (int h = 0; h < kPParts; ++h) {
+          const uint32_t pb = h + 1 < kPParts ? bar(kBarPPart + 3u * (uint32_t)g + (uint32_t)h) : bar(kBarPFull + g);
+          if (!bar_wait(pb, (uint32_t)j & 1u, abort_addr, a.dev_status, wlim, kSusp)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 2 * p_begin(h); kk < 2 * p_begin(h + 1); ++kk)
+            tc_mma_ts(d_o, d_s + 8u * kk, v_desc + (uint64_t)(kk * 2048 / 16), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        }
         return true;
       };
       for (int j = 0; j <= n_iter && ok; ++j) {
@@ -327,7 +349,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       const int jt = key_tile(j);
       if (!bar_wait(bar(kBarSFull + grp), (uint32_t)j & 1u, abort_addr, a.dev_status, wlim)) break;
       tc_fence_after();
-      if (!idle) {
       // the thread's whole S row, 32 columns (one TMEM load) at a time
       uint32_t sr[4][32];
       // mask (raw scores; the scale is folded into the exponent below)
@@ -401,43 +422,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const float nr = (ref == -INFINITY) ? 0.f : -ref;
         return f2_pack(nr, nr);
       };
-      bool move;
       float alpha = 1.f;
-#if KVATTN_PREFILL_TWO_PASS
-      {
-        // Two passes over TMEM, 32 columns at a time with the next chunk's
-        // load in flight: the row max, then the exponentials from a second
-        // load of each chunk (a TMEM reload is cheaper than keeping the whole
-        // 128-column row in registers).  P chunk c2 goes to columns
-        // 16c2 .. 16c2+15, which the second pass has already read.
-        uint32_t cb[2][32];
-        tmem_ld32(lane_addr + col_s, cb[0]);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c2 = 0; c2 < 4; ++c2) {
-          if (c2 < 3) tmem_ld32(lane_addr + col_s + 32u * (c2 + 1), cb[(c2 + 1) & 1]);
-          mask_regs(cb[c2 & 1], c2);
-          max_regs(cb[c2 & 1]);
-          if (c2 < 3) tmem_wait_ld();
-        }
-        const float mx = row_max();
-        move = mx > ref + 8.f;
-        const float ref_new = move ? mx : ref;
-        alpha = move ? fast_exp2(ref - ref_new) : 1.f;
-        ref = ref_new;
-        const uint64_t nr2 = neg_ref2();
-        tmem_ld32(lane_addr + col_s, cb[0]);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c2 = 0; c2 < 4; ++c2) {
-          if (c2 < 3) tmem_ld32(lane_addr + col_s + 32u * (c2 + 1), cb[(c2 + 1) & 1]);
-          mask_regs(cb[c2 & 1], c2);
-          exp_regs(cb[c2 & 1], c2, nr2);
-          if (c2 < 3) tmem_wait_ld();
-        }
-      }
-#else
-      {
+      uint64_t nr2 = 0ull;
+      if (!idle) {
         // load the row, take its max, then exponentiate
 #pragma unroll
         for (int c2 = 0; c2 < 4; ++c2) tmem_ld32(lane_addr + col_s + 32u * c2, sr[c2]);
@@ -448,33 +435,28 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           max_chunk(c2);
         }
         const float mx = row_max();
-        move = mx > ref + 8.f;
+        const bool move = mx > ref + 8.f;
         const float ref_new = move ? mx : ref;
         alpha = move ? fast_exp2(ref - ref_new) : 1.f;
         ref = ref_new;
-        const uint64_t nr2 = neg_ref2();
+        nr2 = neg_ref2();
+        // P of the first part's keys; then O's rescale, if the reference
+        // moved, before P_g(j) V_j adds to O (PV_g(j-1) has finished: QK_g(j)
+        // was issued after it)
 #pragma unroll
-        for (int c2 = 0; c2 < 4; ++c2) exp_chunk(c2, nr2);
-      }
-#endif
-      float sa, sb;
-      f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), sa, sb);
-      l = l * alpha + (sa + sb);
-
-      if (j > 0 && __any_sync(0xffffffffu, move)) {
-        // a row's reference moved: rescale its O (PV_g(j-1) has finished:
-        // QK_g(j) was issued after it)
+        for (int c2 = 0; c2 < p_begin(1); ++c2) exp_chunk(c2, nr2);
+        if (j > 0 && __any_sync(0xffffffffu, move)) {
 #pragma unroll
-        for (int c2 = 0; c2 < 4; ++c2) {
-          uint32_t r[32];
-          tmem_ld32(lane_addr + col_o + 32u * c2, r);
-          tmem_wait_ld();
+          for (int c2 = 0; c2 < 4; ++c2) {
+            uint32_t r[32];
+            tmem_ld32(lane_addr + col_o + 32u * c2, r);
+            tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
-          tmem_st32(lane_addr + col_o + 32u * c2, r);
+            for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
+            tmem_st32(lane_addr + col_o + 32u * c2, r);
+          }
         }
       }
-      }  // !idle
       if (j == n_all - 1 && Lmax < jt * kBN + kBN) {
         // rows of the last V tile past the last visible key may hold any bits;
         // zero them so that 0 * (garbage) cannot reach O (both Q tiles' groups
@@ -492,6 +474,24 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         // the zeroed rows, written through the generic proxy, before the
         // tensor cores read the stage (only this tile needs the fence)
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      }
+      // each part of P (the first with O's rescale) goes out as soon as it is
+      // in TMEM: the issuer runs P.V on it while the next part is computed
+#pragma unroll
+      for (int h = 1; h < kPParts; ++h) {
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) bar_arrive(bar(kBarPPart + 3 * grp + (h - 1)));
+        if (!idle) {
+#pragma unroll
+          for (int c2 = p_begin(h); c2 < p_begin(h + 1); ++c2) exp_chunk(c2, nr2);
+        }
+      }
+      if (!idle) {
+        float sa, sb;
+        f2_unpack(f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3])), sa, sb);
+        l = l * alpha + (sa + sb);
       }
       tmem_wait_st();
       tc_fence_before();
