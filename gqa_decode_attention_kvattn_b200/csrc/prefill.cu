@@ -393,13 +393,21 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       // packed sums in four accumulators; 32 keys (16 P columns) at a time,
       // written over the S columns already read
       uint64_t sum2[4] = {0ull, 0ull, 0ull, 0ull};
-      auto exp_regs = [&](const uint32_t (&r)[32], int c2, uint64_t nr2) {
-        uint32_t pk[16];
+      auto exp_regs = [&](uint32_t (&r)[32], int c2, uint64_t nr2) {
+        // in stages over the chunk's 16 pairs, each stage's steps independent
+        // of one another: the exponent arguments, the exponentials, then the
+        // sums and the bf16 packing (the scores are dead after the first)
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
           const uint64_t sv = ((uint64_t)r[c + 1] << 32) | r[c];
           float x0, x1;
           f2_unpack(f2_fma(sv, sc2, nr2), x0, x1);
+          r[c] = __float_as_uint(x0);
+          r[c + 1] = __float_as_uint(x1);
+        }
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          const float x0 = __uint_as_float(r[c]), x1 = __uint_as_float(r[c + 1]);
           float p0, p1;
           if (((c >> 1) & 3) < 4 - KVATTN_PREFILL_POLY_PAIRS) {
             p0 = fast_exp2(x0);
@@ -412,6 +420,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
               p1 = x1 == -INFINITY ? 0.f : p1;
             }
           }
+          r[c] = __float_as_uint(p0);
+          r[c + 1] = __float_as_uint(p1);
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          const float p0 = __uint_as_float(r[c]), p1 = __uint_as_float(r[c + 1]);
           sum2[(c >> 1) & 3] = f2_add(sum2[(c >> 1) & 3], f2_pack(p0, p1));
           pk[c >> 1] = pack_bf16x2_p(p0, p1);
         }
