@@ -14,7 +14,8 @@
 // one (b, t), so a small decode batch still spreads over the SMs, and for
 // many tokens a CTA takes a whole token.  The CTA builds the (cos,
 // sin) pairs of its position in shared memory, rotates its vectors' 64 slots
-// (coalesced 4-byte accesses in the interleaved full-width layout), and a CTA
+// (coalesced 16-byte accesses of four pairs in the interleaved full-width
+// layout, 2-byte accesses in the others), and a CTA
 // holding key vectors also copies those heads' value rows (16-byte
 // accesses).  The kernel moves B*T*(2H + 3Hkv)*256 bytes, a negligible share
 // of a decode step.
@@ -60,22 +61,28 @@ __global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(RopeAppendArg
   const int rp = tab.rotary_dim / 2;  // rotated pairs
   const bool full_meta = tab.layout == 0 && rp == kPairs;
 
-  // Each thread loads a batch of its words before it stores any: q_rot may be
+  // Each thread loads a batch of its chunks before it stores any: q_rot may be
   // q itself, so the compiler cannot move a load above an earlier store, and
-  // one word at a time would pay a full memory latency per word.  Every word
-  // is read and written by the same thread, so rotating in place is safe.  The
-  // first batch (the whole of a decode token's share) is loaded before the
-  // (cos, sin) table is built, so its latency overlaps the fp64 sincos.
-  constexpr int kBatch = 8;
+  // one chunk at a time would pay a full memory latency per chunk.  Every
+  // chunk is read and written by the same thread, so rotating in place is
+  // safe.  The first batch (the whole of a decode token's share) is loaded
+  // before the (cos, sin) table is built, so its latency overlaps the fp64
+  // sincos.  In the interleaved full-width layout a 16-byte chunk holds four
+  // whole pairs (a head vector is 16 chunks), so the addressing and the memory
+  // instructions are paid once per four pairs.
+  constexpr int kBatch = 4;
+  constexpr int kChunks = kHeadDim / 8;  // 16-byte chunks per head vector
   const int n_slots = nv * kPairs;
-  auto load_batch = [&](int base_idx, uint32_t (&w)[kBatch]) {
+  const int n_chunks = nv * kChunks;
+  auto load_batch = [&](int base_idx, uint4 (&w)[kBatch]) {
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       const int idx = base_idx + u * blockDim.x;
-      w[u] = idx < n_slots ? reinterpret_cast<const uint32_t*>(vec_in(v0 + idx / kPairs))[idx & (kPairs - 1)] : 0u;
+      w[u] = idx < n_chunks ? reinterpret_cast<const uint4*>(vec_in(v0 + idx / kChunks))[idx & (kChunks - 1)]
+                            : make_uint4(0u, 0u, 0u, 0u);
     }
   };
-  uint32_t w_first[kBatch];
+  uint4 w_first[kBatch];
   if (full_meta) load_batch(threadIdx.x, w_first);
   // values: bit copy of the 256-byte rows of this CTA's key heads, the first
   // batch of 16-byte chunks also in flight before the table
@@ -103,9 +110,10 @@ __global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(RopeAppendArg
   __syncthreads();
 
   if (full_meta) {
-    // Meta layout over the whole head: each pair is one 32-bit word
-    for (int base_idx = threadIdx.x; base_idx < n_slots; base_idx += blockDim.x * kBatch) {
-      uint32_t w[kBatch];
+    // Meta layout over the whole head: each pair is one 32-bit word, four
+    // pairs 4c .. 4c+3 per 16-byte chunk c of the head vector
+    for (int base_idx = threadIdx.x; base_idx < n_chunks; base_idx += blockDim.x * kBatch) {
+      uint4 w[kBatch];
       if (base_idx == (int)threadIdx.x) {
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) w[u] = w_first[u];
@@ -115,11 +123,18 @@ __global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(RopeAppendArg
 #pragma unroll
       for (int u = 0; u < kBatch; ++u) {
         const int idx = base_idx + u * blockDim.x;
-        if (idx < n_slots) {
-          const int i = idx & (kPairs - 1);
-          uint16_t y0, y1;
-          rope_rotate_bits(true, s_cos[i], s_sin[i], (uint16_t)(w[u] & 0xFFFFu), (uint16_t)(w[u] >> 16), y0, y1);
-          reinterpret_cast<uint32_t*>(vec_out(v0 + idx / kPairs))[i] = (uint32_t)y0 | ((uint32_t)y1 << 16);
+        if (idx < n_chunks) {
+          const int c = idx & (kChunks - 1);
+          const uint32_t in[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+          uint32_t o[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = 4 * c + e;
+            uint16_t y0, y1;
+            rope_rotate_bits(true, s_cos[i], s_sin[i], (uint16_t)(in[e] & 0xFFFFu), (uint16_t)(in[e] >> 16), y0, y1);
+            o[e] = (uint32_t)y0 | ((uint32_t)y1 << 16);
+          }
+          reinterpret_cast<uint4*>(vec_out(v0 + idx / kChunks))[c] = make_uint4(o[0], o[1], o[2], o[3]);
         }
       }
     }
