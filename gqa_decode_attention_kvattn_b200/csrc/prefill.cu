@@ -84,6 +84,8 @@ constexpr uint32_t kOffAbort = kOffTmemSlot + 8;
 constexpr uint32_t kPrefillSmemBytes = kOffAbort + 8 + 1024;  // + alignment slack
 static_assert(kPrefillSmemBytes <= 227 * 1024, "shared memory per CTA");
 
+// every wait of the producer and the MMA issuer polls without the suspend
+// hint (1), or those waits may suspend (0); measured within noise
 #ifndef KVATTN_PREFILL_SPIN_ALL
 #define KVATTN_PREFILL_SPIN_ALL 1
 #endif
