@@ -78,6 +78,12 @@ def test_decode_step_in_place_rotation():
     _check_step(12, 2, 1, 32, 8, 96, [5, 70], kv.LLAMA3, "decode", in_place=True)
 
 
+def test_prefill_step_in_place_rotation_whole_tokens():
+    # 600 tokens: rope_append gives each CTA a whole token (32 query and 8 key
+    # heads) and rotates q into itself in 16-byte chunks of four pairs
+    _check_step(14, 2, 300, 32, 8, 1024, [100, 500], kv.LLAMA3_1, "prefill", in_place=True)
+
+
 @pytest.mark.parametrize("hint", [0, 1500, 3000, 4096])
 def test_decode_split_sizes_agree(hint):
     # different hints give different split sizes; each must match the oracle
