@@ -122,7 +122,8 @@ extern "C" KVATTN_API int kvattn_decode_noalloc(const kvattn_dims* dims, const u
   if (!aligned16(q_rot) || !aligned16(cache_k) || !aligned16(cache_v) || !aligned16(out) ||
       (reinterpret_cast<uintptr_t>(start_pos) & 3u))
     return KVATTN_ERR_INVALID_ARG;
-  // the merge kernel's grid is (sequences, heads)
+  // the merge kernel's grid is (sequences, groups of four heads); the same
+  // limits as kvattn_decode
   if (dims->batch > (1 << 24) || dims->n_heads > 65535) return KVATTN_ERR_UNSUPPORTED;
   const int hint = max_kv_len_hint <= 0 ? dims->max_seq_len : max_kv_len_hint;
   if (hint > dims->max_seq_len || hint < 1) return KVATTN_ERR_OUT_OF_RANGE;

@@ -228,8 +228,9 @@ int run_attention(const kvattn_dims* dims, int32_t T, const uint16_t* q_rot, con
   if (hint > dims->max_seq_len || hint < T) return KVATTN_ERR_OUT_OF_RANGE;
   if (!(scale > 0.f)) scale = 1.0f / std::sqrt((float)kHeadDim);
   if (!std::isfinite(scale)) return KVATTN_ERR_INVALID_ARG;
-  // the merge kernel's grid is (row sets, heads): at most 2^24 row sets and
-  // 65535 heads, checked before anything is launched
+  // the merge kernel's grid is (row sets, groups of four heads): at most 2^24
+  // row sets; heads are capped at 65535 (the grid's y extent would allow
+  // four times more), checked before anything is launched
   if ((long long)dims->batch * T > (1LL << 24) || dims->n_heads > 65535) return KVATTN_ERR_UNSUPPORTED;
 
   int sms = 0;

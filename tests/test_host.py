@@ -166,10 +166,11 @@ def test_masked_entry_points_validate_the_mask(lib):
 
 
 def test_merge_grid_limits_refused_before_launch(lib):
-    # The split-K merge runs one CTA per (row set, head): row sets on the
-    # grid's x extent (B*T at most 2^24 here), heads on its y extent (at most
-    # 65535).  Larger calls are refused on the host, before the split kernel
-    # could be launched without the merge that clears its work counter.
+    # The split-K merge runs one CTA per (row set, four heads): row sets on the
+    # grid's x extent (B*T at most 2^24 here), head groups on its y extent
+    # (heads capped at 65535).  Larger calls are refused on the host, before
+    # the split kernel could be launched without the merge that clears its
+    # work counter.
     P = [FAKE] * 4
     big_b = _dims(batch=(1 << 24) + 1)
     assert lib.kvattn_decode(ctypes.byref(big_b), *P, 0, 0.0, FAKE, None, 0, None, None) == 2
