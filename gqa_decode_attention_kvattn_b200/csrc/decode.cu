@@ -1,8 +1,8 @@
 // K2 + K3: split-K grouped-query attention over the KV cache, on CUDA cores.
 //
 // What it computes ("Llama 3.1 8B KV cache", section "The cache itself is
-// concatenation"; "Llama 3.1 8B · Repeat heads"; the mask comment of model.py
-// 281-302 in "Llama 3 8B · KV cache"): for query token t of sequence b and
+// concatenation"; "Llama 3.1 8B · Repeat heads"; the comment in the "mask"
+// code excerpt of "Llama 3 8B · KV cache"): for query token t of sequence b and
 // query head h, with G = H / Hkv and j = floor(h / G),
 //   out[b,t,h,:] = sum_{r < L} softmax_r(scale * q[b,t,h,:] . K[b,r,j,:]) V[b,r,j,:]
 // over the L = start_pos[b] + t + 1 visible cache rows.

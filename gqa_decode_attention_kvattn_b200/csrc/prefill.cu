@@ -1,7 +1,7 @@
 // K4: chunked-prefill attention on the 5th-generation tensor cores (tcgen05,
 // accumulators in tensor memory).
 //
-// What it computes ("Llama 3 8B · KV cache", model.py 281-302 excerpt: the
+// What it computes ("Llama 3 8B · KV cache", its "mask" code excerpt: the
 // scores of T new tokens against cache_len + T keys, where entry (i, j) is
 // masked iff j > cache_len + i; softmax(q K^T / sqrt(d)) V of "Llama 3.1 8B KV
 // cache", section "The cache itself is concatenation"; KV head floor(h/G) of

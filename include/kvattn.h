@@ -2,8 +2,8 @@
  * kvattn.h -- C ABI of libkvattn.so: the cached grouped-query-attention step
  * of a Llama-3.1-style decoder on NVIDIA B200 (sm_100a).
  *
- * One call of the step, as "Llama 3 8B · KV cache" (model.py 160-177 and
- * 281-302 excerpts) and "Llama 3.1 8B KV cache" (sections "RoPE has to know
+ * One call of the step, as "Llama 3 8B · KV cache" (its "update" and
+ * "mask" code excerpts) and "Llama 3.1 8B KV cache" (sections "RoPE has to know
  * where it is" and "The cache itself is concatenation") describe it:
  *   1. rotate the new queries and keys with RoPE at absolute positions
  *      start_pos .. start_pos+T-1                    -> kvattn_rope_append
@@ -295,8 +295,8 @@ KVATTN_API size_t kvattn_prefill_workspace_bytes(const kvattn_dims* dims, int32_
 /* Step 3 for a chunk of T new tokens per sequence (chunked prefill into an
  * existing cache).  Row t of the chunk sits at position start_pos[b]+t and
  * sees cache rows 0 .. start_pos[b]+t: the rectangular causal mask whose only
- * masked entries are (t, r) with r > start_pos + t (comment in model.py
- * 281-302 of "Llama 3 8B · KV cache").
+ * masked entries are (t, r) with r > start_pos + t (comment in the
+ * "mask" code excerpt of "Llama 3 8B · KV cache").
  *   out[b,t,h,:] = sum_{r <= start_pos[b]+t} softmax_r(scale * q_rot[b,t,h,:] .
  *                  cache_k[b,r,floor(h/G),:]) * cache_v[b,r,floor(h/G),:]
  * q_rot and out are bf16 [B,T,H,d]; the chunk's rows must already be in the

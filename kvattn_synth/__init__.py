@@ -23,8 +23,8 @@ host, a CUDA kernel in ``synth.cu`` for large device-resident caches):
 The pages' workloads draw cache contents and new q/k/v i.i.d. N(0,1) in bf16
 and start positions uniform over an inclusive range; these helpers give
 exactly that.  Cache rows at or beyond a sequence's start position stay zero,
-as a freshly allocated cache would (Meta ``model.py`` allocates the cache with
-``torch.zeros``: "Llama 3 8B · KV cache", model.py 129-145 excerpt).
+as a freshly allocated cache would (the model allocates the cache with
+``torch.zeros``: "Llama 3 8B · KV cache", its "storage" code excerpt).
 """
 from __future__ import annotations
 

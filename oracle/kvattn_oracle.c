@@ -20,9 +20,9 @@
  *  2. Positions p = start_pos[b] + t: the past length is the offset, so the
  *     token after 4096 cached ones is rotated at angle 4097*f_i (same section
  *     of "Llama 3.1 8B KV cache"; freqs_cis[start_pos:start_pos+seqlen] in the
- *     model.py 281-302 excerpt of "Llama 3 8B · KV cache").
+ *     "mask" code excerpt of "Llama 3 8B · KV cache").
  *  3. Rotation of each pair of q and k by angle p*f_i, as the complex product
- *     (x_a + i x_b) e^{i p f_i}: Meta's apply_rotary_emb (model.py 160-177
+ *     (x_a + i x_b) e^{i p f_i}: Meta's apply_rotary_emb (the "update" code
  *     excerpt of "Llama 3 8B · KV cache"; its body is not printed;
  *     interleaved pairs (a, b) = (2i, 2i+1) and the counter-clockwise sense
  *     are the reading taken).  "The Modern Decoder Block" (module L7.3) also
@@ -32,16 +32,16 @@
  *     in fp64.
  *  4. Storage: q_rot and k_rot rounded to bf16 (round to nearest even), the
  *     cache dtype following the activations (cache.to(xq), bf16 default
- *     tensor type: "Llama 3 8B · KV cache", model.py 160-177 and
- *     generation.py 105-109 excerpts).  cache_k[b, p] <- k_rot,
+ *     tensor type: "Llama 3 8B · KV cache", its "update" and
+ *     "dtype" code excerpts).  cache_k[b, p] <- k_rot,
  *     cache_v[b, p] <- v_new; no other row changes (same page, KV-cache
  *     formulas and the write cache_k[:bsz, start_pos:start_pos+seqlen]).
  *  5. Attention for query token t of sequence b and query head h: KV head
  *     j = floor(h / G), G = H / Hkv ("Llama 3.1 8B · Repeat heads":
  *     K_G[h] = K_r[floor(h/4)]; "Grouped-query attention: a smaller KV cache",
  *     6:47).  Visible rows r = 0 .. start_pos[b] + t, the rectangular causal
- *     mask (entry (t, r) masked iff r > cache_len + t: comment in model.py
- *     281-302 of "Llama 3 8B · KV cache").  Scores s_r = q.K_r * scale,
+ *     mask (entry (t, r) masked iff r > cache_len + t: comment in the
+ *     "mask" code excerpt of "Llama 3 8B · KV cache").  Scores s_r = q.K_r * scale,
  *     scale = 1/sqrt(d); w = softmax(s) with the maximum subtracted;
  *     out = sum_r w_r V_r -- all in fp64 ("Llama 3.1 8B KV cache", section
  *     "The cache itself is concatenation").  The output is fp64, unrounded.
