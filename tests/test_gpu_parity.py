@@ -68,6 +68,12 @@ def _check_step(seed, B, T, H, Hkv, S, sp, rope, kind, hint=0, in_place=False):
     (40, 64, 2, 700, [0, 127, 128, 699] + [int(x) for x in np.random.RandomState(8).randint(0, 700, 36)],
      kv.LLAMA3_1),
     (2, 64, 1, 900, [899, 33], kv.LLAMA3_1),            # G = 64 (MQA, 64 heads)
+    # fewer than four query heads, or not a multiple of four: the merge runs
+    # four heads per CTA and its last CTA has heads to spare (long rows, so
+    # every sequence is split)
+    (3, 2, 1, 3000, [2999, 100, 1500], kv.LLAMA3),     # H = 2, G = 2
+    (2, 6, 3, 4000, [3999, 2000], kv.LLAMA3_1),        # H = 6, G = 2
+    (2, 1, 1, 5000, [4999, 64], kv.LLAMA3),            # H = 1 (one head)
 ])
 def test_decode_step_small(case):
     B, H, Hkv, S, sp, rope = case
